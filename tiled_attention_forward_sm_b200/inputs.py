@@ -1,0 +1,104 @@
+"""Seeded synthetic inputs for the attention forward pass.
+
+This module holds no attention arithmetic.  It only draws Q, K, V (and names
+the workloads); the CUDA path and the CPU oracle both take their inputs from
+here, so they see the same bf16 bits.
+
+Recipe: ``torch.Generator('cpu').manual_seed(seed)``; draw fp32 ``randn`` for
+Q, then K, then V, each [B, H, N, d]; multiply Q by ``q_std``; round to bf16
+(round to nearest even, torch's cast).
+"""
+from __future__ import annotations
+
+import math
+from dataclasses import dataclass
+
+import torch
+
+
+@dataclass(frozen=True)
+class Workload:
+    """One attention forward problem: shapes, mask, scale and input law."""
+    name: str
+    B: int
+    H: int
+    N: int
+    d: int
+    causal: bool
+    q_std: float
+    seed: int
+
+    @property
+    def scale(self) -> float:
+        return 1.0 / math.sqrt(self.d)
+
+    @property
+    def flops(self) -> float:
+        """Reported FLOPs: 4*B*H*N^2*d (two products of 2*N^2*d each per
+        head), halved under the causal mask."""
+        f = 4.0 * self.B * self.H * self.N * self.N * self.d
+        return f / 2.0 if self.causal else f
+
+    @property
+    def rows(self) -> int:
+        return self.B * self.H * self.N
+
+
+# The five workloads the attention forward is measured and checked on.
+WORKLOADS = {
+    w.name: w for w in [
+        Workload("b1h2n256d64", 1, 2, 256, 64, False, 1.0, 1001),
+        Workload("b4h16n2048d128_causal", 4, 16, 2048, 128, True, 1.0, 1002),
+        Workload("b2h32n8192d128_causal", 2, 32, 8192, 128, True, 1.0, 1003),
+        Workload("b8h16n4096d128_peaky", 8, 16, 4096, 128, False, 3.0, 1004),
+        Workload("b1h16n32768d128_causal", 1, 16, 32768, 128, True, 1.0, 1005),
+    ]
+}
+
+# The workload bench.py times by default: the largest causal d=128 case of
+# the sequence-length range the throughput target is stated for (N >= 8192).
+BENCH_WORKLOAD = "b2h32n8192d128_causal"
+
+
+def make_qkv(B: int, H: int, N: int, d: int, seed: int, q_std: float = 1.0):
+    """Return bf16 CPU tensors (q, k, v), each [B, H, N, d], contiguous."""
+    g = torch.Generator(device="cpu")
+    g.manual_seed(int(seed))
+    shape = (B, H, N, d)
+    q = torch.randn(shape, generator=g, dtype=torch.float32)
+    k = torch.randn(shape, generator=g, dtype=torch.float32)
+    v = torch.randn(shape, generator=g, dtype=torch.float32)
+    if q_std != 1.0:
+        q = q * q_std
+    return (q.to(torch.bfloat16).contiguous(), k.to(torch.bfloat16).contiguous(),
+            v.to(torch.bfloat16).contiguous())
+
+
+def make_workload_inputs(w: Workload):
+    return make_qkv(w.B, w.H, w.N, w.d, w.seed, w.q_std)
+
+
+def bf16_bits(t: torch.Tensor):
+    """bf16 tensor -> numpy uint16 array of its bit patterns (no copy of
+    values, just a reinterpretation)."""
+    assert t.dtype == torch.bfloat16
+    return t.contiguous().view(torch.int16).numpy().view("uint16")
+
+
+def sample_rows(w: Workload, n_random: int = 256, seed: int = 7):
+    """Deterministic row sample (flat indices (b*H+h)*N + i) for checking a
+    large workload: in every (b, h), the first and last 128 rows and both rows
+    at every 4th 128-row tile boundary; plus ``n_random`` seeded random rows
+    over the whole problem."""
+    import numpy as np
+    per_bh = set(range(min(128, w.N)))
+    per_bh.update(range(max(0, w.N - 128), w.N))
+    for t in range(0, w.N, 4 * 128):
+        for i in (t - 1, t):
+            if 0 <= i < w.N:
+                per_bh.add(i)
+    per_bh = np.array(sorted(per_bh), dtype=np.int64)
+    rows = [bh * w.N + per_bh for bh in range(w.B * w.H)]
+    rng = np.random.default_rng(seed)
+    rows.append(rng.integers(0, w.rows, size=n_random, dtype=np.int64))
+    return np.unique(np.concatenate(rows))
