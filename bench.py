@@ -1,0 +1,354 @@
+#!/usr/bin/env python
+"""Benchmark of the B200 attention forward pass.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl {b200,reference}]
+                    [--workload NAME]
+
+One step = one attention forward pass (the whole hot path: one kernel launch)
+over the workload's batch, inputs resident in HBM.  Prints ONE JSON line on
+rank 0.  Multi-GPU (under torchrun): every rank runs its own copy of the
+workload (independent batches, no collective on the data path, weak
+scaling); the time is the max over ranks.
+
+``--impl reference`` times the CPU oracle (fp64 plain definition) on the
+host cores instead, on bounded row samples of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from tiled_attention_forward_sm_b200.inputs import (BENCH_WORKLOAD, WORKLOADS,  # noqa: E402
+                                                    bf16_bits, make_workload_inputs)
+
+METRIC = "attention fwd TFLOPS (bf16, d=128) and % of B200 dense BF16 peak, 1 GPU"
+UNIT = "TFLOPS"
+FALLBACK_PEAK = {"bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "hbm_gbs": 6650.0}
+DATASHEET_BF16_TFLOPS = 2250.0
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "attn_fwd_traffic.json")
+KERNEL_SOURCES = [os.path.join(ROOT, "tiled_attention_forward_sm_b200", "csrc", f)
+                  for f in ("attn_fwd_kernel.cuh", "ptx.cuh", "attn_fwd.cu")]
+CLOCK_QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+
+def kernel_sha() -> str:
+    h = hashlib.sha256()
+    for p in KERNEL_SOURCES:
+        with open(p, "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAK), "fallback"
+
+
+def load_traffic(launch_rows_scale: float):
+    """dram read+write bytes per launch from the committed ncu summary, if it
+    was taken on the current kernel sources; else None."""
+    if not os.path.exists(TRAFFIC_FILE):
+        return None
+    with open(TRAFFIC_FILE) as f:
+        t = json.load(f)
+    if t.get("kernel_sha") != kernel_sha():
+        return None
+    return float(t["dram_bytes_per_launch"]) * launch_rows_scale / float(t.get("rows_scale", 1.0))
+
+
+# ----------------------------------------------------------------- clocks ---
+class ClockSampler:
+    """nvidia-smi sampling (200 ms) while the GPU is busy."""
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        out = os.path.join(ROOT, "gpurun_out") if os.path.isdir(os.path.join(ROOT, "gpurun_out")) else "/tmp"
+        self.path = os.path.join(out, f"clocks_rank{self.gpu}_{os.getpid()}.csv")
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={CLOCK_QUERY}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"],
+                    "samples": 0}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        smax = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i] == "Active"})
+        load = [s for s in sm if s > 0.5 * max(sm)] if sm else []
+        return {"sm_mhz": statistics.median(load) if load else None,
+                "sm_max_mhz": max(smax) if smax else None,
+                "reasons": reasons, "samples": len(rows),
+                "power_w_max": max((float(r[3]) for r in rows
+                                    if r[3].replace(".", "").isdigit()), default=None)}
+
+
+# ------------------------------------------------------------ distributed ---
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+# ---------------------------------------------------------- CPU baseline ---
+def oracle_sample_rows(w, n_rows: int, seed: int):
+    rng = np.random.default_rng(seed)
+    return np.sort(rng.choice(w.rows, size=min(n_rows, w.rows), replace=False)).astype(np.int64)
+
+
+def row_flops(w, rows) -> float:
+    """Metric FLOPs attributable to the listed rows: 4*d per visible key
+    (the 4*N^2*d total, halved under the mask, is the sum over rows)."""
+    i = rows % w.N
+    keys = (i + 1) if w.causal else np.full_like(i, w.N)
+    return float(4.0 * w.d * keys.astype(np.float64).sum())
+
+
+def time_oracle(w, bits, target_s: float, seed: int = 123):
+    """Run the oracle on growing seeded row batches until about target_s of
+    CPU work; return (TFLOPS, rows, seconds, threads)."""
+    import oracle  # CPU baseline leg only
+    qb, kb, vb = bits
+    total_rows, total_t, total_f = 0, 0.0, 0.0
+    batch = 1024
+    k = 0
+    while total_t < target_s and total_rows < w.rows:
+        rows = oracle_sample_rows(w, batch, seed + k)
+        t0 = time.perf_counter()
+        oracle.attn_ref(qb, kb, vb, w.causal, w.scale, rows=rows)
+        dt = time.perf_counter() - t0
+        total_t += dt
+        total_f += row_flops(w, rows)
+        total_rows += len(rows)
+        k += 1
+        if dt < 0.5 * target_s:
+            batch = min(batch * 2, 65536)
+    return total_f / total_t / 1e12, total_rows, total_t, oracle.max_threads()
+
+
+# ------------------------------------------------------------- GPU arm -----
+def run_b200(args, w):
+    import tiled_attention_forward_sm_b200 as tab
+    world, rank, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    pg = None
+    if world > 1:
+        import datetime
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=dev)
+        pg = True
+
+    q_h, k_h, v_h = make_workload_inputs(w)
+    q, k, v = (t.to(dev) for t in (q_h, k_h, v_h))
+    o = torch.empty_like(q)
+    lse = torch.empty((w.B, w.H, w.N), dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        tab.attn_fwd_into(q, k, v, o, lse, causal=w.causal, scale=w.scale, stream=stream)
+
+    sampler = ClockSampler(local)
+    sampler.start()
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    if pg:
+        torch.distributed.barrier()
+    torch.cuda.synchronize(dev)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    clocks = sampler.stop()
+    if pg:
+        torch.distributed.barrier()
+    ms_total = e0.elapsed_time(e1)
+    status = tab.last_device_error(stream)
+    if status != 0:
+        raise SystemExit(f"device status {status}: {tab.strerror(status)}")
+
+    # end to end: host buffers through the C ABI host entry point
+    q_p, k_p, v_p = (t.pin_memory() for t in (q_h, k_h, v_h))
+    o_p = torch.empty_like(q_p).pin_memory()
+    lse_p = torch.empty((w.B, w.H, w.N), dtype=torch.float32).pin_memory()
+    e2e_steps = max(1, min(args.steps, args.e2e_steps))
+    for _ in range(min(args.warmup, 3)):
+        tab.attn_fwd_host(q_p, k_p, v_p, o_p, lse_p, q, k, v, o, lse, w.causal, w.scale, stream)
+    if pg:
+        torch.distributed.barrier()
+    torch.cuda.synchronize(dev)
+    f0 = torch.cuda.Event(enable_timing=True)
+    f1 = torch.cuda.Event(enable_timing=True)
+    f0.record(stream)
+    for _ in range(e2e_steps):
+        tab.attn_fwd_host(q_p, k_p, v_p, o_p, lse_p, q, k, v, o, lse, w.causal, w.scale, stream)
+    f1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = f0.elapsed_time(f1) / e2e_steps
+
+    t = torch.tensor([ms_total, e2e_ms], dtype=torch.float64, device=dev)
+    if pg:
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    ms_total, e2e_ms = float(t[0]), float(t[1])
+    if pg:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+    if rank != 0:
+        return None
+
+    ms_step = ms_total / args.steps
+    value = world * w.flops / (ms_step * 1e-3) / 1e12
+    e2e_value = world * w.flops / (e2e_ms * 1e-3) / 1e12
+    peaks, peak_kind = load_peaks()
+    peak = float(peaks["bf16_tflops"])
+    achieved = w.flops / (ms_step * 1e-3) / 1e12  # per launch, this GPU
+    tb = w.rows * w.d * 2
+    traffic = load_traffic(1.0)
+    line = {
+        "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded N(0,1) bf16 Q/K/V, see inputs.py)",
+        "config": {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d,
+                   "causal": w.causal, "scale": w.scale, "q_std": w.q_std,
+                   "flops_per_step": w.flops,
+                   "l2": f"inputs larger than L2: Q+K+V {3 * tb / 1e6:.0f} MB vs 126 MB; no flush",
+                   "parallelism": f"replica x{world} (independent batches)"},
+        "roofline": {"bound": "tensor", "achieved": round(achieved, 2),
+                     "peak": peak, "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
+                     "peak_source": f"{peak_kind} bf16 burst (MEASURED_PEAKS.json)"
+                     if peak_kind == "measured" else "fallback 1.59 PFLOP/s",
+                     "frac_of_sustained": round(achieved / float(peaks.get(
+                         "bf16_tflops_sustained", FALLBACK_PEAK["bf16_tflops_sustained"])), 4),
+                     "frac_of_datasheet_2250": round(achieved / DATASHEET_BF16_TFLOPS, 4),
+                     "traffic": traffic,
+                     "algorithmic_bytes": 4 * tb + w.rows * 4},
+        "e2e": {"value": round(e2e_value, 2), "unit": UNIT,
+                "h2d_bytes_per_step": 3 * tb, "d2h_bytes_per_step": tb + w.rows * 4,
+                "steps": e2e_steps, "ms_per_step": round(e2e_ms, 4),
+                "api": "attn_fwd_host (pinned host buffers, copies in the timed region)"},
+        "gpu_launches": args.steps,
+        "clocks": clocks,
+        "kernel_sha": kernel_sha(),
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        bits = (bf16_bits(q_h), bf16_bits(k_h), bf16_bits(v_h))
+        tf, nrows, secs, cores = time_oracle(w, bits, args.cpu_seconds)
+        line["cpu_baseline"] = {
+            "value": round(tf, 6), "unit": UNIT, "cores": cores, "kind": "oracle",
+            "sample": f"{nrows} seeded random rows of {w.rows} ({secs:.1f} s); "
+                      "TFLOPS from the rows' exact share of the metric FLOPs"}
+    return line
+
+
+# ------------------------------------------------------- reference arm -----
+def run_reference(args, w):
+    world, rank, _ = dist_env()
+    if rank != 0:
+        return None
+    import oracle
+    q_h, k_h, v_h = make_workload_inputs(w)
+    bits = (bf16_bits(q_h), bf16_bits(k_h), bf16_bits(v_h))
+    qb, kb, vb = bits
+    # each step: a bounded row sample, sized so the whole run stays ~1 minute
+    t0 = time.perf_counter()
+    probe_rows = oracle_sample_rows(w, 256, 999)
+    oracle.attn_ref(qb, kb, vb, w.causal, w.scale, rows=probe_rows)
+    per_flop = (time.perf_counter() - t0) / row_flops(w, probe_rows)
+    budget = 60.0 / max(1, args.steps + args.warmup)
+    avg_row = row_flops(w, oracle_sample_rows(w, 4096, 5)) / 4096
+    n_rows = int(max(64, min(w.rows, budget / (per_flop * avg_row))))
+    for s in range(args.warmup):
+        oracle.attn_ref(qb, kb, vb, w.causal, w.scale, rows=oracle_sample_rows(w, n_rows, 10_000 + s))
+    flops, secs = 0.0, 0.0
+    for s in range(args.steps):
+        rows = oracle_sample_rows(w, n_rows, 20_000 + s)
+        t0 = time.perf_counter()
+        oracle.attn_ref(qb, kb, vb, w.causal, w.scale, rows=rows)
+        secs += time.perf_counter() - t0
+        flops += row_flops(w, rows)
+    value = flops / secs / 1e12
+    cores = oracle.max_threads()
+    return {
+        "impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": UNIT,
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(1e3 * secs / args.steps, 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d,
+                   "causal": w.causal, "scale": w.scale, "q_std": w.q_std},
+        "cpu_baseline": {"value": round(value, 6), "unit": UNIT, "cores": cores,
+                         "kind": "oracle",
+                         "sample": f"{n_rows} seeded random rows per step of {w.rows}"},
+        "e2e": {"value": round(value, 6), "unit": UNIT, "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+        "gpu_launches": 0,
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["b200", "reference"], default="b200")
+    ap.add_argument("--workload", default=BENCH_WORKLOAD, choices=sorted(WORKLOADS))
+    ap.add_argument("--e2e-steps", type=int, default=20)
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    w = WORKLOADS[args.workload]
+    line = run_reference(args, w) if args.impl == "reference" else run_b200(args, w)
+    if line is not None:
+        print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()

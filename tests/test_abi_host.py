@@ -1,0 +1,104 @@
+"""Host-side tests of the C ABI: the library loads without a GPU, exports
+every symbol include/attn_b200.h declares, and rejects bad arguments before
+any CUDA call."""
+import math
+import os
+import re
+
+import pytest
+
+import tiled_attention_forward_sm_b200 as tab
+from tiled_attention_forward_sm_b200 import build as tab_build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    tab_build.build()
+    return tab.library()
+
+
+def declared_symbols():
+    names = []
+    inc = os.path.join(ROOT, "include")
+    for fn in sorted(os.listdir(inc)):
+        if fn.endswith(".h"):
+            text = open(os.path.join(inc, fn)).read()
+            text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+            names += re.findall(r"\b(attn_[a-z0-9_]+)\s*\(", text)
+    return sorted(set(names))
+
+
+def test_header_declares_entry_points():
+    syms = declared_symbols()
+    for s in ["attn_fwd", "attn_fwd_host", "attn_last_device_error", "attn_strerror",
+              "attn_check_args", "attn_version"]:
+        assert s in syms
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for s in declared_symbols():
+        assert hasattr(lib, s), f"{s} declared in include/ but not exported"
+
+
+def test_strerror_and_version(lib):
+    assert tab.strerror(0) == "ok"
+    for code in (-1, -2, -3, -4, -5, -7, 12345):
+        assert isinstance(tab.strerror(code), str) and tab.strerror(code)
+    assert lib.attn_version() > 0
+
+
+A = 1 << 20  # a 16-byte aligned fake address; check_args never dereferences
+
+
+def ptrs(d=128, B=1, H=1, N=128):
+    tb = B * H * N * d * 2
+    return [A, A + tb, A + 2 * tb, A + 3 * tb, A + 4 * tb]
+
+
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("N", [128, 256, 384, 32768])
+def test_check_args_accepts_supported(lib, d, N):
+    assert tab.check_args(*ptrs(d, 2, 3, N), 2, 3, N, d, 1 / math.sqrt(d)) == 0
+
+
+def test_check_args_rejections(lib):
+    p = ptrs()
+    assert tab.check_args(0, *p[1:], 1, 1, 128, 128, 0.1) == -1        # null q
+    assert tab.check_args(*p[:4], 0, 1, 1, 128, 128, 0.1) == -1        # null lse
+    assert tab.check_args(*p, 0, 1, 128, 128, 0.1) == -1               # B = 0
+    assert tab.check_args(*p, 1, -1, 128, 128, 0.1) == -1              # H < 0
+    assert tab.check_args(*p, 1, 1, 0, 128, 0.1) == -1                 # N = 0
+    assert tab.check_args(*p, 1, 1, 128, 128, 0.0) == -1               # scale 0
+    assert tab.check_args(*p, 1, 1, 128, 128, -1.0) == -1              # scale < 0
+    assert tab.check_args(*p, 1, 1, 128, 128, float("nan")) == -1
+    assert tab.check_args(*p, 1, 1, 128, 128, float("inf")) == -1
+    assert tab.check_args(*p, 1, 1, 128, 96, 0.1) == -2                # d unsupported
+    assert tab.check_args(*p, 1, 1, 100, 128, 0.1) == -2               # N % 128
+    assert tab.check_args(*p, 1 << 12, 1 << 12, 1 << 8, 128, 0.1) == -2  # rows >= 2^31
+    q, k, v, o, l = p
+    assert tab.check_args(q + 8, k, v, o, l, 1, 1, 128, 128, 0.1) == -3   # misaligned q
+    assert tab.check_args(q, k, v, o + 2, l, 1, 1, 128, 128, 0.1) == -3   # misaligned o
+    assert tab.check_args(q, k, v, o, l + 2, 1, 1, 128, 128, 0.1) == -3   # misaligned lse
+    assert tab.check_args(q, k, v, q, l, 1, 1, 128, 128, 0.1) == -1       # o aliases q
+    assert tab.check_args(q, k, v, o, v + 64, 1, 1, 128, 128, 0.1) == -1  # lse inside v
+    assert tab.check_args(q, q, q, o, l, 1, 1, 128, 128, 0.1) == 0        # inputs may alias
+
+
+def test_binding_rejects_cpu_tensors(lib):
+    import torch
+    x = torch.zeros(1, 1, 128, 128, dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        tab.attn_fwd(x, x, x)
+
+
+def test_product_does_not_import_oracle():
+    """The product package never imports or names the oracle."""
+    pkg = os.path.join(ROOT, "tiled_attention_forward_sm_b200")
+    for dirpath, _, files in os.walk(pkg):
+        for fn in files:
+            if fn.endswith((".py", ".cu", ".cuh", ".h")):
+                text = open(os.path.join(dirpath, fn)).read()
+                assert not re.search(r"^\s*(import|from)\s+oracle\b", text, re.M), fn
+                assert "attn_ref" not in text and "libattn_ref" not in text, fn

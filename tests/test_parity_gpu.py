@@ -1,0 +1,141 @@
+"""GPU parity: the CUDA path (through the C ABI) against the fp64 oracle on
+the same seeded bf16 inputs.
+
+Tolerance (bf16 I/O, fp32 accumulation): |O_gpu - O_ref| <= 2e-2 + 1e-2 |O_ref|
+elementwise and |LSE_gpu - LSE_ref| <= 1e-3.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import tiled_attention_forward_sm_b200 as tab
+from tiled_attention_forward_sm_b200.inputs import (WORKLOADS, bf16_bits, make_qkv,
+                                                    make_workload_inputs, sample_rows)
+
+pytestmark = pytest.mark.gpu
+
+ATOL_O, RTOL_O, ATOL_LSE = 2e-2, 1e-2, 1e-3
+
+
+def gpu_run(q, k, v, causal, scale):
+    qd, kd, vd = (t.cuda() for t in (q, k, v))
+    o, lse = tab.attn_fwd(qd, kd, vd, causal=causal, scale=scale)
+    assert tab.last_device_error() == 0
+    return o.float().cpu().numpy().astype(np.float64), lse.cpu().numpy().astype(np.float64)
+
+
+def check(o_gpu, lse_gpu, o_ref, lse_ref, what=""):
+    assert np.isfinite(o_gpu).all() and np.isfinite(lse_gpu).all(), what
+    err_o = np.abs(o_gpu - o_ref)
+    bad = err_o > ATOL_O + RTOL_O * np.abs(o_ref)
+    assert not bad.any(), f"{what}: {bad.sum()} O elements out of tolerance, max err {err_o.max():.3g}"
+    err_l = np.abs(lse_gpu - lse_ref)
+    assert err_l.max() <= ATOL_LSE, f"{what}: LSE max err {err_l.max():.3g}"
+    return err_o.max(), err_l.max()
+
+
+def full_parity(oracle_mod, B, H, N, d, causal, seed, q_std=1.0, scale=None):
+    scale = 1 / math.sqrt(d) if scale is None else scale
+    q, k, v = make_qkv(B, H, N, d, seed, q_std)
+    o, lse = gpu_run(q, k, v, causal, scale)
+    o_ref, lse_ref = oracle_mod.attn_ref(bf16_bits(q), bf16_bits(k), bf16_bits(v), causal, scale)
+    return check(o, lse, o_ref, lse_ref, f"B{B} H{H} N{N} d{d} causal={causal}")
+
+
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("N", [128, 256, 384, 640])
+def test_small_shapes(oracle_mod, d, causal, N):
+    """Single tile, one pair, an odd number of 128-row tiles (a CTA with one
+    Q tile), several K/V tiles with a ragged pair count."""
+    full_parity(oracle_mod, 2, 3, N, d, causal, seed=N + d + causal)
+
+
+@pytest.mark.parametrize("name", ["b1h2n256d64", "b4h16n2048d128_causal"])
+def test_workload_full(oracle_mod, name):
+    w = WORKLOADS[name]
+    full_parity(oracle_mod, w.B, w.H, w.N, w.d, w.causal, w.seed, w.q_std)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_peaky_scores_exercise_lazy_rescale(oracle_mod, causal):
+    """Q ~ 3 N(0,1): the running maximum jumps often; several K/V tiles."""
+    full_parity(oracle_mod, 1, 4, 1024, 128, causal, seed=77, q_std=3.0)
+
+
+@pytest.mark.parametrize("scale", [0.01, 0.5, 2.0])
+def test_other_scales(oracle_mod, scale):
+    full_parity(oracle_mod, 1, 2, 512, 128, True, seed=5, scale=scale)
+
+
+def test_large_magnitude_scores(oracle_mod):
+    """Scores spanning ~+-200 (log2 units): weights underflow to exactly 0
+    for all but a few keys; no overflow, LSE still exact."""
+    full_parity(oracle_mod, 1, 2, 512, 64, False, seed=6, q_std=8.0, scale=0.5)
+
+
+@pytest.mark.parametrize("name", ["b2h32n8192d128_causal", "b8h16n4096d128_peaky",
+                                  "b1h16n32768d128_causal"])
+def test_workload_sampled_rows(oracle_mod, name):
+    """Full-size workloads in the launch configuration the benchmark uses;
+    the oracle computes a deterministic row sample (first/last 128 rows of
+    every head, rows at every 4th tile boundary, 256 random rows)."""
+    w = WORKLOADS[name]
+    q, k, v = make_workload_inputs(w)
+    o, lse = gpu_run(q, k, v, w.causal, w.scale)
+    rows = sample_rows(w, n_random=256)
+    if w.N >= 32768:
+        rows = rows[rows % w.N >= w.N - 256]  # keep the oracle to seconds: last rows
+        rows = np.concatenate([rows, np.arange(0, 128, dtype=np.int64)])
+    o_ref, lse_ref = oracle_mod.attn_ref(bf16_bits(q), bf16_bits(k), bf16_bits(v), w.causal,
+                                         w.scale, rows=rows)
+    check(o.reshape(-1, w.d)[rows], lse.reshape(-1)[rows], o_ref, lse_ref, name)
+
+
+def test_deterministic_bitwise():
+    q, k, v = (t.cuda() for t in make_qkv(2, 4, 1024, 128, 9))
+    o1, l1 = tab.attn_fwd(q, k, v, causal=True)
+    for _ in range(5):
+        o2, l2 = tab.attn_fwd(q, k, v, causal=True)
+        assert torch.equal(o1, o2) and torch.equal(l1, l2)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_every_output_written_and_guards_intact(causal):
+    """O and LSE pre-filled with NaN inside guard bands: every element is
+    written and no guard byte changes."""
+    B, H, N, d = 1, 3, 384, 128
+    q, k, v = (t.cuda() for t in make_qkv(B, H, N, d, 10))
+    g = 4096
+    o_buf = torch.full((g + B * H * N * d + g,), float("nan"), dtype=torch.bfloat16, device="cuda")
+    l_buf = torch.full((g + B * H * N + g,), float("nan"), dtype=torch.float32, device="cuda")
+    o = o_buf[g:g + B * H * N * d].view(B, H, N, d)
+    lse = l_buf[g:g + B * H * N].view(B, H, N)
+    tab.attn_fwd_into(q, k, v, o, lse, causal=causal)
+    assert tab.last_device_error() == 0
+    assert torch.isfinite(o).all() and torch.isfinite(lse).all()
+    assert torch.isnan(o_buf[:g]).all() and torch.isnan(o_buf[-g:]).all()
+    assert torch.isnan(l_buf[:g]).all() and torch.isnan(l_buf[-g:]).all()
+
+
+def test_host_entry_point_matches_device_entry_point():
+    B, H, N, d = 1, 2, 512, 128
+    q, k, v = make_qkv(B, H, N, d, 12)
+    qd, kd, vd = (t.cuda() for t in (q, k, v))
+    o_ref, l_ref = tab.attn_fwd(qd, kd, vd, causal=True)
+    qh, kh, vh = (t.pin_memory() for t in (q, k, v))
+    oh = torch.empty_like(qh).pin_memory()
+    lh = torch.empty((B, H, N), dtype=torch.float32).pin_memory()
+    od = torch.empty_like(qd); ld = torch.empty((B, H, N), dtype=torch.float32, device="cuda")
+    tab.attn_fwd_host(qh, kh, vh, oh, lh, qd, kd, vd, od, ld, causal=True)
+    assert torch.equal(oh, o_ref.cpu()) and torch.equal(lh, l_ref.cpu())
+
+
+def test_rejected_arguments_launch_nothing():
+    q = torch.zeros(1, 1, 100, 128, dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(tab.AttnError) as e:
+        tab.attn_fwd(q, q, q)
+    assert e.value.status == -2
+    assert tab.last_device_error() == 0

@@ -1,0 +1,15 @@
+"""B200 (sm_100a) dense attention forward: O = softmax(scale Q K^T [causal]) V.
+
+Thin Python binding over the C ABI in ``include/attn_b200.h``: it marshals
+torch tensors into pointers and sizes and raises on a non-zero status.  Every
+step of the computation runs in the CUDA kernels of ``libattn_b200.so``;
+there is no CPU or PyTorch fallback: without the library or an sm_100 device
+the calls raise.
+"""
+from __future__ import annotations
+
+from ._abi import (ATTN_OK, AttnError, attn_fwd, attn_fwd_host, attn_fwd_into,
+                   check_args, last_device_error, library, library_path, strerror)
+
+__all__ = ["ATTN_OK", "AttnError", "attn_fwd", "attn_fwd_into", "attn_fwd_host",
+           "check_args", "last_device_error", "library", "library_path", "strerror"]

@@ -1,0 +1,129 @@
+"""ctypes binding of ``libattn_b200.so`` (see ``include/attn_b200.h``).
+
+Argument marshalling only.  The library is loaded on first use; if it is
+missing the call raises (run ``python -m tiled_attention_forward_sm_b200.build``).
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+
+import torch
+
+from .build import LIB
+
+ATTN_OK = 0
+_lib = None
+
+
+class AttnError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        super().__init__(f"{what}: {strerror(status)} (status {status})")
+        self.status = status
+
+
+def library_path() -> str:
+    return LIB
+
+
+def library():
+    """Load (once) and return the ctypes handle of the CUDA library."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB):
+            raise RuntimeError(
+                f"CUDA library {LIB} not built; run python -m tiled_attention_forward_sm_b200.build")
+        lib = ctypes.CDLL(LIB)
+        vp, i, f = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
+        lib.attn_fwd.restype = i
+        lib.attn_fwd.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, f, vp]
+        lib.attn_fwd_host.restype = i
+        lib.attn_fwd_host.argtypes = [vp] * 10 + [i, i, i, i, i, f, vp]
+        lib.attn_last_device_error.restype = i
+        lib.attn_last_device_error.argtypes = [vp]
+        lib.attn_strerror.restype = ctypes.c_char_p
+        lib.attn_strerror.argtypes = [i]
+        lib.attn_check_args.restype = i
+        lib.attn_check_args.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, f]
+        lib.attn_version.restype = i
+        lib.attn_version.argtypes = []
+        _lib = lib
+    return _lib
+
+
+def strerror(status: int) -> str:
+    return library().attn_strerror(int(status)).decode()
+
+
+def check_args(q_ptr: int, k_ptr: int, v_ptr: int, o_ptr: int, lse_ptr: int,
+               B: int, H: int, N: int, d: int, scale: float) -> int:
+    """The library's precondition check on raw pointer values (no CUDA call)."""
+    return library().attn_check_args(q_ptr, k_ptr, v_ptr, o_ptr, lse_ptr, B, H, N, d, scale)
+
+
+def _stream_handle(stream) -> int:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return int(stream.cuda_stream) if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def _shape(q: torch.Tensor):
+    if q.dim() != 4:
+        raise ValueError("q, k, v must be [B, H, N, d]")
+    return tuple(int(x) for x in q.shape)
+
+
+def attn_fwd_into(q, k, v, o, lse, causal: bool = False, scale: float | None = None,
+                  stream=None) -> None:
+    """Enqueue the forward pass writing into ``o`` (bf16 [B,H,N,d]) and ``lse``
+    (fp32 [B,H,N]).  Inputs: CUDA bf16 contiguous [B,H,N,d] tensors."""
+    B, H, N, d = _shape(q)
+    for name, t, dt in (("q", q, torch.bfloat16), ("k", k, torch.bfloat16),
+                        ("v", v, torch.bfloat16), ("o", o, torch.bfloat16)):
+        if not t.is_cuda or t.dtype != dt or not t.is_contiguous() or tuple(t.shape) != (B, H, N, d):
+            raise ValueError(f"{name} must be a contiguous CUDA bf16 tensor of shape {(B, H, N, d)}")
+    if not lse.is_cuda or lse.dtype != torch.float32 or not lse.is_contiguous() or \
+            tuple(lse.shape) != (B, H, N):
+        raise ValueError(f"lse must be a contiguous CUDA fp32 tensor of shape {(B, H, N)}")
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    rc = library().attn_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
+                            lse.data_ptr(), B, H, N, d, int(bool(causal)), float(scale),
+                            _stream_handle(stream))
+    if rc != ATTN_OK:
+        raise AttnError(rc, "attn_fwd")
+
+
+def attn_fwd(q, k, v, causal: bool = False, scale: float | None = None, stream=None):
+    """Return ``(o, lse)`` for CUDA bf16 [B,H,N,d] inputs (enqueued on the
+    current or given stream)."""
+    B, H, N, d = _shape(q)
+    o = torch.empty_like(q)
+    lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
+    attn_fwd_into(q, k, v, o, lse, causal, scale, stream)
+    return o, lse
+
+
+def attn_fwd_host(q_h, k_h, v_h, o_h, lse_h, q_d, k_d, v_d, o_d, lse_d,
+                  causal: bool = False, scale: float | None = None, stream=None) -> None:
+    """Forward pass on HOST tensors through the C ABI's host entry point:
+    copies in, computes, copies out, and synchronises the stream.  The
+    ``*_d`` tensors are the caller's device buffers of the same shapes."""
+    B, H, N, d = _shape(q_h)
+    for t in (q_h, k_h, v_h, o_h, lse_h):
+        if t.is_cuda or not t.is_contiguous():
+            raise ValueError("host tensors must be contiguous CPU tensors")
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    rc = library().attn_fwd_host(
+        q_h.data_ptr(), k_h.data_ptr(), v_h.data_ptr(), o_h.data_ptr(), lse_h.data_ptr(),
+        q_d.data_ptr(), k_d.data_ptr(), v_d.data_ptr(), o_d.data_ptr(), lse_d.data_ptr(),
+        B, H, N, d, int(bool(causal)), float(scale), _stream_handle(stream))
+    if rc != ATTN_OK:
+        raise AttnError(rc, "attn_fwd_host")
+
+
+def last_device_error(stream=None) -> int:
+    """Synchronise the stream and return (and clear) the device status word."""
+    return int(library().attn_last_device_error(_stream_handle(stream)))

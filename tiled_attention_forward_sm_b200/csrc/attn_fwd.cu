@@ -1,0 +1,239 @@
+// C-ABI launcher for the sm_100a attention forward kernel: argument checks,
+// TMA tensor maps, launch configuration and the device status word.
+//
+// The operation and the ABI contract are documented in include/attn_b200.h.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "attn_b200.h"
+#include "attn_fwd_kernel.cuh"
+
+namespace attn_b200 {
+
+// Written (first error wins) by kernels whose bounded waits ran out.
+__device__ int g_attn_status = 0;
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+
+struct DeviceState {
+  bool checked = false;
+  bool usable = false;
+  int* status = nullptr;  // device address of g_attn_status
+  int num_sms = 0;
+};
+
+std::mutex g_mu;
+DeviceState g_dev[kMaxDevices];
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+
+// Per-device one-time set-up: capability check and the status word address.
+int device_state(DeviceState** out) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+    cudaGetLastError();
+    return ATTN_ERR_NO_DEVICE;
+  }
+  std::lock_guard<std::mutex> lock(g_mu);
+  DeviceState& st = g_dev[dev];
+  if (!st.checked) {
+    int major = 0, minor = 0, sms = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+      cudaGetLastError();
+      return ATTN_ERR_NO_DEVICE;
+    }
+    st.usable = (major == 10 && minor == 0);
+    st.num_sms = sms;
+    if (st.usable) {
+      void* p = nullptr;
+      if (cudaGetSymbolAddress(&p, g_attn_status) != cudaSuccess) {
+        cudaGetLastError();
+        return ATTN_ERR_CUDA;
+      }
+      st.status = static_cast<int*>(p);
+    }
+    if (!g_encode) {
+      cudaDriverEntryPointQueryResult q;
+      void* fn = nullptr;
+      if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) !=
+              cudaSuccess ||
+          q != cudaDriverEntryPointSuccess || fn == nullptr) {
+        cudaGetLastError();
+        return ATTN_ERR_CUDA;
+      }
+      g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+    }
+    st.checked = true;
+  }
+  if (!st.usable) return ATTN_ERR_NO_DEVICE;
+  *out = &st;
+  return ATTN_OK;
+}
+
+// 2-D view [rows, d] of a [B,H,N,d] bf16 tensor; 128-row x 64-column boxes
+// with the 128-byte swizzle the tcgen05 shared-memory descriptors expect.
+int make_tmap(CUtensorMap* m, const void* ptr, uint64_t rows, int d) {
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(d) * 2};
+  cuuint32_t box[2] = {64, 128};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims,
+                        strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+bool ranges_overlap(const void* a, size_t na, const void* b, size_t nb) {
+  const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
+  return x < y + nb && y < x + na;
+}
+
+template <int D, bool CAUSAL>
+int launch(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
+           int N, float scale, cudaStream_t stream, const DeviceState& st) {
+  using C = Config<D>;
+  const uint64_t rows = static_cast<uint64_t>(B) * H * N;
+  CUtensorMap tq, tk, tv;
+  if (make_tmap(&tq, q, rows, D) || make_tmap(&tk, k, rows, D) || make_tmap(&tv, v, rows, D))
+    return ATTN_ERR_CUDA;
+
+  KernelArgs args;
+  args.o = static_cast<__nv_bfloat16*>(o);
+  args.lse = lse;
+  args.N = N;
+  args.n_qtiles = N / kBlockM;
+  args.n_qpairs = (args.n_qtiles + 1) / 2;
+  args.scale_log2 = scale * 1.4426950408889634f;
+  args.status = st.status;
+
+  auto kern = attn_fwd_kernel<D, CAUSAL>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes) !=
+      cudaSuccess) {
+    cudaGetLastError();
+    return ATTN_ERR_CUDA;
+  }
+  cudaLaunchConfig_t cfg;
+  std::memset(&cfg, 0, sizeof cfg);
+  cfg.gridDim = dim3(static_cast<unsigned>(B * H), static_cast<unsigned>(args.n_qpairs), 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = C::kSmemBytes;
+  cfg.stream = stream;
+  if (cudaLaunchKernelEx(&cfg, kern, tq, tk, tv, args) != cudaSuccess) {
+    cudaGetLastError();
+    return ATTN_ERR_CUDA;
+  }
+  return ATTN_OK;
+}
+
+}  // namespace
+}  // namespace attn_b200
+
+using namespace attn_b200;
+
+extern "C" int attn_check_args(const void* q, const void* k, const void* v, const void* o,
+                               const float* lse, int B, int H, int N, int d, float scale) {
+  if (!q || !k || !v || !o || !lse) return ATTN_ERR_INVALID_ARG;
+  if (B <= 0 || H <= 0 || N <= 0) return ATTN_ERR_INVALID_ARG;
+  if (!std::isfinite(scale) || !(scale > 0.f)) return ATTN_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
+  if (N % kBlockM != 0) return ATTN_ERR_UNSUPPORTED;
+  const uint64_t rows = static_cast<uint64_t>(B) * H * N;
+  if (rows >= (1ull << 31) || static_cast<uint64_t>(B) * H > 0x7FFFFFFFull ||
+      N / (2 * kBlockM) + 1 > 65535)
+    return ATTN_ERR_UNSUPPORTED;
+  const uintptr_t al = reinterpret_cast<uintptr_t>(q) | reinterpret_cast<uintptr_t>(k) |
+                       reinterpret_cast<uintptr_t>(v) | reinterpret_cast<uintptr_t>(o);
+  if (al & 15u) return ATTN_ERR_MISALIGNED;
+  if (reinterpret_cast<uintptr_t>(lse) & 3u) return ATTN_ERR_MISALIGNED;
+  const size_t tb = rows * static_cast<size_t>(d) * 2, lb = rows * 4;
+  if (ranges_overlap(o, tb, q, tb) || ranges_overlap(o, tb, k, tb) ||
+      ranges_overlap(o, tb, v, tb) || ranges_overlap(lse, lb, q, tb) ||
+      ranges_overlap(lse, lb, k, tb) || ranges_overlap(lse, lb, v, tb) ||
+      ranges_overlap(lse, lb, o, tb))
+    return ATTN_ERR_INVALID_ARG;
+  return ATTN_OK;
+}
+
+extern "C" int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B,
+                        int H, int N, int d, int causal, float scale, attn_stream_t stream) {
+  int rc = attn_check_args(q, k, v, o, lse, B, H, N, d, scale);
+  if (rc != ATTN_OK) return rc;
+  DeviceState* st = nullptr;
+  rc = device_state(&st);
+  if (rc != ATTN_OK) return rc;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (d == 128)
+    return causal ? launch<128, true>(q, k, v, o, lse, B, H, N, scale, s, *st)
+                  : launch<128, false>(q, k, v, o, lse, B, H, N, scale, s, *st);
+  return causal ? launch<64, true>(q, k, v, o, lse, B, H, N, scale, s, *st)
+                : launch<64, false>(q, k, v, o, lse, B, H, N, scale, s, *st);
+}
+
+extern "C" int attn_last_device_error(attn_stream_t stream) {
+  DeviceState* st = nullptr;
+  int rc = device_state(&st);
+  if (rc != ATTN_OK) return rc;
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) {
+    cudaGetLastError();
+    return ATTN_ERR_CUDA;
+  }
+  int val = 0;
+  const int zero = 0;
+  if (cudaMemcpyFromSymbol(&val, g_attn_status, sizeof(int)) != cudaSuccess ||
+      cudaMemcpyToSymbol(g_attn_status, &zero, sizeof(int)) != cudaSuccess) {
+    cudaGetLastError();
+    return ATTN_ERR_CUDA;
+  }
+  return val;
+}
+
+extern "C" int attn_fwd_host(const void* q_h, const void* k_h, const void* v_h, void* o_h,
+                             float* lse_h, void* q_d, void* k_d, void* v_d, void* o_d,
+                             float* lse_d, int B, int H, int N, int d, int causal, float scale,
+                             attn_stream_t stream) {
+  if (!q_h || !k_h || !v_h || !o_h || !lse_h) return ATTN_ERR_INVALID_ARG;
+  int rc = attn_check_args(q_d, k_d, v_d, o_d, lse_d, B, H, N, d, scale);
+  if (rc != ATTN_OK) return rc;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const size_t rows = static_cast<size_t>(B) * H * N;
+  const size_t tb = rows * static_cast<size_t>(d) * 2;
+  if (cudaMemcpyAsync(q_d, q_h, tb, cudaMemcpyHostToDevice, s) != cudaSuccess ||
+      cudaMemcpyAsync(k_d, k_h, tb, cudaMemcpyHostToDevice, s) != cudaSuccess ||
+      cudaMemcpyAsync(v_d, v_h, tb, cudaMemcpyHostToDevice, s) != cudaSuccess) {
+    cudaGetLastError();
+    return ATTN_ERR_CUDA;
+  }
+  rc = attn_fwd(q_d, k_d, v_d, o_d, lse_d, B, H, N, d, causal, scale, stream);
+  if (rc != ATTN_OK) return rc;
+  if (cudaMemcpyAsync(o_h, o_d, tb, cudaMemcpyDeviceToHost, s) != cudaSuccess ||
+      cudaMemcpyAsync(lse_h, lse_d, rows * 4, cudaMemcpyDeviceToHost, s) != cudaSuccess) {
+    cudaGetLastError();
+    return ATTN_ERR_CUDA;
+  }
+  return attn_last_device_error(stream);
+}
+
+extern "C" const char* attn_strerror(int status) {
+  switch (status) {
+    case ATTN_OK: return "ok";
+    case ATTN_ERR_INVALID_ARG: return "invalid argument";
+    case ATTN_ERR_UNSUPPORTED: return "unsupported shape (d must be 64 or 128, N a multiple of 128)";
+    case ATTN_ERR_MISALIGNED: return "misaligned pointer (q, k, v, o need 16 bytes, lse 4)";
+    case ATTN_ERR_CUDA: return "CUDA call failed";
+    case ATTN_ERR_DEVICE_TIMEOUT: return "device-side wait timed out";
+    case ATTN_ERR_NO_DEVICE: return "no usable sm_100 device";
+    default: return "unknown status";
+  }
+}
+
+extern "C" int attn_version(void) { return (0 << 16) | (1 << 8) | 0; }
