@@ -38,7 +38,7 @@ METRIC = "attention fwd TFLOPS (bf16, d=128) and % of B200 dense BF16 peak, 1 GP
 UNIT = "TFLOPS"
 FALLBACK_PEAK = {"bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "hbm_gbs": 6650.0}
 DATASHEET_BF16_TFLOPS = 2250.0
-TRAFFIC_FILE = os.path.join(ROOT, "profiles", "attn_fwd_traffic.json")
+PROFILE_FILE = os.path.join(ROOT, "profiles", "attn_fwd_b2h32n8192d128_causal.txt")
 KERNEL_SOURCES = [os.path.join(ROOT, "tiled_attention_forward_sm_b200", "csrc", f)
                   for f in ("attn_fwd_kernel.cuh", "ptx.cuh", "attn_fwd.cu")]
 CLOCK_QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
@@ -63,24 +63,31 @@ def load_peaks():
     return dict(FALLBACK_PEAK), "fallback"
 
 
-def load_traffic(launch_rows_scale: float):
-    """dram read+write bytes per launch from the committed ncu summary, if it
-    was taken on the current kernel sources; else None."""
-    if not os.path.exists(TRAFFIC_FILE):
+def load_traffic(workload_name: str):
+    """dram read+write bytes per launch from the committed ncu summary of the
+    bench workload, if it was taken on the current kernel sources; else None."""
+    if workload_name != BENCH_WORKLOAD or not os.path.exists(PROFILE_FILE):
         return None
-    with open(TRAFFIC_FILE) as f:
-        t = json.load(f)
-    if t.get("kernel_sha") != kernel_sha():
+    fields = {}
+    with open(PROFILE_FILE) as f:
+        for line in f:
+            if ":" in line and not line.startswith("#"):
+                k, v = line.split(":", 1)
+                fields[k.strip()] = v.strip()
+    if fields.get("kernel_sha") != kernel_sha():
         return None
-    return float(t["dram_bytes_per_launch"]) * launch_rows_scale / float(t.get("rows_scale", 1.0))
+    try:
+        return int(fields["dram_read_write_bytes_per_launch"])
+    except (KeyError, ValueError):
+        return None
 
 
 # ----------------------------------------------------------------- clocks ---
 class ClockSampler:
-    """nvidia-smi sampling (200 ms) while the GPU is busy."""
+    """nvidia-smi sampling (100 ms) while the GPU is busy."""
 
-    def __init__(self, gpu_index: int):
-        self.gpu = gpu_index
+    def __init__(self, gpu_id: str):
+        self.gpu = gpu_id  # nvidia-smi --id: index or UUID of the physical GPU
         self.proc = None
         self.path = None
 
@@ -90,7 +97,7 @@ class ClockSampler:
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={CLOCK_QUERY}",
-                 "--format=csv,noheader,nounits", "-lms", "200"],
+                 "--format=csv,noheader,nounits", "-lms", "100"],
                 stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
         except (OSError, FileNotFoundError):
             self.proc = None
@@ -190,11 +197,13 @@ def run_b200(args, w):
     def step():
         tab.attn_fwd_into(q, k, v, o, lse, causal=w.causal, scale=w.scale, stream=stream)
 
-    sampler = ClockSampler(local)
-    sampler.start()
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES", "")
+    smi_id = vis.split(",")[local].strip() if vis and len(vis.split(",")) > local else str(local)
+    sampler = ClockSampler(smi_id)
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize(dev)
+    sampler.start()
     if pg:
         torch.distributed.barrier()
     torch.cuda.synchronize(dev)
@@ -249,7 +258,7 @@ def run_b200(args, w):
     peak = float(peaks["bf16_tflops"])
     achieved = w.flops / (ms_step * 1e-3) / 1e12  # per launch, this GPU
     tb = w.rows * w.d * 2
-    traffic = load_traffic(1.0)
+    traffic = load_traffic(w.name)
     line = {
         "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 4),
@@ -334,7 +343,7 @@ def run_reference(args, w):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--steps", type=int, default=1000)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["b200", "reference"], default="b200")
     ap.add_argument("--workload", default=BENCH_WORKLOAD, choices=sorted(WORKLOADS))
