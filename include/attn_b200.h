@@ -70,6 +70,28 @@ int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
              attn_stream_t stream);
 
 /*
+ * Tuning options for attn_fwd_ex.  Every option only changes how the same
+ * result is computed (rounding differs within the documented tolerance).
+ *   exp2_poly_pairs  of every 4 pairs of score columns, how many take their
+ *                    exponential from an FMA-pipe polynomial instead of the
+ *                    special-function unit (the split described on the page's
+ *                    section "Deplacer une partie des exponentielles");
+ *                    0, 1 or 2, or -1 for the library default.
+ */
+typedef struct {
+  int exp2_poly_pairs;
+} attn_opts;
+
+/*
+ * attn_fwd_ex -- attn_fwd with tuning options (opts may be NULL: defaults).
+ * Same contract as attn_fwd; an out-of-range option returns
+ * ATTN_ERR_INVALID_ARG before anything is enqueued.
+ */
+int attn_fwd_ex(const void* q, const void* k, const void* v, void* o, float* lse,
+                int B, int H, int N, int d, int causal, float scale,
+                const attn_opts* opts, attn_stream_t stream);
+
+/*
  * attn_fwd_host -- the same operation on HOST buffers: copies q, k, v from
  * host to the caller's device buffers, runs attn_fwd, and copies o and lse
  * back, all enqueued on `stream` (pinned host memory makes the copies

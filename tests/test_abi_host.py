@@ -32,8 +32,8 @@ def declared_symbols():
 
 def test_header_declares_entry_points():
     syms = declared_symbols()
-    for s in ["attn_fwd", "attn_fwd_host", "attn_last_device_error", "attn_strerror",
-              "attn_check_args", "attn_version"]:
+    for s in ["attn_fwd", "attn_fwd_ex", "attn_fwd_host", "attn_last_device_error",
+              "attn_strerror", "attn_check_args", "attn_version"]:
         assert s in syms
 
 
@@ -102,3 +102,38 @@ def test_product_does_not_import_oracle():
                 text = open(os.path.join(dirpath, fn)).read()
                 assert not re.search(r"^\s*(import|from)\s+oracle\b", text, re.M), fn
                 assert "attn_ref" not in text and "libattn_ref" not in text, fn
+
+
+def test_fwd_ex_rejects_bad_option_before_any_cuda_call(lib):
+    import ctypes
+    p = ptrs()
+    for bad in (-2, 3, 100):
+        opts = tab.AttnOpts(bad)
+        rc = lib.attn_fwd_ex(*p, 1, 1, 128, 128, 0, 0.1, ctypes.byref(opts), None)
+        assert rc == -1
+
+
+def test_exp2_polynomial_coefficients_and_error():
+    """The kernel's exp2 polynomial literals are the ones the generator
+    derives, and the fp32 instruction sequence stays within 1e-4 relative
+    error of 2^x over the clamped range (far below bf16's 2^-9)."""
+    import importlib.util
+    import numpy as np
+    gen_path = os.path.join(ROOT, "tiled_attention_forward_sm_b200", "csrc", "gen_exp2_poly.py")
+    spec = importlib.util.spec_from_file_location("gen_exp2_poly", gen_path)
+    gen = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(gen)
+    c = [float(np.float32(v)) for v in gen.remez_relative()]
+    src = open(os.path.join(ROOT, "tiled_attention_forward_sm_b200", "csrc",
+                            "attn_fwd_kernel.cuh")).read()
+    lits = [float(x) for x in re.findall(r"kC[0-3] = ([0-9.]+)f", src)]
+    assert len(lits) == 4
+    assert np.allclose(lits, c, rtol=0, atol=1e-9)
+    xs = np.linspace(-125.0, 8.0, 400001).astype(np.float32)
+    rel = np.abs(gen.fp32_exp2_emulation(xs, lits).astype(np.float64) /
+                 np.exp2(xs.astype(np.float64)) - 1.0)
+    assert rel.max() < 1e-4
+    # integers are exact up to the polynomial's value at f = 0
+    ints = np.arange(-125, 9).astype(np.float32)
+    np.testing.assert_allclose(gen.fp32_exp2_emulation(ints, lits), np.exp2(ints) * lits[0],
+                               rtol=1e-7)

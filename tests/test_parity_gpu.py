@@ -19,9 +19,9 @@ pytestmark = pytest.mark.gpu
 ATOL_O, RTOL_O, ATOL_LSE = 2e-2, 1e-2, 1e-3
 
 
-def gpu_run(q, k, v, causal, scale):
+def gpu_run(q, k, v, causal, scale, poly=None):
     qd, kd, vd = (t.cuda() for t in (q, k, v))
-    o, lse = tab.attn_fwd(qd, kd, vd, causal=causal, scale=scale)
+    o, lse = tab.attn_fwd(qd, kd, vd, causal=causal, scale=scale, exp2_poly_pairs=poly)
     assert tab.last_device_error() == 0
     return o.float().cpu().numpy().astype(np.float64), lse.cpu().numpy().astype(np.float64)
 
@@ -36,10 +36,10 @@ def check(o_gpu, lse_gpu, o_ref, lse_ref, what=""):
     return err_o.max(), err_l.max()
 
 
-def full_parity(oracle_mod, B, H, N, d, causal, seed, q_std=1.0, scale=None):
+def full_parity(oracle_mod, B, H, N, d, causal, seed, q_std=1.0, scale=None, poly=None):
     scale = 1 / math.sqrt(d) if scale is None else scale
     q, k, v = make_qkv(B, H, N, d, seed, q_std)
-    o, lse = gpu_run(q, k, v, causal, scale)
+    o, lse = gpu_run(q, k, v, causal, scale, poly)
     o_ref, lse_ref = oracle_mod.attn_ref(bf16_bits(q), bf16_bits(k), bf16_bits(v), causal, scale)
     return check(o, lse, o_ref, lse_ref, f"B{B} H{H} N{N} d{d} causal={causal}")
 
@@ -51,6 +51,15 @@ def test_small_shapes(oracle_mod, d, causal, N):
     """Single tile, one pair, an odd number of 128-row tiles (a CTA with one
     Q tile), several K/V tiles with a ragged pair count."""
     full_parity(oracle_mod, 2, 3, N, d, causal, seed=N + d + causal)
+
+
+@pytest.mark.parametrize("poly", [0, 1, 2])
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("causal", [False, True])
+def test_exp2_split_variants(oracle_mod, poly, d, causal):
+    """Every split of the exponentials between the special-function unit and
+    the FMA polynomial meets the same tolerance (peaky scores, masked tiles)."""
+    full_parity(oracle_mod, 1, 3, 640, d, causal, seed=31 + poly, q_std=3.0, poly=poly)
 
 
 @pytest.mark.parametrize("name", ["b1h2n256d64", "b4h16n2048d128_causal"])

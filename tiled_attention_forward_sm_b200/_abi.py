@@ -17,6 +17,11 @@ ATTN_OK = 0
 _lib = None
 
 
+class AttnOpts(ctypes.Structure):
+    """Mirror of attn_opts in include/attn_b200.h."""
+    _fields_ = [("exp2_poly_pairs", ctypes.c_int)]
+
+
 class AttnError(RuntimeError):
     def __init__(self, status: int, what: str):
         super().__init__(f"{what}: {strerror(status)} (status {status})")
@@ -38,6 +43,8 @@ def library():
         vp, i, f = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
         lib.attn_fwd.restype = i
         lib.attn_fwd.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, f, vp]
+        lib.attn_fwd_ex.restype = i
+        lib.attn_fwd_ex.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, f, vp, vp]
         lib.attn_fwd_host.restype = i
         lib.attn_fwd_host.argtypes = [vp] * 10 + [i, i, i, i, i, f, vp]
         lib.attn_last_device_error.restype = i
@@ -75,9 +82,10 @@ def _shape(q: torch.Tensor):
 
 
 def attn_fwd_into(q, k, v, o, lse, causal: bool = False, scale: float | None = None,
-                  stream=None) -> None:
+                  stream=None, exp2_poly_pairs: int | None = None) -> None:
     """Enqueue the forward pass writing into ``o`` (bf16 [B,H,N,d]) and ``lse``
-    (fp32 [B,H,N]).  Inputs: CUDA bf16 contiguous [B,H,N,d] tensors."""
+    (fp32 [B,H,N]).  Inputs: CUDA bf16 contiguous [B,H,N,d] tensors.
+    ``exp2_poly_pairs`` (0..2) selects the attn_fwd_ex tuning option."""
     B, H, N, d = _shape(q)
     for name, t, dt in (("q", q, torch.bfloat16), ("k", k, torch.bfloat16),
                         ("v", v, torch.bfloat16), ("o", o, torch.bfloat16)):
@@ -88,20 +96,25 @@ def attn_fwd_into(q, k, v, o, lse, causal: bool = False, scale: float | None = N
         raise ValueError(f"lse must be a contiguous CUDA fp32 tensor of shape {(B, H, N)}")
     if scale is None:
         scale = 1.0 / math.sqrt(d)
-    rc = library().attn_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
-                            lse.data_ptr(), B, H, N, d, int(bool(causal)), float(scale),
-                            _stream_handle(stream))
+    args = (q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
+            B, H, N, d, int(bool(causal)), float(scale))
+    if exp2_poly_pairs is None:
+        rc = library().attn_fwd(*args, _stream_handle(stream))
+    else:
+        opts = AttnOpts(int(exp2_poly_pairs))
+        rc = library().attn_fwd_ex(*args, ctypes.byref(opts), _stream_handle(stream))
     if rc != ATTN_OK:
         raise AttnError(rc, "attn_fwd")
 
 
-def attn_fwd(q, k, v, causal: bool = False, scale: float | None = None, stream=None):
+def attn_fwd(q, k, v, causal: bool = False, scale: float | None = None, stream=None,
+             exp2_poly_pairs: int | None = None):
     """Return ``(o, lse)`` for CUDA bf16 [B,H,N,d] inputs (enqueued on the
     current or given stream)."""
     B, H, N, d = _shape(q)
     o = torch.empty_like(q)
     lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
-    attn_fwd_into(q, k, v, o, lse, causal, scale, stream)
+    attn_fwd_into(q, k, v, o, lse, causal, scale, stream, exp2_poly_pairs)
     return o, lse
 
 

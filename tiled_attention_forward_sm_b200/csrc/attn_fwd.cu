@@ -98,7 +98,7 @@ bool ranges_overlap(const void* a, size_t na, const void* b, size_t nb) {
   return x < y + nb && y < x + na;
 }
 
-template <int D, bool CAUSAL>
+template <int D, bool CAUSAL, int kPolyPairs>
 int launch(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
            int N, float scale, cudaStream_t stream, const DeviceState& st) {
   using C = Config<D>;
@@ -116,7 +116,19 @@ int launch(const void* q, const void* k, const void* v, void* o, float* lse, int
   args.scale_log2 = scale * 1.4426950408889634f;
   args.status = st.status;
 
-  auto kern = attn_fwd_kernel<D, CAUSAL>;
+  auto kern = attn_fwd_kernel<D, CAUSAL, kPolyPairs>;
+  // The kernel's register split (setmaxnreg) hands the softmax warpgroups
+  // registers released by the producer/MMA warpgroup; it is only valid if
+  // the kernel was built with the full per-thread budget it assumes.
+  static const bool regs_ok = [&] {
+    cudaFuncAttributes fa;
+    if (cudaFuncGetAttributes(&fa, kern) != cudaSuccess) {
+      cudaGetLastError();
+      return false;
+    }
+    return fa.numRegs * kThreads >= kRegSplitTotal;
+  }();
+  if (!regs_ok) return ATTN_ERR_CUDA;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes) !=
       cudaSuccess) {
     cudaGetLastError();
@@ -124,7 +136,11 @@ int launch(const void* q, const void* k, const void* v, void* o, float* lse, int
   }
   cudaLaunchConfig_t cfg;
   std::memset(&cfg, 0, sizeof cfg);
+#if ATTN_HEAD_MAJOR
+  cfg.gridDim = dim3(static_cast<unsigned>(args.n_qpairs), static_cast<unsigned>(B * H), 1);
+#else
   cfg.gridDim = dim3(static_cast<unsigned>(B * H), static_cast<unsigned>(args.n_qpairs), 1);
+#endif
   cfg.blockDim = dim3(kThreads, 1, 1);
   cfg.dynamicSmemBytes = C::kSmemBytes;
   cfg.stream = stream;
@@ -134,6 +150,24 @@ int launch(const void* q, const void* k, const void* v, void* o, float* lse, int
   }
   return ATTN_OK;
 }
+
+// Default share of exponentials computed by the FMA polynomial (pairs per 4):
+// measured on B200, the special-function unit alone is fastest for this
+// kernel (see the exp2 split sweep in the design notes).
+constexpr int kDefaultPolyPairs = 0;
+
+template <int D, bool CAUSAL>
+int launch_poly(int poly_pairs, const void* q, const void* k, const void* v, void* o, float* lse,
+                int B, int H, int N, float scale, cudaStream_t s, const DeviceState& st) {
+  switch (poly_pairs) {
+    case 0: return launch<D, CAUSAL, 0>(q, k, v, o, lse, B, H, N, scale, s, st);
+    case 2: return launch<D, CAUSAL, 2>(q, k, v, o, lse, B, H, N, scale, s, st);
+    default: return launch<D, CAUSAL, 1>(q, k, v, o, lse, B, H, N, scale, s, st);
+  }
+}
+
+int fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N,
+             int d, int causal, float scale, int poly_pairs, attn_stream_t stream);
 
 }  // namespace
 }  // namespace attn_b200
@@ -149,7 +183,7 @@ extern "C" int attn_check_args(const void* q, const void* k, const void* v, cons
   if (N % kBlockM != 0) return ATTN_ERR_UNSUPPORTED;
   const uint64_t rows = static_cast<uint64_t>(B) * H * N;
   if (rows >= (1ull << 31) || static_cast<uint64_t>(B) * H > 0x7FFFFFFFull ||
-      N / (2 * kBlockM) + 1 > 65535)
+      N / (2 * kBlockM) + 1 > 65535 || (ATTN_HEAD_MAJOR && static_cast<uint64_t>(B) * H > 65535))
     return ATTN_ERR_UNSUPPORTED;
   const uintptr_t al = reinterpret_cast<uintptr_t>(q) | reinterpret_cast<uintptr_t>(k) |
                        reinterpret_cast<uintptr_t>(v) | reinterpret_cast<uintptr_t>(o);
@@ -164,8 +198,10 @@ extern "C" int attn_check_args(const void* q, const void* k, const void* v, cons
   return ATTN_OK;
 }
 
-extern "C" int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B,
-                        int H, int N, int d, int causal, float scale, attn_stream_t stream) {
+namespace attn_b200 {
+namespace {
+int fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N,
+             int d, int causal, float scale, int poly_pairs, attn_stream_t stream) {
   int rc = attn_check_args(q, k, v, o, lse, B, H, N, d, scale);
   if (rc != ATTN_OK) return rc;
   DeviceState* st = nullptr;
@@ -173,10 +209,28 @@ extern "C" int attn_fwd(const void* q, const void* k, const void* v, void* o, fl
   if (rc != ATTN_OK) return rc;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (d == 128)
-    return causal ? launch<128, true>(q, k, v, o, lse, B, H, N, scale, s, *st)
-                  : launch<128, false>(q, k, v, o, lse, B, H, N, scale, s, *st);
-  return causal ? launch<64, true>(q, k, v, o, lse, B, H, N, scale, s, *st)
-                : launch<64, false>(q, k, v, o, lse, B, H, N, scale, s, *st);
+    return causal ? launch_poly<128, true>(poly_pairs, q, k, v, o, lse, B, H, N, scale, s, *st)
+                  : launch_poly<128, false>(poly_pairs, q, k, v, o, lse, B, H, N, scale, s, *st);
+  return causal ? launch_poly<64, true>(poly_pairs, q, k, v, o, lse, B, H, N, scale, s, *st)
+                : launch_poly<64, false>(poly_pairs, q, k, v, o, lse, B, H, N, scale, s, *st);
+}
+}  // namespace
+}  // namespace attn_b200
+
+extern "C" int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B,
+                        int H, int N, int d, int causal, float scale, attn_stream_t stream) {
+  return fwd_impl(q, k, v, o, lse, B, H, N, d, causal, scale, kDefaultPolyPairs, stream);
+}
+
+extern "C" int attn_fwd_ex(const void* q, const void* k, const void* v, void* o, float* lse, int B,
+                           int H, int N, int d, int causal, float scale, const attn_opts* opts,
+                           attn_stream_t stream) {
+  int poly = kDefaultPolyPairs;
+  if (opts) {
+    if (opts->exp2_poly_pairs < -1 || opts->exp2_poly_pairs > 2) return ATTN_ERR_INVALID_ARG;
+    if (opts->exp2_poly_pairs >= 0) poly = opts->exp2_poly_pairs;
+  }
+  return fwd_impl(q, k, v, o, lse, B, H, N, d, causal, scale, poly, stream);
 }
 
 extern "C" int attn_last_device_error(attn_stream_t stream) {
@@ -235,5 +289,14 @@ extern "C" const char* attn_strerror(int status) {
     default: return "unknown status";
   }
 }
+
+#ifdef ATTN_TRACE_ENABLED
+// Tracing builds only: register the device buffer (kTraceCtas x kTrNumEvents
+// x kTraceSteps uint64) that kernels stamp; nullptr turns stamping off.
+extern "C" int attn_trace_set_buffer(void* dev_buf) {
+  unsigned long long* p = static_cast<unsigned long long*>(dev_buf);
+  return cudaMemcpyToSymbol(g_trace_buf, &p, sizeof p) == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+#endif
 
 extern "C" int attn_version(void) { return (0 << 16) | (1 << 8) | 0; }

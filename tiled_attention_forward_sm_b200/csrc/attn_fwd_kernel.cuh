@@ -23,7 +23,8 @@
 //               the lazy O rescale and the epilogue for Q0
 //   warps 4-7   softmax group 1 (Q1), same for Q1
 //   warp  8     TMA producer: Q0/Q1 once, then K_j, V_j through a ring
-//   warp  9     TMEM allocator and single-thread tcgen05 MMA issuer
+//   warp  9     TMEM allocator and tcgen05 MMA issuer (warp-uniform control,
+//               one elected lane issues)
 //   warps 10-11 idle
 //
 // Tensor Memory plan (512 columns x 128 lanes x 32 bit):
@@ -53,14 +54,65 @@ constexpr int kStatusDeviceTimeout = -5;
 // status word and the CTA's abort flag, and every role then leaves its loop.
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s
 
+// The two softmax groups take turns on the special-function units: group 0
+// runs its exponentials for step j, then group 1 for step j, then group 0
+// for step j+1, ...  Without the ordering both groups' exponential phases
+// overlap and each runs at half rate, lengthening the per-tile critical path.
+#ifndef ATTN_SOFTMAX_ORDER
+#define ATTN_SOFTMAX_ORDER 0
+#endif
+
+// K/V ring depth for d = 128 (each stage holds one 128 x 128 bf16 tile).
+#ifndef ATTN_KV_STAGES_D128
+#define ATTN_KV_STAGES_D128 4
+#endif
+
+// CTA launch order: head-major (all query pairs of one head adjacent, so the
+// CTAs that stream the same K/V run together and share it through L2) or
+// pair-major (every head's heaviest pair first).
+#ifndef ATTN_HEAD_MAJOR
+#define ATTN_HEAD_MAJOR 0
+#endif
+
 constexpr int kBlockM = 128;  // query rows per Q tile
 constexpr int kBlockN = 128;  // keys per K/V tile
 constexpr int kThreads = 384;
+// Register split: softmax warpgroups (256 threads) grow to kRegsSoftmax,
+// the producer/MMA warpgroup (128 threads) shrinks to kRegsOther.  The sum
+// must not exceed what the CTA was launched with (384 threads x 168).
+constexpr int kRegsSoftmax = 200;
+constexpr int kRegsOther = 104;
+constexpr int kRegSplitTotal = 256 * kRegsSoftmax + 128 * kRegsOther;
+static_assert(kRegSplitTotal <= kThreads * 168, "register split exceeds the launch budget");
 
 // Lazy-rescale threshold in log2 units: the running maximum is raised only
 // when a tile's maximum exceeds it by more than this, so every weight stays
 // at most 2^8 (fp32 row sums and bf16 weights stay far from overflow).
 constexpr float kRescaleTau = 8.0f;
+
+// Optional timeline tracing (compiled in only with ATTN_TRACE_ENABLED; the
+// library build leaves it out): clock64 stamps at each role's hand-off for
+// the first kTraceCtas CTAs and kTraceSteps K/V steps, written to a device
+// buffer registered by the tracing build's host code.
+enum TraceEvent : int {
+  kTrMmaS0 = 0, kTrMmaPV0a, kTrMmaPV0b, kTrMmaS1, kTrMmaPV1a, kTrMmaPV1b, kTrMmaV,
+  kTrSm0Full, kTrSm0Ld, kTrSm0Max, kTrSm0Pa, kTrSm0Pb,
+  kTrSm1Full, kTrSm1Ld, kTrSm1Max, kTrSm1Pa, kTrSm1Pb,
+  kTrProdK, kTrProdV, kTrStart, kTrEnd, kTrMmaS0end, kTrMmaS1end, kTrMmaPV0end, kTrNumEvents
+};
+constexpr int kTraceCtas = 64;
+constexpr int kTraceSteps = 72;
+#ifdef ATTN_TRACE_ENABLED
+__device__ unsigned long long* g_trace_buf = nullptr;
+__device__ __forceinline__ void trace_stamp(int ev, int j) {
+  const int cta = blockIdx.x + blockIdx.y * gridDim.x;
+  if (g_trace_buf != nullptr && cta < kTraceCtas && j >= 0 && j < kTraceSteps)
+    g_trace_buf[(static_cast<size_t>(cta) * kTrNumEvents + ev) * kTraceSteps + j] = clock64();
+}
+#define ATTN_TRACE(ev, j) ::attn_b200::trace_stamp((ev), (j))
+#else
+#define ATTN_TRACE(ev, j) ((void)0)
+#endif
 
 struct KernelArgs {
   __nv_bfloat16* o;   // [B*H*N, D]
@@ -78,13 +130,14 @@ struct Config {
   static constexpr int kTileBytes = kBlockM * D * 2;        // one 128 x D bf16 tile
   static constexpr int kBoxes = D / 64;                      // 64-column TMA boxes per tile
   static constexpr int kBoxBytes = kBlockM * 64 * 2;         // 16 KB
-  static constexpr int kStages = D == 128 ? 4 : 8;           // K/V ring depth
+  static constexpr int kStages = D == 128 ? ATTN_KV_STAGES_D128 : 8;  // K/V ring depth
   static constexpr int kQOff = 0;
   static constexpr int kKVOff = 2 * kTileBytes;
   static constexpr int kBarOff = kKVOff + kStages * kTileBytes;
-  // barriers: q_full, kv_full[S], kv_empty[S], s_full[2], p_ready[2],
-  // o_final[2], drain
-  static constexpr int kNumBars = 1 + 2 * kStages + 2 + 2 + 2 + 1;
+  // barriers: q_full, kv_full[S], kv_empty[S], s_full[2], p_ready[2 tiles][2
+  // halves], o_final[2], drain
+  // + exp_token[2] (softmax group s may run its exponentials)
+  static constexpr int kNumBars = 1 + 2 * kStages + 2 + 4 + 2 + 1 + 2;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;
   static constexpr int kSmemBytes = kMiscOff + 16 + 1024;  // + alignment slack
   static constexpr uint32_t kIdescQK = ptx::idesc_bf16_f32(128, kBlockN, 0, 0);
@@ -99,6 +152,7 @@ struct Shared {
   uint64_t* p_ready;
   uint64_t* o_final;
   uint64_t* drain;
+  uint64_t* exp_token;
   uint32_t* tmem_base;
   volatile int* abort_flag;
 };
@@ -129,7 +183,7 @@ __device__ __forceinline__ bool wait_one(const Shared& sh, int* status, uint64_t
 // Warp-uniform bounded wait (every lane returns the same answer), for roles
 // whose next instructions are warp-collective tcgen05 loads/stores.
 __device__ __forceinline__ bool wait_warp(const Shared& sh, int* status, uint64_t* bar,
-                                          uint32_t parity) {
+                                          uint32_t parity, bool drain = false) {
   uint64_t t0 = 0;
   for (uint32_t it = 0;; ++it) {
     const bool ok = ptx::mbar_try_wait(bar, parity);
@@ -139,7 +193,7 @@ __device__ __forceinline__ bool wait_warp(const Shared& sh, int* status, uint64_
       if (ptx::lane_id() == 0) {
         const uint64_t now = ptx::globaltimer_ns();
         if (t0 == 0) t0 = now;
-        if (*sh.abort_flag) {
+        if (!drain && *sh.abort_flag) {
           stop = 1;
         } else if (now - t0 > kWaitLimitNs) {
           raise_status(sh, status, kStatusDeviceTimeout);
@@ -188,6 +242,7 @@ __device__ void producer_role(const Shared& sh, const KernelArgs& a, uint8_t* sm
       const uint32_t ph = (issued / C::kStages) & 1;
       if (!wait_one(sh, a.status, &sh.kv_empty[st], ph ^ 1)) { ok = false; break; }
       uint8_t* dst = smem + C::kKVOff + st * C::kTileBytes;
+      ATTN_TRACE(which == 0 ? kTrProdK : kTrProdV, j);
       ptx::mbar_arrive_expect_tx(&sh.kv_full[st], C::kTileBytes);
       const CUtensorMap* m = which == 0 ? tk : tv;
       for (int b = 0; b < C::kBoxes; ++b)
@@ -203,6 +258,11 @@ __device__ void producer_role(const Shared& sh, const KernelArgs& a, uint8_t* sm
 }
 
 // ---------------------------------------------------------------------- MMA
+// Executed by the whole MMA warp so descriptors stay warp-uniform; each
+// tcgen05.mma / tcgen05.commit is issued by one elected lane.  Descriptors
+// are built once and advanced by constant offsets (the start-address field
+// is the low 14 bits, in 16-byte units; no carry can leave it because
+// shared memory is below 256 KB).
 template <int D, bool CAUSAL>
 __device__ void mma_role(const Shared& sh, const KernelArgs& a, uint8_t* smem, uint32_t tmem,
                          int qpair) {
@@ -210,98 +270,156 @@ __device__ void mma_role(const Shared& sh, const KernelArgs& a, uint8_t* smem, u
   const int n0 = kv_tiles_for<CAUSAL>(2 * qpair, a.n_qtiles);
   const int n1 = kv_tiles_for<CAUSAL>(2 * qpair + 1, a.n_qtiles);
   const int n = n0 > n1 ? n0 : n1;
-  const uint32_t q_addr = ptx::smem_u32(smem + C::kQOff);
-  const uint32_t kv_addr = ptx::smem_u32(smem + C::kKVOff);
   const uint32_t t_s[2] = {tmem + 0, tmem + 128};
   const uint32_t t_o[2] = {tmem + 256, tmem + 384};
+  // K-major (Q, K): SBO = 1024 B between 8-row groups; MN-major (V):
+  // LBO = one 64-column box (16 KB), SBO = 1024 B between 8-key groups.
+  const uint64_t q_desc = ptx::sdesc_sw128(ptx::smem_u32(smem + C::kQOff), 16, 1024);
+  const uint64_t k_desc = ptx::sdesc_sw128(ptx::smem_u32(smem + C::kKVOff), 16, 1024);
+  const uint64_t v_desc = ptx::sdesc_sw128(ptx::smem_u32(smem + C::kKVOff), C::kBoxBytes, 1024);
+  constexpr uint64_t kTileUnits = C::kTileBytes >> 4;
 
-  // S_s = Q_s K^T over D (K-major operands, D/16 MMAs of K-depth 16)
-  auto issue_qk = [&](int s, uint32_t k_addr) {
-    const uint32_t qa = q_addr + s * C::kTileBytes;
+  // S_s = Q_s K^T over D (D/16 MMAs of K-depth 16; a 16-deep step moves 32 B
+  // inside the 128 B swizzle row, a 64-deep step moves one box)
+  auto issue_qk = [&](int s, int stage) {
+    const uint64_t qd = q_desc + s * kTileUnits;
+    const uint64_t kd = k_desc + stage * kTileUnits;
 #pragma unroll
     for (int kk = 0; kk < D / 16; ++kk) {
-      const uint32_t off = (kk / 4) * C::kBoxBytes + (kk % 4) * 32;
-      ptx::mma_ss(t_s[s], ptx::sdesc_sw128(qa + off, 16, 1024),
-                  ptx::sdesc_sw128(k_addr + off, 16, 1024), C::kIdescQK, kk > 0 ? 1u : 0u);
+      const uint64_t off = static_cast<uint64_t>(((kk / 4) * C::kBoxBytes + (kk % 4) * 32) >> 4);
+      ptx::mma_ss_elect(t_s[s], qd + off, kd + off, C::kIdescQK, kk > 0 ? 1u : 0u);
     }
   };
-  // O_s (+)= P_s V over the 128 keys (P from TMEM, V MN-major)
-  auto issue_pv = [&](int s, uint32_t v_addr, bool accumulate) {
+  // O_s (+)= P_s V over keys [64*half, 64*half + 64): P from TMEM (8 columns
+  // per 16 keys), V MN-major (2 KB per 16 keys)
+  auto issue_pv_half = [&](int s, int half, int stage, uint32_t accumulate) {
+    const uint64_t vd = v_desc + stage * kTileUnits;
 #pragma unroll
-    for (int kk = 0; kk < kBlockN / 16; ++kk) {
-      ptx::mma_ts(t_o[s], t_s[s] + 8 * kk, ptx::sdesc_sw128(v_addr + kk * 2048, C::kBoxBytes, 1024),
-                  C::kIdescPV, (accumulate || kk > 0) ? 1u : 0u);
+    for (int k4 = 0; k4 < 4; ++k4) {
+      const int kk = 4 * half + k4;
+      ptx::mma_ts_elect(t_o[s], t_s[s] + 8 * kk, vd + static_cast<uint64_t>((kk * 2048) >> 4),
+                        C::kIdescPV, (accumulate | static_cast<uint32_t>(kk > 0)));
     }
+  };
+  int trace_j = 0;
+  (void)trace_j;
+  // Both halves of PV_s(j); the first half is issued as soon as the softmax
+  // has published keys 0-63 of P, before keys 64-127 are ready.
+  auto issue_pv = [&](int s, int stage, uint32_t accumulate, uint32_t parity) -> bool {
+    if (!wait_warp(sh, a.status, &sh.p_ready[2 * s], parity)) return false;
+    ptx::tc_fence_after_sync();
+    ATTN_TRACE(s == 0 ? kTrMmaPV0a : kTrMmaPV1a, trace_j);
+    issue_pv_half(s, 0, stage, accumulate);
+    if (!wait_warp(sh, a.status, &sh.p_ready[2 * s + 1], parity)) return false;
+    ptx::tc_fence_after_sync();
+    ATTN_TRACE(s == 0 ? kTrMmaPV0b : kTrMmaPV1b, trace_j);
+    issue_pv_half(s, 1, stage, accumulate);
+    return true;
   };
 
   int consumed = 0;
   auto stage_of = [&](int c) { return c % C::kStages; };
   auto phase_of = [&](int c) { return static_cast<uint32_t>((c / C::kStages) & 1); };
 
-  if (!wait_one(sh, a.status, sh.q_full, 0)) goto done;
+  if (!wait_warp(sh, a.status, sh.q_full, 0)) goto done;
   {
     // step 0: S0(0), S1(0)
-    int ck = consumed++;
-    if (!wait_one(sh, a.status, &sh.kv_full[stage_of(ck)], phase_of(ck))) goto done;
+    const int ck = consumed++;
+    if (!wait_warp(sh, a.status, &sh.kv_full[stage_of(ck)], phase_of(ck))) goto done;
     ptx::tc_fence_after_sync();
-    const uint32_t k_addr0 = kv_addr + stage_of(ck) * C::kTileBytes;
-    if (n0 > 0) { issue_qk(0, k_addr0); ptx::tc_commit(&sh.s_full[0]); }
-    if (n1 > 0) { issue_qk(1, k_addr0); ptx::tc_commit(&sh.s_full[1]); }
-    ptx::tc_commit(&sh.kv_empty[stage_of(ck)]);
+    ATTN_TRACE(kTrMmaS0, 0);
+    if (n0 > 0) { issue_qk(0, stage_of(ck)); ptx::commit_elect(&sh.s_full[0]); }
+    ATTN_TRACE(kTrMmaS1, 0);
+    if (n1 > 0) { issue_qk(1, stage_of(ck)); ptx::commit_elect(&sh.s_full[1]); }
+    ptx::commit_elect(&sh.kv_empty[stage_of(ck)]);
 
+    // Per step j: both K/V waits come first (the tiles are normally resident
+    // long before), so that PV_s(j) and S_s(j+1) issue back to back and no
+    // barrier round trip sits on a tile's S -> softmax -> PV -> S chain.
     for (int j = 0; j < n; ++j) {
       const int cv = consumed++;
-      if (!wait_one(sh, a.status, &sh.kv_full[stage_of(cv)], phase_of(cv))) goto done;
-      const uint32_t v_addr = kv_addr + stage_of(cv) * C::kTileBytes;
+      trace_j = j;
+      if (!wait_warp(sh, a.status, &sh.kv_full[stage_of(cv)], phase_of(cv))) goto done;
+      const int ck2 = (j + 1 < n) ? consumed++ : -1;
+      if (ck2 >= 0 &&
+          !wait_warp(sh, a.status, &sh.kv_full[stage_of(ck2)], phase_of(ck2)))
+        goto done;
+      ptx::tc_fence_after_sync();
+      ATTN_TRACE(kTrMmaV, j);
       const uint32_t pj = static_cast<uint32_t>(j & 1);
+      const uint32_t acc = j > 0 ? 1u : 0u;
       if (j < n0) {
-        if (!wait_one(sh, a.status, &sh.p_ready[0], pj)) goto done;
-        ptx::tc_fence_after_sync();
-        issue_pv(0, v_addr, j > 0);
-        if (j == n0 - 1) ptx::tc_commit(&sh.o_final[0]);
+        if (!issue_pv(0, stage_of(cv), acc, pj)) goto done;
+        ATTN_TRACE(kTrMmaPV0end, j);
+        if (j == n0 - 1) ptx::commit_elect(&sh.o_final[0]);
       }
-      int ck2 = -1;
-      uint32_t k_addr = 0;
-      if (j + 1 < n) {
-        ck2 = consumed++;
-        if (!wait_one(sh, a.status, &sh.kv_full[stage_of(ck2)], phase_of(ck2))) goto done;
-        ptx::tc_fence_after_sync();
-        k_addr = kv_addr + stage_of(ck2) * C::kTileBytes;
-        if (j + 1 < n0) { issue_qk(0, k_addr); ptx::tc_commit(&sh.s_full[0]); }
+      if (ck2 >= 0) {
+        ATTN_TRACE(kTrMmaS0, j + 1);
+        if (j + 1 < n0) { issue_qk(0, stage_of(ck2)); ptx::commit_elect(&sh.s_full[0]); }
+        ATTN_TRACE(kTrMmaS0end, j + 1);
       }
       if (j < n1) {
-        if (!wait_one(sh, a.status, &sh.p_ready[1], pj)) goto done;
-        ptx::tc_fence_after_sync();
-        issue_pv(1, v_addr, j > 0);
-        if (j == n1 - 1) ptx::tc_commit(&sh.o_final[1]);
+        if (!issue_pv(1, stage_of(cv), acc, pj)) goto done;
+        if (j == n1 - 1) ptx::commit_elect(&sh.o_final[1]);
       }
-      ptx::tc_commit(&sh.kv_empty[stage_of(cv)]);
+      ptx::commit_elect(&sh.kv_empty[stage_of(cv)]);
       if (ck2 >= 0) {
-        if (j + 1 < n1) { issue_qk(1, k_addr); ptx::tc_commit(&sh.s_full[1]); }
-        ptx::tc_commit(&sh.kv_empty[stage_of(ck2)]);
+        ATTN_TRACE(kTrMmaS1, j + 1);
+        if (j + 1 < n1) { issue_qk(1, stage_of(ck2)); ptx::commit_elect(&sh.s_full[1]); }
+        ATTN_TRACE(kTrMmaS1end, j + 1);
+        ptx::commit_elect(&sh.kv_empty[stage_of(ck2)]);
       }
     }
   }
 done:
-  // Drain: every MMA this thread issued completes before TMEM is released.
-  ptx::tc_commit(sh.drain);
-  wait_one(sh, a.status, sh.drain, 0, true);
+  // Drain: every MMA this warp issued completes before TMEM is released.
+  ptx::commit_elect(sh.drain);
+  wait_warp(sh, a.status, sh.drain, 0, true);
 }
 
 // ------------------------------------------------------------------ softmax
+// exp2 on the FMA pipe for a pair of inputs: 2^x = 2^j * 2^f with j the
+// nearest integer (1.5*2^23 rounding trick) and f in [-1/2, 1/2]; 2^f by a
+// degree-3 polynomial minimising relative error (coefficients from
+// csrc/gen_exp2_poly.py, max relative error 7.5e-5); 2^j added to the
+// exponent field.  Inputs are clamped at -125 so the exponent stays normal.
+__device__ __forceinline__ uint64_t exp2_poly2(uint64_t x2) {
+  constexpr float kC0 = 0.9999280571937561f, kC1 = 0.6932609677314758f;
+  constexpr float kC2 = 0.2426111251115799f, kC3 = 0.0551716685295105f;
+  constexpr float kMagic = 12582912.0f;  // 1.5 * 2^23
+  float x0, x1;
+  ptx::f2unpack(x2, x0, x1);
+  x2 = ptx::f2pack(fmaxf(x0, -125.f), fmaxf(x1, -125.f));
+  const uint64_t magic = ptx::f2pack(kMagic, kMagic);
+  const uint64_t t = ptx::fadd2(x2, magic);
+  const uint64_t f = ptx::fsub2(x2, ptx::fsub2(t, magic));
+  uint64_t p = ptx::ffma2(f, ptx::f2pack(kC3, kC3), ptx::f2pack(kC2, kC2));
+  p = ptx::ffma2(f, p, ptx::f2pack(kC1, kC1));
+  p = ptx::ffma2(f, p, ptx::f2pack(kC0, kC0));
+  float p0, p1, t0, t1;
+  ptx::f2unpack(p, p0, p1);
+  ptx::f2unpack(t, t0, t1);
+  return ptx::f2pack(__uint_as_float(__float_as_uint(p0) + (__float_as_uint(t0) << 23)),
+                     __uint_as_float(__float_as_uint(p1) + (__float_as_uint(t1) << 23)));
+}
+
 // One thread per query row; warp w of the group reads TMEM lanes
 // [32*(w%4), 32*(w%4)+32), so row r = 32*(w%4) + lane is the tile row.
-template <int D, bool CAUSAL>
+// Of every 4 column pairs, kPolyPairs go through exp2_poly2 (FMA pipe) and
+// the rest through ex2.approx (MUFU), so both units share the exponentials.
+template <int D, bool CAUSAL, int kPolyPairs>
 __device__ void softmax_role(const Shared& sh, const KernelArgs& a, uint32_t tmem, int s, int bh,
                              int qpair, int warp_in_group) {
   const int qt = 2 * qpair + s;
   const int n_s = kv_tiles_for<CAUSAL>(qt, a.n_qtiles);
   if (n_s == 0) return;
-  const int r = warp_in_group * 32 + static_cast<int>(ptx::lane_id());
+  const int lane = static_cast<int>(ptx::lane_id());
+  const int r = warp_in_group * 32 + lane;
   const uint32_t lane_off = static_cast<uint32_t>(warp_in_group * 32) << 16;
   const uint32_t t_s = tmem + lane_off + 128u * s;
   const uint32_t t_o = tmem + lane_off + 256u + 128u * s;
   const float sl2 = a.scale_log2;
+  const uint64_t sl2x2 = ptx::f2pack(sl2, sl2);
 
   float m = -INFINITY;  // running max of scale*log2(e)*score (log2 units)
   float l = 0.f;        // running sum of weights, relative to 2^m
@@ -309,6 +427,7 @@ __device__ void softmax_role(const Shared& sh, const KernelArgs& a, uint32_t tme
   for (int j = 0; j < n_s; ++j) {
     if (!wait_warp(sh, a.status, &sh.s_full[s], static_cast<uint32_t>(j & 1))) return;
     ptx::tc_fence_after_sync();
+    if (r == 0) ATTN_TRACE(s == 0 ? kTrSm0Full : kTrSm1Full, j);
 
     uint32_t sr[128];
     ptx::tmem_ld32(t_s + 0, sr + 0);
@@ -323,24 +442,30 @@ __device__ void softmax_role(const Shared& sh, const KernelArgs& a, uint32_t tme
     float x[128];
 #pragma unroll
     for (int c = 0; c < 128; ++c) x[c] = __uint_as_float(sr[c]);
+    if (r == 0) ATTN_TRACE(s == 0 ? kTrSm0Ld : kTrSm1Ld, j);
 
     // Causal: the last visited tile is the diagonal one (key tile == query
     // tile); key c of it is visible to row r iff c <= r.
-    if (CAUSAL && j == n_s - 1) {
+    const bool diag = CAUSAL && j == n_s - 1;
+    if (diag) {
 #pragma unroll
       for (int c = 0; c < 128; ++c)
         if (c > r) x[c] = -INFINITY;
     }
 
+    // Row max: four independent chains of three-input maxima.
     float mx0 = x[0], mx1 = x[1], mx2 = x[2], mx3 = x[3];
 #pragma unroll
-    for (int c = 4; c < 128; c += 4) {
-      mx0 = fmaxf(mx0, x[c]);
-      mx1 = fmaxf(mx1, x[c + 1]);
-      mx2 = fmaxf(mx2, x[c + 2]);
-      mx3 = fmaxf(mx3, x[c + 3]);
+    for (int c = 4; c + 8 <= 128; c += 8) {
+      mx0 = ptx::max3(mx0, x[c], x[c + 1]);
+      mx1 = ptx::max3(mx1, x[c + 2], x[c + 3]);
+      mx2 = ptx::max3(mx2, x[c + 4], x[c + 5]);
+      mx3 = ptx::max3(mx3, x[c + 6], x[c + 7]);
     }
+    mx0 = ptx::max3(mx0, x[124], x[125]);
+    mx1 = ptx::max3(mx1, x[126], x[127]);
     const float tile_max = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * sl2;
+    if (r == 0) ATTN_TRACE(s == 0 ? kTrSm0Max : kTrSm1Max, j);
 
     // Lazy rescale: raise the running max only when it moves by > tau.
     float alpha = 1.f;
@@ -350,28 +475,9 @@ __device__ void softmax_role(const Shared& sh, const KernelArgs& a, uint32_t tme
       m = tile_max;
       rescale = (j > 0);
     }
-    const float neg_m = -m;
-
-    float l0 = 0.f, l1 = 0.f, l2 = 0.f, l3 = 0.f;
-    uint32_t pk[64];
-#pragma unroll
-    for (int c = 0; c < 128; c += 4) {
-      const float p0 = ptx::ex2_approx(fmaf(x[c], sl2, neg_m));
-      const float p1 = ptx::ex2_approx(fmaf(x[c + 1], sl2, neg_m));
-      const float p2 = ptx::ex2_approx(fmaf(x[c + 2], sl2, neg_m));
-      const float p3 = ptx::ex2_approx(fmaf(x[c + 3], sl2, neg_m));
-      l0 += p0; l1 += p1; l2 += p2; l3 += p3;
-      pk[c / 2] = ptx::pack_bf16x2(p0, p1);
-      pk[c / 2 + 1] = ptx::pack_bf16x2(p2, p3);
-    }
-    l = l * alpha + ((l0 + l1) + (l2 + l3));
-
-    // P_s (bf16 pairs) over the first 64 columns of the S_s region.
-    ptx::tmem_st32(t_s + 0, pk + 0);
-    ptx::tmem_st32(t_s + 32, pk + 32);
-
     // O_s *= alpha for the rows whose max moved (PV_s(j-1) is complete: its
-    // commit preceded the one that published S_s(j)).
+    // commit preceded the one that published S_s(j)).  Done before any P is
+    // published, so the first half of PV_s(j) sees the rescaled O.
     if (__any_sync(0xffffffffu, rescale)) {
 #pragma unroll 1
       for (int c0 = 0; c0 < D; c0 += 32) {
@@ -383,9 +489,61 @@ __device__ void softmax_role(const Shared& sh, const KernelArgs& a, uint32_t tme
         ptx::tmem_st32(t_o + c0, ov);
       }
     }
-    ptx::tmem_st_wait();
-    ptx::tc_fence_before_sync();
-    ptx::mbar_arrive(&sh.p_ready[s]);
+    const uint64_t negm2 = ptx::f2pack(-m, -m);
+#if ATTN_SOFTMAX_ORDER
+    // Turn order: group 0 waits for group 1's step j-1, group 1 for group
+    // 0's step j (if group 0 has a step j: under the causal mask group 1
+    // visits one more K/V tile than group 0).
+    {
+      const int other_n = kv_tiles_for<CAUSAL>(2 * qpair + (1 - s), a.n_qtiles);
+      const bool must_wait = (s == 0) ? (j >= 1 && j - 1 < other_n) : (j < other_n);
+      const uint32_t par = static_cast<uint32_t>(((s == 0) ? (j - 1) : j) & 1);
+      if (must_wait && !wait_warp(sh, a.status, &sh.exp_token[s], par)) return;
+    }
+#endif
+
+    uint64_t lsum2a = ptx::f2pack(0.f, 0.f), lsum2b = lsum2a;
+#pragma unroll
+    for (int half = 0; half < 2; ++half) {
+      uint32_t pk[32];
+#pragma unroll
+      for (int q = 0; q < 32; ++q) {
+        const int c = 64 * half + 2 * q;
+        const uint64_t y2 = ptx::ffma2(ptx::f2pack(x[c], x[c + 1]), sl2x2, negm2);
+        uint64_t p2;
+        if ((q & 3) < kPolyPairs) {
+          // A masked key (-inf) comes out as 2^-125 rather than 0: against a
+          // row sum l >= 1 and O entries summed in fp32 that weight is far
+          // below one unit in the last place, so it cannot change O or LSE.
+          p2 = exp2_poly2(y2);
+        } else {
+          float y0, y1;
+          ptx::f2unpack(y2, y0, y1);
+          p2 = ptx::f2pack(ptx::ex2_approx(y0), ptx::ex2_approx(y1));
+        }
+        if (q & 1) lsum2b = ptx::fadd2(lsum2b, p2);
+        else lsum2a = ptx::fadd2(lsum2a, p2);
+        float p0, p1;
+        ptx::f2unpack(p2, p0, p1);
+        pk[q] = ptx::pack_bf16x2(p0, p1);
+      }
+      // P_s keys [64*half, 64*half+64) as bf16 pairs over TMEM columns
+      // [32*half, 32*half+32) of the S_s region; publish this half at once.
+      ptx::tmem_st32(t_s + 32 * half, pk);
+      ptx::tmem_st_wait();
+      ptx::tc_fence_before_sync();
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive(&sh.p_ready[2 * s + half]);
+      if (r == 0) ATTN_TRACE(s == 0 ? (half ? kTrSm0Pb : kTrSm0Pa) : (half ? kTrSm1Pb : kTrSm1Pa), j);
+    }
+#if ATTN_SOFTMAX_ORDER
+    __syncwarp();
+    if (lane == 0) ptx::mbar_arrive(&sh.exp_token[1 - s]);
+#endif
+    float la0, la1, lb0, lb1;
+    ptx::f2unpack(lsum2a, la0, la1);
+    ptx::f2unpack(lsum2b, lb0, lb1);
+    l = l * alpha + ((la0 + la1) + (lb0 + lb1));
   }
 
   // Epilogue: O_s / l -> bf16 rows; LSE = (m + log2 l) * ln 2.
@@ -413,7 +571,7 @@ __device__ void softmax_role(const Shared& sh, const KernelArgs& a, uint32_t tme
 }
 
 // ------------------------------------------------------------------- kernel
-template <int D, bool CAUSAL>
+template <int D, bool CAUSAL, int kPolyPairs>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap_q,
                     const __grid_constant__ CUtensorMap tmap_k,
@@ -430,17 +588,23 @@ __global__ void __launch_bounds__(kThreads, 1)
   sh.kv_empty = bars + 1 + C::kStages;
   sh.s_full = bars + 1 + 2 * C::kStages;
   sh.p_ready = sh.s_full + 2;
-  sh.o_final = sh.p_ready + 2;
+  sh.o_final = sh.p_ready + 4;
   sh.drain = sh.o_final + 2;
+  sh.exp_token = sh.drain + 1;
   sh.tmem_base = reinterpret_cast<uint32_t*>(smem + C::kMiscOff);
   sh.abort_flag = reinterpret_cast<volatile int*>(smem + C::kMiscOff + 4);
 
   const int warp = threadIdx.x / 32;
   // Heaviest query tiles first under the causal mask (blockIdx.y = 0 runs
   // first and takes the last pair).
+#if ATTN_HEAD_MAJOR
+  const int bh = blockIdx.y;
+  const int qp_idx = blockIdx.x;
+#else
   const int bh = blockIdx.x;
-  const int qpair = CAUSAL ? (args.n_qpairs - 1 - static_cast<int>(blockIdx.y))
-                           : static_cast<int>(blockIdx.y);
+  const int qp_idx = blockIdx.y;
+#endif
+  const int qpair = CAUSAL ? (args.n_qpairs - 1 - qp_idx) : qp_idx;
 
   if (threadIdx.x == 0) {
     ptx::mbar_init(sh.q_full, 1);
@@ -450,10 +614,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int i = 0; i < 2; ++i) {
       ptx::mbar_init(&sh.s_full[i], 1);
-      ptx::mbar_init(&sh.p_ready[i], 128);
+      ptx::mbar_init(&sh.p_ready[2 * i], 4);
+      ptx::mbar_init(&sh.p_ready[2 * i + 1], 4);
       ptx::mbar_init(&sh.o_final[i], 1);
     }
     ptx::mbar_init(sh.drain, 1);
+    ptx::mbar_init(&sh.exp_token[0], 4);
+    ptx::mbar_init(&sh.exp_token[1], 4);
     *sh.abort_flag = 0;
     ptx::fence_barrier_init();
   }
@@ -466,24 +633,29 @@ __global__ void __launch_bounds__(kThreads, 1)
     ptx::tmem_alloc(sh.tmem_base, 512);
     ptx::tmem_relinquish();
   }
+  if (warp >= 8) ptx::setmaxnreg_dec<kRegsOther>();
   ptx::tc_fence_before_sync();
   __syncthreads();
   ptx::tc_fence_after_sync();
   const uint32_t tmem = *sh.tmem_base;
+  if (threadIdx.x == 0) ATTN_TRACE(kTrStart, 0);
 
+  // Register split (see kRegsSoftmax): the producer/MMA warpgroup released
+  // its share before the CTA-wide barrier above.
   if (warp < 8) {
-    softmax_role<D, CAUSAL>(sh, args, tmem, warp / 4, bh, qpair, warp % 4);
+    ptx::setmaxnreg_inc<kRegsSoftmax>();
+    softmax_role<D, CAUSAL, kPolyPairs>(sh, args, tmem, warp / 4, bh, qpair, warp % 4);
   } else if (warp == 8) {
     if (ptx::lane_id() == 0)
       producer_role<D, CAUSAL>(sh, args, smem, &tmap_q, &tmap_k, &tmap_v, bh, qpair);
     __syncwarp();
   } else if (warp == 9) {
-    if (ptx::lane_id() == 0) mma_role<D, CAUSAL>(sh, args, smem, tmem, qpair);
-    __syncwarp();
+    mma_role<D, CAUSAL>(sh, args, smem, tmem, qpair);
   }
 
   ptx::tc_fence_before_sync();
   __syncthreads();
+  if (threadIdx.x == 0) ATTN_TRACE(kTrEnd, 0);
   if (warp == 9) {
     ptx::tc_fence_after_sync();
     ptx::tmem_dealloc(tmem, 512);
