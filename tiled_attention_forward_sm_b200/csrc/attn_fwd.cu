@@ -113,6 +113,8 @@ int launch(const void* q, const void* k, const void* v, void* o, float* lse, int
   args.N = N;
   args.n_qtiles = N / kBlockM;
   args.n_qpairs = (args.n_qtiles + 1) / 2;
+  args.BH = B * H;
+  args.n_items = args.BH * args.n_qpairs;
   args.scale_log2 = scale * 1.4426950408889634f;
   args.status = st.status;
 
@@ -136,11 +138,9 @@ int launch(const void* q, const void* k, const void* v, void* o, float* lse, int
   }
   cudaLaunchConfig_t cfg;
   std::memset(&cfg, 0, sizeof cfg);
-#if ATTN_HEAD_MAJOR
-  cfg.gridDim = dim3(static_cast<unsigned>(args.n_qpairs), static_cast<unsigned>(B * H), 1);
-#else
-  cfg.gridDim = dim3(static_cast<unsigned>(B * H), static_cast<unsigned>(args.n_qpairs), 1);
-#endif
+  // Persistent: one CTA per SM (at most one per work item).
+  const int grid = args.n_items < st.num_sms ? args.n_items : st.num_sms;
+  cfg.gridDim = dim3(static_cast<unsigned>(grid), 1, 1);
   cfg.blockDim = dim3(kThreads, 1, 1);
   cfg.dynamicSmemBytes = C::kSmemBytes;
   cfg.stream = stream;
@@ -182,9 +182,8 @@ extern "C" int attn_check_args(const void* q, const void* k, const void* v, cons
   if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
   if (N % kBlockM != 0) return ATTN_ERR_UNSUPPORTED;
   const uint64_t rows = static_cast<uint64_t>(B) * H * N;
-  if (rows >= (1ull << 31) || static_cast<uint64_t>(B) * H > 0x7FFFFFFFull ||
-      N / (2 * kBlockM) + 1 > 65535 || (ATTN_HEAD_MAJOR && static_cast<uint64_t>(B) * H > 65535))
-    return ATTN_ERR_UNSUPPORTED;
+  // Work items (B*H*ceil(N/256)) are numbered in int.
+  if (rows >= (1ull << 31)) return ATTN_ERR_UNSUPPORTED;
   const uintptr_t al = reinterpret_cast<uintptr_t>(q) | reinterpret_cast<uintptr_t>(k) |
                        reinterpret_cast<uintptr_t>(v) | reinterpret_cast<uintptr_t>(o);
   if (al & 15u) return ATTN_ERR_MISALIGNED;

@@ -10,19 +10,24 @@
 //  * section "Faire avancer plusieurs tuiles sans ecraser leurs donnees":
 //    thread groups with distinct roles (data loading, softmax, MMA issue),
 //    one tile in softmax while another occupies the tensor cores, several
-//    result regions in Tensor Memory each with a producer/consumer lifetime;
+//    result regions in Tensor Memory each with a producer/consumer lifetime,
+//    and the first part of the weights announced before the rest;
 //  * section "Deplacer une partie des exponentielles": a common scale kept
 //    between old and new contributions, with some rescalings skipped under a
-//    condition that keeps sums consistent and values in range.
+//    condition that keeps sums consistent and values in range; part of the
+//    exponentials can be computed with ordinary multiply-adds.
 //
-// CTA work unit: two 128-row Q tiles (Q0, Q1) of one (batch, head), i.e.
-// 256 query rows, against the K/V tiles they can see (128 keys per tile).
+// Work item: two 128-row Q tiles (Q0, Q1) of one (batch, head), i.e. 256
+// query rows, against the K/V tiles they can see (128 keys per tile).  The
+// kernel is persistent: one CTA per SM walks a static list of work items
+// (heaviest first under the causal mask, dealt out in a snake order so every
+// CTA gets a similar total), and all barrier phases run on across items.
 //
 // Roles (12 warps, 384 threads):
 //   warps 0-3   softmax group 0 (Q0): one thread per query row; also applies
 //               the lazy O rescale and the epilogue for Q0
 //   warps 4-7   softmax group 1 (Q1), same for Q1
-//   warp  8     TMA producer: Q0/Q1 once, then K_j, V_j through a ring
+//   warp  8     TMA producer: Q0/Q1 per item, then K_j, V_j through a ring
 //   warp  9     TMEM allocator and tcgen05 MMA issuer (warp-uniform control,
 //               one elected lane issues)
 //   warps 10-11 idle
@@ -33,7 +38,7 @@
 //   cols [256,256+D) O0 accumulator (fp32)
 //   cols [384,384+D) O1 accumulator
 //
-// MMA issue order per K/V step j (single thread, in-order tensor pipe):
+// MMA issue order per K/V step j (one thread, in-order tensor pipe):
 //   PV0(j-1) ... S0(j) ... PV1(j-1) ... S1(j)
 // so the commit that publishes S_s(j) also guarantees PV_s(j-1) finished:
 // the softmax group may rescale O_s in place as soon as it sees S_s(j).
@@ -54,24 +59,15 @@ constexpr int kStatusDeviceTimeout = -5;
 // status word and the CTA's abort flag, and every role then leaves its loop.
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s
 
-// The two softmax groups take turns on the special-function units: group 0
-// runs its exponentials for step j, then group 1 for step j, then group 0
-// for step j+1, ...  Without the ordering both groups' exponential phases
-// overlap and each runs at half rate, lengthening the per-tile critical path.
-#ifndef ATTN_SOFTMAX_ORDER
-#define ATTN_SOFTMAX_ORDER 0
+// Softmax arithmetic form: packed f32x2 FMA/ADD (1) or scalar FMA/ADD (0).
+// Measured on B200 the packed form is faster.
+#ifndef ATTN_PACKED_SOFTMAX
+#define ATTN_PACKED_SOFTMAX 1
 #endif
 
 // K/V ring depth for d = 128 (each stage holds one 128 x 128 bf16 tile).
 #ifndef ATTN_KV_STAGES_D128
 #define ATTN_KV_STAGES_D128 4
-#endif
-
-// CTA launch order: head-major (all query pairs of one head adjacent, so the
-// CTAs that stream the same K/V run together and share it through L2) or
-// pair-major (every head's heaviest pair first).
-#ifndef ATTN_HEAD_MAJOR
-#define ATTN_HEAD_MAJOR 0
 #endif
 
 constexpr int kBlockM = 128;  // query rows per Q tile
@@ -92,8 +88,8 @@ constexpr float kRescaleTau = 8.0f;
 
 // Optional timeline tracing (compiled in only with ATTN_TRACE_ENABLED; the
 // library build leaves it out): clock64 stamps at each role's hand-off for
-// the first kTraceCtas CTAs and kTraceSteps K/V steps, written to a device
-// buffer registered by the tracing build's host code.
+// the first work item of the first kTraceCtas CTAs and kTraceSteps K/V
+// steps, written to a device buffer registered by the tracing build.
 enum TraceEvent : int {
   kTrMmaS0 = 0, kTrMmaPV0a, kTrMmaPV0b, kTrMmaS1, kTrMmaPV1a, kTrMmaPV1b, kTrMmaV,
   kTrSm0Full, kTrSm0Ld, kTrSm0Max, kTrSm0Pa, kTrSm0Pb,
@@ -105,7 +101,7 @@ constexpr int kTraceSteps = 72;
 #ifdef ATTN_TRACE_ENABLED
 __device__ unsigned long long* g_trace_buf = nullptr;
 __device__ __forceinline__ void trace_stamp(int ev, int j) {
-  const int cta = blockIdx.x + blockIdx.y * gridDim.x;
+  const int cta = blockIdx.x;
   if (g_trace_buf != nullptr && cta < kTraceCtas && j >= 0 && j < kTraceSteps)
     g_trace_buf[(static_cast<size_t>(cta) * kTrNumEvents + ev) * kTraceSteps + j] = clock64();
 }
@@ -120,6 +116,8 @@ struct KernelArgs {
   int N;              // keys/queries per head (multiple of 128)
   int n_qtiles;       // N / 128
   int n_qpairs;       // ceil(n_qtiles / 2)
+  int BH;             // B * H
+  int n_items;        // BH * n_qpairs work items
   float scale_log2;   // scale * log2(e)
   int* status;        // device status word
 };
@@ -134,10 +132,9 @@ struct Config {
   static constexpr int kQOff = 0;
   static constexpr int kKVOff = 2 * kTileBytes;
   static constexpr int kBarOff = kKVOff + kStages * kTileBytes;
-  // barriers: q_full, kv_full[S], kv_empty[S], s_full[2], p_ready[2 tiles][2
-  // halves], o_final[2], drain
-  // + exp_token[2] (softmax group s may run its exponentials)
-  static constexpr int kNumBars = 1 + 2 * kStages + 2 + 4 + 2 + 1 + 2;
+  // barriers: q_full[2], q_empty[2], kv_full[S], kv_empty[S], s_full[2],
+  // p_ready[2 tiles][2 halves], o_final[2], drain
+  static constexpr int kNumBars = 4 + 2 * kStages + 2 + 4 + 2 + 1;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;
   static constexpr int kSmemBytes = kMiscOff + 16 + 1024;  // + alignment slack
   static constexpr uint32_t kIdescQK = ptx::idesc_bf16_f32(128, kBlockN, 0, 0);
@@ -145,14 +142,14 @@ struct Config {
 };
 
 struct Shared {
-  uint64_t* q_full;
-  uint64_t* kv_full;
-  uint64_t* kv_empty;
-  uint64_t* s_full;
-  uint64_t* p_ready;
-  uint64_t* o_final;
+  uint64_t* q_full;    // [2] Q_s landed in shared memory
+  uint64_t* q_empty;   // [2] last S_s of the item done: Q_s buffer reusable
+  uint64_t* kv_full;   // [kStages]
+  uint64_t* kv_empty;  // [kStages]
+  uint64_t* s_full;    // [2] S_s(j) in TMEM
+  uint64_t* p_ready;   // [2*s + half] half of P_s(j) in TMEM
+  uint64_t* o_final;   // [2] last PV_s of the item done
   uint64_t* drain;
-  uint64_t* exp_token;
   uint32_t* tmem_base;
   volatile int* abort_flag;
 };
@@ -212,47 +209,80 @@ __device__ __forceinline__ int kv_tiles_for(int qt, int n_qtiles) {
   return CAUSAL ? qt + 1 : n_qtiles;
 }
 
+// ------------------------------------------------------------ work schedule
+struct Item {
+  int bh;     // batch * H + head
+  int qpair;  // Q tiles 2*qpair and 2*qpair + 1
+  int n0;     // K/V tiles Q0 visits (0: no such tile)
+  int n1;     // K/V tiles Q1 visits
+};
+
+// Items are numbered pair-major with the heaviest pairs first under the
+// causal mask; round r deals items [r*G, r*G + G) to the G CTAs, reversing
+// the direction every other round (snake), so each CTA's total work is
+// nearly the same.  Returns false once this CTA has no item in round r.
+template <bool CAUSAL>
+__device__ __forceinline__ bool item_for(int r, const KernelArgs& a, Item& it) {
+  const int G = static_cast<int>(gridDim.x), c = static_cast<int>(blockIdx.x);
+  const int idx = r * G + ((r & 1) ? (G - 1 - c) : c);
+  if (idx >= a.n_items) return false;
+  const int qp_idx = idx / a.BH;
+  it.bh = idx - qp_idx * a.BH;
+  it.qpair = CAUSAL ? (a.n_qpairs - 1 - qp_idx) : qp_idx;
+  it.n0 = kv_tiles_for<CAUSAL>(2 * it.qpair, a.n_qtiles);
+  it.n1 = kv_tiles_for<CAUSAL>(2 * it.qpair + 1, a.n_qtiles);
+  return true;
+}
+
 // ----------------------------------------------------------------- producer
 template <int D, bool CAUSAL>
 __device__ void producer_role(const Shared& sh, const KernelArgs& a, uint8_t* smem,
                               const CUtensorMap* tq, const CUtensorMap* tk,
-                              const CUtensorMap* tv, int bh, int qpair) {
+                              const CUtensorMap* tv) {
   using C = Config<D>;
-  const int qt0 = 2 * qpair, qt1 = 2 * qpair + 1;
-  const int n0 = kv_tiles_for<CAUSAL>(qt0, a.n_qtiles);
-  const int n1 = kv_tiles_for<CAUSAL>(qt1, a.n_qtiles);
-  const int n = n0 > n1 ? n0 : n1;
-  const int row0 = bh * a.N;  // first row of this (b, h) in the 2-D views
   const uint64_t pol_q = ptx::policy_evict_first();
   const uint64_t pol_kv = ptx::policy_evict_last();
-
-  // Q tiles (Q1 only if it exists)
-  const int nq = (n1 > 0) ? 2 : 1;
-  ptx::mbar_arrive_expect_tx(sh.q_full, nq * C::kTileBytes);
-  for (int s = 0; s < nq; ++s)
-    for (int b = 0; b < C::kBoxes; ++b)
-      ptx::tma_load_2d(tq, sh.q_full, smem + C::kQOff + s * C::kTileBytes + b * C::kBoxBytes,
-                       64 * b, row0 + (2 * qpair + s) * kBlockM, pol_q);
-
-  int issued = 0;
+  int q_loads[2] = {0, 0};  // loads into Q buffer s so far
+  int issued = 0;           // K/V tiles issued into the ring so far
   bool ok = true;
-  for (int j = 0; j < n && ok; ++j) {
-    for (int which = 0; which < 2; ++which) {  // 0: K_j, 1: V_j
-      const int st = issued % C::kStages;
-      const uint32_t ph = (issued / C::kStages) & 1;
-      if (!wait_one(sh, a.status, &sh.kv_empty[st], ph ^ 1)) { ok = false; break; }
-      uint8_t* dst = smem + C::kKVOff + st * C::kTileBytes;
-      ATTN_TRACE(which == 0 ? kTrProdK : kTrProdV, j);
-      ptx::mbar_arrive_expect_tx(&sh.kv_full[st], C::kTileBytes);
-      const CUtensorMap* m = which == 0 ? tk : tv;
+  Item it;
+  for (int r = 0; ok && item_for<CAUSAL>(r, a, it); ++r) {
+    const int n = it.n0 > it.n1 ? it.n0 : it.n1;
+    const int row0 = it.bh * a.N;  // first row of this (b, h) in the 2-D views
+    // Q_s, once the previous item's last S_s no longer needs the buffer.
+    for (int s = 0; s < 2 && ok; ++s) {
+      if ((s == 0 ? it.n0 : it.n1) == 0) continue;
+      if (q_loads[s] > 0 &&
+          !wait_one(sh, a.status, &sh.q_empty[s], static_cast<uint32_t>((q_loads[s] - 1) & 1))) {
+        ok = false;
+        break;
+      }
+      ptx::mbar_arrive_expect_tx(&sh.q_full[s], C::kTileBytes);
       for (int b = 0; b < C::kBoxes; ++b)
-        ptx::tma_load_2d(m, &sh.kv_full[st], dst + b * C::kBoxBytes, 64 * b,
-                         row0 + j * kBlockN, pol_kv);
-      ++issued;
+        ptx::tma_load_2d(tq, &sh.q_full[s], smem + C::kQOff + s * C::kTileBytes + b * C::kBoxBytes,
+                         64 * b, row0 + (2 * it.qpair + s) * kBlockM, pol_q);
+      ++q_loads[s];
+    }
+    for (int j = 0; j < n && ok; ++j) {
+      for (int which = 0; which < 2; ++which) {  // 0: K_j, 1: V_j
+        const int st = issued % C::kStages;
+        const uint32_t ph = (issued / C::kStages) & 1;
+        if (!wait_one(sh, a.status, &sh.kv_empty[st], ph ^ 1)) { ok = false; break; }
+        uint8_t* dst = smem + C::kKVOff + st * C::kTileBytes;
+        ATTN_TRACE(which == 0 ? kTrProdK : kTrProdV, r == 0 ? j : -1);
+        ptx::mbar_arrive_expect_tx(&sh.kv_full[st], C::kTileBytes);
+        const CUtensorMap* m = which == 0 ? tk : tv;
+        for (int b = 0; b < C::kBoxes; ++b)
+          ptx::tma_load_2d(m, &sh.kv_full[st], dst + b * C::kBoxBytes, 64 * b,
+                           row0 + j * kBlockN, pol_kv);
+        ++issued;
+      }
     }
   }
   // Drain: every load issued must land before the CTA may exit.
-  wait_one(sh, a.status, sh.q_full, 0, true);
+  for (int s = 0; s < 2; ++s)
+    if (q_loads[s] > 0)
+      wait_one(sh, a.status, &sh.q_full[s], static_cast<uint32_t>((q_loads[s] - 1) & 1), true);
   for (int t = (issued > C::kStages ? issued - C::kStages : 0); t < issued; ++t)
     wait_one(sh, a.status, &sh.kv_full[t % C::kStages], (t / C::kStages) & 1, true);
 }
@@ -264,12 +294,8 @@ __device__ void producer_role(const Shared& sh, const KernelArgs& a, uint8_t* sm
 // is the low 14 bits, in 16-byte units; no carry can leave it because
 // shared memory is below 256 KB).
 template <int D, bool CAUSAL>
-__device__ void mma_role(const Shared& sh, const KernelArgs& a, uint8_t* smem, uint32_t tmem,
-                         int qpair) {
+__device__ void mma_role(const Shared& sh, const KernelArgs& a, uint8_t* smem, uint32_t tmem) {
   using C = Config<D>;
-  const int n0 = kv_tiles_for<CAUSAL>(2 * qpair, a.n_qtiles);
-  const int n1 = kv_tiles_for<CAUSAL>(2 * qpair + 1, a.n_qtiles);
-  const int n = n0 > n1 ? n0 : n1;
   const uint32_t t_s[2] = {tmem + 0, tmem + 128};
   const uint32_t t_o[2] = {tmem + 256, tmem + 384};
   // K-major (Q, K): SBO = 1024 B between 8-row groups; MN-major (V):
@@ -301,11 +327,14 @@ __device__ void mma_role(const Shared& sh, const KernelArgs& a, uint8_t* smem, u
                         C::kIdescPV, (accumulate | static_cast<uint32_t>(kk > 0)));
     }
   };
-  int trace_j = 0;
+  int trace_j = -1;
   (void)trace_j;
+  int p_count[2] = {0, 0};  // P_s publications consumed so far (all items)
   // Both halves of PV_s(j); the first half is issued as soon as the softmax
   // has published keys 0-63 of P, before keys 64-127 are ready.
-  auto issue_pv = [&](int s, int stage, uint32_t accumulate, uint32_t parity) -> bool {
+  auto issue_pv = [&](int s, int stage, uint32_t accumulate) -> bool {
+    const uint32_t parity = static_cast<uint32_t>(p_count[s] & 1);
+    ++p_count[s];
     if (!wait_warp(sh, a.status, &sh.p_ready[2 * s], parity)) return false;
     ptx::tc_fence_after_sync();
     ATTN_TRACE(s == 0 ? kTrMmaPV0a : kTrMmaPV1a, trace_j);
@@ -316,58 +345,76 @@ __device__ void mma_role(const Shared& sh, const KernelArgs& a, uint8_t* smem, u
     issue_pv_half(s, 1, stage, accumulate);
     return true;
   };
+  // S_s(j) of an item visiting n_s K/V tiles; after its last S the Q_s
+  // buffer is handed back to the producer.
+  auto issue_s = [&](int s, int j, int n_s, int stage) {
+    issue_qk(s, stage);
+    ptx::commit_elect(&sh.s_full[s]);
+    if (j == n_s - 1) ptx::commit_elect(&sh.q_empty[s]);
+  };
 
   int consumed = 0;
+  int q_uses[2] = {0, 0};
   auto stage_of = [&](int c) { return c % C::kStages; };
   auto phase_of = [&](int c) { return static_cast<uint32_t>((c / C::kStages) & 1); };
 
-  if (!wait_warp(sh, a.status, sh.q_full, 0)) goto done;
-  {
-    // step 0: S0(0), S1(0)
-    const int ck = consumed++;
-    if (!wait_warp(sh, a.status, &sh.kv_full[stage_of(ck)], phase_of(ck))) goto done;
-    ptx::tc_fence_after_sync();
-    ATTN_TRACE(kTrMmaS0, 0);
-    if (n0 > 0) { issue_qk(0, stage_of(ck)); ptx::commit_elect(&sh.s_full[0]); }
-    ATTN_TRACE(kTrMmaS1, 0);
-    if (n1 > 0) { issue_qk(1, stage_of(ck)); ptx::commit_elect(&sh.s_full[1]); }
-    ptx::commit_elect(&sh.kv_empty[stage_of(ck)]);
-
-    // Per step j: both K/V waits come first (the tiles are normally resident
-    // long before), so that PV_s(j) and S_s(j+1) issue back to back and no
-    // barrier round trip sits on a tile's S -> softmax -> PV -> S chain.
-    for (int j = 0; j < n; ++j) {
-      const int cv = consumed++;
-      trace_j = j;
-      if (!wait_warp(sh, a.status, &sh.kv_full[stage_of(cv)], phase_of(cv))) goto done;
-      const int ck2 = (j + 1 < n) ? consumed++ : -1;
-      if (ck2 >= 0 &&
-          !wait_warp(sh, a.status, &sh.kv_full[stage_of(ck2)], phase_of(ck2)))
+  Item it;
+  for (int r = 0; item_for<CAUSAL>(r, a, it); ++r) {
+    const int n0 = it.n0, n1 = it.n1;
+    const int n = n0 > n1 ? n0 : n1;
+    for (int s = 0; s < 2; ++s) {
+      if ((s == 0 ? n0 : n1) == 0) continue;
+      if (!wait_warp(sh, a.status, &sh.q_full[s], static_cast<uint32_t>(q_uses[s] & 1)))
         goto done;
+      ++q_uses[s];
+    }
+    {
+      // step 0: S0(0), S1(0)
+      const int ck = consumed++;
+      if (!wait_warp(sh, a.status, &sh.kv_full[stage_of(ck)], phase_of(ck))) goto done;
       ptx::tc_fence_after_sync();
-      ATTN_TRACE(kTrMmaV, j);
-      const uint32_t pj = static_cast<uint32_t>(j & 1);
-      const uint32_t acc = j > 0 ? 1u : 0u;
-      if (j < n0) {
-        if (!issue_pv(0, stage_of(cv), acc, pj)) goto done;
-        ATTN_TRACE(kTrMmaPV0end, j);
-        if (j == n0 - 1) ptx::commit_elect(&sh.o_final[0]);
-      }
-      if (ck2 >= 0) {
-        ATTN_TRACE(kTrMmaS0, j + 1);
-        if (j + 1 < n0) { issue_qk(0, stage_of(ck2)); ptx::commit_elect(&sh.s_full[0]); }
-        ATTN_TRACE(kTrMmaS0end, j + 1);
-      }
-      if (j < n1) {
-        if (!issue_pv(1, stage_of(cv), acc, pj)) goto done;
-        if (j == n1 - 1) ptx::commit_elect(&sh.o_final[1]);
-      }
-      ptx::commit_elect(&sh.kv_empty[stage_of(cv)]);
-      if (ck2 >= 0) {
-        ATTN_TRACE(kTrMmaS1, j + 1);
-        if (j + 1 < n1) { issue_qk(1, stage_of(ck2)); ptx::commit_elect(&sh.s_full[1]); }
-        ATTN_TRACE(kTrMmaS1end, j + 1);
-        ptx::commit_elect(&sh.kv_empty[stage_of(ck2)]);
+      ATTN_TRACE(kTrMmaS0, r == 0 ? 0 : -1);
+      if (n0 > 0) issue_s(0, 0, n0, stage_of(ck));
+      ATTN_TRACE(kTrMmaS1, r == 0 ? 0 : -1);
+      if (n1 > 0) issue_s(1, 0, n1, stage_of(ck));
+      ptx::commit_elect(&sh.kv_empty[stage_of(ck)]);
+
+      // Per step j: both K/V waits come first (the tiles are normally
+      // resident long before), so that PV_s(j) and S_s(j+1) issue back to
+      // back and no barrier round trip sits on a tile's S -> softmax -> PV
+      // -> S chain.
+      for (int j = 0; j < n; ++j) {
+        const int cv = consumed++;
+        trace_j = r == 0 ? j : -1;
+        if (!wait_warp(sh, a.status, &sh.kv_full[stage_of(cv)], phase_of(cv))) goto done;
+        const int ck2 = (j + 1 < n) ? consumed++ : -1;
+        if (ck2 >= 0 &&
+            !wait_warp(sh, a.status, &sh.kv_full[stage_of(ck2)], phase_of(ck2)))
+          goto done;
+        ptx::tc_fence_after_sync();
+        ATTN_TRACE(kTrMmaV, trace_j);
+        const uint32_t acc = j > 0 ? 1u : 0u;
+        if (j < n0) {
+          if (!issue_pv(0, stage_of(cv), acc)) goto done;
+          ATTN_TRACE(kTrMmaPV0end, trace_j);
+          if (j == n0 - 1) ptx::commit_elect(&sh.o_final[0]);
+        }
+        if (ck2 >= 0) {
+          ATTN_TRACE(kTrMmaS0, r == 0 ? j + 1 : -1);
+          if (j + 1 < n0) issue_s(0, j + 1, n0, stage_of(ck2));
+          ATTN_TRACE(kTrMmaS0end, r == 0 ? j + 1 : -1);
+        }
+        if (j < n1) {
+          if (!issue_pv(1, stage_of(cv), acc)) goto done;
+          if (j == n1 - 1) ptx::commit_elect(&sh.o_final[1]);
+        }
+        ptx::commit_elect(&sh.kv_empty[stage_of(cv)]);
+        if (ck2 >= 0) {
+          ATTN_TRACE(kTrMmaS1, r == 0 ? j + 1 : -1);
+          if (j + 1 < n1) issue_s(1, j + 1, n1, stage_of(ck2));
+          ATTN_TRACE(kTrMmaS1end, r == 0 ? j + 1 : -1);
+          ptx::commit_elect(&sh.kv_empty[stage_of(ck2)]);
+        }
       }
     }
   }
@@ -403,171 +450,217 @@ __device__ __forceinline__ uint64_t exp2_poly2(uint64_t x2) {
                      __uint_as_float(__float_as_uint(p1) + (__float_as_uint(t1) << 23)));
 }
 
+// Scalar form of exp2_poly2 (same steps, one input).
+__device__ __forceinline__ float exp2_poly1(float x) {
+  constexpr float kC0 = 0.9999280571937561f, kC1 = 0.6932609677314758f;
+  constexpr float kC2 = 0.2426111251115799f, kC3 = 0.0551716685295105f;
+  constexpr float kMagic = 12582912.0f;  // 1.5 * 2^23
+  x = fmaxf(x, -125.f);
+  const float t = x + kMagic;
+  const float f = x - (t - kMagic);
+  float p = fmaf(f, kC3, kC2);
+  p = fmaf(f, p, kC1);
+  p = fmaf(f, p, kC0);
+  return __uint_as_float(__float_as_uint(p) + (__float_as_uint(t) << 23));
+}
+
+// One K/V step of the online softmax for one query row (one thread):
+// S_s(j) from TMEM -> running max (lazy rule) -> weights -> P_s(j) back to
+// TMEM in two published halves; m and l are the row's running max (log2
+// units) and sum.
+template <int D, bool CAUSAL, int kPolyPairs>
+__device__ __forceinline__ bool softmax_step(const Shared& sh, const KernelArgs& a, int s,
+                                             uint32_t t_s, uint32_t t_o, int r, int lane,
+                                             bool diag, bool first, uint32_t s_parity, int tj,
+                                             float& m, float& l) {
+  const float sl2 = a.scale_log2;
+  if (!wait_warp(sh, a.status, &sh.s_full[s], s_parity)) return false;
+  ptx::tc_fence_after_sync();
+  if (r == 0) ATTN_TRACE(s == 0 ? kTrSm0Full : kTrSm1Full, tj);
+
+  uint32_t sr[128];
+  ptx::tmem_ld32(t_s + 0, sr + 0);
+  ptx::tmem_ld32(t_s + 32, sr + 32);
+  ptx::tmem_ld32(t_s + 64, sr + 64);
+  ptx::tmem_ld32(t_s + 96, sr + 96);
+  ptx::tmem_ld_wait_tie(sr + 0);
+  ptx::reg_tie32(sr + 32);
+  ptx::reg_tie32(sr + 64);
+  ptx::reg_tie32(sr + 96);
+
+  float x[128];
+#pragma unroll
+  for (int c = 0; c < 128; ++c) x[c] = __uint_as_float(sr[c]);
+  if (r == 0) ATTN_TRACE(s == 0 ? kTrSm0Ld : kTrSm1Ld, tj);
+
+  // Causal: the last visited tile is the diagonal one (key tile == query
+  // tile); key c of it is visible to row r iff c <= r.
+  if (diag) {
+#pragma unroll
+    for (int c = 0; c < 128; ++c)
+      if (c > r) x[c] = -INFINITY;
+  }
+
+  // Row max: eight independent chains of three-input maxima.
+  float mx[8];
+#pragma unroll
+  for (int k = 0; k < 8; ++k) mx[k] = x[k];
+#pragma unroll
+  for (int c = 8; c + 16 <= 128; c += 16) {
+#pragma unroll
+    for (int k = 0; k < 8; ++k) mx[k] = ptx::max3(mx[k], x[c + 2 * k], x[c + 2 * k + 1]);
+  }
+#pragma unroll
+  for (int k = 0; k < 4; ++k) mx[k] = ptx::max3(mx[k], x[120 + 2 * k], x[121 + 2 * k]);
+  const float tile_max =
+      ptx::max3(ptx::max3(mx[0], mx[1], mx[2]), ptx::max3(mx[3], mx[4], mx[5]), fmaxf(mx[6], mx[7])) *
+      sl2;
+  if (r == 0) ATTN_TRACE(s == 0 ? kTrSm0Max : kTrSm1Max, tj);
+
+  // Lazy rescale: raise the running max only when it moves by > tau.
+  float alpha = 1.f;
+  bool rescale = false;
+  if (tile_max - m > kRescaleTau) {  // also true on the first tile (m = -inf)
+    alpha = ptx::ex2_approx(m - tile_max);  // 0 on the first tile
+    m = tile_max;
+    rescale = !first;
+  }
+  // O_s *= alpha for the rows whose max moved (PV_s(j-1) is complete: its
+  // commit preceded the one that published S_s(j)).  Done before any P is
+  // published, so the first half of PV_s(j) sees the rescaled O.
+  if (__any_sync(0xffffffffu, rescale)) {
+#pragma unroll 1
+    for (int c0 = 0; c0 < D; c0 += 32) {
+      uint32_t ov[32];
+      ptx::tmem_ld32(t_o + c0, ov);
+      ptx::tmem_ld_wait_tie(ov);
+#pragma unroll
+      for (int c = 0; c < 32; ++c) ov[c] = __float_as_uint(__uint_as_float(ov[c]) * alpha);
+      ptx::tmem_st32(t_o + c0, ov);
+    }
+  }
+  const uint64_t sl2x2 = ptx::f2pack(sl2, sl2);
+  const uint64_t negm2 = ptx::f2pack(-m, -m);
+  (void)sl2x2;
+  (void)negm2;
+
+#if ATTN_PACKED_SOFTMAX
+  uint64_t lsum2a = ptx::f2pack(0.f, 0.f), lsum2b = lsum2a;
+#else
+  float ls0 = 0.f, ls1 = 0.f, ls2 = 0.f, ls3 = 0.f;
+#endif
+#pragma unroll
+  for (int half = 0; half < 2; ++half) {
+    uint32_t pk[32];
+#pragma unroll
+    for (int q = 0; q < 32; ++q) {
+      const int c = 64 * half + 2 * q;
+#if ATTN_PACKED_SOFTMAX
+      const uint64_t y2 = ptx::ffma2(ptx::f2pack(x[c], x[c + 1]), sl2x2, negm2);
+      uint64_t p2;
+      if ((q & 3) < kPolyPairs) {
+        // A masked key (-inf) comes out as 2^-125 rather than 0: against a
+        // row sum l >= 1 and O entries summed in fp32 that weight is far
+        // below one unit in the last place, so it cannot change O or LSE.
+        p2 = exp2_poly2(y2);
+      } else {
+        float y0, y1;
+        ptx::f2unpack(y2, y0, y1);
+        p2 = ptx::f2pack(ptx::ex2_approx(y0), ptx::ex2_approx(y1));
+      }
+      if (q & 1) lsum2b = ptx::fadd2(lsum2b, p2);
+      else lsum2a = ptx::fadd2(lsum2a, p2);
+      float p0, p1;
+      ptx::f2unpack(p2, p0, p1);
+#else
+      const float y0 = fmaf(x[c], sl2, -m), y1 = fmaf(x[c + 1], sl2, -m);
+      float p0, p1;
+      if ((q & 3) < kPolyPairs) {
+        p0 = exp2_poly1(y0);
+        p1 = exp2_poly1(y1);
+      } else {
+        p0 = ptx::ex2_approx(y0);
+        p1 = ptx::ex2_approx(y1);
+      }
+      if (q & 1) { ls2 += p0; ls3 += p1; } else { ls0 += p0; ls1 += p1; }
+#endif
+      pk[q] = ptx::pack_bf16x2(p0, p1);
+    }
+    // P_s keys [64*half, 64*half+64) as bf16 pairs over TMEM columns
+    // [32*half, 32*half+32) of the S_s region; publish this half at once.
+    ptx::tmem_st32(t_s + 32 * half, pk);
+    ptx::tmem_st_wait();
+    ptx::tc_fence_before_sync();
+    __syncwarp();
+    if (lane == 0) ptx::mbar_arrive(&sh.p_ready[2 * s + half]);
+    if (r == 0) ATTN_TRACE(s == 0 ? (half ? kTrSm0Pb : kTrSm0Pa) : (half ? kTrSm1Pb : kTrSm1Pa), tj);
+  }
+#if ATTN_PACKED_SOFTMAX
+  float la0, la1, lb0, lb1;
+  ptx::f2unpack(lsum2a, la0, la1);
+  ptx::f2unpack(lsum2b, lb0, lb1);
+  l = l * alpha + ((la0 + la1) + (lb0 + lb1));
+#else
+  l = l * alpha + ((ls0 + ls1) + (ls2 + ls3));
+#endif
+  return true;
+}
+
 // One thread per query row; warp w of the group reads TMEM lanes
 // [32*(w%4), 32*(w%4)+32), so row r = 32*(w%4) + lane is the tile row.
-// Of every 4 column pairs, kPolyPairs go through exp2_poly2 (FMA pipe) and
-// the rest through ex2.approx (MUFU), so both units share the exponentials.
 template <int D, bool CAUSAL, int kPolyPairs>
-__device__ void softmax_role(const Shared& sh, const KernelArgs& a, uint32_t tmem, int s, int bh,
-                             int qpair, int warp_in_group) {
-  const int qt = 2 * qpair + s;
-  const int n_s = kv_tiles_for<CAUSAL>(qt, a.n_qtiles);
-  if (n_s == 0) return;
+__device__ void softmax_role(const Shared& sh, const KernelArgs& a, uint32_t tmem, int s,
+                             int warp_in_group) {
   const int lane = static_cast<int>(ptx::lane_id());
   const int r = warp_in_group * 32 + lane;
   const uint32_t lane_off = static_cast<uint32_t>(warp_in_group * 32) << 16;
   const uint32_t t_s = tmem + lane_off + 128u * s;
   const uint32_t t_o = tmem + lane_off + 256u + 128u * s;
-  const float sl2 = a.scale_log2;
-  const uint64_t sl2x2 = ptx::f2pack(sl2, sl2);
+  int s_count = 0;  // S_s tiles consumed so far (all items)
+  int o_count = 0;  // items finished by this group
 
-  float m = -INFINITY;  // running max of scale*log2(e)*score (log2 units)
-  float l = 0.f;        // running sum of weights, relative to 2^m
+  Item it;
+  for (int rr = 0; item_for<CAUSAL>(rr, a, it); ++rr) {
+    const int n_s = s == 0 ? it.n0 : it.n1;
+    if (n_s == 0) continue;
+    const int qt = 2 * it.qpair + s;
+    float m = -INFINITY;  // running max of scale*log2(e)*score (log2 units)
+    float l = 0.f;        // running sum of weights, relative to 2^m
+    for (int j = 0; j < n_s; ++j) {
+      const bool diag = CAUSAL && j == n_s - 1;
+      if (!softmax_step<D, CAUSAL, kPolyPairs>(sh, a, s, t_s, t_o, r, lane, diag, j == 0,
+                                               static_cast<uint32_t>(s_count & 1),
+                                               rr == 0 ? j : -1, m, l))
+        return;
+      ++s_count;
+    }
 
-  for (int j = 0; j < n_s; ++j) {
-    if (!wait_warp(sh, a.status, &sh.s_full[s], static_cast<uint32_t>(j & 1))) return;
+    // Epilogue: O_s / l -> bf16 rows; LSE = (m + log2 l) * ln 2.  The next
+    // item's first PV_s (which overwrites O_s) is only issued after this
+    // thread publishes that item's P, i.e. after these loads completed.
+    if (!wait_warp(sh, a.status, &sh.o_final[s], static_cast<uint32_t>(o_count & 1))) return;
+    ++o_count;
     ptx::tc_fence_after_sync();
-    if (r == 0) ATTN_TRACE(s == 0 ? kTrSm0Full : kTrSm1Full, j);
-
-    uint32_t sr[128];
-    ptx::tmem_ld32(t_s + 0, sr + 0);
-    ptx::tmem_ld32(t_s + 32, sr + 32);
-    ptx::tmem_ld32(t_s + 64, sr + 64);
-    ptx::tmem_ld32(t_s + 96, sr + 96);
-    ptx::tmem_ld_wait_tie(sr + 0);
-    ptx::reg_tie32(sr + 32);
-    ptx::reg_tie32(sr + 64);
-    ptx::reg_tie32(sr + 96);
-
-    float x[128];
-#pragma unroll
-    for (int c = 0; c < 128; ++c) x[c] = __uint_as_float(sr[c]);
-    if (r == 0) ATTN_TRACE(s == 0 ? kTrSm0Ld : kTrSm1Ld, j);
-
-    // Causal: the last visited tile is the diagonal one (key tile == query
-    // tile); key c of it is visible to row r iff c <= r.
-    const bool diag = CAUSAL && j == n_s - 1;
-    if (diag) {
-#pragma unroll
-      for (int c = 0; c < 128; ++c)
-        if (c > r) x[c] = -INFINITY;
-    }
-
-    // Row max: four independent chains of three-input maxima.
-    float mx0 = x[0], mx1 = x[1], mx2 = x[2], mx3 = x[3];
-#pragma unroll
-    for (int c = 4; c + 8 <= 128; c += 8) {
-      mx0 = ptx::max3(mx0, x[c], x[c + 1]);
-      mx1 = ptx::max3(mx1, x[c + 2], x[c + 3]);
-      mx2 = ptx::max3(mx2, x[c + 4], x[c + 5]);
-      mx3 = ptx::max3(mx3, x[c + 6], x[c + 7]);
-    }
-    mx0 = ptx::max3(mx0, x[124], x[125]);
-    mx1 = ptx::max3(mx1, x[126], x[127]);
-    const float tile_max = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * sl2;
-    if (r == 0) ATTN_TRACE(s == 0 ? kTrSm0Max : kTrSm1Max, j);
-
-    // Lazy rescale: raise the running max only when it moves by > tau.
-    float alpha = 1.f;
-    bool rescale = false;
-    if (tile_max - m > kRescaleTau) {  // also true on the first tile (m = -inf)
-      alpha = ptx::ex2_approx(m - tile_max);  // 0 on the first tile
-      m = tile_max;
-      rescale = (j > 0);
-    }
-    // O_s *= alpha for the rows whose max moved (PV_s(j-1) is complete: its
-    // commit preceded the one that published S_s(j)).  Done before any P is
-    // published, so the first half of PV_s(j) sees the rescaled O.
-    if (__any_sync(0xffffffffu, rescale)) {
+    const float inv_l = 1.f / l;
+    const size_t row_g = static_cast<size_t>(it.bh) * a.N + static_cast<size_t>(qt) * kBlockM + r;
+    __nv_bfloat16* orow = a.o + row_g * D;
 #pragma unroll 1
-      for (int c0 = 0; c0 < D; c0 += 32) {
-        uint32_t ov[32];
-        ptx::tmem_ld32(t_o + c0, ov);
-        ptx::tmem_ld_wait_tie(ov);
+    for (int c0 = 0; c0 < D; c0 += 32) {
+      uint32_t ov[32];
+      ptx::tmem_ld32(t_o + c0, ov);
+      ptx::tmem_ld_wait_tie(ov);
+      uint32_t pk[16];
 #pragma unroll
-        for (int c = 0; c < 32; ++c) ov[c] = __float_as_uint(__uint_as_float(ov[c]) * alpha);
-        ptx::tmem_st32(t_o + c0, ov);
-      }
-    }
-    const uint64_t negm2 = ptx::f2pack(-m, -m);
-#if ATTN_SOFTMAX_ORDER
-    // Turn order: group 0 waits for group 1's step j-1, group 1 for group
-    // 0's step j (if group 0 has a step j: under the causal mask group 1
-    // visits one more K/V tile than group 0).
-    {
-      const int other_n = kv_tiles_for<CAUSAL>(2 * qpair + (1 - s), a.n_qtiles);
-      const bool must_wait = (s == 0) ? (j >= 1 && j - 1 < other_n) : (j < other_n);
-      const uint32_t par = static_cast<uint32_t>(((s == 0) ? (j - 1) : j) & 1);
-      if (must_wait && !wait_warp(sh, a.status, &sh.exp_token[s], par)) return;
-    }
-#endif
-
-    uint64_t lsum2a = ptx::f2pack(0.f, 0.f), lsum2b = lsum2a;
+      for (int c = 0; c < 16; ++c)
+        pk[c] = ptx::pack_bf16x2(__uint_as_float(ov[2 * c]) * inv_l,
+                                 __uint_as_float(ov[2 * c + 1]) * inv_l);
+      uint4* dst = reinterpret_cast<uint4*>(orow + c0);
 #pragma unroll
-    for (int half = 0; half < 2; ++half) {
-      uint32_t pk[32];
-#pragma unroll
-      for (int q = 0; q < 32; ++q) {
-        const int c = 64 * half + 2 * q;
-        const uint64_t y2 = ptx::ffma2(ptx::f2pack(x[c], x[c + 1]), sl2x2, negm2);
-        uint64_t p2;
-        if ((q & 3) < kPolyPairs) {
-          // A masked key (-inf) comes out as 2^-125 rather than 0: against a
-          // row sum l >= 1 and O entries summed in fp32 that weight is far
-          // below one unit in the last place, so it cannot change O or LSE.
-          p2 = exp2_poly2(y2);
-        } else {
-          float y0, y1;
-          ptx::f2unpack(y2, y0, y1);
-          p2 = ptx::f2pack(ptx::ex2_approx(y0), ptx::ex2_approx(y1));
-        }
-        if (q & 1) lsum2b = ptx::fadd2(lsum2b, p2);
-        else lsum2a = ptx::fadd2(lsum2a, p2);
-        float p0, p1;
-        ptx::f2unpack(p2, p0, p1);
-        pk[q] = ptx::pack_bf16x2(p0, p1);
-      }
-      // P_s keys [64*half, 64*half+64) as bf16 pairs over TMEM columns
-      // [32*half, 32*half+32) of the S_s region; publish this half at once.
-      ptx::tmem_st32(t_s + 32 * half, pk);
-      ptx::tmem_st_wait();
-      ptx::tc_fence_before_sync();
-      __syncwarp();
-      if (lane == 0) ptx::mbar_arrive(&sh.p_ready[2 * s + half]);
-      if (r == 0) ATTN_TRACE(s == 0 ? (half ? kTrSm0Pb : kTrSm0Pa) : (half ? kTrSm1Pb : kTrSm1Pa), j);
+      for (int v = 0; v < 4; ++v)
+        dst[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
     }
-#if ATTN_SOFTMAX_ORDER
-    __syncwarp();
-    if (lane == 0) ptx::mbar_arrive(&sh.exp_token[1 - s]);
-#endif
-    float la0, la1, lb0, lb1;
-    ptx::f2unpack(lsum2a, la0, la1);
-    ptx::f2unpack(lsum2b, lb0, lb1);
-    l = l * alpha + ((la0 + la1) + (lb0 + lb1));
+    a.lse[row_g] = (m + log2f(l)) * 0.69314718055994531f;
   }
-
-  // Epilogue: O_s / l -> bf16 rows; LSE = (m + log2 l) * ln 2.
-  if (!wait_warp(sh, a.status, &sh.o_final[s], 0)) return;
-  ptx::tc_fence_after_sync();
-  const float inv_l = 1.f / l;
-  const size_t row_g = static_cast<size_t>(bh) * a.N + static_cast<size_t>(qt) * kBlockM + r;
-  __nv_bfloat16* orow = a.o + row_g * D;
-#pragma unroll 1
-  for (int c0 = 0; c0 < D; c0 += 32) {
-    uint32_t ov[32];
-    ptx::tmem_ld32(t_o + c0, ov);
-    ptx::tmem_ld_wait_tie(ov);
-    uint32_t pk[16];
-#pragma unroll
-    for (int c = 0; c < 16; ++c)
-      pk[c] = ptx::pack_bf16x2(__uint_as_float(ov[2 * c]) * inv_l,
-                               __uint_as_float(ov[2 * c + 1]) * inv_l);
-    uint4* dst = reinterpret_cast<uint4*>(orow + c0);
-#pragma unroll
-    for (int v = 0; v < 4; ++v)
-      dst[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
-  }
-  a.lse[row_g] = (m + log2f(l)) * 0.69314718055994531f;
 }
 
 // ------------------------------------------------------------------- kernel
@@ -584,43 +677,31 @@ __global__ void __launch_bounds__(kThreads, 1)
   Shared sh;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kBarOff);
   sh.q_full = bars;
-  sh.kv_full = bars + 1;
-  sh.kv_empty = bars + 1 + C::kStages;
-  sh.s_full = bars + 1 + 2 * C::kStages;
+  sh.q_empty = bars + 2;
+  sh.kv_full = bars + 4;
+  sh.kv_empty = sh.kv_full + C::kStages;
+  sh.s_full = sh.kv_empty + C::kStages;
   sh.p_ready = sh.s_full + 2;
   sh.o_final = sh.p_ready + 4;
   sh.drain = sh.o_final + 2;
-  sh.exp_token = sh.drain + 1;
   sh.tmem_base = reinterpret_cast<uint32_t*>(smem + C::kMiscOff);
   sh.abort_flag = reinterpret_cast<volatile int*>(smem + C::kMiscOff + 4);
 
   const int warp = threadIdx.x / 32;
-  // Heaviest query tiles first under the causal mask (blockIdx.y = 0 runs
-  // first and takes the last pair).
-#if ATTN_HEAD_MAJOR
-  const int bh = blockIdx.y;
-  const int qp_idx = blockIdx.x;
-#else
-  const int bh = blockIdx.x;
-  const int qp_idx = blockIdx.y;
-#endif
-  const int qpair = CAUSAL ? (args.n_qpairs - 1 - qp_idx) : qp_idx;
-
   if (threadIdx.x == 0) {
-    ptx::mbar_init(sh.q_full, 1);
-    for (int i = 0; i < C::kStages; ++i) {
-      ptx::mbar_init(&sh.kv_full[i], 1);
-      ptx::mbar_init(&sh.kv_empty[i], 1);
-    }
     for (int i = 0; i < 2; ++i) {
+      ptx::mbar_init(&sh.q_full[i], 1);
+      ptx::mbar_init(&sh.q_empty[i], 1);
       ptx::mbar_init(&sh.s_full[i], 1);
       ptx::mbar_init(&sh.p_ready[2 * i], 4);
       ptx::mbar_init(&sh.p_ready[2 * i + 1], 4);
       ptx::mbar_init(&sh.o_final[i], 1);
     }
+    for (int i = 0; i < C::kStages; ++i) {
+      ptx::mbar_init(&sh.kv_full[i], 1);
+      ptx::mbar_init(&sh.kv_empty[i], 1);
+    }
     ptx::mbar_init(sh.drain, 1);
-    ptx::mbar_init(&sh.exp_token[0], 4);
-    ptx::mbar_init(&sh.exp_token[1], 4);
     *sh.abort_flag = 0;
     ptx::fence_barrier_init();
   }
@@ -644,13 +725,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   // its share before the CTA-wide barrier above.
   if (warp < 8) {
     ptx::setmaxnreg_inc<kRegsSoftmax>();
-    softmax_role<D, CAUSAL, kPolyPairs>(sh, args, tmem, warp / 4, bh, qpair, warp % 4);
+    softmax_role<D, CAUSAL, kPolyPairs>(sh, args, tmem, warp / 4, warp % 4);
   } else if (warp == 8) {
-    if (ptx::lane_id() == 0)
-      producer_role<D, CAUSAL>(sh, args, smem, &tmap_q, &tmap_k, &tmap_v, bh, qpair);
+    if (ptx::lane_id() == 0) producer_role<D, CAUSAL>(sh, args, smem, &tmap_q, &tmap_k, &tmap_v);
     __syncwarp();
   } else if (warp == 9) {
-    mma_role<D, CAUSAL>(sh, args, smem, tmem, qpair);
+    mma_role<D, CAUSAL>(sh, args, smem, tmem);
   }
 
   ptx::tc_fence_before_sync();
