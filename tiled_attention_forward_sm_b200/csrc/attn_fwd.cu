@@ -9,6 +9,7 @@
 #include <cmath>
 #include <cstdint>
 #include <cstring>
+#include <atomic>
 #include <mutex>
 
 #include "attn_b200.h"
@@ -19,6 +20,13 @@ namespace attn_b200 {
 // Written (first error wins) by kernels whose bounded waits ran out.
 __device__ int g_attn_status = 0;
 
+// Work-queue slots: each launch takes the next slot ({next item, CTAs
+// finished}); the launch's last CTA resets it to zero.  Launches that run
+// at the same time use different slots as long as fewer than kQueueSlots
+// of them overlap.
+constexpr int kQueueSlots = 256;
+__device__ int g_attn_queue[2 * kQueueSlots];
+
 namespace {
 
 constexpr int kMaxDevices = 64;
@@ -27,7 +35,9 @@ struct DeviceState {
   bool checked = false;
   bool usable = false;
   int* status = nullptr;  // device address of g_attn_status
+  int* queue = nullptr;   // device address of g_attn_queue
   int num_sms = 0;
+  std::atomic<unsigned> launches{0};
 };
 
 std::mutex g_mu;
@@ -60,6 +70,11 @@ int device_state(DeviceState** out) {
         return ATTN_ERR_CUDA;
       }
       st.status = static_cast<int*>(p);
+      if (cudaGetSymbolAddress(&p, g_attn_queue) != cudaSuccess) {
+        cudaGetLastError();
+        return ATTN_ERR_CUDA;
+      }
+      st.queue = static_cast<int*>(p);
     }
     if (!g_encode) {
       cudaDriverEntryPointQueryResult q;
@@ -100,7 +115,7 @@ bool ranges_overlap(const void* a, size_t na, const void* b, size_t nb) {
 
 template <int D, bool CAUSAL, int kPolyPairs>
 int launch(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
-           int N, float scale, cudaStream_t stream, const DeviceState& st) {
+           int N, float scale, cudaStream_t stream, DeviceState& st) {
   using C = Config<D>;
   const uint64_t rows = static_cast<uint64_t>(B) * H * N;
   CUtensorMap tq, tk, tv;
@@ -115,6 +130,14 @@ int launch(const void* q, const void* k, const void* v, void* o, float* lse, int
   args.n_qpairs = (args.n_qtiles + 1) / 2;
   args.BH = B * H;
   args.n_items = args.BH * args.n_qpairs;
+  // Scheduling window: enough heads that a window holds about two rounds of
+  // items (so its light tail evens out the CTAs), few enough that the
+  // window's K/V stays in L2 while its CTAs run.
+  {
+    const int want = (2 * st.num_sms + args.n_qpairs - 1) / args.n_qpairs;
+    args.win_heads = want < 1 ? 1 : (want > args.BH ? args.BH : want);
+  }
+  args.queue = st.queue + 2 * static_cast<int>(st.launches.fetch_add(1) % kQueueSlots);
   args.scale_log2 = scale * 1.4426950408889634f;
   args.status = st.status;
 
@@ -158,7 +181,7 @@ constexpr int kDefaultPolyPairs = 0;
 
 template <int D, bool CAUSAL>
 int launch_poly(int poly_pairs, const void* q, const void* k, const void* v, void* o, float* lse,
-                int B, int H, int N, float scale, cudaStream_t s, const DeviceState& st) {
+                int B, int H, int N, float scale, cudaStream_t s, DeviceState& st) {
   switch (poly_pairs) {
     case 0: return launch<D, CAUSAL, 0>(q, k, v, o, lse, B, H, N, scale, s, st);
     case 2: return launch<D, CAUSAL, 2>(q, k, v, o, lse, B, H, N, scale, s, st);

@@ -19,9 +19,12 @@
 //
 // Work item: two 128-row Q tiles (Q0, Q1) of one (batch, head), i.e. 256
 // query rows, against the K/V tiles they can see (128 keys per tile).  The
-// kernel is persistent: one CTA per SM walks a static list of work items
-// (heaviest first under the causal mask, dealt out in a snake order so every
-// CTA gets a similar total), and all barrier phases run on across items.
+// kernel is persistent: one CTA per SM takes work items from a shared queue
+// (page lecompute.fr/en/kernel-perf/flapping-airplanes-thunderkittens-
+// megakernels, section "Choose between predetermined work and a shared work
+// queue": a queue rebalances, at the cost of one atomic per item), in an
+// order that keeps the running CTAs on a few heads, and all barrier phases
+// run on across items.
 //
 // Roles (12 warps, 384 threads):
 //   warps 0-3   softmax group 0 (Q0): one thread per query row; also applies
@@ -65,10 +68,23 @@ constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s
 #define ATTN_PACKED_SOFTMAX 1
 #endif
 
+// Work distribution: items are claimed from a per-launch counter in global
+// memory (1, a shared work queue: a CTA that finishes early takes the next
+// item) or dealt statically in a snake order (0).
+#ifndef ATTN_DYNAMIC_QUEUE
+#define ATTN_DYNAMIC_QUEUE 1
+#endif
+
 // K/V ring depth for d = 128 (each stage holds one 128 x 128 bf16 tile).
 #ifndef ATTN_KV_STAGES_D128
 #define ATTN_KV_STAGES_D128 4
 #endif
+
+// Work items announced by the producer to the MMA and softmax warps through
+// a small ring in shared memory.
+constexpr int kItemSlots = 4;
+// Readers of each ring slot: the MMA warp and the 8 softmax warps.
+constexpr int kItemReaders = 9;
 
 constexpr int kBlockM = 128;  // query rows per Q tile
 constexpr int kBlockN = 128;  // keys per K/V tile
@@ -118,8 +134,10 @@ struct KernelArgs {
   int n_qpairs;       // ceil(n_qtiles / 2)
   int BH;             // B * H
   int n_items;        // BH * n_qpairs work items
+  int win_heads;      // heads per scheduling window (item order, see decode_item)
   float scale_log2;   // scale * log2(e)
   int* status;        // device status word
+  int* queue;         // {next item, CTAs finished}: this launch's queue slot
 };
 
 template <int D>
@@ -133,10 +151,11 @@ struct Config {
   static constexpr int kKVOff = 2 * kTileBytes;
   static constexpr int kBarOff = kKVOff + kStages * kTileBytes;
   // barriers: q_full[2], q_empty[2], kv_full[S], kv_empty[S], s_full[2],
-  // p_ready[2 tiles][2 halves], o_final[2], drain
-  static constexpr int kNumBars = 4 + 2 * kStages + 2 + 4 + 2 + 1;
+  // p_ready[2 tiles][2 halves], o_final[2], drain, item_full[R], item_empty[R]
+  static constexpr int kNumBars = 4 + 2 * kStages + 2 + 4 + 2 + 1 + 2 * kItemSlots;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;
-  static constexpr int kSmemBytes = kMiscOff + 16 + 1024;  // + alignment slack
+  // misc: tmem base, abort flag, item ring
+  static constexpr int kSmemBytes = kMiscOff + 8 + 4 * kItemSlots + 1024;  // + alignment slack
   static constexpr uint32_t kIdescQK = ptx::idesc_bf16_f32(128, kBlockN, 0, 0);
   static constexpr uint32_t kIdescPV = ptx::idesc_bf16_f32(128, D, 0, 1);
 };
@@ -150,6 +169,9 @@ struct Shared {
   uint64_t* p_ready;   // [2*s + half] half of P_s(j) in TMEM
   uint64_t* o_final;   // [2] last PV_s of the item done
   uint64_t* drain;
+  uint64_t* item_full;   // [kItemSlots] item index written
+  uint64_t* item_empty;  // [kItemSlots] every reader has taken it
+  volatile int* item_ring;
   uint32_t* tmem_base;
   volatile int* abort_flag;
 };
@@ -217,20 +239,65 @@ struct Item {
   int n1;     // K/V tiles Q1 visits
 };
 
-// Items are numbered pair-major with the heaviest pairs first under the
-// causal mask; round r deals items [r*G, r*G + G) to the G CTAs, reversing
-// the direction every other round (snake), so each CTA's total work is
-// nearly the same.  Returns false once this CTA has no item in round r.
+// Item numbering: heads are taken in windows of win_heads; inside a window
+// the pairs are numbered heaviest first under the causal mask (pair-major
+// over the window's heads).  Items handed out in this order keep the CTAs
+// that run together on a few heads, whose K/V then stays in L2, while the
+// light pairs at the end of each window even out the CTAs' finishing times.
 template <bool CAUSAL>
-__device__ __forceinline__ bool item_for(int r, const KernelArgs& a, Item& it) {
-  const int G = static_cast<int>(gridDim.x), c = static_cast<int>(blockIdx.x);
-  const int idx = r * G + ((r & 1) ? (G - 1 - c) : c);
-  if (idx >= a.n_items) return false;
-  const int qp_idx = idx / a.BH;
-  it.bh = idx - qp_idx * a.BH;
+__device__ __forceinline__ Item decode_item(int idx, const KernelArgs& a) {
+  const int per_win = a.win_heads * a.n_qpairs;
+  const int w = idx / per_win;
+  const int k = idx - w * per_win;
+  const int h0 = w * a.win_heads;
+  const int wh = (a.BH - h0) < a.win_heads ? (a.BH - h0) : a.win_heads;
+  const int qp_idx = k / wh;
+  Item it;
+  it.bh = h0 + (k - qp_idx * wh);
   it.qpair = CAUSAL ? (a.n_qpairs - 1 - qp_idx) : qp_idx;
   it.n0 = kv_tiles_for<CAUSAL>(2 * it.qpair, a.n_qtiles);
   it.n1 = kv_tiles_for<CAUSAL>(2 * it.qpair + 1, a.n_qtiles);
+  return it;
+}
+
+// The producer's r-th item: claimed from the launch's queue counter, or
+// dealt statically (round r gives CTA c item r*G + c, reversed every other
+// round).  Returns an index >= n_items when there is no more work.
+__device__ __forceinline__ int claim_item(int r, const KernelArgs& a) {
+#if ATTN_DYNAMIC_QUEUE
+  (void)r;
+  return atomicAdd(a.queue, 1);
+#else
+  const int G = static_cast<int>(gridDim.x), c = static_cast<int>(blockIdx.x);
+  return r * G + ((r & 1) ? (G - 1 - c) : c);
+#endif
+}
+
+// Producer: announce its r-th item (or the end, idx < 0) in ring slot r % R.
+__device__ __forceinline__ bool post_item(const Shared& sh, const KernelArgs& a, int r, int idx) {
+  const int slot = r % kItemSlots;
+  const uint32_t ph = static_cast<uint32_t>((r / kItemSlots) & 1);
+  if (!wait_one(sh, a.status, &sh.item_empty[slot], ph ^ 1)) return false;
+  sh.item_ring[slot] = idx;
+  ptx::mbar_arrive(&sh.item_full[slot]);  // release: the write is seen by waiters
+  return true;
+}
+
+// Reader warp: its r-th item.  Returns false at the end of the work (or on
+// abort, with ok cleared).
+template <bool CAUSAL>
+__device__ __forceinline__ bool read_item(const Shared& sh, const KernelArgs& a, int r, Item& it,
+                                          bool& ok) {
+  const int slot = r % kItemSlots;
+  if (!wait_warp(sh, a.status, &sh.item_full[slot], static_cast<uint32_t>((r / kItemSlots) & 1))) {
+    ok = false;
+    return false;
+  }
+  const int idx = sh.item_ring[slot];
+  __syncwarp();
+  if (ptx::lane_id() == 0) ptx::mbar_arrive(&sh.item_empty[slot]);
+  if (idx < 0) return false;
+  it = decode_item<CAUSAL>(idx, a);
   return true;
 }
 
@@ -245,8 +312,14 @@ __device__ void producer_role(const Shared& sh, const KernelArgs& a, uint8_t* sm
   int q_loads[2] = {0, 0};  // loads into Q buffer s so far
   int issued = 0;           // K/V tiles issued into the ring so far
   bool ok = true;
-  Item it;
-  for (int r = 0; ok && item_for<CAUSAL>(r, a, it); ++r) {
+  int idx = claim_item(0, a);
+  for (int r = 0; ok; ++r) {
+    if (idx >= a.n_items) {
+      post_item(sh, a, r, -1);
+      break;
+    }
+    if (!post_item(sh, a, r, idx)) break;
+    const Item it = decode_item<CAUSAL>(idx, a);
     const int n = it.n0 > it.n1 ? it.n0 : it.n1;
     const int row0 = it.bh * a.N;  // first row of this (b, h) in the 2-D views
     // Q_s, once the previous item's last S_s no longer needs the buffer.
@@ -278,6 +351,10 @@ __device__ void producer_role(const Shared& sh, const KernelArgs& a, uint8_t* sm
         ++issued;
       }
     }
+    // Claim the next item only now: the ring holds the last K/V steps of
+    // this one, so the claim's latency overlaps them, and a CTA never holds
+    // an item it cannot start soon (which would lengthen the tail).
+    idx = claim_item(r + 1, a);
   }
   // Drain: every load issued must land before the CTA may exit.
   for (int s = 0; s < 2; ++s)
@@ -359,7 +436,8 @@ __device__ void mma_role(const Shared& sh, const KernelArgs& a, uint8_t* smem, u
   auto phase_of = [&](int c) { return static_cast<uint32_t>((c / C::kStages) & 1); };
 
   Item it;
-  for (int r = 0; item_for<CAUSAL>(r, a, it); ++r) {
+  bool ok = true;
+  for (int r = 0; read_item<CAUSAL>(sh, a, r, it, ok); ++r) {
     const int n0 = it.n0, n1 = it.n1;
     const int n = n0 > n1 ? n0 : n1;
     for (int s = 0; s < 2; ++s) {
@@ -620,7 +698,8 @@ __device__ void softmax_role(const Shared& sh, const KernelArgs& a, uint32_t tme
   int o_count = 0;  // items finished by this group
 
   Item it;
-  for (int rr = 0; item_for<CAUSAL>(rr, a, it); ++rr) {
+  bool ok = true;
+  for (int rr = 0; read_item<CAUSAL>(sh, a, rr, it, ok); ++rr) {
     const int n_s = s == 0 ? it.n0 : it.n1;
     if (n_s == 0) continue;
     const int qt = 2 * it.qpair + s;
@@ -684,8 +763,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   sh.p_ready = sh.s_full + 2;
   sh.o_final = sh.p_ready + 4;
   sh.drain = sh.o_final + 2;
+  sh.item_full = sh.drain + 1;
+  sh.item_empty = sh.item_full + kItemSlots;
   sh.tmem_base = reinterpret_cast<uint32_t*>(smem + C::kMiscOff);
   sh.abort_flag = reinterpret_cast<volatile int*>(smem + C::kMiscOff + 4);
+  sh.item_ring = reinterpret_cast<volatile int*>(smem + C::kMiscOff + 8);
 
   const int warp = threadIdx.x / 32;
   if (threadIdx.x == 0) {
@@ -702,6 +784,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       ptx::mbar_init(&sh.kv_empty[i], 1);
     }
     ptx::mbar_init(sh.drain, 1);
+    for (int i = 0; i < kItemSlots; ++i) {
+      ptx::mbar_init(&sh.item_full[i], 1);
+      ptx::mbar_init(&sh.item_empty[i], kItemReaders);
+    }
     *sh.abort_flag = 0;
     ptx::fence_barrier_init();
   }
@@ -735,7 +821,18 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   ptx::tc_fence_before_sync();
   __syncthreads();
-  if (threadIdx.x == 0) ATTN_TRACE(kTrEnd, 0);
+  if (threadIdx.x == 0) {
+    ATTN_TRACE(kTrEnd, 0);
+#if ATTN_DYNAMIC_QUEUE
+    // The last CTA to finish resets this launch's queue slot for its next
+    // user (every CTA's claims precede its arrival here).
+    __threadfence();
+    if (atomicAdd(args.queue + 1, 1) == static_cast<int>(gridDim.x) - 1) {
+      atomicExch(args.queue, 0);
+      atomicExch(args.queue + 1, 0);
+    }
+#endif
+  }
   if (warp == 9) {
     ptx::tc_fence_after_sync();
     ptx::tmem_dealloc(tmem, 512);
