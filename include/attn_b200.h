@@ -92,6 +92,31 @@ int attn_fwd_ex(const void* q, const void* k, const void* v, void* o, float* lse
                 const attn_opts* opts, attn_stream_t stream);
 
 /*
+ * attn_fwd_noalloc -- attn_fwd for callers that cannot allocate device
+ * memory, e.g. code running under global-mode CUDA stream capture (where
+ * cudaMalloc is refused) or inside a framework whose allocator owns all
+ * device memory.  There is no counterpart on the source pages: it is a
+ * property of this library, not of the method.
+ *
+ * Same arguments, results and errors as attn_fwd; nothing is allocated.
+ * The kernel's only scratch, its work-queue counter (8 bytes), lives in a
+ * fixed 256-byte array the library holds in device memory on every GPU that
+ * loads it, until the process exits.  The call clears that counter on
+ * `stream` before its kernel, so each call starts clean, but every call
+ * shares the same array: calls that overlap on the GPU (other streams, or
+ * other threads' streams) race and must be serialised by the caller.
+ * Problems whose work-item count plus the number of SMs would overflow the
+ * 32-bit counter return ATTN_ERR_UNSUPPORTED.
+ *
+ * The first call of any entry point on a device (this one included) looks
+ * up the scratch array's device address for that device; make that first
+ * call before beginning any stream capture.
+ */
+int attn_fwd_noalloc(const void* q, const void* k, const void* v, void* o, float* lse,
+                     int B, int H, int N, int d, int causal, float scale,
+                     attn_stream_t stream);
+
+/*
  * attn_fwd_host -- the same operation on HOST buffers: copies q, k, v from
  * host to the caller's device buffers, runs attn_fwd, and copies o and lse
  * back, all enqueued on `stream` (pinned host memory makes the copies

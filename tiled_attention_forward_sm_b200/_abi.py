@@ -45,6 +45,8 @@ def library():
         lib.attn_fwd.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, f, vp]
         lib.attn_fwd_ex.restype = i
         lib.attn_fwd_ex.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, f, vp, vp]
+        lib.attn_fwd_noalloc.restype = i
+        lib.attn_fwd_noalloc.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, f, vp]
         lib.attn_fwd_host.restype = i
         lib.attn_fwd_host.argtypes = [vp] * 10 + [i, i, i, i, i, f, vp]
         lib.attn_last_device_error.restype = i
@@ -116,6 +118,27 @@ def attn_fwd(q, k, v, causal: bool = False, scale: float | None = None, stream=N
     lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
     attn_fwd_into(q, k, v, o, lse, causal, scale, stream, exp2_poly_pairs)
     return o, lse
+
+
+def attn_fwd_noalloc_into(q, k, v, o, lse, causal: bool = False, scale: float | None = None,
+                          stream=None) -> None:
+    """The allocation-free entry point (see attn_fwd_noalloc in the header):
+    same contract as attn_fwd_into; calls that overlap on the GPU race."""
+    B, H, N, d = _shape(q)
+    for name, t in (("q", q), ("k", k), ("v", v), ("o", o)):
+        if not t.is_cuda or t.dtype != torch.bfloat16 or not t.is_contiguous() or \
+                tuple(t.shape) != (B, H, N, d):
+            raise ValueError(f"{name} must be a contiguous CUDA bf16 tensor of shape {(B, H, N, d)}")
+    if not lse.is_cuda or lse.dtype != torch.float32 or not lse.is_contiguous() or \
+            tuple(lse.shape) != (B, H, N):
+        raise ValueError(f"lse must be a contiguous CUDA fp32 tensor of shape {(B, H, N)}")
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    rc = library().attn_fwd_noalloc(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
+                                    lse.data_ptr(), B, H, N, d, int(bool(causal)), float(scale),
+                                    _stream_handle(stream))
+    if rc != ATTN_OK:
+        raise AttnError(rc, "attn_fwd_noalloc")
 
 
 def attn_fwd_host(q_h, k_h, v_h, o_h, lse_h, q_d, k_d, v_d, o_d, lse_d,

@@ -27,6 +27,17 @@ __device__ int g_attn_status = 0;
 constexpr int kQueueSlots = 256;
 __device__ int g_attn_queue[2 * kQueueSlots];
 
+// Scratch of attn_fwd_noalloc: a fixed array this library owns for as long
+// as it is loaded (every GPU that loads it keeps these bytes until exit).
+// The call needs one work-queue slot ({next item, CTAs finished}, 8 bytes)
+// out of it, for any problem size.  Host code must not pass the symbol
+// itself to a kernel (on the host it is only a stand-in); each device's
+// address comes from cudaGetSymbolAddress in device_state().
+constexpr int kNoAllocScratchBytes = 256;
+constexpr int kNoAllocQueueBytes = 2 * static_cast<int>(sizeof(int));
+static_assert(kNoAllocQueueBytes <= kNoAllocScratchBytes, "queue slot must fit the scratch");
+static __device__ __align__(256) int g_attn_noalloc_scratch[kNoAllocScratchBytes / sizeof(int)];
+
 namespace {
 
 constexpr int kMaxDevices = 64;
@@ -36,6 +47,7 @@ struct DeviceState {
   bool usable = false;
   int* status = nullptr;  // device address of g_attn_status
   int* queue = nullptr;   // device address of g_attn_queue
+  int* noalloc_scratch = nullptr;  // device address of g_attn_noalloc_scratch
   int num_sms = 0;
   std::atomic<unsigned> launches{0};
 };
@@ -75,6 +87,11 @@ int device_state(DeviceState** out) {
         return ATTN_ERR_CUDA;
       }
       st.queue = static_cast<int*>(p);
+      if (cudaGetSymbolAddress(&p, g_attn_noalloc_scratch) != cudaSuccess) {
+        cudaGetLastError();
+        return ATTN_ERR_CUDA;
+      }
+      st.noalloc_scratch = static_cast<int*>(p);
     }
     if (!g_encode) {
       cudaDriverEntryPointQueryResult q;
@@ -115,7 +132,7 @@ bool ranges_overlap(const void* a, size_t na, const void* b, size_t nb) {
 
 template <int D, bool CAUSAL, int kPolyPairs>
 int launch(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
-           int N, float scale, cudaStream_t stream, DeviceState& st) {
+           int N, float scale, cudaStream_t stream, DeviceState& st, int* queue = nullptr) {
   using C = Config<D>;
   const uint64_t rows = static_cast<uint64_t>(B) * H * N;
   CUtensorMap tq, tk, tv;
@@ -137,7 +154,9 @@ int launch(const void* q, const void* k, const void* v, void* o, float* lse, int
     const int want = (2 * st.num_sms + args.n_qpairs - 1) / args.n_qpairs;
     args.win_heads = want < 1 ? 1 : (want > args.BH ? args.BH : want);
   }
-  args.queue = st.queue + 2 * static_cast<int>(st.launches.fetch_add(1) % kQueueSlots);
+  args.queue = queue != nullptr
+                   ? queue
+                   : st.queue + 2 * static_cast<int>(st.launches.fetch_add(1) % kQueueSlots);
   args.scale_log2 = scale * 1.4426950408889634f;
   args.status = st.status;
 
@@ -253,6 +272,33 @@ extern "C" int attn_fwd_ex(const void* q, const void* k, const void* v, void* o,
     if (opts->exp2_poly_pairs >= 0) poly = opts->exp2_poly_pairs;
   }
   return fwd_impl(q, k, v, o, lse, B, H, N, d, causal, scale, poly, stream);
+}
+
+// Allocation-free entry point (include/attn_b200.h): same kernel, work
+// queue in the library's fixed scratch array, cleared on every call.
+extern "C" int attn_fwd_noalloc(const void* q, const void* k, const void* v, void* o, float* lse,
+                                int B, int H, int N, int d, int causal, float scale,
+                                attn_stream_t stream) {
+  int rc = attn_check_args(q, k, v, o, lse, B, H, N, d, scale);
+  if (rc != ATTN_OK) return rc;
+  DeviceState* st = nullptr;
+  rc = device_state(&st);  // first call on a device: resolves the scratch address
+  if (rc != ATTN_OK) return rc;
+  // The queue counter is a 32-bit int that every CTA pushes once past the
+  // last item: items + CTAs must stay representable.
+  const int64_t items = static_cast<int64_t>(B) * H * ((N / kBlockM + 1) / 2);
+  if (items + st->num_sms > 0x7FFFFFFFll) return ATTN_ERR_UNSUPPORTED;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (cudaMemsetAsync(st->noalloc_scratch, 0, kNoAllocQueueBytes, s) != cudaSuccess) {
+    cudaGetLastError();
+    return ATTN_ERR_CUDA;
+  }
+  int* qs = st->noalloc_scratch;
+  if (d == 128)
+    return causal ? launch<128, true, kDefaultPolyPairs>(q, k, v, o, lse, B, H, N, scale, s, *st, qs)
+                  : launch<128, false, kDefaultPolyPairs>(q, k, v, o, lse, B, H, N, scale, s, *st, qs);
+  return causal ? launch<64, true, kDefaultPolyPairs>(q, k, v, o, lse, B, H, N, scale, s, *st, qs)
+                : launch<64, false, kDefaultPolyPairs>(q, k, v, o, lse, B, H, N, scale, s, *st, qs);
 }
 
 extern "C" int attn_last_device_error(attn_stream_t stream) {
