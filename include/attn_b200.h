@@ -33,7 +33,7 @@ extern "C" {
 typedef enum {
   ATTN_OK = 0,
   ATTN_ERR_INVALID_ARG = -1,   /* null pointer, non-positive size, bad scale */
-  ATTN_ERR_UNSUPPORTED = -2,   /* d not in {64,128}, N not a multiple of 128, too large */
+  ATTN_ERR_UNSUPPORTED = -2,   /* d not in {64,128}, or B*H*N >= 2^31 */
   ATTN_ERR_MISALIGNED = -3,    /* a device pointer is not 16-byte aligned */
   ATTN_ERR_CUDA = -4,          /* a CUDA runtime/driver call failed */
   ATTN_ERR_DEVICE_TIMEOUT = -5,/* a bounded wait inside the kernel ran out */
@@ -52,7 +52,7 @@ typedef void* attn_stream_t;
  *   lse      device, fp32 [B, H, N].  Written (natural log of the softmax
  *            denominator of the scaled, masked scores).
  *   o and lse must not overlap q, k, v or each other.
- *   B, H, N  > 0; N a multiple of 128; B*H*N < 2^31.
+ *   B, H, N  > 0 (any N; tiles past N are masked); B*H*N < 2^31.
  *   d        64 or 128.
  *   causal   0: every key visible; non-zero: key j visible to query i iff j <= i.
  *   scale    finite and > 0 (typically 1/sqrt(d)).
@@ -142,6 +142,18 @@ int attn_fwd_host(const void* q_h, const void* k_h, const void* v_h, void* o_h, 
  * the read fails.
  */
 int attn_last_device_error(attn_stream_t stream);
+
+/*
+ * attn_selftest_wait_timeout -- exercises the kernels' failure detection
+ * without a fault: enqueues on `stream` one warp that waits, through the
+ * same bounded wait the attention kernel uses, on a barrier nothing ever
+ * completes.  After limit_us microseconds (1 .. 10^7) the wait gives up and
+ * records ATTN_ERR_DEVICE_TIMEOUT in the device status word, which the next
+ * attn_last_device_error(stream) returns (and clears); the context stays
+ * usable.  Returns ATTN_OK once enqueued, ATTN_ERR_INVALID_ARG for an
+ * out-of-range limit.
+ */
+int attn_selftest_wait_timeout(int limit_us, attn_stream_t stream);
 
 /* Static string for a status code (never NULL). */
 const char* attn_strerror(int status);

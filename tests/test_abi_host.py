@@ -58,7 +58,7 @@ def ptrs(d=128, B=1, H=1, N=128):
 
 
 @pytest.mark.parametrize("d", [64, 128])
-@pytest.mark.parametrize("N", [128, 256, 384, 32768])
+@pytest.mark.parametrize("N", [1, 100, 128, 129, 256, 384, 1000, 32768])
 def test_check_args_accepts_supported(lib, d, N):
     assert tab.check_args(*ptrs(d, 2, 3, N), 2, 3, N, d, 1 / math.sqrt(d)) == 0
 
@@ -75,7 +75,7 @@ def test_check_args_rejections(lib):
     assert tab.check_args(*p, 1, 1, 128, 128, float("nan")) == -1
     assert tab.check_args(*p, 1, 1, 128, 128, float("inf")) == -1
     assert tab.check_args(*p, 1, 1, 128, 96, 0.1) == -2                # d unsupported
-    assert tab.check_args(*p, 1, 1, 100, 128, 0.1) == -2               # N % 128
+    assert tab.check_args(*p, 1, 1, 128, 256, 0.1) == -2               # d unsupported
     assert tab.check_args(*p, 1 << 12, 1 << 12, 1 << 8, 128, 0.1) == -2  # rows >= 2^31
     q, k, v, o, l = p
     assert tab.check_args(q + 8, k, v, o, l, 1, 1, 128, 128, 0.1) == -3   # misaligned q
@@ -140,3 +140,9 @@ def test_exp2_polynomial_coefficients_and_error():
     ints = np.arange(-125, 9).astype(np.float32)
     np.testing.assert_allclose(gen.fp32_exp2_emulation(ints, lits), np.exp2(ints) * lits[0],
                                rtol=1e-7)
+
+
+def test_selftest_rejects_bad_limit(lib):
+    assert lib.attn_selftest_wait_timeout(0, None) == -1
+    assert lib.attn_selftest_wait_timeout(-5, None) == -1
+    assert lib.attn_selftest_wait_timeout(20000000, None) == -1

@@ -53,6 +53,33 @@ def test_small_shapes(oracle_mod, d, causal, N):
     full_parity(oracle_mod, 2, 3, N, d, causal, seed=N + d + causal)
 
 
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("N", [1, 7, 100, 129, 255, 300, 1000])
+def test_ragged_lengths(oracle_mod, d, causal, N):
+    """N not a multiple of 128: the last K/V tile is masked past N and the
+    rows past N are neither computed into nor written."""
+    full_parity(oracle_mod, 2, 3, N, d, causal, seed=900 + N + d, q_std=2.0)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_ragged_length_writes_nothing_past_the_rows(causal):
+    """B*H heads of N = 200 rows, packed back to back inside guard bands: no
+    head's last, partial tile writes into the next head or past the end."""
+    B, H, N, d = 1, 3, 200, 128
+    q, k, v = (t.cuda() for t in make_qkv(B, H, N, d, 11))
+    g = 4096
+    o_buf = torch.full((g + B * H * N * d + g,), float("nan"), dtype=torch.bfloat16, device="cuda")
+    l_buf = torch.full((g + B * H * N + g,), float("nan"), dtype=torch.float32, device="cuda")
+    o = o_buf[g:g + B * H * N * d].view(B, H, N, d)
+    lse = l_buf[g:g + B * H * N].view(B, H, N)
+    tab.attn_fwd_into(q, k, v, o, lse, causal=causal)
+    assert tab.last_device_error() == 0
+    assert torch.isfinite(o).all() and torch.isfinite(lse).all()
+    assert torch.isnan(o_buf[:g]).all() and torch.isnan(o_buf[-g:]).all()
+    assert torch.isnan(l_buf[:g]).all() and torch.isnan(l_buf[-g:]).all()
+
+
 @pytest.mark.parametrize("poly", [0, 1, 2])
 @pytest.mark.parametrize("d", [64, 128])
 @pytest.mark.parametrize("causal", [False, True])
@@ -143,8 +170,17 @@ def test_host_entry_point_matches_device_entry_point():
 
 
 def test_rejected_arguments_launch_nothing():
-    q = torch.zeros(1, 1, 100, 128, dtype=torch.bfloat16, device="cuda")
+    q = torch.zeros(1, 1, 128, 96, dtype=torch.bfloat16, device="cuda")  # d = 96: unsupported
     with pytest.raises(tab.AttnError) as e:
         tab.attn_fwd(q, q, q)
     assert e.value.status == -2
     assert tab.last_device_error() == 0
+
+
+def test_bounded_wait_reports_timeout_and_context_stays_usable(oracle_mod):
+    """A wait on a barrier that nothing completes gives up after its limit,
+    the status word reports the timeout, and the next launch is correct."""
+    tab.selftest_wait_timeout(20000)  # 20 ms
+    assert tab.last_device_error() == -5
+    assert tab.last_device_error() == 0  # read-and-clear
+    full_parity(oracle_mod, 1, 2, 256, 128, True, seed=3)

@@ -49,6 +49,8 @@ def library():
         lib.attn_fwd_noalloc.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, f, vp]
         lib.attn_fwd_host.restype = i
         lib.attn_fwd_host.argtypes = [vp] * 10 + [i, i, i, i, i, f, vp]
+        lib.attn_selftest_wait_timeout.restype = i
+        lib.attn_selftest_wait_timeout.argtypes = [i, vp]
         lib.attn_last_device_error.restype = i
         lib.attn_last_device_error.argtypes = [vp]
         lib.attn_strerror.restype = ctypes.c_char_p
@@ -158,6 +160,14 @@ def attn_fwd_host(q_h, k_h, v_h, o_h, lse_h, q_d, k_d, v_d, o_d, lse_d,
         B, H, N, d, int(bool(causal)), float(scale), _stream_handle(stream))
     if rc != ATTN_OK:
         raise AttnError(rc, "attn_fwd_host")
+
+
+def selftest_wait_timeout(limit_us: int, stream=None) -> None:
+    """Enqueue the bounded-wait self-test (see the header); the next
+    last_device_error() should report the timeout status."""
+    rc = library().attn_selftest_wait_timeout(int(limit_us), _stream_handle(stream))
+    if rc != ATTN_OK:
+        raise AttnError(rc, "attn_selftest_wait_timeout")
 
 
 def last_device_error(stream=None) -> int:

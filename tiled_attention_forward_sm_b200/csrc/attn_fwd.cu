@@ -111,14 +111,18 @@ int device_state(DeviceState** out) {
   return ATTN_OK;
 }
 
-// 2-D view [rows, d] of a [B,H,N,d] bf16 tensor; 128-row x 64-column boxes
-// with the 128-byte swizzle the tcgen05 shared-memory descriptors expect.
-int make_tmap(CUtensorMap* m, const void* ptr, uint64_t rows, int d) {
-  cuuint64_t dims[2] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(rows)};
-  cuuint64_t strides[1] = {static_cast<cuuint64_t>(d) * 2};
-  cuuint32_t box[2] = {64, 128};
-  cuuint32_t estr[2] = {1, 1};
-  CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims,
+// 3-D view [B*H][N][d] of a [B,H,N,d] bf16 tensor; boxes of 128 rows x 64
+// columns of one head, with the 128-byte swizzle the tcgen05 shared-memory
+// descriptors expect.  Rows past N of a head are outside the view and read
+// as zero, so a tile never picks up the next head's rows.
+int make_tmap(CUtensorMap* m, const void* ptr, int BH, int N, int d) {
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(N),
+                        static_cast<cuuint64_t>(BH)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2,
+                           static_cast<cuuint64_t>(N) * static_cast<cuuint64_t>(d) * 2};
+  cuuint32_t box[3] = {64, 128, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims,
                         strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                         CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
@@ -134,16 +138,16 @@ template <int D, bool CAUSAL, int kPolyPairs>
 int launch(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
            int N, float scale, cudaStream_t stream, DeviceState& st, int* queue = nullptr) {
   using C = Config<D>;
-  const uint64_t rows = static_cast<uint64_t>(B) * H * N;
   CUtensorMap tq, tk, tv;
-  if (make_tmap(&tq, q, rows, D) || make_tmap(&tk, k, rows, D) || make_tmap(&tv, v, rows, D))
+  if (make_tmap(&tq, q, B * H, N, D) || make_tmap(&tk, k, B * H, N, D) ||
+      make_tmap(&tv, v, B * H, N, D))
     return ATTN_ERR_CUDA;
 
   KernelArgs args;
   args.o = static_cast<__nv_bfloat16*>(o);
   args.lse = lse;
   args.N = N;
-  args.n_qtiles = N / kBlockM;
+  args.n_qtiles = (N + kBlockM - 1) / kBlockM;
   args.n_qpairs = (args.n_qtiles + 1) / 2;
   args.BH = B * H;
   args.n_items = args.BH * args.n_qpairs;
@@ -222,7 +226,6 @@ extern "C" int attn_check_args(const void* q, const void* k, const void* v, cons
   if (B <= 0 || H <= 0 || N <= 0) return ATTN_ERR_INVALID_ARG;
   if (!std::isfinite(scale) || !(scale > 0.f)) return ATTN_ERR_INVALID_ARG;
   if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
-  if (N % kBlockM != 0) return ATTN_ERR_UNSUPPORTED;
   const uint64_t rows = static_cast<uint64_t>(B) * H * N;
   // Work items (B*H*ceil(N/256)) are numbered in int.
   if (rows >= (1ull << 31)) return ATTN_ERR_UNSUPPORTED;
@@ -286,7 +289,7 @@ extern "C" int attn_fwd_noalloc(const void* q, const void* k, const void* v, voi
   if (rc != ATTN_OK) return rc;
   // The queue counter is a 32-bit int that every CTA pushes once past the
   // last item: items + CTAs must stay representable.
-  const int64_t items = static_cast<int64_t>(B) * H * ((N / kBlockM + 1) / 2);
+  const int64_t items = static_cast<int64_t>(B) * H * (((N + kBlockM - 1) / kBlockM + 1) / 2);
   if (items + st->num_sms > 0x7FFFFFFFll) return ATTN_ERR_UNSUPPORTED;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (cudaMemsetAsync(st->noalloc_scratch, 0, kNoAllocQueueBytes, s) != cudaSuccess) {
@@ -299,6 +302,17 @@ extern "C" int attn_fwd_noalloc(const void* q, const void* k, const void* v, voi
                   : launch<128, false, kDefaultPolyPairs>(q, k, v, o, lse, B, H, N, scale, s, *st, qs);
   return causal ? launch<64, true, kDefaultPolyPairs>(q, k, v, o, lse, B, H, N, scale, s, *st, qs)
                 : launch<64, false, kDefaultPolyPairs>(q, k, v, o, lse, B, H, N, scale, s, *st, qs);
+}
+
+extern "C" int attn_selftest_wait_timeout(int limit_us, attn_stream_t stream) {
+  if (limit_us <= 0 || limit_us > 10000000) return ATTN_ERR_INVALID_ARG;
+  DeviceState* st = nullptr;
+  int rc = device_state(&st);
+  if (rc != ATTN_OK) return rc;
+  wait_timeout_selftest_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(
+      st->status, static_cast<uint64_t>(limit_us) * 1000ull);
+  if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
+  return ATTN_OK;
 }
 
 extern "C" int attn_last_device_error(attn_stream_t stream) {
@@ -349,7 +363,7 @@ extern "C" const char* attn_strerror(int status) {
   switch (status) {
     case ATTN_OK: return "ok";
     case ATTN_ERR_INVALID_ARG: return "invalid argument";
-    case ATTN_ERR_UNSUPPORTED: return "unsupported shape (d must be 64 or 128, N a multiple of 128)";
+    case ATTN_ERR_UNSUPPORTED: return "unsupported shape (d must be 64 or 128; B*H*N below 2^31)";
     case ATTN_ERR_MISALIGNED: return "misaligned pointer (q, k, v, o need 16 bytes, lse 4)";
     case ATTN_ERR_CUDA: return "CUDA call failed";
     case ATTN_ERR_DEVICE_TIMEOUT: return "device-side wait timed out";

@@ -129,8 +129,8 @@ __device__ __forceinline__ void trace_stamp(int ev, int j) {
 struct KernelArgs {
   __nv_bfloat16* o;   // [B*H*N, D]
   float* lse;         // [B*H*N]
-  int N;              // keys/queries per head (multiple of 128)
-  int n_qtiles;       // N / 128
+  int N;              // keys/queries per head (any N >= 1)
+  int n_qtiles;       // ceil(N / 128)
   int n_qpairs;       // ceil(n_qtiles / 2)
   int BH;             // B * H
   int n_items;        // BH * n_qpairs work items
@@ -184,14 +184,15 @@ __device__ __forceinline__ void raise_status(const Shared& sh, int* status, int 
 // Single-thread bounded wait.  A drain wait (for this thread's own copies or
 // MMAs in flight) ignores the abort flag but keeps the time limit.
 __device__ __forceinline__ bool wait_one(const Shared& sh, int* status, uint64_t* bar,
-                                         uint32_t parity, bool drain = false) {
+                                         uint32_t parity, bool drain = false,
+                                         uint64_t limit_ns = kWaitLimitNs) {
   if (ptx::mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = ptx::globaltimer_ns();
   for (uint32_t it = 1;; ++it) {
     if (ptx::mbar_try_wait(bar, parity)) return true;
     if ((it & 63u) == 0) {
       if (!drain && *sh.abort_flag) return false;
-      if (ptx::globaltimer_ns() - t0 > kWaitLimitNs) {
+      if (ptx::globaltimer_ns() - t0 > limit_ns) {
         raise_status(sh, status, kStatusDeviceTimeout);
         return false;
       }
@@ -202,7 +203,8 @@ __device__ __forceinline__ bool wait_one(const Shared& sh, int* status, uint64_t
 // Warp-uniform bounded wait (every lane returns the same answer), for roles
 // whose next instructions are warp-collective tcgen05 loads/stores.
 __device__ __forceinline__ bool wait_warp(const Shared& sh, int* status, uint64_t* bar,
-                                          uint32_t parity, bool drain = false) {
+                                          uint32_t parity, bool drain = false,
+                                          uint64_t limit_ns = kWaitLimitNs) {
   uint64_t t0 = 0;
   for (uint32_t it = 0;; ++it) {
     const bool ok = ptx::mbar_try_wait(bar, parity);
@@ -214,7 +216,7 @@ __device__ __forceinline__ bool wait_warp(const Shared& sh, int* status, uint64_
         if (t0 == 0) t0 = now;
         if (!drain && *sh.abort_flag) {
           stop = 1;
-        } else if (now - t0 > kWaitLimitNs) {
+        } else if (now - t0 > limit_ns) {
           raise_status(sh, status, kStatusDeviceTimeout);
           stop = 1;
         }
@@ -321,7 +323,6 @@ __device__ void producer_role(const Shared& sh, const KernelArgs& a, uint8_t* sm
     if (!post_item(sh, a, r, idx)) break;
     const Item it = decode_item<CAUSAL>(idx, a);
     const int n = it.n0 > it.n1 ? it.n0 : it.n1;
-    const int row0 = it.bh * a.N;  // first row of this (b, h) in the 2-D views
     // Q_s, once the previous item's last S_s no longer needs the buffer.
     for (int s = 0; s < 2 && ok; ++s) {
       if ((s == 0 ? it.n0 : it.n1) == 0) continue;
@@ -332,8 +333,8 @@ __device__ void producer_role(const Shared& sh, const KernelArgs& a, uint8_t* sm
       }
       ptx::mbar_arrive_expect_tx(&sh.q_full[s], C::kTileBytes);
       for (int b = 0; b < C::kBoxes; ++b)
-        ptx::tma_load_2d(tq, &sh.q_full[s], smem + C::kQOff + s * C::kTileBytes + b * C::kBoxBytes,
-                         64 * b, row0 + (2 * it.qpair + s) * kBlockM, pol_q);
+        ptx::tma_load_3d(tq, &sh.q_full[s], smem + C::kQOff + s * C::kTileBytes + b * C::kBoxBytes,
+                         64 * b, (2 * it.qpair + s) * kBlockM, it.bh, pol_q);
       ++q_loads[s];
     }
     for (int j = 0; j < n && ok; ++j) {
@@ -346,8 +347,8 @@ __device__ void producer_role(const Shared& sh, const KernelArgs& a, uint8_t* sm
         ptx::mbar_arrive_expect_tx(&sh.kv_full[st], C::kTileBytes);
         const CUtensorMap* m = which == 0 ? tk : tv;
         for (int b = 0; b < C::kBoxes; ++b)
-          ptx::tma_load_2d(m, &sh.kv_full[st], dst + b * C::kBoxBytes, 64 * b,
-                           row0 + j * kBlockN, pol_kv);
+          ptx::tma_load_3d(m, &sh.kv_full[st], dst + b * C::kBoxBytes, 64 * b, j * kBlockN,
+                           it.bh, pol_kv);
         ++issued;
       }
     }
@@ -549,8 +550,8 @@ __device__ __forceinline__ float exp2_poly1(float x) {
 template <int D, bool CAUSAL, int kPolyPairs>
 __device__ __forceinline__ bool softmax_step(const Shared& sh, const KernelArgs& a, int s,
                                              uint32_t t_s, uint32_t t_o, int r, int lane,
-                                             bool diag, bool first, uint32_t s_parity, int tj,
-                                             float& m, float& l) {
+                                             int key_limit, bool first, uint32_t s_parity,
+                                             int tj, float& m, float& l) {
   const float sl2 = a.scale_log2;
   if (!wait_warp(sh, a.status, &sh.s_full[s], s_parity)) return false;
   ptx::tc_fence_after_sync();
@@ -571,12 +572,14 @@ __device__ __forceinline__ bool softmax_step(const Shared& sh, const KernelArgs&
   for (int c = 0; c < 128; ++c) x[c] = __uint_as_float(sr[c]);
   if (r == 0) ATTN_TRACE(s == 0 ? kTrSm0Ld : kTrSm1Ld, tj);
 
-  // Causal: the last visited tile is the diagonal one (key tile == query
-  // tile); key c of it is visible to row r iff c <= r.
-  if (diag) {
+  // Keys c >= key_limit of this tile are invisible to row r: under the
+  // causal mask on the diagonal tile (key tile == query tile) key_limit is
+  // r + 1; on the last tile of a length that is not a multiple of 128 it is
+  // the number of keys that exist.  Elsewhere it is 128 and nothing is masked.
+  if (__any_sync(0xffffffffu, key_limit < 128)) {
 #pragma unroll
     for (int c = 0; c < 128; ++c)
-      if (c > r) x[c] = -INFINITY;
+      if (c >= key_limit) x[c] = -INFINITY;
   }
 
   // Row max: eight independent chains of three-input maxima.
@@ -705,9 +708,11 @@ __device__ void softmax_role(const Shared& sh, const KernelArgs& a, uint32_t tme
     const int qt = 2 * it.qpair + s;
     float m = -INFINITY;  // running max of scale*log2(e)*score (log2 units)
     float l = 0.f;        // running sum of weights, relative to 2^m
+    const int keys_in_last = a.N - (a.n_qtiles - 1) * kBlockN;  // 1..128
     for (int j = 0; j < n_s; ++j) {
-      const bool diag = CAUSAL && j == n_s - 1;
-      if (!softmax_step<D, CAUSAL, kPolyPairs>(sh, a, s, t_s, t_o, r, lane, diag, j == 0,
+      int key_limit = (j == a.n_qtiles - 1) ? keys_in_last : kBlockN;
+      if (CAUSAL && j == qt) key_limit = r + 1 < key_limit ? r + 1 : key_limit;
+      if (!softmax_step<D, CAUSAL, kPolyPairs>(sh, a, s, t_s, t_o, r, lane, key_limit, j == 0,
                                                static_cast<uint32_t>(s_count & 1),
                                                rr == 0 ? j : -1, m, l))
         return;
@@ -721,6 +726,9 @@ __device__ void softmax_role(const Shared& sh, const KernelArgs& a, uint32_t tme
     ++o_count;
     ptx::tc_fence_after_sync();
     const float inv_l = 1.f / l;
+    // Rows past N (last tile of a ragged length) are computed on zero
+    // queries and not stored.
+    const bool row_ok = qt * kBlockM + r < a.N;
     const size_t row_g = static_cast<size_t>(it.bh) * a.N + static_cast<size_t>(qt) * kBlockM + r;
     __nv_bfloat16* orow = a.o + row_g * D;
 #pragma unroll 1
@@ -733,12 +741,14 @@ __device__ void softmax_role(const Shared& sh, const KernelArgs& a, uint32_t tme
       for (int c = 0; c < 16; ++c)
         pk[c] = ptx::pack_bf16x2(__uint_as_float(ov[2 * c]) * inv_l,
                                  __uint_as_float(ov[2 * c + 1]) * inv_l);
-      uint4* dst = reinterpret_cast<uint4*>(orow + c0);
+      if (row_ok) {
+        uint4* dst = reinterpret_cast<uint4*>(orow + c0);
 #pragma unroll
-      for (int v = 0; v < 4; ++v)
-        dst[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+        for (int v = 0; v < 4; ++v)
+          dst[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+      }
     }
-    a.lse[row_g] = (m + log2f(l)) * 0.69314718055994531f;
+    if (row_ok) a.lse[row_g] = (m + log2f(l)) * 0.69314718055994531f;
   }
 }
 
@@ -837,6 +847,27 @@ __global__ void __launch_bounds__(kThreads, 1)
     ptx::tc_fence_after_sync();
     ptx::tmem_dealloc(tmem, 512);
   }
+}
+
+// ------------------------------------------------------- wait self-test
+// Failure detection without a fault: one warp waits, through the same
+// bounded wait the attention kernel uses, on an mbarrier that nothing ever
+// arrives on.  After limit_ns the wait gives up, writes the timeout code to
+// the status word and returns; the CTA exits normally and the context stays
+// usable.
+__global__ void __launch_bounds__(32, 1) wait_timeout_selftest_kernel(int* status,
+                                                                    uint64_t limit_ns) {
+  __shared__ uint64_t never;
+  __shared__ int abort_flag;
+  Shared sh = {};
+  sh.abort_flag = &abort_flag;
+  if (threadIdx.x == 0) {
+    ptx::mbar_init(&never, 1);
+    abort_flag = 0;
+    ptx::fence_barrier_init();
+  }
+  __syncwarp();
+  wait_warp(sh, status, &never, 0, false, limit_ns);
 }
 
 }  // namespace attn_b200
