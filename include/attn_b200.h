@@ -33,10 +33,12 @@ extern "C" {
 typedef enum {
   ATTN_OK = 0,
   ATTN_ERR_INVALID_ARG = -1,   /* null pointer, non-positive size, bad scale */
-  ATTN_ERR_UNSUPPORTED = -2,   /* d not in {64,128}, or B*H*N >= 2^31 */
+  ATTN_ERR_UNSUPPORTED = -2,   /* d not in {64,96,128}, or B*H*N >= 2^31 */
   ATTN_ERR_MISALIGNED = -3,    /* a device pointer is not 16-byte aligned */
   ATTN_ERR_CUDA = -4,          /* a CUDA runtime/driver call failed */
   ATTN_ERR_DEVICE_TIMEOUT = -5,/* a bounded wait inside the kernel ran out */
+  ATTN_ERR_DEVICE_BOUNDS = -6, /* device-side check: sequence offsets do not
+                                  fit the buffers (attn_fwd_varlen) */
   ATTN_ERR_NO_DEVICE = -7      /* no usable sm_100 device is current */
 } attn_status;
 
@@ -53,7 +55,7 @@ typedef void* attn_stream_t;
  *            denominator of the scaled, masked scores).
  *   o and lse must not overlap q, k, v or each other.
  *   B, H, N  > 0 (any N; tiles past N are masked); B*H*N < 2^31.
- *   d        64 or 128.
+ *   d        64, 96 or 128.
  *   causal   0: every key visible; non-zero: key j visible to query i iff j <= i.
  *   scale    finite and > 0 (typically 1/sqrt(d)).
  *   stream   CUDA stream the kernel is enqueued on.
@@ -115,6 +117,100 @@ int attn_fwd_ex(const void* q, const void* k, const void* v, void* o, float* lse
 int attn_fwd_noalloc(const void* q, const void* k, const void* v, void* o, float* lse,
                      int B, int H, int N, int d, int causal, float scale,
                      attn_stream_t stream);
+
+/*
+ * attn_fwd_chunk -- attention of N_q queries per head against N_k keys per
+ * head, with an explicit causal offset and shared K/V heads.  This is the
+ * building block for key/value caches (queries are the last N_q positions:
+ * causal_delta = N_k - N_q), for splitting the keys into slices, and for
+ * sharding them over GPUs: a chunk's O and LSE are the exact inputs of
+ * attn_combine.
+ *
+ *   q        device, bf16 [B, H, N_q, d].          k, v  bf16 [B, H_kv, N_k, d].
+ *   o        device, [B, H, N_q, d]: bf16, or fp32 when o_fp32 != 0.  Written.
+ *   lse      device, fp32 [B, H, N_q].  Written.
+ *   H_kv     K/V heads; H % H_kv == 0, query head h reads K/V head h/(H/H_kv).
+ *   N_q, N_k > 0; B*H*N_q < 2^31 and B*H_kv*N_k < 2^31.
+ *   causal   non-zero: key j visible to query i iff j <= i + causal_delta
+ *            (|causal_delta| <= 2^30).  A query that sees no key gets O = 0
+ *            and LSE = -inf.  causal = 0 ignores causal_delta.
+ *   d, scale, stream, alignment, overlap, ownership, errors: as attn_fwd
+ *   (o must be 16-byte aligned in both formats).
+ */
+int attn_fwd_chunk(const void* q, const void* k, const void* v, void* o, float* lse,
+                   int B, int H, int H_kv, int N_q, int N_k, int d, int causal,
+                   int causal_delta, float scale, int o_fp32, attn_stream_t stream);
+
+/*
+ * attn_fwd_varlen -- a batch of sequences of different lengths, packed
+ * token-major without padding.
+ *
+ *   q        device, bf16 [total_q, H, d]: the query tokens of sequence b are
+ *            rows cu_seqlens_q[b] .. cu_seqlens_q[b+1]-1.
+ *   k, v     device, bf16 [total_k, H_kv, d], split by cu_seqlens_k.
+ *   o        device, bf16 [total_q, H, d].  Written for every token of every
+ *            sequence.
+ *   lse      device, fp32 [H, total_q].  Written likewise.
+ *   cu_seqlens_q, cu_seqlens_k  device, int32 [B+1], non-decreasing, from 0
+ *            to total_q / total_k; a sequence may be empty.  Read only.
+ *   max_seqlen_q, max_seqlen_k  upper bounds of the sequence lengths (> 0).
+ *   causal   non-zero: inside sequence b, key j visible to query i iff
+ *            j <= i + (len_k(b) - len_q(b)) (the last query sees the last
+ *            key); a query that sees no key gets O = 0 and LSE = -inf.
+ *   H % H_kv == 0; total_q*H and total_k*H_kv < 2^31.
+ *   d, scale, stream, alignment (q, k, v, o: 16 bytes; lse and the offset
+ *   arrays: 4), overlap, ownership and errors: as attn_fwd.  The offsets are
+ *   device data, so they are checked on the device: a sequence whose offsets
+ *   fall outside [0, total] or whose length exceeds its max_seqlen is skipped
+ *   and attn_last_device_error() reports ATTN_ERR_DEVICE_BOUNDS.
+ */
+int attn_fwd_varlen(const void* q, const void* k, const void* v, void* o, float* lse,
+                    const int* cu_seqlens_q, const int* cu_seqlens_k,
+                    int B, int H, int H_kv, int max_seqlen_q, int max_seqlen_k,
+                    int total_q, int total_k, int d, int causal, float scale,
+                    attn_stream_t stream);
+
+/*
+ * attn_fwd_splitkv -- attn_fwd_chunk with each head's keys cut into
+ * n_splits slices that run as separate work items, merged by attn_combine.
+ * Same result as attn_fwd_chunk with a bf16 O (within its tolerance); it
+ * pays when B*H*ceil(N_q/256) work items are too few to fill the GPU, e.g.
+ * a short block of queries against a long key/value cache.
+ *
+ *   q, k, v, o, lse, B, H, H_kv, N_q, N_k, d, causal, causal_delta, scale,
+ *   stream: as attn_fwd_chunk, with a bf16 O.
+ *   n_splits  1 .. 256; it is reduced so that every slice holds keys
+ *             (at most ceil(N_k/128) slices).  With one slice this is
+ *             attn_fwd_chunk.
+ *   ws_o      device, fp32, n_splits * B*H*N_q*d values, 16-byte aligned.
+ *   ws_lse    device, fp32, n_splits * B*H*N_q values.
+ *             Caller-owned scratch (the call allocates nothing); it must not
+ *             overlap the other buffers.  Unused (may be NULL) with one slice.
+ */
+int attn_fwd_splitkv(const void* q, const void* k, const void* v, void* o, float* lse,
+                     int B, int H, int H_kv, int N_q, int N_k, int d, int causal,
+                     int causal_delta, float scale, int n_splits, float* ws_o,
+                     float* ws_lse, attn_stream_t stream);
+
+/*
+ * attn_combine -- merge G partial results of the same query rows against
+ * disjoint key sets (slices of one sequence, or shards on other GPUs) into
+ * the result against their union:
+ *   LSE = log sum_g exp(LSE_g),   O = sum_g exp(LSE_g - LSE) O_g.
+ * This is the online softmax's common-scale rule (page lecompute.fr/kernel-
+ * perf/flashattention-4-limites-calcul-matriciel, section "Deplacer une
+ * partie des exponentielles") applied across slices instead of tiles.
+ *
+ *   o_parts    device, fp32 [G, rows, d], 16-byte aligned.  Read only.
+ *   lse_parts  device, fp32 [G, rows] (-inf: the part saw no key).
+ *   o          device, [rows, d]: bf16, or fp32 when o_fp32 != 0.  Written.
+ *   lse        device, fp32 [rows].  Written (-inf if no part saw a key,
+ *              with O = 0).
+ *   G          1 .. 256;  rows >= 1;  d 64, 96 or 128.
+ *   Outputs must not overlap the inputs.  Errors and asynchrony as attn_fwd.
+ */
+int attn_combine(const float* o_parts, const float* lse_parts, int G, long long rows, int d,
+                 void* o, float* lse, int o_fp32, attn_stream_t stream);
 
 /*
  * attn_fwd_host -- the same operation on HOST buffers: copies q, k, v from

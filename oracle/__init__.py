@@ -9,6 +9,13 @@ Contents
 --------
 ``attn_ref``            the plain fp64 definition (C, ``attn_ref.c``), see that
                         file's header for the formula and the pages it follows.
+``attn_ref_general``    the same definition for N_q queries against N_k keys,
+                        K/V heads shared by groups of query heads, and a
+                        causal offset (empty rows: O = 0, LSE = -inf).
+``attn_ref_varlen``     ``attn_ref_general`` applied to each sequence of a
+                        packed token-major batch.
+``lse_merge``           the result against a union of disjoint key sets from
+                        the results against each set.
 ``tiled_online_model``  a second fp64 formulation that follows the pages'
                         tiled algorithm step by step (tiles of K/V, a running
                         maximum and running sum, lazy rescale).  It is used to
@@ -55,6 +62,13 @@ def _load():
             ctypes.c_int64, ctypes.c_int64, ctypes.c_int64, ctypes.c_int64,
             ctypes.c_int, ctypes.c_double, ctypes.c_int,
             ctypes.c_void_p, ctypes.c_int64]
+        lib.attn_ref_general_f64.restype = ctypes.c_int
+        lib.attn_ref_general_f64.argtypes = [
+            ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+            ctypes.c_void_p, ctypes.c_void_p,
+            ctypes.c_int64, ctypes.c_int64, ctypes.c_int64, ctypes.c_int64, ctypes.c_int64,
+            ctypes.c_int64, ctypes.c_int, ctypes.c_int64, ctypes.c_double, ctypes.c_int,
+            ctypes.c_void_p, ctypes.c_int64]
         lib.attn_ref_max_threads.restype = ctypes.c_int
         lib.attn_ref_max_threads.argtypes = []
         _lib = lib
@@ -99,6 +113,103 @@ def attn_ref(q_bits, k_bits, v_bits, causal: bool, scale: float,
         float(scale), int(nthreads), rows_p, nrows)
     if rc != 0:
         raise ValueError("attn_ref_f64 rejected its arguments")
+    return o, lse
+
+
+def attn_ref_general(q_bits, k_bits, v_bits, causal: bool, delta: int, scale: float,
+                     rows=None, nthreads: int = 0):
+    """Plain fp64 attention of N_q queries against N_k keys (``attn_ref.c``,
+    ``attn_ref_general_f64``).
+
+    q_bits: uint16 bf16 bits [B, H, N_q, d]; k_bits, v_bits: [B, H_kv, N_k, d]
+    with H a multiple of H_kv (query head h reads K/V head h // (H // H_kv)).
+    Under ``causal`` key j is visible to query i iff j <= i + delta; a query
+    that sees no key gets O = 0 and LSE = -inf.  ``rows``: optional flat row
+    indices ``(b*H + h)*N_q + i``.  Returns ``(o, lse)`` in float64 shaped
+    like ``attn_ref``'s.
+    """
+    q_bits = np.ascontiguousarray(q_bits, dtype=np.uint16)
+    k_bits = np.ascontiguousarray(k_bits, dtype=np.uint16)
+    v_bits = np.ascontiguousarray(v_bits, dtype=np.uint16)
+    if q_bits.ndim != 4 or k_bits.ndim != 4 or k_bits.shape != v_bits.shape:
+        raise ValueError("q [B,H,N_q,d]; k, v one [B,H_kv,N_k,d] shape")
+    B, H, N_q, d = q_bits.shape
+    Bk, H_kv, N_k, dk = k_bits.shape
+    if Bk != B or dk != d:
+        raise ValueError("q and k/v disagree on B or d")
+    if rows is None:
+        o = np.empty((B, H, N_q, d), dtype=np.float64)
+        lse = np.empty((B, H, N_q), dtype=np.float64)
+        rows_p, nrows = None, 0
+    else:
+        rows = np.ascontiguousarray(rows, dtype=np.int64)
+        nrows = rows.shape[0]
+        o = np.empty((nrows, d), dtype=np.float64)
+        lse = np.empty((nrows,), dtype=np.float64)
+        rows_p = rows.ctypes.data
+    rc = _load().attn_ref_general_f64(
+        q_bits.ctypes.data, k_bits.ctypes.data, v_bits.ctypes.data,
+        o.ctypes.data, lse.ctypes.data, B, H, H_kv, N_q, N_k, d, int(bool(causal)),
+        int(delta), float(scale), int(nthreads), rows_p, nrows)
+    if rc != 0:
+        raise ValueError("attn_ref_general_f64 rejected its arguments")
+    return o, lse
+
+
+def attn_ref_varlen(q_bits, k_bits, v_bits, cu_q, cu_k, causal: bool, scale: float):
+    """``attn_ref_general`` on each sequence of a packed batch.
+
+    q_bits [T_q, H, d], k_bits and v_bits [T_k, H_kv, d] (uint16 bf16 bits);
+    sequence b owns query tokens cu_q[b]..cu_q[b+1]-1 and key tokens
+    cu_k[b]..cu_k[b+1]-1.  Under ``causal`` the last query of a sequence
+    sees its last key (delta = len_k - len_q).  Returns o [T_q, H, d] and
+    lse [H, T_q] in float64; tokens of a sequence with no keys get O = 0 and
+    LSE = -inf.
+    """
+    q_bits = np.asarray(q_bits, dtype=np.uint16)
+    k_bits = np.asarray(k_bits, dtype=np.uint16)
+    v_bits = np.asarray(v_bits, dtype=np.uint16)
+    T_q, H, d = q_bits.shape
+    o = np.zeros((T_q, H, d), dtype=np.float64)
+    lse = np.full((H, T_q), -np.inf, dtype=np.float64)
+    for b in range(len(cu_q) - 1):
+        q0, q1, k0, k1 = int(cu_q[b]), int(cu_q[b + 1]), int(cu_k[b]), int(cu_k[b + 1])
+        if q1 == q0 or k1 == k0:
+            continue
+        qs = q_bits[q0:q1].transpose(1, 0, 2)[None]
+        ks = k_bits[k0:k1].transpose(1, 0, 2)[None]
+        vs = v_bits[k0:k1].transpose(1, 0, 2)[None]
+        ob, lb = attn_ref_general(qs, ks, vs, causal, (k1 - k0) - (q1 - q0), scale)
+        o[q0:q1] = ob[0].transpose(1, 0, 2)
+        lse[:, q0:q1] = lb[0]
+    return o, lse
+
+
+def lse_merge(o_parts, lse_parts):
+    """Result against a union of disjoint key sets from the results against
+    each set, in fp64.
+
+    Each part's O is its keys' exp-weighted sum of V divided by exp(LSE), so
+    bringing the parts to one common scale (the rule page lecompute.fr/
+    kernel-perf/flashattention-4-limites-calcul-matriciel states for old and
+    new contributions, section "Deplacer une partie des exponentielles") and
+    adding gives LSE = log sum_g exp(LSE_g) and O = sum_g exp(LSE_g - LSE) O_g.
+    A part with LSE_g = -inf (no key) has weight 0; if every part has none,
+    O = 0 and LSE = -inf.
+
+    o_parts [G, rows, d], lse_parts [G, rows].  Returns (o [rows, d], lse [rows]).
+    """
+    o_parts = np.asarray(o_parts, dtype=np.float64)
+    lse_parts = np.asarray(lse_parts, dtype=np.float64)
+    m = lse_parts.max(axis=0)
+    empty = np.isneginf(m)
+    m_safe = np.where(empty, 0.0, m)
+    w = np.exp(lse_parts - m_safe[None, :])            # 0 for parts with no key
+    total = w.sum(axis=0)
+    with np.errstate(divide="ignore"):
+        lse = np.where(empty, -np.inf, m_safe + np.log(np.where(empty, 1.0, total)))
+    wn = np.where(empty[None, :], 0.0, w / np.where(empty, 1.0, total)[None, :])
+    o = np.einsum("gr,grd->rd", wn, o_parts)
     return o, lse
 
 

@@ -131,6 +131,103 @@ int attn_ref_f64(const uint16_t *q, const uint16_t *k, const uint16_t *v,
   return failed ? -1 : 0;
 }
 
+/*
+ * The same definition for queries and keys of different lengths, with K/V
+ * heads shared by groups of query heads and a causal offset:
+ *
+ *   q [B, H, N_q, d],  k and v [B, H_kv, N_k, d];  query head h reads K/V
+ *   head h / (H / H_kv) of its batch;
+ *   J(i) = {0 .. N_k-1}                   (causal == 0)
+ *        = {j < N_k : j <= i + delta}     (causal != 0)
+ *
+ * A row whose J(i) is empty has no weights to normalise: its result is
+ * O = 0 and LSE = log(0) = -inf (the empty sum).  With N_q = N_k, H_kv = H
+ * and delta = 0 this is attn_ref_f64.
+ */
+static void attn_row_general(const uint16_t *q, const uint16_t *k, const uint16_t *v,
+                             int64_t H, int64_t H_kv, int64_t N_q, int64_t N_k,
+                             int64_t d, int causal, int64_t delta, double scale,
+                             int64_t r, double *s, double *o_row, double *lse_row) {
+  const int64_t bh = r / N_q;
+  const int64_t i = r % N_q;
+  const int64_t b = bh / H, h = bh % H;
+  const int64_t bkv = b * H_kv + h / (H / H_kv);
+  const uint16_t *qi = q + r * d;
+  const uint16_t *kb = k + bkv * N_k * d;
+  const uint16_t *vb = v + bkv * N_k * d;
+  int64_t nj = N_k;
+  if (causal) {
+    const int64_t last = i + delta; /* last visible key */
+    nj = last < 0 ? 0 : (last + 1 < N_k ? last + 1 : N_k);
+  }
+  for (int64_t c = 0; c < d; ++c) o_row[c] = 0.0;
+  if (nj == 0) {
+    *lse_row = -INFINITY;
+    return;
+  }
+  double m = -INFINITY;
+  for (int64_t j = 0; j < nj; ++j) {
+    double acc = 0.0;
+    for (int64_t c = 0; c < d; ++c)
+      acc += bf16_to_double(qi[c]) * bf16_to_double(kb[j * d + c]);
+    s[j] = scale * acc;
+    if (s[j] > m) m = s[j];
+  }
+  double l = 0.0;
+  for (int64_t j = 0; j < nj; ++j) {
+    const double p = exp(s[j] - m);
+    l += p;
+    for (int64_t c = 0; c < d; ++c) o_row[c] += p * bf16_to_double(vb[j * d + c]);
+  }
+  for (int64_t c = 0; c < d; ++c) o_row[c] /= l;
+  *lse_row = m + log(l);
+}
+
+/*
+ * attn_ref_general_f64: q host bf16 bits [B,H,N_q,d]; k, v [B,H_kv,N_k,d].
+ *   rows == NULL: every row; o is [B*H*N_q, d], lse [B*H*N_q].
+ *   rows != NULL: the nrows flat row indices (b*H + h)*N_q + i listed.
+ * Returns 0, or -1 on a bad argument (nothing written).
+ */
+int attn_ref_general_f64(const uint16_t *q, const uint16_t *k, const uint16_t *v,
+                         double *o, double *lse, int64_t B, int64_t H, int64_t H_kv,
+                         int64_t N_q, int64_t N_k, int64_t d, int causal, int64_t delta,
+                         double scale, int nthreads, const int64_t *rows, int64_t nrows) {
+  if (!q || !k || !v || !o || !lse) return -1;
+  if (B <= 0 || H <= 0 || H_kv <= 0 || H % H_kv != 0 || N_q <= 0 || N_k <= 0 || d <= 0)
+    return -1;
+  const int64_t total = B * H * N_q;
+  const int64_t n_out = rows ? nrows : total;
+  if (rows) {
+    if (nrows < 0) return -1;
+    for (int64_t t = 0; t < nrows; ++t)
+      if (rows[t] < 0 || rows[t] >= total) return -1;
+  }
+#ifdef _OPENMP
+  if (nthreads > 0) omp_set_num_threads(nthreads);
+#else
+  (void)nthreads;
+#endif
+  int failed = 0;
+#pragma omp parallel
+  {
+    double *s = (double *)malloc(sizeof(double) * (size_t)N_k);
+    if (!s) {
+#pragma omp atomic write
+      failed = 1;
+    } else {
+#pragma omp for schedule(dynamic, 16)
+      for (int64_t t = 0; t < n_out; ++t) {
+        const int64_t r = rows ? rows[t] : t;
+        attn_row_general(q, k, v, H, H_kv, N_q, N_k, d, causal, delta, scale, r, s,
+                         o + t * d, lse + t);
+      }
+      free(s);
+    }
+  }
+  return failed ? -1 : 0;
+}
+
 /* Number of OpenMP threads a parallel region would use (for reporting). */
 int attn_ref_max_threads(void) {
 #ifdef _OPENMP

@@ -57,7 +57,7 @@ def ptrs(d=128, B=1, H=1, N=128):
     return [A, A + tb, A + 2 * tb, A + 3 * tb, A + 4 * tb]
 
 
-@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("d", [64, 96, 128])
 @pytest.mark.parametrize("N", [1, 100, 128, 129, 256, 384, 1000, 32768])
 def test_check_args_accepts_supported(lib, d, N):
     assert tab.check_args(*ptrs(d, 2, 3, N), 2, 3, N, d, 1 / math.sqrt(d)) == 0
@@ -74,7 +74,8 @@ def test_check_args_rejections(lib):
     assert tab.check_args(*p, 1, 1, 128, 128, -1.0) == -1              # scale < 0
     assert tab.check_args(*p, 1, 1, 128, 128, float("nan")) == -1
     assert tab.check_args(*p, 1, 1, 128, 128, float("inf")) == -1
-    assert tab.check_args(*p, 1, 1, 128, 96, 0.1) == -2                # d unsupported
+    assert tab.check_args(*p, 1, 1, 128, 80, 0.1) == -2                # d unsupported
+    assert tab.check_args(*p, 1, 1, 128, 32, 0.1) == -2                # d unsupported
     assert tab.check_args(*p, 1, 1, 128, 256, 0.1) == -2               # d unsupported
     assert tab.check_args(*p, 1 << 12, 1 << 12, 1 << 8, 128, 0.1) == -2  # rows >= 2^31
     q, k, v, o, l = p
@@ -146,3 +147,69 @@ def test_selftest_rejects_bad_limit(lib):
     assert lib.attn_selftest_wait_timeout(0, None) == -1
     assert lib.attn_selftest_wait_timeout(-5, None) == -1
     assert lib.attn_selftest_wait_timeout(20000000, None) == -1
+
+
+def test_new_entry_points_are_declared():
+    syms = declared_symbols()
+    for s in ["attn_fwd_chunk", "attn_fwd_varlen", "attn_fwd_splitkv", "attn_combine",
+              "attn_fwd_noalloc", "attn_selftest_wait_timeout"]:
+        assert s in syms
+
+
+def test_chunk_rejections_before_any_cuda_call(lib):
+    """attn_fwd_chunk's host checks (no device needed to reach them)."""
+    q, k, v, o, l = ptrs()
+    f = lib.attn_fwd_chunk
+    ok = (1, 4, 2, 128, 256, 128, 1, 128, 0.1, 0)
+    assert f(q, k, v, o, l, 1, 4, 3, 128, 256, 128, 1, 0, 0.1, 0, None) == -1  # H % H_kv
+    assert f(q, k, v, o, l, 1, 4, 0, 128, 256, 128, 1, 0, 0.1, 0, None) == -1  # H_kv = 0
+    assert f(q, k, v, o, l, 1, 4, 2, 0, 256, 128, 1, 0, 0.1, 0, None) == -1    # N_q = 0
+    assert f(q, k, v, o, l, 1, 4, 2, 128, 0, 128, 1, 0, 0.1, 0, None) == -1    # N_k = 0
+    assert f(q, k, v, o, l, 1, 4, 2, 128, 256, 80, 1, 0, 0.1, 0, None) == -2   # d
+    assert f(q, k, v, o, l, 1, 4, 2, 128, 256, 128, 1, (1 << 30) + 1, 0.1, 0, None) == -1
+    assert f(q + 8, k, v, o, l, 1, 4, 2, 128, 256, 128, 1, 0, 0.1, 0, None) == -3
+    # LSE placed right after a bf16 O of 4*128 rows: fine for a bf16 O (the
+    # call then fails only for want of a device), an overlap for an fp32 O
+    big = A + (1 << 28)
+    ob = 4 * 128 * 128 * 2
+    args = (big, big + (1 << 22), big + (1 << 23), big + (1 << 24), big + (1 << 24) + ob,
+            1, 4, 2, 128, 256, 128, 1, 0, 0.1)
+    assert f(*args, 0, None) not in (-1, -2, -3)
+    assert f(*args, 1, None) == -1
+    del ok
+
+
+def test_varlen_rejections_before_any_cuda_call(lib):
+    q, k, v, o, l = ptrs()
+    cq, ck = A + (1 << 26), A + (1 << 26) + 4096
+    f = lib.attn_fwd_varlen
+    base = (q, k, v, o, l, cq, ck)
+    assert f(*base[:5], 0, ck, 2, 4, 2, 64, 64, 100, 100, 128, 1, 0.1, None) == -1  # null offsets
+    assert f(*base, 0, 4, 2, 64, 64, 100, 100, 128, 1, 0.1, None) == -1   # B = 0
+    assert f(*base, 2, 4, 3, 64, 64, 100, 100, 128, 1, 0.1, None) == -1   # H % H_kv
+    assert f(*base, 2, 4, 2, 0, 64, 100, 100, 128, 1, 0.1, None) == -1    # max_seqlen_q
+    assert f(*base, 2, 4, 2, 64, 64, 0, 100, 128, 1, 0.1, None) == -1     # total_q
+    assert f(*base, 2, 4, 2, 64, 64, 100, 100, 96 + 16, 1, 0.1, None) == -2
+    assert f(*base, 2, 4, 2, 64, 64, 100, 100, 128, 1, float("nan"), None) == -1
+    assert f(q, k, v, o, l, cq + 2, ck, 2, 4, 2, 64, 64, 100, 100, 128, 1, 0.1, None) == -3
+    assert f(q, k, v, o, l, cq, o, 2, 4, 2, 64, 64, 100, 100, 128, 1, 0.1, None) == -1  # cu_k in o
+    assert f(*base, 2, 1 << 16, 1, 64, 64, 1 << 15, 1 << 15, 128, 1, 0.1, None) == -2  # rows
+
+
+def test_splitkv_and_combine_rejections_before_any_cuda_call(lib):
+    q, k, v, o, l = ptrs(128, 1, 1, 1024)
+    w_o, w_l = A + (1 << 27), A + (1 << 28)
+    f = lib.attn_fwd_splitkv
+    g = (1, 1, 1, 1024, 1024, 128, 1, 0, 0.1)
+    assert f(q, k, v, o, l, *g, 0, w_o, w_l, None) == -1     # 0 slices
+    assert f(q, k, v, o, l, *g, 257, w_o, w_l, None) == -1   # too many
+    assert f(q, k, v, o, l, *g, 4, None, w_l, None) == -1    # no scratch
+    assert f(q, k, v, o, l, *g, 4, w_o + 4, w_l, None) == -3
+    assert f(q, k, v, o, l, *g, 4, q, w_l, None) == -1       # scratch = q
+    assert f(q, k, v, o, l, 1, 2, 3, 1024, 1024, 128, 1, 0, 0.1, 4, w_o, w_l, None) == -1  # heads
+    c = lib.attn_combine
+    assert c(w_o, w_l, 0, 100, 128, o, l, 0, None) == -1      # G = 0
+    assert c(w_o, w_l, 2, 0, 128, o, l, 0, None) == -1        # rows = 0
+    assert c(w_o, w_l, 2, 100, 80, o, l, 0, None) == -2       # d
+    assert c(w_o + 8, w_l, 2, 100, 128, o, l, 0, None) == -3
+    assert c(w_o, w_l, 2, 100, 128, w_o, l, 0, None) == -1    # output over a part

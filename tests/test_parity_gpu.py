@@ -44,7 +44,7 @@ def full_parity(oracle_mod, B, H, N, d, causal, seed, q_std=1.0, scale=None, pol
     return check(o, lse, o_ref, lse_ref, f"B{B} H{H} N{N} d{d} causal={causal}")
 
 
-@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("d", [64, 96, 128])
 @pytest.mark.parametrize("causal", [False, True])
 @pytest.mark.parametrize("N", [128, 256, 384, 640])
 def test_small_shapes(oracle_mod, d, causal, N):
@@ -53,7 +53,7 @@ def test_small_shapes(oracle_mod, d, causal, N):
     full_parity(oracle_mod, 2, 3, N, d, causal, seed=N + d + causal)
 
 
-@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("d", [64, 96, 128])
 @pytest.mark.parametrize("causal", [False, True])
 @pytest.mark.parametrize("N", [1, 7, 100, 129, 255, 300, 1000])
 def test_ragged_lengths(oracle_mod, d, causal, N):
@@ -62,11 +62,13 @@ def test_ragged_lengths(oracle_mod, d, causal, N):
     full_parity(oracle_mod, 2, 3, N, d, causal, seed=900 + N + d, q_std=2.0)
 
 
+@pytest.mark.parametrize("d", [96, 128])
 @pytest.mark.parametrize("causal", [False, True])
-def test_ragged_length_writes_nothing_past_the_rows(causal):
+def test_ragged_length_writes_nothing_past_the_rows(causal, d):
     """B*H heads of N = 200 rows, packed back to back inside guard bands: no
-    head's last, partial tile writes into the next head or past the end."""
-    B, H, N, d = 1, 3, 200, 128
+    head's last, partial tile writes into the next head or past the end (at
+    d = 96 no row writes past its 96 columns either)."""
+    B, H, N = 1, 3, 200
     q, k, v = (t.cuda() for t in make_qkv(B, H, N, d, 11))
     g = 4096
     o_buf = torch.full((g + B * H * N * d + g,), float("nan"), dtype=torch.bfloat16, device="cuda")
@@ -81,7 +83,7 @@ def test_ragged_length_writes_nothing_past_the_rows(causal):
 
 
 @pytest.mark.parametrize("poly", [0, 1, 2])
-@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("d", [64, 96, 128])
 @pytest.mark.parametrize("causal", [False, True])
 def test_exp2_split_variants(oracle_mod, poly, d, causal):
     """Every split of the exponentials between the special-function unit and
@@ -170,7 +172,7 @@ def test_host_entry_point_matches_device_entry_point():
 
 
 def test_rejected_arguments_launch_nothing():
-    q = torch.zeros(1, 1, 128, 96, dtype=torch.bfloat16, device="cuda")  # d = 96: unsupported
+    q = torch.zeros(1, 1, 128, 80, dtype=torch.bfloat16, device="cuda")  # d = 80: unsupported
     with pytest.raises(tab.AttnError) as e:
         tab.attn_fwd(q, q, q)
     assert e.value.status == -2

@@ -59,6 +59,14 @@ def library():
         lib.attn_check_args.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, f]
         lib.attn_version.restype = i
         lib.attn_version.argtypes = []
+        lib.attn_fwd_chunk.restype = i
+        lib.attn_fwd_chunk.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, i, i, f, i, vp]
+        lib.attn_fwd_varlen.restype = i
+        lib.attn_fwd_varlen.argtypes = [vp] * 7 + [i] * 9 + [f, vp]
+        lib.attn_fwd_splitkv.restype = i
+        lib.attn_fwd_splitkv.argtypes = [vp] * 5 + [i] * 8 + [f, i, vp, vp, vp]
+        lib.attn_combine.restype = i
+        lib.attn_combine.argtypes = [vp, vp, i, ctypes.c_longlong, i, vp, vp, i, vp]
         _lib = lib
     return _lib
 
@@ -173,3 +181,138 @@ def selftest_wait_timeout(limit_us: int, stream=None) -> None:
 def last_device_error(stream=None) -> int:
     """Synchronise the stream and return (and clear) the device status word."""
     return int(library().attn_last_device_error(_stream_handle(stream)))
+
+
+def _check(t, name, dtype, shape):
+    if not t.is_cuda or t.dtype != dtype or not t.is_contiguous() or tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must be a contiguous CUDA {dtype} tensor of shape {tuple(shape)}")
+
+
+def attn_fwd_chunk_into(q, k, v, o, lse, causal: bool = False, causal_delta: int = 0,
+                        scale: float | None = None, stream=None) -> None:
+    """N_q queries against N_k keys per head (see attn_fwd_chunk in the
+    header): q bf16 [B,H,N_q,d]; k, v bf16 [B,H_kv,N_k,d]; o [B,H,N_q,d] in
+    bf16 or fp32 (fp32 keeps partial results exact for attn_combine); lse fp32
+    [B,H,N_q].  Under ``causal`` key j is visible to query i iff
+    j <= i + causal_delta."""
+    if q.dim() != 4 or k.dim() != 4:
+        raise ValueError("q, k, v must be 4-D")
+    B, H, N_q, d = (int(x) for x in q.shape)
+    _, H_kv, N_k, _ = (int(x) for x in k.shape)
+    _check(q, "q", torch.bfloat16, (B, H, N_q, d))
+    _check(k, "k", torch.bfloat16, (B, H_kv, N_k, d))
+    _check(v, "v", torch.bfloat16, (B, H_kv, N_k, d))
+    if o.dtype not in (torch.bfloat16, torch.float32):
+        raise ValueError("o must be bf16 or fp32")
+    _check(o, "o", o.dtype, (B, H, N_q, d))
+    _check(lse, "lse", torch.float32, (B, H, N_q))
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    rc = library().attn_fwd_chunk(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
+                                  lse.data_ptr(), B, H, H_kv, N_q, N_k, d, int(bool(causal)),
+                                  int(causal_delta), float(scale),
+                                  int(o.dtype == torch.float32), _stream_handle(stream))
+    if rc != ATTN_OK:
+        raise AttnError(rc, "attn_fwd_chunk")
+
+
+def attn_fwd_chunk(q, k, v, causal: bool = False, causal_delta: int = 0,
+                   scale: float | None = None, out_dtype=torch.bfloat16, stream=None):
+    """Return ``(o, lse)`` of attn_fwd_chunk_into."""
+    B, H, N_q, d = (int(x) for x in q.shape)
+    o = torch.empty((B, H, N_q, d), dtype=out_dtype, device=q.device)
+    lse = torch.empty((B, H, N_q), dtype=torch.float32, device=q.device)
+    attn_fwd_chunk_into(q, k, v, o, lse, causal, causal_delta, scale, stream)
+    return o, lse
+
+
+def attn_fwd_varlen(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q: int, max_seqlen_k: int,
+                    causal: bool = False, scale: float | None = None, stream=None):
+    """Packed variable-length batch (see attn_fwd_varlen in the header):
+    q bf16 [T_q, H, d]; k, v bf16 [T_k, H_kv, d]; cu_seqlens_* CUDA int32
+    [B+1].  Returns o bf16 [T_q, H, d] and lse fp32 [H, T_q]."""
+    if q.dim() != 3 or k.dim() != 3:
+        raise ValueError("q, k, v must be [tokens, heads, d]")
+    T_q, H, d = (int(x) for x in q.shape)
+    T_k, H_kv, _ = (int(x) for x in k.shape)
+    _check(q, "q", torch.bfloat16, (T_q, H, d))
+    _check(k, "k", torch.bfloat16, (T_k, H_kv, d))
+    _check(v, "v", torch.bfloat16, (T_k, H_kv, d))
+    B = int(cu_seqlens_q.shape[0]) - 1
+    _check(cu_seqlens_q, "cu_seqlens_q", torch.int32, (B + 1,))
+    _check(cu_seqlens_k, "cu_seqlens_k", torch.int32, (B + 1,))
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    o = torch.empty_like(q)
+    lse = torch.empty((H, T_q), dtype=torch.float32, device=q.device)
+    rc = library().attn_fwd_varlen(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
+                                   lse.data_ptr(), cu_seqlens_q.data_ptr(),
+                                   cu_seqlens_k.data_ptr(), B, H, H_kv, int(max_seqlen_q),
+                                   int(max_seqlen_k), T_q, T_k, d, int(bool(causal)),
+                                   float(scale), _stream_handle(stream))
+    if rc != ATTN_OK:
+        raise AttnError(rc, "attn_fwd_varlen")
+    return o, lse
+
+
+def splitkv_slices(N: int, n_splits: int) -> int:
+    """Key slices attn_fwd_splitkv actually uses for N keys (every slice
+    holds keys)."""
+    tiles = (int(N) + 127) // 128
+    per = (tiles + int(n_splits) - 1) // int(n_splits)
+    return (tiles + per - 1) // per
+
+
+def attn_fwd_splitkv(q, k, v, n_splits: int, causal: bool = False, causal_delta: int = 0,
+                     scale: float | None = None, stream=None):
+    """attn_fwd_chunk (bf16 O) with each head's keys cut into ``n_splits``
+    slices that run as separate work items and are merged by the LSE combine
+    kernel (see the header).  q bf16 [B,H,N_q,d]; k, v bf16 [B,H_kv,N_k,d].
+    The fp32 scratch is allocated here from torch's allocator."""
+    if q.dim() != 4 or k.dim() != 4:
+        raise ValueError("q, k, v must be 4-D")
+    B, H, N_q, d = (int(x) for x in q.shape)
+    _, H_kv, N_k, _ = (int(x) for x in k.shape)
+    _check(q, "q", torch.bfloat16, (B, H, N_q, d))
+    _check(k, "k", torch.bfloat16, (B, H_kv, N_k, d))
+    _check(v, "v", torch.bfloat16, (B, H_kv, N_k, d))
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    used = splitkv_slices(N_k, n_splits) if n_splits >= 1 else 0
+    o = torch.empty_like(q)
+    lse = torch.empty((B, H, N_q), dtype=torch.float32, device=q.device)
+    if used > 1:
+        ws_o = torch.empty((used, B * H * N_q, d), dtype=torch.float32, device=q.device)
+        ws_l = torch.empty((used, B * H * N_q), dtype=torch.float32, device=q.device)
+        wp = (ws_o.data_ptr(), ws_l.data_ptr())
+    else:
+        wp = (None, None)
+    rc = library().attn_fwd_splitkv(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
+                                    lse.data_ptr(), B, H, H_kv, N_q, N_k, d, int(bool(causal)),
+                                    int(causal_delta), float(scale), int(n_splits), wp[0], wp[1],
+                                    _stream_handle(stream))
+    if rc != ATTN_OK:
+        raise AttnError(rc, "attn_fwd_splitkv")
+    return o, lse
+
+
+def attn_combine(o_parts, lse_parts, out_dtype=torch.bfloat16, stream=None):
+    """LSE merge of partial results (see attn_combine in the header):
+    o_parts fp32 [G, ..., d], lse_parts fp32 [G, ...] with matching leading
+    shapes.  Returns (o [..., d] in ``out_dtype``, lse fp32 [...])."""
+    if o_parts.dim() < 2 or tuple(o_parts.shape[:-1]) != tuple(lse_parts.shape):
+        raise ValueError("o_parts must be [G, ..., d] and lse_parts [G, ...]")
+    G, d = int(o_parts.shape[0]), int(o_parts.shape[-1])
+    rows = int(lse_parts[0].numel())
+    _check(o_parts, "o_parts", torch.float32, o_parts.shape)
+    _check(lse_parts, "lse_parts", torch.float32, lse_parts.shape)
+    if out_dtype not in (torch.bfloat16, torch.float32):
+        raise ValueError("out_dtype must be bf16 or fp32")
+    o = torch.empty(tuple(o_parts.shape[1:]), dtype=out_dtype, device=o_parts.device)
+    lse = torch.empty(tuple(lse_parts.shape[1:]), dtype=torch.float32, device=o_parts.device)
+    rc = library().attn_combine(o_parts.data_ptr(), lse_parts.data_ptr(), G, rows, d,
+                                o.data_ptr(), lse.data_ptr(), int(out_dtype == torch.float32),
+                                _stream_handle(stream))
+    if rc != ATTN_OK:
+        raise AttnError(rc, "attn_combine")
+    return o, lse

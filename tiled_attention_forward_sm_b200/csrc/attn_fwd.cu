@@ -13,6 +13,7 @@
 #include <mutex>
 
 #include "attn_b200.h"
+#include "attn_combine_kernel.cuh"
 #include "attn_fwd_kernel.cuh"
 
 namespace attn_b200 {
@@ -41,6 +42,8 @@ static __device__ __align__(256) int g_attn_noalloc_scratch[kNoAllocScratchBytes
 namespace {
 
 constexpr int kMaxDevices = 64;
+// Most key slices of one split-KV launch (and parts of one merge).
+constexpr int kMaxSplits = 256;
 
 struct DeviceState {
   bool checked = false;
@@ -111,16 +114,36 @@ int device_state(DeviceState** out) {
   return ATTN_OK;
 }
 
-// 3-D view [B*H][N][d] of a [B,H,N,d] bf16 tensor; boxes of 128 rows x 64
-// columns of one head, with the 128-byte swizzle the tcgen05 shared-memory
-// descriptors expect.  Rows past N of a head are outside the view and read
-// as zero, so a tile never picks up the next head's rows.
-int make_tmap(CUtensorMap* m, const void* ptr, int BH, int N, int d) {
+// Per-head 3-D view [Z][N][d] of a [.., N, d] bf16 tensor (Z = batch x
+// heads); boxes of 128 rows x 64 columns of one head, with the 128-byte
+// swizzle the tcgen05 shared-memory descriptors expect.  Rows past N of a
+// head are outside the view and read as zero, so a tile never picks up the
+// next head's rows.
+int make_tmap_heads(CUtensorMap* m, const void* ptr, int Z, int N, int d) {
   cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(N),
-                        static_cast<cuuint64_t>(BH)};
+                        static_cast<cuuint64_t>(Z)};
   cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2,
                            static_cast<cuuint64_t>(N) * static_cast<cuuint64_t>(d) * 2};
   cuuint32_t box[3] = {64, 128, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims,
+                        strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+// Token-major 3-D view [T][Hx][d] of a packed [T, Hx, d] bf16 tensor; boxes
+// of 64 columns x 1 head x 128 tokens, which land in shared memory exactly
+// like the per-head boxes (128 rows of 128 bytes).  Tokens past T read as
+// zero; tokens of the next sequence inside a tile are masked (keys) or not
+// stored (queries) by the kernel.
+int make_tmap_tokens(CUtensorMap* m, const void* ptr, int T, int Hx, int d) {
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(Hx),
+                        static_cast<cuuint64_t>(T)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2,
+                           static_cast<cuuint64_t>(Hx) * static_cast<cuuint64_t>(d) * 2};
+  cuuint32_t box[3] = {64, 1, 128};
   cuuint32_t estr[3] = {1, 1, 1};
   CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims,
                         strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
@@ -134,34 +157,83 @@ bool ranges_overlap(const void* a, size_t na, const void* b, size_t nb) {
   return x < y + nb && y < x + na;
 }
 
+// One attention launch, in either layout (see KernelArgs).  Checked by the
+// entry points before it reaches launch().
+struct Problem {
+  const void* q = nullptr;
+  const void* k = nullptr;
+  const void* v = nullptr;
+  void* o = nullptr;
+  float* lse = nullptr;
+  const int* cu_q = nullptr;  // packed layout when set
+  const int* cu_k = nullptr;
+  int B = 0, H = 0, H_kv = 0;
+  int N_q = 0, N_k = 0;  // per head, or the longest sequence (packed)
+  int T_q = 0, T_k = 0;  // packed: total tokens
+  int d = 0;
+  int causal = 0;
+  int delta = 0;         // dense causal offset
+  float scale = 0.f;
+  int o_f32 = 0;
+  int n_splits = 1;
+  int split_tiles = 0;   // 0: all K/V tiles in one slice
+  long long split_rows = 0;
+};
+
+// Work items of a problem: (head, Q tile pair, key slice).
+int64_t problem_items(const Problem& p) {
+  const int64_t pairs = ((static_cast<int64_t>(p.N_q) + kBlockM - 1) / kBlockM + 1) / 2;
+  return static_cast<int64_t>(p.B) * p.H * pairs * p.n_splits;
+}
+
 template <int D, bool CAUSAL, int kPolyPairs>
-int launch(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
-           int N, float scale, cudaStream_t stream, DeviceState& st, int* queue = nullptr) {
+int launch(const Problem& p, cudaStream_t stream, DeviceState& st, int* queue = nullptr) {
   using C = Config<D>;
   CUtensorMap tq, tk, tv;
-  if (make_tmap(&tq, q, B * H, N, D) || make_tmap(&tk, k, B * H, N, D) ||
-      make_tmap(&tv, v, B * H, N, D))
-    return ATTN_ERR_CUDA;
+  if (p.cu_q != nullptr) {
+    if (make_tmap_tokens(&tq, p.q, p.T_q, p.H, D) || make_tmap_tokens(&tk, p.k, p.T_k, p.H_kv, D) ||
+        make_tmap_tokens(&tv, p.v, p.T_k, p.H_kv, D))
+      return ATTN_ERR_CUDA;
+  } else {
+    if (make_tmap_heads(&tq, p.q, p.B * p.H, p.N_q, D) ||
+        make_tmap_heads(&tk, p.k, p.B * p.H_kv, p.N_k, D) ||
+        make_tmap_heads(&tv, p.v, p.B * p.H_kv, p.N_k, D))
+      return ATTN_ERR_CUDA;
+  }
 
   KernelArgs args;
-  args.o = static_cast<__nv_bfloat16*>(o);
-  args.lse = lse;
-  args.N = N;
-  args.n_qtiles = (N + kBlockM - 1) / kBlockM;
-  args.n_qpairs = (args.n_qtiles + 1) / 2;
-  args.BH = B * H;
-  args.n_items = args.BH * args.n_qpairs;
+  args.o = p.o;
+  args.lse = p.lse;
+  args.cu_q = p.cu_q;
+  args.cu_k = p.cu_k;
+  args.H = p.H;
+  args.H_kv = p.H_kv;
+  args.q_per_kv = p.H / p.H_kv;
+  args.N_q = p.N_q;
+  args.N_k = p.N_k;
+  args.T_q = p.T_q;
+  args.T_k = p.T_k;
+  args.delta = p.delta;
+  args.n_qpairs = ((p.N_q + kBlockM - 1) / kBlockM + 1) / 2;
+  args.n_splits = p.n_splits;
+  args.split_tiles = p.split_tiles > 0 ? p.split_tiles : (p.N_k + kBlockN - 1) / kBlockN;
+  if (args.split_tiles < 1) args.split_tiles = 1;
+  args.split_rows = p.split_rows;
+  args.o_f32 = p.o_f32;
+  args.BH = p.B * p.H;
+  args.n_items = static_cast<int>(problem_items(p));
   // Scheduling window: enough heads that a window holds about two rounds of
   // items (so its light tail evens out the CTAs), few enough that the
   // window's K/V stays in L2 while its CTAs run.
   {
-    const int want = (2 * st.num_sms + args.n_qpairs - 1) / args.n_qpairs;
+    const int per_head = args.n_qpairs * args.n_splits;
+    const int want = (2 * st.num_sms + per_head - 1) / per_head;
     args.win_heads = want < 1 ? 1 : (want > args.BH ? args.BH : want);
   }
   args.queue = queue != nullptr
                    ? queue
                    : st.queue + 2 * static_cast<int>(st.launches.fetch_add(1) % kQueueSlots);
-  args.scale_log2 = scale * 1.4426950408889634f;
+  args.scale_log2 = p.scale * 1.4426950408889634f;
   args.status = st.status;
 
   auto kern = attn_fwd_kernel<D, CAUSAL, kPolyPairs>;
@@ -203,17 +275,116 @@ int launch(const void* q, const void* k, const void* v, void* o, float* lse, int
 constexpr int kDefaultPolyPairs = 0;
 
 template <int D, bool CAUSAL>
-int launch_poly(int poly_pairs, const void* q, const void* k, const void* v, void* o, float* lse,
-                int B, int H, int N, float scale, cudaStream_t s, DeviceState& st) {
+int launch_poly(int poly_pairs, const Problem& p, cudaStream_t s, DeviceState& st, int* queue) {
   switch (poly_pairs) {
-    case 0: return launch<D, CAUSAL, 0>(q, k, v, o, lse, B, H, N, scale, s, st);
-    case 2: return launch<D, CAUSAL, 2>(q, k, v, o, lse, B, H, N, scale, s, st);
-    default: return launch<D, CAUSAL, 1>(q, k, v, o, lse, B, H, N, scale, s, st);
+    case 0: return launch<D, CAUSAL, 0>(p, s, st, queue);
+    case 2: return launch<D, CAUSAL, 2>(p, s, st, queue);
+    default: return launch<D, CAUSAL, 1>(p, s, st, queue);
   }
 }
 
-int fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N,
-             int d, int causal, float scale, int poly_pairs, attn_stream_t stream);
+template <int D>
+int launch_d(int poly_pairs, const Problem& p, cudaStream_t s, DeviceState& st, int* queue) {
+  return p.causal ? launch_poly<D, true>(poly_pairs, p, s, st, queue)
+                  : launch_poly<D, false>(poly_pairs, p, s, st, queue);
+}
+
+// Launch a checked problem on the calling thread's device.
+int run_problem(const Problem& p, int poly_pairs, attn_stream_t stream, int* queue = nullptr,
+                DeviceState* st = nullptr) {
+  if (st == nullptr) {
+    const int rc = device_state(&st);
+    if (rc != ATTN_OK) return rc;
+  }
+  if (problem_items(p) + st->num_sms > 0x7FFFFFFFll) return ATTN_ERR_UNSUPPORTED;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  switch (p.d) {
+    case 128: return launch_d<128>(poly_pairs, p, s, *st, queue);
+    case 96: return launch_d<96>(poly_pairs, p, s, *st, queue);
+    default: return launch_d<64>(poly_pairs, p, s, *st, queue);
+  }
+}
+
+// LSE merge of G partial results (see attn_combine_kernel.cuh).
+int run_combine(const float* o_parts, const float* lse_parts, int G, long long rows, int d,
+                void* o, float* lse, int o_f32, attn_stream_t stream, const DeviceState& st) {
+  const long long threads = rows * (d / 4);
+  long long blocks = (threads + 255) / 256;
+  const long long cap = static_cast<long long>(st.num_sms) * 8;
+  if (blocks > cap) blocks = cap;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (o_f32)
+    lse_combine_kernel<true><<<static_cast<unsigned>(blocks), 256, 0, s>>>(o_parts, lse_parts, G,
+                                                                          rows, d, o, lse);
+  else
+    lse_combine_kernel<false><<<static_cast<unsigned>(blocks), 256, 0, s>>>(o_parts, lse_parts, G,
+                                                                           rows, d, o, lse);
+  if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
+  return ATTN_OK;
+}
+
+bool head_dim_ok(int d) { return d == 64 || d == 96 || d == 128; }
+
+bool scale_ok(float scale) { return std::isfinite(scale) && scale > 0.f; }
+
+// Output buffers must not overlap the inputs or one another.
+bool outputs_disjoint(const void* const* outs, const size_t* out_bytes, int n_out,
+                      const void* const* ins, const size_t* in_bytes, int n_in) {
+  for (int i = 0; i < n_out; ++i) {
+    for (int j = 0; j < n_in; ++j)
+      if (ranges_overlap(outs[i], out_bytes[i], ins[j], in_bytes[j])) return false;
+    for (int j = i + 1; j < n_out; ++j)
+      if (ranges_overlap(outs[i], out_bytes[i], outs[j], out_bytes[j])) return false;
+  }
+  return true;
+}
+
+// Checks of a dense problem with per-head layout (attn_fwd, attn_fwd_chunk).
+int check_dense(const Problem& p) {
+  if (!p.q || !p.k || !p.v || !p.o || !p.lse) return ATTN_ERR_INVALID_ARG;
+  if (p.B <= 0 || p.H <= 0 || p.H_kv <= 0 || p.N_q <= 0 || p.N_k <= 0) return ATTN_ERR_INVALID_ARG;
+  if (p.H % p.H_kv != 0) return ATTN_ERR_INVALID_ARG;
+  if (!scale_ok(p.scale)) return ATTN_ERR_INVALID_ARG;
+  if (p.delta < -(1 << 30) || p.delta > (1 << 30)) return ATTN_ERR_INVALID_ARG;
+  if (!head_dim_ok(p.d)) return ATTN_ERR_UNSUPPORTED;
+  const uint64_t rows_q = static_cast<uint64_t>(p.B) * p.H * p.N_q;
+  const uint64_t rows_k = static_cast<uint64_t>(p.B) * p.H_kv * p.N_k;
+  // Rows are numbered in int on the device.
+  if (rows_q >= (1ull << 31) || rows_k >= (1ull << 31)) return ATTN_ERR_UNSUPPORTED;
+  const uintptr_t al = reinterpret_cast<uintptr_t>(p.q) | reinterpret_cast<uintptr_t>(p.k) |
+                       reinterpret_cast<uintptr_t>(p.v) | reinterpret_cast<uintptr_t>(p.o);
+  if (al & 15u) return ATTN_ERR_MISALIGNED;
+  if (reinterpret_cast<uintptr_t>(p.lse) & 3u) return ATTN_ERR_MISALIGNED;
+  const size_t qb = rows_q * static_cast<size_t>(p.d) * 2, kb = rows_k * static_cast<size_t>(p.d) * 2;
+  const size_t splits = p.n_splits > 1 ? static_cast<size_t>(p.n_splits) : 1;
+  const size_t ob = splits * rows_q * static_cast<size_t>(p.d) * (p.o_f32 ? 4 : 2);
+  const size_t lb = splits * rows_q * 4;
+  const void* outs[2] = {p.o, p.lse};
+  const size_t out_bytes[2] = {ob, lb};
+  const void* ins[3] = {p.q, p.k, p.v};
+  const size_t in_bytes[3] = {qb, kb, kb};
+  if (!outputs_disjoint(outs, out_bytes, 2, ins, in_bytes, 3)) return ATTN_ERR_INVALID_ARG;
+  return ATTN_OK;
+}
+
+Problem dense_problem(const void* q, const void* k, const void* v, void* o, float* lse, int B,
+                      int H, int N, int d, int causal, float scale) {
+  Problem p;
+  p.q = q;
+  p.k = k;
+  p.v = v;
+  p.o = o;
+  p.lse = lse;
+  p.B = B;
+  p.H = H;
+  p.H_kv = H;
+  p.N_q = N;
+  p.N_k = N;
+  p.d = d;
+  p.causal = causal ? 1 : 0;
+  p.scale = scale;
+  return p;
+}
 
 }  // namespace
 }  // namespace attn_b200
@@ -222,48 +393,16 @@ using namespace attn_b200;
 
 extern "C" int attn_check_args(const void* q, const void* k, const void* v, const void* o,
                                const float* lse, int B, int H, int N, int d, float scale) {
-  if (!q || !k || !v || !o || !lse) return ATTN_ERR_INVALID_ARG;
-  if (B <= 0 || H <= 0 || N <= 0) return ATTN_ERR_INVALID_ARG;
-  if (!std::isfinite(scale) || !(scale > 0.f)) return ATTN_ERR_INVALID_ARG;
-  if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
-  const uint64_t rows = static_cast<uint64_t>(B) * H * N;
-  // Work items (B*H*ceil(N/256)) are numbered in int.
-  if (rows >= (1ull << 31)) return ATTN_ERR_UNSUPPORTED;
-  const uintptr_t al = reinterpret_cast<uintptr_t>(q) | reinterpret_cast<uintptr_t>(k) |
-                       reinterpret_cast<uintptr_t>(v) | reinterpret_cast<uintptr_t>(o);
-  if (al & 15u) return ATTN_ERR_MISALIGNED;
-  if (reinterpret_cast<uintptr_t>(lse) & 3u) return ATTN_ERR_MISALIGNED;
-  const size_t tb = rows * static_cast<size_t>(d) * 2, lb = rows * 4;
-  if (ranges_overlap(o, tb, q, tb) || ranges_overlap(o, tb, k, tb) ||
-      ranges_overlap(o, tb, v, tb) || ranges_overlap(lse, lb, q, tb) ||
-      ranges_overlap(lse, lb, k, tb) || ranges_overlap(lse, lb, v, tb) ||
-      ranges_overlap(lse, lb, o, tb))
-    return ATTN_ERR_INVALID_ARG;
-  return ATTN_OK;
+  return check_dense(dense_problem(q, k, v, const_cast<void*>(o), const_cast<float*>(lse), B, H,
+                                   N, d, 0, scale));
 }
-
-namespace attn_b200 {
-namespace {
-int fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N,
-             int d, int causal, float scale, int poly_pairs, attn_stream_t stream) {
-  int rc = attn_check_args(q, k, v, o, lse, B, H, N, d, scale);
-  if (rc != ATTN_OK) return rc;
-  DeviceState* st = nullptr;
-  rc = device_state(&st);
-  if (rc != ATTN_OK) return rc;
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (d == 128)
-    return causal ? launch_poly<128, true>(poly_pairs, q, k, v, o, lse, B, H, N, scale, s, *st)
-                  : launch_poly<128, false>(poly_pairs, q, k, v, o, lse, B, H, N, scale, s, *st);
-  return causal ? launch_poly<64, true>(poly_pairs, q, k, v, o, lse, B, H, N, scale, s, *st)
-                : launch_poly<64, false>(poly_pairs, q, k, v, o, lse, B, H, N, scale, s, *st);
-}
-}  // namespace
-}  // namespace attn_b200
 
 extern "C" int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B,
                         int H, int N, int d, int causal, float scale, attn_stream_t stream) {
-  return fwd_impl(q, k, v, o, lse, B, H, N, d, causal, scale, kDefaultPolyPairs, stream);
+  const Problem p = dense_problem(q, k, v, o, lse, B, H, N, d, causal, scale);
+  const int rc = check_dense(p);
+  if (rc != ATTN_OK) return rc;
+  return run_problem(p, kDefaultPolyPairs, stream);
 }
 
 extern "C" int attn_fwd_ex(const void* q, const void* k, const void* v, void* o, float* lse, int B,
@@ -274,7 +413,127 @@ extern "C" int attn_fwd_ex(const void* q, const void* k, const void* v, void* o,
     if (opts->exp2_poly_pairs < -1 || opts->exp2_poly_pairs > 2) return ATTN_ERR_INVALID_ARG;
     if (opts->exp2_poly_pairs >= 0) poly = opts->exp2_poly_pairs;
   }
-  return fwd_impl(q, k, v, o, lse, B, H, N, d, causal, scale, poly, stream);
+  const Problem p = dense_problem(q, k, v, o, lse, B, H, N, d, causal, scale);
+  const int rc = check_dense(p);
+  if (rc != ATTN_OK) return rc;
+  return run_problem(p, poly, stream);
+}
+
+extern "C" int attn_fwd_chunk(const void* q, const void* k, const void* v, void* o, float* lse,
+                              int B, int H, int H_kv, int N_q, int N_k, int d, int causal,
+                              int causal_delta, float scale, int o_fp32, attn_stream_t stream) {
+  Problem p = dense_problem(q, k, v, o, lse, B, H, N_q, d, causal, scale);
+  p.H_kv = H_kv;
+  p.N_k = N_k;
+  p.delta = causal_delta;
+  p.o_f32 = o_fp32 ? 1 : 0;
+  const int rc = check_dense(p);
+  if (rc != ATTN_OK) return rc;
+  return run_problem(p, kDefaultPolyPairs, stream);
+}
+
+extern "C" int attn_fwd_varlen(const void* q, const void* k, const void* v, void* o, float* lse,
+                               const int* cu_seqlens_q, const int* cu_seqlens_k, int B, int H,
+                               int H_kv, int max_seqlen_q, int max_seqlen_k, int total_q,
+                               int total_k, int d, int causal, float scale,
+                               attn_stream_t stream) {
+  if (!q || !k || !v || !o || !lse || !cu_seqlens_q || !cu_seqlens_k) return ATTN_ERR_INVALID_ARG;
+  if (B <= 0 || H <= 0 || H_kv <= 0 || H % H_kv != 0) return ATTN_ERR_INVALID_ARG;
+  if (max_seqlen_q <= 0 || max_seqlen_k <= 0 || total_q <= 0 || total_k <= 0)
+    return ATTN_ERR_INVALID_ARG;
+  if (!scale_ok(scale)) return ATTN_ERR_INVALID_ARG;
+  if (!head_dim_ok(d)) return ATTN_ERR_UNSUPPORTED;
+  const uint64_t rows_q = static_cast<uint64_t>(total_q) * H;
+  const uint64_t rows_k = static_cast<uint64_t>(total_k) * H_kv;
+  if (rows_q >= (1ull << 31) || rows_k >= (1ull << 31)) return ATTN_ERR_UNSUPPORTED;
+  const uintptr_t al = reinterpret_cast<uintptr_t>(q) | reinterpret_cast<uintptr_t>(k) |
+                       reinterpret_cast<uintptr_t>(v) | reinterpret_cast<uintptr_t>(o);
+  if (al & 15u) return ATTN_ERR_MISALIGNED;
+  if ((reinterpret_cast<uintptr_t>(lse) | reinterpret_cast<uintptr_t>(cu_seqlens_q) |
+       reinterpret_cast<uintptr_t>(cu_seqlens_k)) & 3u)
+    return ATTN_ERR_MISALIGNED;
+  const size_t qb = rows_q * static_cast<size_t>(d) * 2, kb = rows_k * static_cast<size_t>(d) * 2;
+  const size_t cb = (static_cast<size_t>(B) + 1) * 4;
+  const void* outs[2] = {o, lse};
+  const size_t out_bytes[2] = {qb, rows_q * 4};
+  const void* ins[5] = {q, k, v, cu_seqlens_q, cu_seqlens_k};
+  const size_t in_bytes[5] = {qb, kb, kb, cb, cb};
+  if (!outputs_disjoint(outs, out_bytes, 2, ins, in_bytes, 5)) return ATTN_ERR_INVALID_ARG;
+  Problem p = dense_problem(q, k, v, o, lse, B, H, max_seqlen_q, d, causal, scale);
+  p.H_kv = H_kv;
+  p.N_k = max_seqlen_k;
+  p.cu_q = cu_seqlens_q;
+  p.cu_k = cu_seqlens_k;
+  p.T_q = total_q;
+  p.T_k = total_k;
+  return run_problem(p, kDefaultPolyPairs, stream);
+}
+
+extern "C" int attn_fwd_splitkv(const void* q, const void* k, const void* v, void* o, float* lse,
+                                int B, int H, int H_kv, int N_q, int N_k, int d, int causal,
+                                int causal_delta, float scale, int n_splits, float* ws_o,
+                                float* ws_lse, attn_stream_t stream) {
+  if (n_splits < 1 || n_splits > kMaxSplits) return ATTN_ERR_INVALID_ARG;
+  Problem p = dense_problem(q, k, v, o, lse, B, H, N_q, d, causal, scale);
+  p.H_kv = H_kv;
+  p.N_k = N_k;
+  p.delta = causal_delta;
+  int rc = check_dense(p);
+  if (rc != ATTN_OK) return rc;
+  const int tiles = (N_k + kBlockN - 1) / kBlockN;
+  const int split_tiles = (tiles + n_splits - 1) / n_splits;
+  const int used = (tiles + split_tiles - 1) / split_tiles;  // slices that hold keys
+  if (used <= 1) return run_problem(p, kDefaultPolyPairs, stream);
+  if (!ws_o || !ws_lse) return ATTN_ERR_INVALID_ARG;
+  if (reinterpret_cast<uintptr_t>(ws_o) & 15u) return ATTN_ERR_MISALIGNED;
+  if (reinterpret_cast<uintptr_t>(ws_lse) & 3u) return ATTN_ERR_MISALIGNED;
+  const uint64_t rows = static_cast<uint64_t>(B) * H * N_q;
+  const uint64_t rows_k = static_cast<uint64_t>(B) * H_kv * N_k;
+  const size_t qb = rows * static_cast<size_t>(d) * 2, kb = rows_k * static_cast<size_t>(d) * 2;
+  const size_t wob = static_cast<size_t>(used) * rows * static_cast<size_t>(d) * 4;
+  const size_t wlb = static_cast<size_t>(used) * rows * 4;
+  const void* outs[4] = {o, lse, ws_o, ws_lse};
+  const size_t out_bytes[4] = {qb, rows * 4, wob, wlb};
+  const void* ins[3] = {q, k, v};
+  const size_t in_bytes[3] = {qb, kb, kb};
+  if (!outputs_disjoint(outs, out_bytes, 4, ins, in_bytes, 3)) return ATTN_ERR_INVALID_ARG;
+  DeviceState* st = nullptr;
+  rc = device_state(&st);
+  if (rc != ATTN_OK) return rc;
+  Problem part = p;
+  part.o = ws_o;
+  part.lse = ws_lse;
+  part.o_f32 = 1;
+  part.n_splits = used;
+  part.split_tiles = split_tiles;
+  part.split_rows = static_cast<long long>(rows);
+  rc = run_problem(part, kDefaultPolyPairs, stream, nullptr, st);
+  if (rc != ATTN_OK) return rc;
+  return run_combine(ws_o, ws_lse, used, static_cast<long long>(rows), d, o, lse, 0, stream, *st);
+}
+
+extern "C" int attn_combine(const float* o_parts, const float* lse_parts, int G, long long rows,
+                            int d, void* o, float* lse, int o_fp32, attn_stream_t stream) {
+  if (!o_parts || !lse_parts || !o || !lse) return ATTN_ERR_INVALID_ARG;
+  if (G < 1 || G > kMaxSplits || rows < 1) return ATTN_ERR_INVALID_ARG;
+  if (!head_dim_ok(d)) return ATTN_ERR_UNSUPPORTED;
+  if (static_cast<uint64_t>(G) * static_cast<uint64_t>(rows) >= (1ull << 40))
+    return ATTN_ERR_UNSUPPORTED;
+  if ((reinterpret_cast<uintptr_t>(o_parts) | reinterpret_cast<uintptr_t>(o)) & 15u)
+    return ATTN_ERR_MISALIGNED;
+  if ((reinterpret_cast<uintptr_t>(lse_parts) | reinterpret_cast<uintptr_t>(lse)) & 3u)
+    return ATTN_ERR_MISALIGNED;
+  const size_t pr = static_cast<size_t>(G) * static_cast<size_t>(rows);
+  const void* outs[2] = {o, lse};
+  const size_t out_bytes[2] = {static_cast<size_t>(rows) * d * (o_fp32 ? 4 : 2),
+                               static_cast<size_t>(rows) * 4};
+  const void* ins[2] = {o_parts, lse_parts};
+  const size_t in_bytes[2] = {pr * d * 4, pr * 4};
+  if (!outputs_disjoint(outs, out_bytes, 2, ins, in_bytes, 2)) return ATTN_ERR_INVALID_ARG;
+  DeviceState* st = nullptr;
+  const int rc = device_state(&st);
+  if (rc != ATTN_OK) return rc;
+  return run_combine(o_parts, lse_parts, G, rows, d, o, lse, o_fp32 ? 1 : 0, stream, *st);
 }
 
 // Allocation-free entry point (include/attn_b200.h): same kernel, work
@@ -282,26 +541,21 @@ extern "C" int attn_fwd_ex(const void* q, const void* k, const void* v, void* o,
 extern "C" int attn_fwd_noalloc(const void* q, const void* k, const void* v, void* o, float* lse,
                                 int B, int H, int N, int d, int causal, float scale,
                                 attn_stream_t stream) {
-  int rc = attn_check_args(q, k, v, o, lse, B, H, N, d, scale);
+  const Problem p = dense_problem(q, k, v, o, lse, B, H, N, d, causal, scale);
+  int rc = check_dense(p);
   if (rc != ATTN_OK) return rc;
   DeviceState* st = nullptr;
   rc = device_state(&st);  // first call on a device: resolves the scratch address
   if (rc != ATTN_OK) return rc;
   // The queue counter is a 32-bit int that every CTA pushes once past the
   // last item: items + CTAs must stay representable.
-  const int64_t items = static_cast<int64_t>(B) * H * (((N + kBlockM - 1) / kBlockM + 1) / 2);
-  if (items + st->num_sms > 0x7FFFFFFFll) return ATTN_ERR_UNSUPPORTED;
+  if (problem_items(p) + st->num_sms > 0x7FFFFFFFll) return ATTN_ERR_UNSUPPORTED;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (cudaMemsetAsync(st->noalloc_scratch, 0, kNoAllocQueueBytes, s) != cudaSuccess) {
     cudaGetLastError();
     return ATTN_ERR_CUDA;
   }
-  int* qs = st->noalloc_scratch;
-  if (d == 128)
-    return causal ? launch<128, true, kDefaultPolyPairs>(q, k, v, o, lse, B, H, N, scale, s, *st, qs)
-                  : launch<128, false, kDefaultPolyPairs>(q, k, v, o, lse, B, H, N, scale, s, *st, qs);
-  return causal ? launch<64, true, kDefaultPolyPairs>(q, k, v, o, lse, B, H, N, scale, s, *st, qs)
-                : launch<64, false, kDefaultPolyPairs>(q, k, v, o, lse, B, H, N, scale, s, *st, qs);
+  return run_problem(p, kDefaultPolyPairs, stream, st->noalloc_scratch, st);
 }
 
 extern "C" int attn_selftest_wait_timeout(int limit_us, attn_stream_t stream) {
@@ -363,10 +617,11 @@ extern "C" const char* attn_strerror(int status) {
   switch (status) {
     case ATTN_OK: return "ok";
     case ATTN_ERR_INVALID_ARG: return "invalid argument";
-    case ATTN_ERR_UNSUPPORTED: return "unsupported shape (d must be 64 or 128; B*H*N below 2^31)";
+    case ATTN_ERR_UNSUPPORTED: return "unsupported shape (d must be 64, 96 or 128; B*H*N below 2^31)";
     case ATTN_ERR_MISALIGNED: return "misaligned pointer (q, k, v, o need 16 bytes, lse 4)";
     case ATTN_ERR_CUDA: return "CUDA call failed";
     case ATTN_ERR_DEVICE_TIMEOUT: return "device-side wait timed out";
+    case ATTN_ERR_DEVICE_BOUNDS: return "sequence offsets outside the buffers (device-side check)";
     case ATTN_ERR_NO_DEVICE: return "no usable sm_100 device";
     default: return "unknown status";
   }

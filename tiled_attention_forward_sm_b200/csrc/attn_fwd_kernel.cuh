@@ -18,7 +18,8 @@
 //    exponentials can be computed with ordinary multiply-adds.
 //
 // Work item: two 128-row Q tiles (Q0, Q1) of one (batch, head), i.e. 256
-// query rows, against the K/V tiles they can see (128 keys per tile).  The
+// query rows, against the K/V tiles they can see (128 keys per tile), or
+// against one slice of those tiles when the keys are split.  The
 // kernel is persistent: one CTA per SM takes work items from a shared queue
 // (page lecompute.fr/en/kernel-perf/flapping-airplanes-thunderkittens-
 // megakernels, section "Choose between predetermined work and a shared work
@@ -57,6 +58,7 @@ namespace attn_b200 {
 
 // Device status word codes (mirrors attn_status in include/attn_b200.h).
 constexpr int kStatusDeviceTimeout = -5;
+constexpr int kStatusDeviceBounds = -6;
 
 // Bounded waits: a wait that has not completed after this long sets the
 // status word and the CTA's abort flag, and every role then leaves its loop.
@@ -68,12 +70,20 @@ constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s
 #define ATTN_PACKED_SOFTMAX 1
 #endif
 
-// Work distribution: items are claimed from a per-launch counter in global
-// memory (1, a shared work queue: a CTA that finishes early takes the next
-// item) or dealt statically in a snake order (0).
-#ifndef ATTN_DYNAMIC_QUEUE
-#define ATTN_DYNAMIC_QUEUE 1
+// S load: all 128 columns then one wait (0), or two waits with the row
+// max of the first 64 columns computed while the last 64 load (1).
+#ifndef ATTN_SPLIT_SLOAD
+#define ATTN_SPLIT_SLOAD 0
 #endif
+
+// P publication: the first half of P is announced after its store
+// completes (0), or after this many column pairs of the second half have
+// been computed (the store's completion wait overlaps them).
+#ifndef ATTN_DEFER_PSTORE_WAIT
+#define ATTN_DEFER_PSTORE_WAIT 0
+#endif
+static_assert(ATTN_DEFER_PSTORE_WAIT >= 0 && ATTN_DEFER_PSTORE_WAIT <= 32,
+              "the first half of P must be announced inside the second half's loop");
 
 // K/V ring depth for d = 128 (each stage holds one 128 x 128 bf16 tile).
 #ifndef ATTN_KV_STAGES_D128
@@ -81,8 +91,9 @@ constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s
 #endif
 
 // Work items announced by the producer to the MMA and softmax warps through
-// a small ring in shared memory.
+// a small ring in shared memory (kItemWords ints per slot).
 constexpr int kItemSlots = 4;
+constexpr int kItemWords = 16;
 // Readers of each ring slot: the MMA warp and the 8 softmax warps.
 constexpr int kItemReaders = 9;
 
@@ -126,15 +137,36 @@ __device__ __forceinline__ void trace_stamp(int ev, int j) {
 #define ATTN_TRACE(ev, j) ((void)0)
 #endif
 
+// One launch's problem.  Two layouts:
+//  * per-head ("dense"): Q is [B, H, N_q, D], K and V are [B, H_kv, N_k, D],
+//    O is laid out like Q, LSE is [B, H, N_q];
+//  * packed token-major (cu_q != null): Q is [T_q, H, D], K and V are
+//    [T_k, H_kv, D]; sequence b owns query tokens [cu_q[b], cu_q[b+1]) and
+//    key tokens [cu_k[b], cu_k[b+1]); O is laid out like Q, LSE is [H, T_q].
+// Query head h reads K/V head h / (H / H_kv).  Under the causal mask key j
+// of a sequence is visible to its query i iff j <= i + delta, with delta
+// given (dense) or k_len - q_len of the sequence (packed: the last query
+// sees the last key).  A row that sees no key gets O = 0 and LSE = -inf.
+// With n_splits > 1 the K/V tiles of a head are cut into slices of
+// split_tiles tiles; slice s writes its normalised partial O and LSE at
+// row offset s * split_rows, for a later LSE-weighted merge.
 struct KernelArgs {
-  __nv_bfloat16* o;   // [B*H*N, D]
-  float* lse;         // [B*H*N]
-  int N;              // keys/queries per head (any N >= 1)
-  int n_qtiles;       // ceil(N / 128)
-  int n_qpairs;       // ceil(n_qtiles / 2)
+  void* o;            // bf16 O, or fp32 (o_f32) O; rows of D values
+  float* lse;
+  const int* cu_q;    // packed layout: B+1 query token offsets (else null)
+  const int* cu_k;    // packed layout: B+1 key token offsets
+  int H, H_kv, q_per_kv;  // query heads, K/V heads, H / H_kv
+  int N_q, N_k;       // dense: rows per head; packed: the longest sequence
+  int T_q, T_k;       // packed: total query and key tokens
+  int delta;          // dense causal offset
+  int n_qpairs;       // ceil(ceil(N_q / 128) / 2)
+  int n_splits;       // key slices per (head, Q tile pair)
+  int split_tiles;    // K/V tiles per slice
+  long long split_rows;  // rows of one slice of the outputs (0 without slices)
+  int o_f32;          // store O as fp32 instead of bf16
   int BH;             // B * H
-  int n_items;        // BH * n_qpairs work items
-  int win_heads;      // heads per scheduling window (item order, see decode_item)
+  int n_items;        // BH * n_qpairs * n_splits work items (some may be empty)
+  int win_heads;      // heads per scheduling window (item order, see make_item)
   float scale_log2;   // scale * log2(e)
   int* status;        // device status word
   int* queue;         // {next item, CTAs finished}: this launch's queue slot
@@ -142,11 +174,14 @@ struct KernelArgs {
 
 template <int D>
 struct Config {
-  static_assert(D == 64 || D == 128, "head dim");
-  static constexpr int kTileBytes = kBlockM * D * 2;        // one 128 x D bf16 tile
-  static constexpr int kBoxes = D / 64;                      // 64-column TMA boxes per tile
+  static_assert(D == 64 || D == 96 || D == 128, "head dim");
+  // A tile is kBoxes 64-column TMA boxes of 128 rows; at D = 96 the second
+  // box's columns 96..127 lie outside the tensor and arrive as zeros (the
+  // products below never read them: QK stops at K = D, PV's N is D).
+  static constexpr int kBoxes = (D + 63) / 64;
   static constexpr int kBoxBytes = kBlockM * 64 * 2;         // 16 KB
-  static constexpr int kStages = D == 128 ? ATTN_KV_STAGES_D128 : 8;  // K/V ring depth
+  static constexpr int kTileBytes = kBoxes * kBoxBytes;      // one 128 x 64*kBoxes tile
+  static constexpr int kStages = D > 64 ? ATTN_KV_STAGES_D128 : 8;  // K/V ring depth
   static constexpr int kQOff = 0;
   static constexpr int kKVOff = 2 * kTileBytes;
   static constexpr int kBarOff = kKVOff + kStages * kTileBytes;
@@ -154,8 +189,9 @@ struct Config {
   // p_ready[2 tiles][2 halves], o_final[2], drain, item_full[R], item_empty[R]
   static constexpr int kNumBars = 4 + 2 * kStages + 2 + 4 + 2 + 1 + 2 * kItemSlots;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;
-  // misc: tmem base, abort flag, item ring
-  static constexpr int kSmemBytes = kMiscOff + 8 + 4 * kItemSlots + 1024;  // + alignment slack
+  // misc: tmem base, abort flag; then the item ring
+  static constexpr int kRingOff = kMiscOff + 16;
+  static constexpr int kSmemBytes = kRingOff + 4 * kItemWords * kItemSlots + 1024;  // + alignment slack
   static constexpr uint32_t kIdescQK = ptx::idesc_bf16_f32(128, kBlockN, 0, 0);
   static constexpr uint32_t kIdescPV = ptx::idesc_bf16_f32(128, D, 0, 1);
 };
@@ -226,68 +262,123 @@ __device__ __forceinline__ bool wait_warp(const Shared& sh, int* status, uint64_
   }
 }
 
-// Number of K/V tiles Q tile `qt` visits.
-template <bool CAUSAL>
-__device__ __forceinline__ int kv_tiles_for(int qt, int n_qtiles) {
-  if (qt >= n_qtiles) return 0;
-  return CAUSAL ? qt + 1 : n_qtiles;
-}
-
 // ------------------------------------------------------------ work schedule
 struct Item {
-  int bh;     // batch * H + head
-  int qpair;  // Q tiles 2*qpair and 2*qpair + 1
-  int n0;     // K/V tiles Q0 visits (0: no such tile)
-  int n1;     // K/V tiles Q1 visits
+  int qpair;         // Q tiles 2*qpair and 2*qpair + 1 of the sequence
+  int n0, n1;        // K/V tiles Q0 and Q1 visit in this item (0: none)
+  int kt0;           // the item's first K/V tile
+  int q_len, k_len;  // query rows and keys of the sequence
+  int delta;         // causal: key j visible to query i iff j <= i + delta
+  int qz, kz;        // map coordinate of the (batch, head) of Q and of K/V
+  int q_row0, k_row0;  // row coordinate of query 0 and key 0 in the maps
+  int split;         // key slice (offset of the partial outputs)
 };
 
-// Item numbering: heads are taken in windows of win_heads; inside a window
-// the pairs are numbered heaviest first under the causal mask (pair-major
-// over the window's heads).  Items handed out in this order keep the CTAs
-// that run together on a few heads, whose K/V then stays in L2, while the
-// light pairs at the end of each window even out the CTAs' finishing times.
+// K/V tiles that Q tile `qt` of `it` visits inside the slice starting at
+// tile it.kt0 (at most split_tiles of them).
 template <bool CAUSAL>
-__device__ __forceinline__ Item decode_item(int idx, const KernelArgs& a) {
+__device__ __forceinline__ int tiles_for(int qt, const Item& it, int split_tiles) {
+  const long long row_lo = static_cast<long long>(qt) * kBlockM;
+  if (row_lo >= it.q_len) return 0;
+  long long hi = it.k_len;  // keys [0, hi) can be seen by some row of the tile
+  if (CAUSAL) {
+    const long long q_hi = row_lo + kBlockM < it.q_len ? row_lo + kBlockM : it.q_len;
+    if (q_hi + it.delta < hi) hi = q_hi + it.delta;
+  }
+  if (hi <= 0) return 0;
+  const long long n = (hi + kBlockN - 1) / kBlockN - it.kt0;
+  return n <= 0 ? 0 : (n > split_tiles ? split_tiles : static_cast<int>(n));
+}
+
+// Item numbering: items are (head, Q tile pair, key slice) with the slice
+// innermost.  Heads are taken in windows of win_heads; inside a window the
+// pairs are numbered heaviest first under the causal mask (pair-major over
+// the window's heads).  Items handed out in this order keep the CTAs that
+// run together on a few heads, whose K/V then stays in L2, while the light
+// pairs at the end of each window even out the CTAs' finishing times.
+// Returns false for an item with no query rows (a pair past the end of a
+// shorter sequence) or, after raising the bounds status, for a sequence
+// whose offsets do not fit the buffers.
+template <bool CAUSAL>
+__device__ __forceinline__ bool make_item(int idx, const KernelArgs& a, int* status,
+                                          Item& it) {
+  int base = idx, split = 0;
+  if (a.n_splits > 1) {
+    base = idx / a.n_splits;
+    split = idx - base * a.n_splits;
+  }
   const int per_win = a.win_heads * a.n_qpairs;
-  const int w = idx / per_win;
-  const int k = idx - w * per_win;
+  const int w = base / per_win;
+  const int k = base - w * per_win;
   const int h0 = w * a.win_heads;
   const int wh = (a.BH - h0) < a.win_heads ? (a.BH - h0) : a.win_heads;
   const int qp_idx = k / wh;
-  Item it;
-  it.bh = h0 + (k - qp_idx * wh);
+  const int bh = h0 + (k - qp_idx * wh);
+  const int b = bh / a.H, h = bh - b * a.H;
+  const int hk = h / a.q_per_kv;
   it.qpair = CAUSAL ? (a.n_qpairs - 1 - qp_idx) : qp_idx;
-  it.n0 = kv_tiles_for<CAUSAL>(2 * it.qpair, a.n_qtiles);
-  it.n1 = kv_tiles_for<CAUSAL>(2 * it.qpair + 1, a.n_qtiles);
-  return it;
+  if (a.cu_q != nullptr) {
+    const int q0 = a.cu_q[b], q1 = a.cu_q[b + 1], k0 = a.cu_k[b], k1 = a.cu_k[b + 1];
+    if (q0 < 0 || q1 < q0 || q1 > a.T_q || q1 - q0 > a.N_q || k0 < 0 || k1 < k0 ||
+        k1 > a.T_k || k1 - k0 > a.N_k) {
+      atomicCAS(status, 0, kStatusDeviceBounds);
+      return false;
+    }
+    it.q_row0 = q0;
+    it.q_len = q1 - q0;
+    it.k_row0 = k0;
+    it.k_len = k1 - k0;
+    it.qz = h;
+    it.kz = hk;
+    it.delta = it.k_len - it.q_len;
+  } else {
+    it.q_row0 = 0;
+    it.q_len = a.N_q;
+    it.k_row0 = 0;
+    it.k_len = a.N_k;
+    it.qz = bh;
+    it.kz = b * a.H_kv + hk;
+    it.delta = a.delta;
+  }
+  if (2 * it.qpair * kBlockM >= it.q_len) return false;
+  it.split = split;
+  it.kt0 = split * a.split_tiles;
+  it.n0 = tiles_for<CAUSAL>(2 * it.qpair, it, a.split_tiles);
+  it.n1 = tiles_for<CAUSAL>(2 * it.qpair + 1, it, a.split_tiles);
+  return true;
 }
 
-// The producer's r-th item: claimed from the launch's queue counter, or
-// dealt statically (round r gives CTA c item r*G + c, reversed every other
-// round).  Returns an index >= n_items when there is no more work.
-__device__ __forceinline__ int claim_item(int r, const KernelArgs& a) {
-#if ATTN_DYNAMIC_QUEUE
-  (void)r;
-  return atomicAdd(a.queue, 1);
-#else
-  const int G = static_cast<int>(gridDim.x), c = static_cast<int>(blockIdx.x);
-  return r * G + ((r & 1) ? (G - 1 - c) : c);
-#endif
-}
-
-// Producer: announce its r-th item (or the end, idx < 0) in ring slot r % R.
-__device__ __forceinline__ bool post_item(const Shared& sh, const KernelArgs& a, int r, int idx) {
+// Producer: announce its r-th item (or the end, it == nullptr) in ring slot
+// r % R.
+__device__ __forceinline__ bool post_item(const Shared& sh, const KernelArgs& a, int r,
+                                          const Item* it) {
   const int slot = r % kItemSlots;
   const uint32_t ph = static_cast<uint32_t>((r / kItemSlots) & 1);
   if (!wait_one(sh, a.status, &sh.item_empty[slot], ph ^ 1)) return false;
-  sh.item_ring[slot] = idx;
-  ptx::mbar_arrive(&sh.item_full[slot]);  // release: the write is seen by waiters
+  volatile int* w = sh.item_ring + slot * kItemWords;
+  if (it == nullptr) {
+    w[0] = 0;
+  } else {
+    w[0] = 1;
+    w[1] = it->qpair;
+    w[2] = it->n0;
+    w[3] = it->n1;
+    w[4] = it->kt0;
+    w[5] = it->q_len;
+    w[6] = it->k_len;
+    w[7] = it->delta;
+    w[8] = it->qz;
+    w[9] = it->kz;
+    w[10] = it->q_row0;
+    w[11] = it->k_row0;
+    w[12] = it->split;
+  }
+  ptx::mbar_arrive(&sh.item_full[slot]);  // release: the writes are seen by waiters
   return true;
 }
 
 // Reader warp: its r-th item.  Returns false at the end of the work (or on
 // abort, with ok cleared).
-template <bool CAUSAL>
 __device__ __forceinline__ bool read_item(const Shared& sh, const KernelArgs& a, int r, Item& it,
                                           bool& ok) {
   const int slot = r % kItemSlots;
@@ -295,12 +386,25 @@ __device__ __forceinline__ bool read_item(const Shared& sh, const KernelArgs& a,
     ok = false;
     return false;
   }
-  const int idx = sh.item_ring[slot];
+  const volatile int* w = sh.item_ring + slot * kItemWords;
+  const bool valid = w[0] != 0;
+  if (valid) {
+    it.qpair = w[1];
+    it.n0 = w[2];
+    it.n1 = w[3];
+    it.kt0 = w[4];
+    it.q_len = w[5];
+    it.k_len = w[6];
+    it.delta = w[7];
+    it.qz = w[8];
+    it.kz = w[9];
+    it.q_row0 = w[10];
+    it.k_row0 = w[11];
+    it.split = w[12];
+  }
   __syncwarp();
   if (ptx::lane_id() == 0) ptx::mbar_arrive(&sh.item_empty[slot]);
-  if (idx < 0) return false;
-  it = decode_item<CAUSAL>(idx, a);
-  return true;
+  return valid;
 }
 
 // ----------------------------------------------------------------- producer
@@ -311,17 +415,38 @@ __device__ void producer_role(const Shared& sh, const KernelArgs& a, uint8_t* sm
   using C = Config<D>;
   const uint64_t pol_q = ptx::policy_evict_first();
   const uint64_t pol_kv = ptx::policy_evict_last();
+  const bool packed = a.cu_q != nullptr;
+  // Tile load: per-head maps are indexed (column, row, head), packed maps
+  // (column, head, token).
+  auto load_tile = [&](const CUtensorMap* m, uint64_t* bar, uint8_t* dst, int row, int z,
+                       uint64_t pol) {
+    for (int b = 0; b < C::kBoxes; ++b) {
+      if (packed)
+        ptx::tma_load_3d(m, bar, dst + b * C::kBoxBytes, 64 * b, z, row, pol);
+      else
+        ptx::tma_load_3d(m, bar, dst + b * C::kBoxBytes, 64 * b, row, z, pol);
+    }
+  };
   int q_loads[2] = {0, 0};  // loads into Q buffer s so far
   int issued = 0;           // K/V tiles issued into the ring so far
   bool ok = true;
-  int idx = claim_item(0, a);
+  // The next non-empty item from the launch's queue (one atomic per claim;
+  // an index >= n_items means the work is done).
+  Item it;
+  auto claim = [&]() -> bool {
+    for (;;) {
+      const int idx = atomicAdd(a.queue, 1);
+      if (idx >= a.n_items) return false;
+      if (make_item<CAUSAL>(idx, a, a.status, it)) return true;
+    }
+  };
+  bool have = claim();
   for (int r = 0; ok; ++r) {
-    if (idx >= a.n_items) {
-      post_item(sh, a, r, -1);
+    if (!have) {
+      post_item(sh, a, r, nullptr);
       break;
     }
-    if (!post_item(sh, a, r, idx)) break;
-    const Item it = decode_item<CAUSAL>(idx, a);
+    if (!post_item(sh, a, r, &it)) break;
     const int n = it.n0 > it.n1 ? it.n0 : it.n1;
     // Q_s, once the previous item's last S_s no longer needs the buffer.
     for (int s = 0; s < 2 && ok; ++s) {
@@ -332,9 +457,8 @@ __device__ void producer_role(const Shared& sh, const KernelArgs& a, uint8_t* sm
         break;
       }
       ptx::mbar_arrive_expect_tx(&sh.q_full[s], C::kTileBytes);
-      for (int b = 0; b < C::kBoxes; ++b)
-        ptx::tma_load_3d(tq, &sh.q_full[s], smem + C::kQOff + s * C::kTileBytes + b * C::kBoxBytes,
-                         64 * b, (2 * it.qpair + s) * kBlockM, it.bh, pol_q);
+      load_tile(tq, &sh.q_full[s], smem + C::kQOff + s * C::kTileBytes,
+                it.q_row0 + (2 * it.qpair + s) * kBlockM, it.qz, pol_q);
       ++q_loads[s];
     }
     for (int j = 0; j < n && ok; ++j) {
@@ -345,17 +469,15 @@ __device__ void producer_role(const Shared& sh, const KernelArgs& a, uint8_t* sm
         uint8_t* dst = smem + C::kKVOff + st * C::kTileBytes;
         ATTN_TRACE(which == 0 ? kTrProdK : kTrProdV, r == 0 ? j : -1);
         ptx::mbar_arrive_expect_tx(&sh.kv_full[st], C::kTileBytes);
-        const CUtensorMap* m = which == 0 ? tk : tv;
-        for (int b = 0; b < C::kBoxes; ++b)
-          ptx::tma_load_3d(m, &sh.kv_full[st], dst + b * C::kBoxBytes, 64 * b, j * kBlockN,
-                           it.bh, pol_kv);
+        load_tile(which == 0 ? tk : tv, &sh.kv_full[st], dst,
+                  it.k_row0 + (it.kt0 + j) * kBlockN, it.kz, pol_kv);
         ++issued;
       }
     }
     // Claim the next item only now: the ring holds the last K/V steps of
     // this one, so the claim's latency overlaps them, and a CTA never holds
     // an item it cannot start soon (which would lengthen the tail).
-    idx = claim_item(r + 1, a);
+    if (ok) have = claim();
   }
   // Drain: every load issued must land before the CTA may exit.
   for (int s = 0; s < 2; ++s)
@@ -438,9 +560,10 @@ __device__ void mma_role(const Shared& sh, const KernelArgs& a, uint8_t* smem, u
 
   Item it;
   bool ok = true;
-  for (int r = 0; read_item<CAUSAL>(sh, a, r, it, ok); ++r) {
+  for (int r = 0; read_item(sh, a, r, it, ok); ++r) {
     const int n0 = it.n0, n1 = it.n1;
     const int n = n0 > n1 ? n0 : n1;
+    if (n == 0) continue;  // rows that see no key: the softmax groups write them
     for (int s = 0; s < 2; ++s) {
       if ((s == 0 ? n0 : n1) == 0) continue;
       if (!wait_warp(sh, a.status, &sh.q_full[s], static_cast<uint32_t>(q_uses[s] & 1)))
@@ -557,7 +680,54 @@ __device__ __forceinline__ bool softmax_step(const Shared& sh, const KernelArgs&
   ptx::tc_fence_after_sync();
   if (r == 0) ATTN_TRACE(s == 0 ? kTrSm0Full : kTrSm1Full, tj);
 
+  // Keys c >= key_limit of this tile are invisible to row r: under the
+  // causal mask on the tiles the diagonal crosses, and on the last tile of a
+  // key sequence whose length is not a multiple of 128.  Elsewhere key_limit
+  // is at least 128 and nothing is masked.
+  const bool masked = __any_sync(0xffffffffu, key_limit < 128);
   uint32_t sr[128];
+  float x[128];
+  // Row max: eight independent chains of three-input maxima.
+  float mx[8];
+#if ATTN_SPLIT_SLOAD
+  ptx::tmem_ld32(t_s + 0, sr + 0);
+  ptx::tmem_ld32(t_s + 32, sr + 32);
+  ptx::tmem_ld_wait_tie(sr + 0);
+  ptx::reg_tie32(sr + 32);
+  ptx::tmem_ld32(t_s + 64, sr + 64);
+  ptx::tmem_ld32(t_s + 96, sr + 96);
+#pragma unroll
+  for (int c = 0; c < 64; ++c) x[c] = __uint_as_float(sr[c]);
+  if (masked) {
+#pragma unroll
+    for (int c = 0; c < 64; ++c)
+      if (c >= key_limit) x[c] = -INFINITY;
+  }
+#pragma unroll
+  for (int k = 0; k < 8; ++k) mx[k] = x[k];
+#pragma unroll
+  for (int c = 8; c + 16 <= 64; c += 16) {
+#pragma unroll
+    for (int k = 0; k < 8; ++k) mx[k] = ptx::max3(mx[k], x[c + 2 * k], x[c + 2 * k + 1]);
+  }
+#pragma unroll
+  for (int k = 0; k < 4; ++k) mx[k] = ptx::max3(mx[k], x[56 + 2 * k], x[57 + 2 * k]);
+  ptx::tmem_ld_wait_tie(sr + 64);
+  ptx::reg_tie32(sr + 96);
+#pragma unroll
+  for (int c = 64; c < 128; ++c) x[c] = __uint_as_float(sr[c]);
+  if (r == 0) ATTN_TRACE(s == 0 ? kTrSm0Ld : kTrSm1Ld, tj);
+  if (masked) {
+#pragma unroll
+    for (int c = 64; c < 128; ++c)
+      if (c >= key_limit) x[c] = -INFINITY;
+  }
+#pragma unroll
+  for (int c = 64; c < 128; c += 16) {
+#pragma unroll
+    for (int k = 0; k < 8; ++k) mx[k] = ptx::max3(mx[k], x[c + 2 * k], x[c + 2 * k + 1]);
+  }
+#else
   ptx::tmem_ld32(t_s + 0, sr + 0);
   ptx::tmem_ld32(t_s + 32, sr + 32);
   ptx::tmem_ld32(t_s + 64, sr + 64);
@@ -566,24 +736,14 @@ __device__ __forceinline__ bool softmax_step(const Shared& sh, const KernelArgs&
   ptx::reg_tie32(sr + 32);
   ptx::reg_tie32(sr + 64);
   ptx::reg_tie32(sr + 96);
-
-  float x[128];
 #pragma unroll
   for (int c = 0; c < 128; ++c) x[c] = __uint_as_float(sr[c]);
   if (r == 0) ATTN_TRACE(s == 0 ? kTrSm0Ld : kTrSm1Ld, tj);
-
-  // Keys c >= key_limit of this tile are invisible to row r: under the
-  // causal mask on the diagonal tile (key tile == query tile) key_limit is
-  // r + 1; on the last tile of a length that is not a multiple of 128 it is
-  // the number of keys that exist.  Elsewhere it is 128 and nothing is masked.
-  if (__any_sync(0xffffffffu, key_limit < 128)) {
+  if (masked) {
 #pragma unroll
     for (int c = 0; c < 128; ++c)
       if (c >= key_limit) x[c] = -INFINITY;
   }
-
-  // Row max: eight independent chains of three-input maxima.
-  float mx[8];
 #pragma unroll
   for (int k = 0; k < 8; ++k) mx[k] = x[k];
 #pragma unroll
@@ -593,6 +753,7 @@ __device__ __forceinline__ bool softmax_step(const Shared& sh, const KernelArgs&
   }
 #pragma unroll
   for (int k = 0; k < 4; ++k) mx[k] = ptx::max3(mx[k], x[120 + 2 * k], x[121 + 2 * k]);
+#endif
   const float tile_max =
       ptx::max3(ptx::max3(mx[0], mx[1], mx[2]), ptx::max3(mx[3], mx[4], mx[5]), fmaxf(mx[6], mx[7])) *
       sl2;
@@ -621,7 +782,10 @@ __device__ __forceinline__ bool softmax_step(const Shared& sh, const KernelArgs&
     }
   }
   const uint64_t sl2x2 = ptx::f2pack(sl2, sl2);
-  const uint64_t negm2 = ptx::f2pack(-m, -m);
+  // A row that has seen no visible key yet keeps m = -inf; its weights are
+  // then computed against 0 (all masked scores give 0, never NaN).
+  const float negm = m == -INFINITY ? 0.f : -m;
+  const uint64_t negm2 = ptx::f2pack(negm, negm);
   (void)sl2x2;
   (void)negm2;
 
@@ -654,7 +818,7 @@ __device__ __forceinline__ bool softmax_step(const Shared& sh, const KernelArgs&
       float p0, p1;
       ptx::f2unpack(p2, p0, p1);
 #else
-      const float y0 = fmaf(x[c], sl2, -m), y1 = fmaf(x[c + 1], sl2, -m);
+      const float y0 = fmaf(x[c], sl2, negm), y1 = fmaf(x[c + 1], sl2, negm);
       float p0, p1;
       if ((q & 3) < kPolyPairs) {
         p0 = exp2_poly1(y0);
@@ -666,15 +830,25 @@ __device__ __forceinline__ bool softmax_step(const Shared& sh, const KernelArgs&
       if (q & 1) { ls2 += p0; ls3 += p1; } else { ls0 += p0; ls1 += p1; }
 #endif
       pk[q] = ptx::pack_bf16x2(p0, p1);
+      if (ATTN_DEFER_PSTORE_WAIT > 0 && half == 1 && q == ATTN_DEFER_PSTORE_WAIT - 1) {
+        // announce the first half now that its store has had time to land
+        ptx::tmem_st_wait();
+        ptx::tc_fence_before_sync();
+        __syncwarp();
+        if (lane == 0) ptx::mbar_arrive(&sh.p_ready[2 * s]);
+        if (r == 0) ATTN_TRACE(s == 0 ? kTrSm0Pa : kTrSm1Pa, tj);
+      }
     }
     // P_s keys [64*half, 64*half+64) as bf16 pairs over TMEM columns
-    // [32*half, 32*half+32) of the S_s region; publish this half at once.
+    // [32*half, 32*half+32) of the S_s region.
     ptx::tmem_st32(t_s + 32 * half, pk);
-    ptx::tmem_st_wait();
-    ptx::tc_fence_before_sync();
-    __syncwarp();
-    if (lane == 0) ptx::mbar_arrive(&sh.p_ready[2 * s + half]);
-    if (r == 0) ATTN_TRACE(s == 0 ? (half ? kTrSm0Pb : kTrSm0Pa) : (half ? kTrSm1Pb : kTrSm1Pa), tj);
+    if (ATTN_DEFER_PSTORE_WAIT == 0 || half == 1) {
+      ptx::tmem_st_wait();
+      ptx::tc_fence_before_sync();
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive(&sh.p_ready[2 * s + half]);
+      if (r == 0) ATTN_TRACE(s == 0 ? (half ? kTrSm0Pb : kTrSm0Pa) : (half ? kTrSm1Pb : kTrSm1Pa), tj);
+    }
   }
 #if ATTN_PACKED_SOFTMAX
   float la0, la1, lb0, lb1;
@@ -702,16 +876,22 @@ __device__ void softmax_role(const Shared& sh, const KernelArgs& a, uint32_t tme
 
   Item it;
   bool ok = true;
-  for (int rr = 0; read_item<CAUSAL>(sh, a, rr, it, ok); ++rr) {
-    const int n_s = s == 0 ? it.n0 : it.n1;
-    if (n_s == 0) continue;
+  for (int rr = 0; read_item(sh, a, rr, it, ok); ++rr) {
     const int qt = 2 * it.qpair + s;
+    const int row = qt * kBlockM + r;  // query row in the sequence
+    if (qt * kBlockM >= it.q_len) continue;  // the item has no such tile
+    const int n_s = s == 0 ? it.n0 : it.n1;
     float m = -INFINITY;  // running max of scale*log2(e)*score (log2 units)
     float l = 0.f;        // running sum of weights, relative to 2^m
-    const int keys_in_last = a.N - (a.n_qtiles - 1) * kBlockN;  // 1..128
     for (int j = 0; j < n_s; ++j) {
-      int key_limit = (j == a.n_qtiles - 1) ? keys_in_last : kBlockN;
-      if (CAUSAL && j == qt) key_limit = r + 1 < key_limit ? r + 1 : key_limit;
+      // Keys of tile kt0 + j visible to this row: those that exist and,
+      // under the causal mask, those at or before row + delta.
+      const int key0 = (it.kt0 + j) * kBlockN;
+      int key_limit = it.k_len - key0;
+      if (CAUSAL) {
+        const long long lim = static_cast<long long>(row) + it.delta + 1 - key0;
+        if (lim < key_limit) key_limit = lim < -1 ? -1 : static_cast<int>(lim);
+      }
       if (!softmax_step<D, CAUSAL, kPolyPairs>(sh, a, s, t_s, t_o, r, lane, key_limit, j == 0,
                                                static_cast<uint32_t>(s_count & 1),
                                                rr == 0 ? j : -1, m, l))
@@ -719,36 +899,62 @@ __device__ void softmax_role(const Shared& sh, const KernelArgs& a, uint32_t tme
       ++s_count;
     }
 
-    // Epilogue: O_s / l -> bf16 rows; LSE = (m + log2 l) * ln 2.  The next
+    // Epilogue: O_s / l -> rows of O; LSE = (m + log2 l) * ln 2.  The next
     // item's first PV_s (which overwrites O_s) is only issued after this
     // thread publishes that item's P, i.e. after these loads completed.
-    if (!wait_warp(sh, a.status, &sh.o_final[s], static_cast<uint32_t>(o_count & 1))) return;
-    ++o_count;
-    ptx::tc_fence_after_sync();
-    const float inv_l = 1.f / l;
-    // Rows past N (last tile of a ragged length) are computed on zero
-    // queries and not stored.
-    const bool row_ok = qt * kBlockM + r < a.N;
-    const size_t row_g = static_cast<size_t>(it.bh) * a.N + static_cast<size_t>(qt) * kBlockM + r;
-    __nv_bfloat16* orow = a.o + row_g * D;
+    // Rows past the end of the sequence (last tile of a ragged length) are
+    // computed on whatever the tile holds and not stored; a row that saw no
+    // key (m = -inf) stores O = 0 and LSE = -inf.
+    if (n_s > 0) {
+      if (!wait_warp(sh, a.status, &sh.o_final[s], static_cast<uint32_t>(o_count & 1))) return;
+      ++o_count;
+      ptx::tc_fence_after_sync();
+    }
+    const bool row_ok = row < it.q_len;
+    const bool empty = m == -INFINITY;
+    const float inv_l = empty ? 0.f : 1.f / l;
+    size_t o_row, l_row;
+    if (a.cu_q != nullptr) {
+      o_row = (static_cast<size_t>(it.q_row0) + row) * a.H + it.qz;
+      l_row = static_cast<size_t>(it.qz) * a.T_q + it.q_row0 + row;
+    } else {
+      o_row = static_cast<size_t>(it.qz) * a.N_q + row;
+      l_row = o_row;
+    }
+    o_row += static_cast<size_t>(it.split) * a.split_rows;
+    l_row += static_cast<size_t>(it.split) * a.split_rows;
 #pragma unroll 1
     for (int c0 = 0; c0 < D; c0 += 32) {
       uint32_t ov[32];
-      ptx::tmem_ld32(t_o + c0, ov);
-      ptx::tmem_ld_wait_tie(ov);
-      uint32_t pk[16];
+      if (n_s > 0) {
+        ptx::tmem_ld32(t_o + c0, ov);
+        ptx::tmem_ld_wait_tie(ov);
 #pragma unroll
-      for (int c = 0; c < 16; ++c)
-        pk[c] = ptx::pack_bf16x2(__uint_as_float(ov[2 * c]) * inv_l,
-                                 __uint_as_float(ov[2 * c + 1]) * inv_l);
-      if (row_ok) {
-        uint4* dst = reinterpret_cast<uint4*>(orow + c0);
+        for (int c = 0; c < 32; ++c)
+          ov[c] = __float_as_uint(empty ? 0.f : __uint_as_float(ov[c]) * inv_l);
+      } else {
+#pragma unroll
+        for (int c = 0; c < 32; ++c) ov[c] = 0u;
+      }
+      if (!row_ok) continue;
+      if (a.o_f32) {
+        uint4* dst = reinterpret_cast<uint4*>(static_cast<float*>(a.o) + o_row * D + c0);
+#pragma unroll
+        for (int v = 0; v < 8; ++v)
+          dst[v] = make_uint4(ov[4 * v], ov[4 * v + 1], ov[4 * v + 2], ov[4 * v + 3]);
+      } else {
+        uint32_t pk[16];
+#pragma unroll
+        for (int c = 0; c < 16; ++c)
+          pk[c] = ptx::pack_bf16x2(__uint_as_float(ov[2 * c]), __uint_as_float(ov[2 * c + 1]));
+        uint4* dst =
+            reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.o) + o_row * D + c0);
 #pragma unroll
         for (int v = 0; v < 4; ++v)
           dst[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
       }
     }
-    if (row_ok) a.lse[row_g] = (m + log2f(l)) * 0.69314718055994531f;
+    if (row_ok) a.lse[l_row] = empty ? -INFINITY : (m + log2f(l)) * 0.69314718055994531f;
   }
 }
 
@@ -777,7 +983,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   sh.item_empty = sh.item_full + kItemSlots;
   sh.tmem_base = reinterpret_cast<uint32_t*>(smem + C::kMiscOff);
   sh.abort_flag = reinterpret_cast<volatile int*>(smem + C::kMiscOff + 4);
-  sh.item_ring = reinterpret_cast<volatile int*>(smem + C::kMiscOff + 8);
+  sh.item_ring = reinterpret_cast<volatile int*>(smem + C::kRingOff);
 
   const int warp = threadIdx.x / 32;
   if (threadIdx.x == 0) {
@@ -833,7 +1039,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   if (threadIdx.x == 0) {
     ATTN_TRACE(kTrEnd, 0);
-#if ATTN_DYNAMIC_QUEUE
     // The last CTA to finish resets this launch's queue slot for its next
     // user (every CTA's claims precede its arrival here).
     __threadfence();
@@ -841,7 +1046,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       atomicExch(args.queue, 0);
       atomicExch(args.queue + 1, 0);
     }
-#endif
   }
   if (warp == 9) {
     ptx::tc_fence_after_sync();
