@@ -70,21 +70,6 @@ constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s
 #define ATTN_PACKED_SOFTMAX 1
 #endif
 
-// S load: all 128 columns then one wait (0), or two waits with the row
-// max of the first 64 columns computed while the last 64 load (1).
-#ifndef ATTN_SPLIT_SLOAD
-#define ATTN_SPLIT_SLOAD 0
-#endif
-
-// P publication: the first half of P is announced after its store
-// completes (0), or after this many column pairs of the second half have
-// been computed (the store's completion wait overlaps them).
-#ifndef ATTN_DEFER_PSTORE_WAIT
-#define ATTN_DEFER_PSTORE_WAIT 0
-#endif
-static_assert(ATTN_DEFER_PSTORE_WAIT >= 0 && ATTN_DEFER_PSTORE_WAIT <= 32,
-              "the first half of P must be announced inside the second half's loop");
-
 // K/V ring depth for d = 128 (each stage holds one 128 x 128 bf16 tile).
 #ifndef ATTN_KV_STAGES_D128
 #define ATTN_KV_STAGES_D128 4
@@ -689,45 +674,6 @@ __device__ __forceinline__ bool softmax_step(const Shared& sh, const KernelArgs&
   float x[128];
   // Row max: eight independent chains of three-input maxima.
   float mx[8];
-#if ATTN_SPLIT_SLOAD
-  ptx::tmem_ld32(t_s + 0, sr + 0);
-  ptx::tmem_ld32(t_s + 32, sr + 32);
-  ptx::tmem_ld_wait_tie(sr + 0);
-  ptx::reg_tie32(sr + 32);
-  ptx::tmem_ld32(t_s + 64, sr + 64);
-  ptx::tmem_ld32(t_s + 96, sr + 96);
-#pragma unroll
-  for (int c = 0; c < 64; ++c) x[c] = __uint_as_float(sr[c]);
-  if (masked) {
-#pragma unroll
-    for (int c = 0; c < 64; ++c)
-      if (c >= key_limit) x[c] = -INFINITY;
-  }
-#pragma unroll
-  for (int k = 0; k < 8; ++k) mx[k] = x[k];
-#pragma unroll
-  for (int c = 8; c + 16 <= 64; c += 16) {
-#pragma unroll
-    for (int k = 0; k < 8; ++k) mx[k] = ptx::max3(mx[k], x[c + 2 * k], x[c + 2 * k + 1]);
-  }
-#pragma unroll
-  for (int k = 0; k < 4; ++k) mx[k] = ptx::max3(mx[k], x[56 + 2 * k], x[57 + 2 * k]);
-  ptx::tmem_ld_wait_tie(sr + 64);
-  ptx::reg_tie32(sr + 96);
-#pragma unroll
-  for (int c = 64; c < 128; ++c) x[c] = __uint_as_float(sr[c]);
-  if (r == 0) ATTN_TRACE(s == 0 ? kTrSm0Ld : kTrSm1Ld, tj);
-  if (masked) {
-#pragma unroll
-    for (int c = 64; c < 128; ++c)
-      if (c >= key_limit) x[c] = -INFINITY;
-  }
-#pragma unroll
-  for (int c = 64; c < 128; c += 16) {
-#pragma unroll
-    for (int k = 0; k < 8; ++k) mx[k] = ptx::max3(mx[k], x[c + 2 * k], x[c + 2 * k + 1]);
-  }
-#else
   ptx::tmem_ld32(t_s + 0, sr + 0);
   ptx::tmem_ld32(t_s + 32, sr + 32);
   ptx::tmem_ld32(t_s + 64, sr + 64);
@@ -753,7 +699,6 @@ __device__ __forceinline__ bool softmax_step(const Shared& sh, const KernelArgs&
   }
 #pragma unroll
   for (int k = 0; k < 4; ++k) mx[k] = ptx::max3(mx[k], x[120 + 2 * k], x[121 + 2 * k]);
-#endif
   const float tile_max =
       ptx::max3(ptx::max3(mx[0], mx[1], mx[2]), ptx::max3(mx[3], mx[4], mx[5]), fmaxf(mx[6], mx[7])) *
       sl2;
@@ -830,25 +775,15 @@ __device__ __forceinline__ bool softmax_step(const Shared& sh, const KernelArgs&
       if (q & 1) { ls2 += p0; ls3 += p1; } else { ls0 += p0; ls1 += p1; }
 #endif
       pk[q] = ptx::pack_bf16x2(p0, p1);
-      if (ATTN_DEFER_PSTORE_WAIT > 0 && half == 1 && q == ATTN_DEFER_PSTORE_WAIT - 1) {
-        // announce the first half now that its store has had time to land
-        ptx::tmem_st_wait();
-        ptx::tc_fence_before_sync();
-        __syncwarp();
-        if (lane == 0) ptx::mbar_arrive(&sh.p_ready[2 * s]);
-        if (r == 0) ATTN_TRACE(s == 0 ? kTrSm0Pa : kTrSm1Pa, tj);
-      }
     }
     // P_s keys [64*half, 64*half+64) as bf16 pairs over TMEM columns
-    // [32*half, 32*half+32) of the S_s region.
+    // [32*half, 32*half+32) of the S_s region; publish this half at once.
     ptx::tmem_st32(t_s + 32 * half, pk);
-    if (ATTN_DEFER_PSTORE_WAIT == 0 || half == 1) {
-      ptx::tmem_st_wait();
-      ptx::tc_fence_before_sync();
-      __syncwarp();
-      if (lane == 0) ptx::mbar_arrive(&sh.p_ready[2 * s + half]);
-      if (r == 0) ATTN_TRACE(s == 0 ? (half ? kTrSm0Pb : kTrSm0Pa) : (half ? kTrSm1Pb : kTrSm1Pa), tj);
-    }
+    ptx::tmem_st_wait();
+    ptx::tc_fence_before_sync();
+    __syncwarp();
+    if (lane == 0) ptx::mbar_arrive(&sh.p_ready[2 * s + half]);
+    if (r == 0) ATTN_TRACE(s == 0 ? (half ? kTrSm0Pb : kTrSm0Pa) : (half ? kTrSm1Pb : kTrSm1Pa), tj);
   }
 #if ATTN_PACKED_SOFTMAX
   float la0, la1, lb0, lb1;
