@@ -12,6 +12,12 @@ scaling); the time is the max over ranks.
 
 ``--impl reference`` times the CPU oracle (fp64 plain definition) on the
 host cores instead, on bounded row samples of the same workload.
+
+``--workload`` also takes the general problems of ``inputs.GENERAL_WORKLOADS``
+(a query block against a key/value cache, split keys, a packed
+variable-length batch); their line reports the same metric from the exact
+number of visible (query, key) pairs, with the roofline bound chosen by
+arithmetic intensity.
 """
 from __future__ import annotations
 
@@ -31,8 +37,9 @@ import torch
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-from tiled_attention_forward_sm_b200.inputs import (BENCH_WORKLOAD, WORKLOADS,  # noqa: E402
-                                                    bf16_bits, make_workload_inputs)
+from tiled_attention_forward_sm_b200.inputs import (BENCH_WORKLOAD,  # noqa: E402
+                                                    GENERAL_WORKLOADS, WORKLOADS, bf16_bits,
+                                                    make_general_inputs, make_workload_inputs)
 
 METRIC = "attention fwd TFLOPS (bf16, d=128) and % of B200 dense BF16 peak, 1 GPU"
 UNIT = "TFLOPS"
@@ -296,6 +303,126 @@ def run_b200(args, w):
     return line
 
 
+# ------------------------------------------- general entry points (GPU) ---
+def visible_pairs(w) -> int:
+    """(query, key) pairs the mask lets through, summed over heads: the
+    queries are the last positions of their key sequence under the mask."""
+    def per_seq(nq: int, nk: int) -> int:
+        if not w.causal:
+            return nq * nk
+        delta = nk - nq
+        i = np.arange(nq, dtype=np.int64)
+        return int(np.clip(i + delta + 1, 0, nk).sum())
+    if w.kind == "varlen":
+        return w.H * sum(per_seq(a, b) for a, b in zip(w.lens_q, w.lens_k))
+    return w.B * w.H * per_seq(w.N_q, w.N_k)
+
+
+def run_general(args, w):
+    import ctypes
+    import tiled_attention_forward_sm_b200 as tab
+    world, rank, local = dist_env()
+    if world > 1:
+        raise SystemExit("general workloads run on one GPU")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    q_h, k_h, v_h = make_general_inputs(w)
+    q, k, v = (t.to(dev) for t in (q_h, k_h, v_h))
+    stream = torch.cuda.current_stream(dev)
+    lib = tab.library()
+    sh = stream.cuda_stream
+    launches = 1
+    if w.kind == "varlen":
+        lens_q = np.array(w.lens_q, dtype=np.int32)
+        lens_k = np.array(w.lens_k, dtype=np.int32)
+        cu_q = torch.from_numpy(np.concatenate([[0], np.cumsum(lens_q)]).astype(np.int32)).to(dev)
+        cu_k = torch.from_numpy(np.concatenate([[0], np.cumsum(lens_k)]).astype(np.int32)).to(dev)
+        o = torch.empty_like(q)
+        lse = torch.empty((w.H, q.shape[0]), dtype=torch.float32, device=dev)
+
+        def step():
+            rc = lib.attn_fwd_varlen(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
+                                     lse.data_ptr(), cu_q.data_ptr(), cu_k.data_ptr(), w.B, w.H,
+                                     w.H_kv, w.N_q, w.N_k, int(q.shape[0]), int(k.shape[0]),
+                                     w.d, int(w.causal), ctypes.c_float(w.scale), sh)
+            assert rc == 0, rc
+    elif w.kind == "chunk":
+        o = torch.empty_like(q)
+        lse = torch.empty((w.B, w.H, w.N_q), dtype=torch.float32, device=dev)
+
+        def step():
+            rc = lib.attn_fwd_chunk(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
+                                    lse.data_ptr(), w.B, w.H, w.H_kv, w.N_q, w.N_k, w.d,
+                                    int(w.causal), w.N_k - w.N_q, ctypes.c_float(w.scale), 0, sh)
+            assert rc == 0, rc
+    else:
+        slices = tab.splitkv_slices(w.N_k, w.n_splits)
+        o = torch.empty_like(q)
+        lse = torch.empty((w.B, w.H, w.N_q), dtype=torch.float32, device=dev)
+        rows = w.B * w.H * w.N_q
+        ws_o = torch.empty((max(slices, 1), rows, w.d), dtype=torch.float32, device=dev)
+        ws_l = torch.empty((max(slices, 1), rows), dtype=torch.float32, device=dev)
+        launches = 2 if slices > 1 else 1
+
+        def step():
+            rc = lib.attn_fwd_splitkv(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
+                                      lse.data_ptr(), w.B, w.H, w.H_kv, w.N_q, w.N_k, w.d,
+                                      int(w.causal), w.N_k - w.N_q, ctypes.c_float(w.scale),
+                                      w.n_splits, ws_o.data_ptr(), ws_l.data_ptr(), sh)
+            assert rc == 0, rc
+
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES", "")
+    smi_id = vis.split(",")[local].strip() if vis and len(vis.split(",")) > local else str(local)
+    sampler = ClockSampler(smi_id)
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    sampler.start()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    clocks = sampler.stop()
+    status = tab.last_device_error(stream)
+    if status != 0:
+        raise SystemExit(f"device status {status}: {tab.strerror(status)}")
+    ms_step = e0.elapsed_time(e1) / args.steps
+    flops = 4.0 * w.d * visible_pairs(w)
+    bytes_alg = 2 * (q.numel() + k.numel() + v.numel() + o.numel()) + 4 * lse.numel()
+    peaks, peak_kind = load_peaks()
+    tflops = flops / (ms_step * 1e-3) / 1e12
+    gbs = bytes_alg / (ms_step * 1e-3) / 1e9
+    ridge = float(peaks["bf16_tflops"]) * 1e12 / (float(peaks["hbm_gbs"]) * 1e9)
+    if flops / bytes_alg >= ridge:
+        roof = {"bound": "tensor", "achieved": round(tflops, 2), "peak": float(peaks["bf16_tflops"]),
+                "unit": "TFLOP/s", "frac": round(tflops / float(peaks["bf16_tflops"]), 4)}
+    else:
+        roof = {"bound": "hbm", "achieved": round(gbs, 1), "peak": float(peaks["hbm_gbs"]),
+                "unit": "GB/s", "frac": round(gbs / float(peaks["hbm_gbs"]), 4)}
+    roof.update({"traffic": None, "algorithmic_bytes": bytes_alg,
+                 "arithmetic_intensity": round(flops / bytes_alg, 1),
+                 "peak_source": f"{peak_kind} (MEASURED_PEAKS.json)"})
+    cfg = {k_: getattr(w, k_) for k_ in ("name", "kind", "B", "H", "H_kv", "N_q", "N_k", "d",
+                                          "causal", "n_splits")}
+    cfg["workload"] = cfg.pop("name")
+    if w.kind == "varlen":
+        cfg["lens"] = list(w.lens_q)
+    cfg.update({"flops_per_step": flops, "l2": "inputs larger than L2; no flush"
+                if bytes_alg > 126e6 else "inputs fit in L2 (126 MB); no flush"})
+    return {
+        "metric": METRIC, "value": round(tflops, 2), "unit": UNIT, "n_gpus": 1,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded N(0,1) bf16 Q/K/V, see inputs.py)", "config": cfg,
+        "roofline": roof,
+        "e2e": None, "gpu_launches": launches * args.steps, "clocks": clocks,
+        "kernel_sha": kernel_sha(),
+    }
+
+
 # ------------------------------------------------------- reference arm -----
 def run_reference(args, w):
     world, rank, _ = dist_env()
@@ -346,15 +473,21 @@ def main():
     ap.add_argument("--steps", type=int, default=1000)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["b200", "reference"], default="b200")
-    ap.add_argument("--workload", default=BENCH_WORKLOAD, choices=sorted(WORKLOADS))
+    ap.add_argument("--workload", default=BENCH_WORKLOAD,
+                    choices=sorted(WORKLOADS) + sorted(GENERAL_WORKLOADS))
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
-    w = WORKLOADS[args.workload]
-    line = run_reference(args, w) if args.impl == "reference" else run_b200(args, w)
+    if args.workload in GENERAL_WORKLOADS:
+        if args.impl == "reference":
+            ap.error("--impl reference times the square workloads only")
+        line = run_general(args, GENERAL_WORKLOADS[args.workload])
+    else:
+        w = WORKLOADS[args.workload]
+        line = run_reference(args, w) if args.impl == "reference" else run_b200(args, w)
     if line is not None:
         print(json.dumps(line), flush=True)
 

@@ -179,3 +179,49 @@ def test_chunks_over_key_slices_combine_to_the_whole(oracle_mod):
     o_ref, l_ref = oracle_mod.attn_ref(bf16_bits(q), bf16_bits(k), bf16_bits(v), True,
                                        1 / math.sqrt(d))
     check(o.float().cpu().numpy(), lse.cpu().numpy(), o_ref, l_ref, "chunks + combine")
+
+
+# ------------------------------------------ measured general workloads ---
+@pytest.mark.parametrize("name", sorted(__import__(
+    "tiled_attention_forward_sm_b200.inputs", fromlist=["GENERAL_WORKLOADS"]).GENERAL_WORKLOADS))
+def test_general_workloads_sampled_parity(oracle_mod, name):
+    """The measured general workloads at their full sizes, through the same
+    entry points bench.py times, on seeded sampled rows against the oracle."""
+    from tiled_attention_forward_sm_b200.inputs import GENERAL_WORKLOADS, make_general_inputs
+    w = GENERAL_WORKLOADS[name]
+    q, k, v = make_general_inputs(w)
+    qd, kd, vd = q.cuda(), k.cuda(), v.cuda()
+    rng = np.random.default_rng(77)
+    if w.kind == "varlen":
+        cu_q = np.concatenate([[0], np.cumsum(w.lens_q)]).astype(np.int32)
+        cu_k = np.concatenate([[0], np.cumsum(w.lens_k)]).astype(np.int32)
+        o, lse = tab.attn_fwd_varlen(qd, kd, vd, torch.from_numpy(cu_q).cuda(),
+                                     torch.from_numpy(cu_k).cuda(), w.N_q, w.N_k, w.causal, w.scale)
+        assert tab.last_device_error() == 0
+        o, lse = o.float().cpu().numpy(), lse.cpu().numpy()
+        qb, kb, vb = bf16_bits(q), bf16_bits(k), bf16_bits(v)
+        for b in range(w.B):
+            q0, q1, k0, k1 = cu_q[b], cu_q[b + 1], cu_k[b], cu_k[b + 1]
+            nq = q1 - q0
+            toks = np.unique(np.concatenate([[0, nq - 1], rng.integers(0, nq, 6)]))
+            rows = np.concatenate([h * nq + toks for h in range(w.H)]).astype(np.int64)
+            o_ref, l_ref = oracle_mod.attn_ref_general(
+                qb[q0:q1].transpose(1, 0, 2)[None], kb[k0:k1].transpose(1, 0, 2)[None],
+                vb[k0:k1].transpose(1, 0, 2)[None], w.causal, (k1 - k0) - nq, w.scale, rows=rows)
+            o_g = np.concatenate([o[q0 + toks, h] for h in range(w.H)])
+            l_g = np.concatenate([lse[h, q0 + toks] for h in range(w.H)])
+            check(o_g, l_g, o_ref, l_ref, f"{name} sequence {b}")
+        return
+    delta = w.N_k - w.N_q
+    if w.kind == "chunk":
+        o, lse = tab.attn_fwd_chunk(qd, kd, vd, w.causal, delta, w.scale)
+    else:
+        o, lse = tab.attn_fwd_splitkv(qd, kd, vd, w.n_splits, w.causal, delta, w.scale)
+    assert tab.last_device_error() == 0
+    total = w.B * w.H * w.N_q
+    rows = np.unique(np.concatenate([np.arange(0, total, w.N_q), np.arange(w.N_q - 1, total, w.N_q),
+                                     rng.integers(0, total, 512)])).astype(np.int64)
+    o_ref, l_ref = oracle_mod.attn_ref_general(bf16_bits(q), bf16_bits(k), bf16_bits(v), w.causal,
+                                               delta, w.scale, rows=rows)
+    check(o.float().cpu().numpy().reshape(-1, w.d)[rows], lse.cpu().numpy().reshape(-1)[rows],
+          o_ref, l_ref, name)

@@ -60,6 +60,76 @@ WORKLOADS = {
 BENCH_WORKLOAD = "b2h32n8192d128_causal"
 
 
+@dataclass(frozen=True)
+class GeneralWorkload:
+    """A problem for the general entry points: queries and keys of different
+    lengths (a block of queries at the end of a key/value cache, the last
+    query seeing the last key), shared K/V heads, split keys, or a packed
+    batch of sequences of different lengths (``lens_q``/``lens_k``)."""
+    name: str
+    kind: str           # "chunk", "splitkv" or "varlen"
+    B: int
+    H: int
+    H_kv: int
+    N_q: int            # per sequence (varlen: the longest)
+    N_k: int
+    d: int
+    causal: bool
+    seed: int
+    n_splits: int = 1
+    lens_q: tuple = ()
+    lens_k: tuple = ()
+
+    @property
+    def scale(self) -> float:
+        return 1.0 / math.sqrt(self.d)
+
+
+def _varlen_lengths(n: int, lo: int, hi: int, seed: int):
+    g = torch.Generator(device="cpu")
+    g.manual_seed(int(seed))
+    return tuple(int(x) for x in torch.randint(lo, hi + 1, (n,), generator=g))
+
+
+_LENS = _varlen_lengths(16, 512, 8192, 2103)
+
+# Problems for the general entry points (parity tests and measurement).
+GENERAL_WORKLOADS = {
+    w.name: w for w in [
+        # 512 new queries against a 16K-token cache, 4 query heads per K/V head
+        GeneralWorkload("kvcache_b4h32kv8_q512_k16384_d128", "chunk", 4, 32, 8, 512, 16384,
+                        128, True, 2101),
+        # a 128-query block against a 32K-token cache: 64 items without
+        # splitting the keys, 512 with 8 slices
+        GeneralWorkload("kvcache_b2h32kv8_q128_k32768_d128_split8", "splitkv", 2, 32, 8, 128,
+                        32768, 128, True, 2102, n_splits=8),
+        GeneralWorkload("kvcache_b2h32kv8_q128_k32768_d128_split1", "splitkv", 2, 32, 8, 128,
+                        32768, 128, True, 2102, n_splits=1),
+        # 16 sequences of 512..8192 tokens (seeded), packed without padding
+        GeneralWorkload("varlen_b16h16_d128_causal", "varlen", 16, 16, 16, max(_LENS),
+                        max(_LENS), 128, True, 2103, lens_q=_LENS, lens_k=_LENS),
+    ]
+}
+
+
+def make_general_inputs(w: GeneralWorkload):
+    """bf16 CPU tensors for a general workload: per-head [B, H, N_q, d] and
+    [B, H_kv, N_k, d], or packed [T_q, H, d] and [T_k, H_kv, d] for varlen
+    (same draw order: Q, then K, then V)."""
+    g = torch.Generator(device="cpu")
+    g.manual_seed(int(w.seed))
+    if w.kind == "varlen":
+        tq, tk = sum(w.lens_q), sum(w.lens_k)
+        q = torch.randn((tq, w.H, w.d), generator=g, dtype=torch.float32)
+        k = torch.randn((tk, w.H_kv, w.d), generator=g, dtype=torch.float32)
+        v = torch.randn((tk, w.H_kv, w.d), generator=g, dtype=torch.float32)
+    else:
+        q = torch.randn((w.B, w.H, w.N_q, w.d), generator=g, dtype=torch.float32)
+        k = torch.randn((w.B, w.H_kv, w.N_k, w.d), generator=g, dtype=torch.float32)
+        v = torch.randn((w.B, w.H_kv, w.N_k, w.d), generator=g, dtype=torch.float32)
+    return tuple(t.to(torch.bfloat16).contiguous() for t in (q, k, v))
+
+
 def make_qkv(B: int, H: int, N: int, d: int, seed: int, q_std: float = 1.0):
     """Return bf16 CPU tensors (q, k, v), each [B, H, N, d], contiguous."""
     g = torch.Generator(device="cpu")
