@@ -33,7 +33,7 @@ extern "C" {
 typedef enum {
   ATTN_OK = 0,
   ATTN_ERR_INVALID_ARG = -1,   /* null pointer, non-positive size, bad scale */
-  ATTN_ERR_UNSUPPORTED = -2,   /* d not in {64,96,128}, or B*H*N >= 2^31 */
+  ATTN_ERR_UNSUPPORTED = -2,   /* d not in {64,96,128,256}, or B*H*N >= 2^31 */
   ATTN_ERR_MISALIGNED = -3,    /* a device pointer is not 16-byte aligned */
   ATTN_ERR_CUDA = -4,          /* a CUDA runtime/driver call failed */
   ATTN_ERR_DEVICE_TIMEOUT = -5,/* a bounded wait inside the kernel ran out */
@@ -55,7 +55,7 @@ typedef void* attn_stream_t;
  *            denominator of the scaled, masked scores).
  *   o and lse must not overlap q, k, v or each other.
  *   B, H, N  > 0 (any N; tiles past N are masked); B*H*N < 2^31.
- *   d        64, 96 or 128.
+ *   d        64, 96, 128 or 256.
  *   causal   0: every key visible; non-zero: key j visible to query i iff j <= i.
  *   scale    finite and > 0 (typically 1/sqrt(d)).
  *   stream   CUDA stream the kernel is enqueued on.
@@ -206,7 +206,7 @@ int attn_fwd_splitkv(const void* q, const void* k, const void* v, void* o, float
  *   o          device, [rows, d]: bf16, or fp32 when o_fp32 != 0.  Written.
  *   lse        device, fp32 [rows].  Written (-inf if no part saw a key,
  *              with O = 0).
- *   G          1 .. 256;  rows >= 1;  d 64, 96 or 128.
+ *   G          1 .. 256;  rows >= 1;  d 64, 96, 128 or 256.
  *   Outputs must not overlap the inputs.  Errors and asynchrony as attn_fwd.
  */
 int attn_combine(const float* o_parts, const float* lse_parts, int G, long long rows, int d,

@@ -57,7 +57,7 @@ def ptrs(d=128, B=1, H=1, N=128):
     return [A, A + tb, A + 2 * tb, A + 3 * tb, A + 4 * tb]
 
 
-@pytest.mark.parametrize("d", [64, 96, 128])
+@pytest.mark.parametrize("d", [64, 96, 128, 256])
 @pytest.mark.parametrize("N", [1, 100, 128, 129, 256, 384, 1000, 32768])
 def test_check_args_accepts_supported(lib, d, N):
     assert tab.check_args(*ptrs(d, 2, 3, N), 2, 3, N, d, 1 / math.sqrt(d)) == 0
@@ -76,7 +76,7 @@ def test_check_args_rejections(lib):
     assert tab.check_args(*p, 1, 1, 128, 128, float("inf")) == -1
     assert tab.check_args(*p, 1, 1, 128, 80, 0.1) == -2                # d unsupported
     assert tab.check_args(*p, 1, 1, 128, 32, 0.1) == -2                # d unsupported
-    assert tab.check_args(*p, 1, 1, 128, 256, 0.1) == -2               # d unsupported
+    assert tab.check_args(*p, 1, 1, 128, 512, 0.1) == -2               # d unsupported
     assert tab.check_args(*p, 1 << 12, 1 << 12, 1 << 8, 128, 0.1) == -2  # rows >= 2^31
     q, k, v, o, l = p
     assert tab.check_args(q + 8, k, v, o, l, 1, 1, 128, 128, 0.1) == -3   # misaligned q

@@ -50,6 +50,7 @@ def draw(B, H, H_kv, N_q, N_k, d, seed, q_std=1.0):
     (1, 3, 1, 640, 256, 64, -384),    # more queries than keys: early rows see nothing
     (2, 2, 2, 257, 257, 96, 64),      # diagonal offset by half a tile
     (1, 2, 1, 200, 700, 128, -100),   # negative offset: rows 0..99 see nothing
+    (1, 4, 2, 300, 900, 256, 600),    # head dim 256
 ])
 def test_chunk_matches_oracle(oracle_mod, out, causal, B, H, H_kv, N_q, N_k, d, delta):
     scale = 1 / math.sqrt(d)
@@ -78,6 +79,7 @@ def test_chunk_square_equals_attn_fwd():
     (128, 4, 2, [300, 0, 1, 1024, 77], [300, 5, 700, 1024, 77]),
     (64, 2, 2, [129, 513, 3], [129, 513, 3]),
     (96, 6, 3, [256, 40], [1000, 0]),
+    (256, 2, 1, [700, 130], [700, 900]),
 ])
 def test_varlen_matches_oracle(oracle_mod, causal, d, H, H_kv, lens_q, lens_k):
     scale = 1 / math.sqrt(d)
@@ -121,6 +123,7 @@ def test_varlen_bad_offsets_are_caught_on_the_device():
     (1, 2, 2, 640, 640, 128, 64),   # more slices asked for than tiles: one tile each
     (1, 8, 2, 128, 8192, 128, 16),  # a block of queries against a long cache
     (2, 4, 4, 1, 3000, 128, 7),     # one query per head
+    (1, 2, 1, 256, 4096, 256, 6),   # head dim 256
 ])
 def test_splitkv_matches_oracle(oracle_mod, causal, B, H, H_kv, N_q, N_k, d, n_splits):
     scale = 1 / math.sqrt(d)
@@ -142,7 +145,7 @@ def test_splitkv_one_slice_is_attn_fwd():
 
 
 # ------------------------------------------------------------ combine ---
-@pytest.mark.parametrize("d", [64, 96, 128])
+@pytest.mark.parametrize("d", [64, 96, 128, 256])
 def test_combine_matches_oracle_merge(oracle_mod, d):
     """Random parts (with some parts and some whole rows unseen, LSE = -inf)
     merged on the GPU against the oracle's merge."""

@@ -44,7 +44,7 @@ def full_parity(oracle_mod, B, H, N, d, causal, seed, q_std=1.0, scale=None, pol
     return check(o, lse, o_ref, lse_ref, f"B{B} H{H} N{N} d{d} causal={causal}")
 
 
-@pytest.mark.parametrize("d", [64, 96, 128])
+@pytest.mark.parametrize("d", [64, 96, 128, 256])
 @pytest.mark.parametrize("causal", [False, True])
 @pytest.mark.parametrize("N", [128, 256, 384, 640])
 def test_small_shapes(oracle_mod, d, causal, N):
@@ -53,7 +53,7 @@ def test_small_shapes(oracle_mod, d, causal, N):
     full_parity(oracle_mod, 2, 3, N, d, causal, seed=N + d + causal)
 
 
-@pytest.mark.parametrize("d", [64, 96, 128])
+@pytest.mark.parametrize("d", [64, 96, 128, 256])
 @pytest.mark.parametrize("causal", [False, True])
 @pytest.mark.parametrize("N", [1, 7, 100, 129, 255, 300, 1000])
 def test_ragged_lengths(oracle_mod, d, causal, N):
@@ -62,7 +62,7 @@ def test_ragged_lengths(oracle_mod, d, causal, N):
     full_parity(oracle_mod, 2, 3, N, d, causal, seed=900 + N + d, q_std=2.0)
 
 
-@pytest.mark.parametrize("d", [96, 128])
+@pytest.mark.parametrize("d", [96, 128, 256])
 @pytest.mark.parametrize("causal", [False, True])
 def test_ragged_length_writes_nothing_past_the_rows(causal, d):
     """B*H heads of N = 200 rows, packed back to back inside guard bands: no
@@ -83,7 +83,7 @@ def test_ragged_length_writes_nothing_past_the_rows(causal, d):
 
 
 @pytest.mark.parametrize("poly", [0, 1, 2])
-@pytest.mark.parametrize("d", [64, 96, 128])
+@pytest.mark.parametrize("d", [64, 96, 128, 256])
 @pytest.mark.parametrize("causal", [False, True])
 def test_exp2_split_variants(oracle_mod, poly, d, causal):
     """Every split of the exponentials between the special-function unit and

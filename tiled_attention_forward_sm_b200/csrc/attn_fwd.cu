@@ -15,6 +15,7 @@
 #include "attn_b200.h"
 #include "attn_combine_kernel.cuh"
 #include "attn_fwd_kernel.cuh"
+#include "attn_fwd_wide_kernel.cuh"
 
 namespace attn_b200 {
 
@@ -188,7 +189,6 @@ int64_t problem_items(const Problem& p) {
 
 template <int D, bool CAUSAL, int kPolyPairs>
 int launch(const Problem& p, cudaStream_t stream, DeviceState& st, int* queue = nullptr) {
-  using C = Config<D>;
   CUtensorMap tq, tk, tv;
   if (p.cu_q != nullptr) {
     if (make_tmap_tokens(&tq, p.q, p.T_q, p.H, D) || make_tmap_tokens(&tk, p.k, p.T_k, p.H_kv, D) ||
@@ -236,20 +236,31 @@ int launch(const Problem& p, cudaStream_t stream, DeviceState& st, int* queue = 
   args.scale_log2 = p.scale * 1.4426950408889634f;
   args.status = st.status;
 
-  auto kern = attn_fwd_kernel<D, CAUSAL, kPolyPairs>;
-  // The kernel's register split (setmaxnreg) hands the softmax warpgroups
-  // registers released by the producer/MMA warpgroup; it is only valid if
-  // the kernel was built with the full per-thread budget it assumes.
-  static const bool regs_ok = [&] {
-    cudaFuncAttributes fa;
-    if (cudaFuncGetAttributes(&fa, kern) != cudaSuccess) {
-      cudaGetLastError();
-      return false;
-    }
-    return fa.numRegs * kThreads >= kRegSplitTotal;
-  }();
-  if (!regs_ok) return ATTN_ERR_CUDA;
-  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes) !=
+  // d = 256 runs the wide kernel (one Q tile at a time, 256-column O).
+  void (*kern)(CUtensorMap, CUtensorMap, CUtensorMap, KernelArgs);
+  int threads, smem_bytes;
+  if constexpr (D == wide::kD) {
+    kern = wide::attn_fwd_wide_kernel<CAUSAL, kPolyPairs>;
+    threads = wide::kThreads;
+    smem_bytes = wide::kSmemBytes;
+  } else {
+    kern = attn_fwd_kernel<D, CAUSAL, kPolyPairs>;
+    threads = kThreads;
+    smem_bytes = Config<D>::kSmemBytes;
+    // The kernel's register split (setmaxnreg) hands the softmax warpgroups
+    // registers released by the producer/MMA warpgroup; it is only valid if
+    // the kernel was built with the full per-thread budget it assumes.
+    static const bool regs_ok = [&] {
+      cudaFuncAttributes fa;
+      if (cudaFuncGetAttributes(&fa, kern) != cudaSuccess) {
+        cudaGetLastError();
+        return false;
+      }
+      return fa.numRegs * kThreads >= kRegSplitTotal;
+    }();
+    if (!regs_ok) return ATTN_ERR_CUDA;
+  }
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes) !=
       cudaSuccess) {
     cudaGetLastError();
     return ATTN_ERR_CUDA;
@@ -259,8 +270,8 @@ int launch(const Problem& p, cudaStream_t stream, DeviceState& st, int* queue = 
   // Persistent: one CTA per SM (at most one per work item).
   const int grid = args.n_items < st.num_sms ? args.n_items : st.num_sms;
   cfg.gridDim = dim3(static_cast<unsigned>(grid), 1, 1);
-  cfg.blockDim = dim3(kThreads, 1, 1);
-  cfg.dynamicSmemBytes = C::kSmemBytes;
+  cfg.blockDim = dim3(static_cast<unsigned>(threads), 1, 1);
+  cfg.dynamicSmemBytes = static_cast<size_t>(smem_bytes);
   cfg.stream = stream;
   if (cudaLaunchKernelEx(&cfg, kern, tq, tk, tv, args) != cudaSuccess) {
     cudaGetLastError();
@@ -299,6 +310,7 @@ int run_problem(const Problem& p, int poly_pairs, attn_stream_t stream, int* que
   if (problem_items(p) + st->num_sms > 0x7FFFFFFFll) return ATTN_ERR_UNSUPPORTED;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   switch (p.d) {
+    case 256: return launch_d<256>(poly_pairs, p, s, *st, queue);
     case 128: return launch_d<128>(poly_pairs, p, s, *st, queue);
     case 96: return launch_d<96>(poly_pairs, p, s, *st, queue);
     default: return launch_d<64>(poly_pairs, p, s, *st, queue);
@@ -323,7 +335,7 @@ int run_combine(const float* o_parts, const float* lse_parts, int G, long long r
   return ATTN_OK;
 }
 
-bool head_dim_ok(int d) { return d == 64 || d == 96 || d == 128; }
+bool head_dim_ok(int d) { return d == 64 || d == 96 || d == 128 || d == 256; }
 
 bool scale_ok(float scale) { return std::isfinite(scale) && scale > 0.f; }
 
@@ -617,7 +629,7 @@ extern "C" const char* attn_strerror(int status) {
   switch (status) {
     case ATTN_OK: return "ok";
     case ATTN_ERR_INVALID_ARG: return "invalid argument";
-    case ATTN_ERR_UNSUPPORTED: return "unsupported shape (d must be 64, 96 or 128; B*H*N below 2^31)";
+    case ATTN_ERR_UNSUPPORTED: return "unsupported shape (d must be 64, 96, 128 or 256; B*H*N below 2^31)";
     case ATTN_ERR_MISALIGNED: return "misaligned pointer (q, k, v, o need 16 bytes, lse 4)";
     case ATTN_ERR_CUDA: return "CUDA call failed";
     case ATTN_ERR_DEVICE_TIMEOUT: return "device-side wait timed out";
