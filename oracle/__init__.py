@@ -16,6 +16,8 @@ Contents
                         packed token-major batch.
 ``lse_merge``           the result against a union of disjoint key sets from
                         the results against each set.
+``kmeans_assign``       the k-means assignment step: nearest centroid of each
+                        point and its squared distance (``kmeans_ref.c``).
 ``tiled_online_model``  a second fp64 formulation that follows the pages'
                         tiled algorithm step by step (tiles of K/V, a running
                         maximum and running sum, lazy rescale).  It is used to
@@ -37,17 +39,64 @@ import numpy as np
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "attn_ref.c")
 _LIB = os.path.join(_HERE, "libattn_ref.so")
+_KM_SRC = os.path.join(_HERE, "kmeans_ref.c")
+_KM_LIB = os.path.join(_HERE, "libkmeans_ref.so")
 _lib = None
+_km_lib = None
 
 
 def build(force: bool = False) -> str:
-    """Compile ``attn_ref.c`` into ``libattn_ref.so`` beside it (gcc, OpenMP,
-    -O2, no fast-math so exp/log keep their IEEE behaviour)."""
-    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
-        cmd = ["gcc", "-O2", "-fno-fast-math", "-fopenmp", "-fPIC", "-shared",
-               "-std=c11", _SRC, "-o", _LIB, "-lm"]
-        subprocess.check_call(cmd)
+    """Compile ``attn_ref.c`` and ``kmeans_ref.c`` into shared libraries
+    beside them (gcc, OpenMP, -O2, no fast-math so exp/log keep their IEEE
+    behaviour)."""
+    for src, lib in ((_SRC, _LIB), (_KM_SRC, _KM_LIB)):
+        if force or not os.path.exists(lib) or os.path.getmtime(lib) < os.path.getmtime(src):
+            cmd = ["gcc", "-O2", "-fno-fast-math", "-fopenmp", "-fPIC", "-shared",
+                   "-std=c11", src, "-o", lib, "-lm"]
+            subprocess.check_call(cmd)
     return _LIB
+
+
+def _load_kmeans():
+    global _km_lib
+    if _km_lib is None:
+        build()
+        lib = ctypes.CDLL(_KM_LIB)
+        lib.kmeans_assign_f64.restype = ctypes.c_int
+        lib.kmeans_assign_f64.argtypes = [
+            ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64, ctypes.c_int64, ctypes.c_int64,
+            ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64,
+            ctypes.c_int]
+        _km_lib = lib
+    return _km_lib
+
+
+def kmeans_assign(x_bits, c_bits, rows=None, with_dist: bool = False, nthreads: int = 0):
+    """k-means assignment in fp64 (``kmeans_ref.c``): for each point the
+    nearest centroid (smallest index among equal distances) and that squared
+    distance.  x_bits [N, d], c_bits [K, d]: uint16 bf16 bit patterns.
+    Returns (assign int32 [n], best float64 [n]) and, with ``with_dist``,
+    the distance rows float64 [n, K] too."""
+    x_bits = np.ascontiguousarray(x_bits, dtype=np.uint16)
+    c_bits = np.ascontiguousarray(c_bits, dtype=np.uint16)
+    N, d = x_bits.shape
+    K, dc = c_bits.shape
+    if dc != d:
+        raise ValueError("points and centroids disagree on d")
+    if rows is None:
+        n, rows_p, nrows = N, None, 0
+    else:
+        rows = np.ascontiguousarray(rows, dtype=np.int64)
+        n, rows_p, nrows = rows.shape[0], rows.ctypes.data, rows.shape[0]
+    assign = np.empty(n, dtype=np.int32)
+    best = np.empty(n, dtype=np.float64)
+    dist = np.empty((n, K), dtype=np.float64) if with_dist else None
+    rc = _load_kmeans().kmeans_assign_f64(
+        x_bits.ctypes.data, c_bits.ctypes.data, N, K, d, assign.ctypes.data, best.ctypes.data,
+        dist.ctypes.data if with_dist else None, rows_p, nrows, int(nthreads))
+    if rc != 0:
+        raise ValueError("kmeans_assign_f64 rejected its arguments")
+    return (assign, best, dist) if with_dist else (assign, best)
 
 
 def _load():
