@@ -38,8 +38,9 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 from tiled_attention_forward_sm_b200.inputs import (BENCH_WORKLOAD,  # noqa: E402
-                                                    GENERAL_WORKLOADS, WORKLOADS, bf16_bits,
-                                                    make_general_inputs, make_workload_inputs)
+                                                    GENERAL_WORKLOADS, KMEANS_WORKLOADS,
+                                                    WORKLOADS, bf16_bits, make_general_inputs,
+                                                    make_kmeans_inputs, make_workload_inputs)
 
 METRIC = "attention fwd TFLOPS (bf16, d=128) and % of B200 dense BF16 peak, 1 GPU"
 UNIT = "TFLOPS"
@@ -423,6 +424,70 @@ def run_general(args, w):
     }
 
 
+# ------------------------------------------------- k-means assignment -----
+def run_kmeans(args, w):
+    import ctypes
+    import tiled_attention_forward_sm_b200 as tab
+    world, rank, local = dist_env()
+    if world > 1:
+        raise SystemExit("k-means workloads run on one GPU")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    x_h, c_h = make_kmeans_inputs(w)
+    x, c = x_h.to(dev), c_h.to(dev)
+    lib = tab.library()
+    ws = torch.empty(int(lib.attn_kmeans_workspace_floats(w.N, w.K)), dtype=torch.float32,
+                     device=dev)
+    assign = torch.empty(w.N, dtype=torch.int32, device=dev)
+    best = torch.empty(w.N, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        rc = lib.attn_kmeans_assign(x.data_ptr(), c.data_ptr(), ws.data_ptr(), assign.data_ptr(),
+                                    best.data_ptr(), w.N, w.K, w.d, stream.cuda_stream)
+        assert rc == 0, rc
+
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES", "")
+    smi_id = vis.split(",")[local].strip() if vis and len(vis.split(",")) > local else str(local)
+    sampler = ClockSampler(smi_id)
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    sampler.start()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    clocks = sampler.stop()
+    status = tab.last_device_error(stream)
+    if status != 0:
+        raise SystemExit(f"device status {status}: {tab.strerror(status)}")
+    ms_step = e0.elapsed_time(e1) / args.steps
+    bytes_alg = 2 * (x.numel() + c.numel()) + 8 * w.N
+    tflops = w.flops / (ms_step * 1e-3) / 1e12
+    peaks, peak_kind = load_peaks()
+    return {
+        "metric": "k-means assignment TFLOPS (2*N*K*d point-centroid products, bf16)",
+        "value": round(tflops, 2), "unit": UNIT, "n_gpus": 1, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms_step, 4), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded centroids and points around them, see inputs.py)",
+        "config": {"workload": w.name, "N": w.N, "K": w.K, "d": w.d, "flops_per_step": w.flops,
+                   "l2": "inputs fit in L2 (126 MB); no flush" if bytes_alg < 126e6
+                   else "inputs larger than L2; no flush"},
+        "roofline": {"bound": "tensor", "achieved": round(tflops, 2),
+                     "peak": float(peaks["bf16_tflops"]), "unit": "TFLOP/s",
+                     "frac": round(tflops / float(peaks["bf16_tflops"]), 4), "traffic": None,
+                     "algorithmic_bytes": bytes_alg,
+                     "peak_source": f"{peak_kind} (MEASURED_PEAKS.json)"},
+        "e2e": None, "gpu_launches": 3 * args.steps, "clocks": clocks,
+        "kernel_sha": kernel_sha(),
+    }
+
+
 # ------------------------------------------------------- reference arm -----
 def run_reference(args, w):
     world, rank, _ = dist_env()
@@ -474,14 +539,19 @@ def main():
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["b200", "reference"], default="b200")
     ap.add_argument("--workload", default=BENCH_WORKLOAD,
-                    choices=sorted(WORKLOADS) + sorted(GENERAL_WORKLOADS))
+                    choices=sorted(WORKLOADS) + sorted(GENERAL_WORKLOADS) +
+                    sorted(KMEANS_WORKLOADS))
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
-    if args.workload in GENERAL_WORKLOADS:
+    if args.workload in KMEANS_WORKLOADS:
+        if args.impl == "reference":
+            ap.error("--impl reference times the attention workloads only")
+        line = run_kmeans(args, KMEANS_WORKLOADS[args.workload])
+    elif args.workload in GENERAL_WORKLOADS:
         if args.impl == "reference":
             ap.error("--impl reference times the square workloads only")
         line = run_general(args, GENERAL_WORKLOADS[args.workload])

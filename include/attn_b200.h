@@ -213,6 +213,32 @@ int attn_combine(const float* o_parts, const float* lse_parts, int G, long long 
                  void* o, float* lse, int o_fp32, attn_stream_t stream);
 
 /*
+ * attn_kmeans_assign -- the assignment step of k-means (page lefilia.fr,
+ * Flash-KMeans item, "FlashAssign"): every point goes to its nearest
+ * centroid, computed tile by tile without writing the N x K distance
+ * matrix.  Same tile machinery as the attention forward, with a running
+ * argmin where attention keeps a running softmax.
+ *
+ *   x          device, bf16 [N, d] points, contiguous.  Read only.
+ *   centroids  device, bf16 [K, d], contiguous.  Read only.
+ *   ws         device, fp32 scratch of attn_kmeans_workspace_floats(N, K)
+ *              values, 16-byte aligned, caller-owned; overwritten.
+ *   assign     device, int32 [N].  Written: the index of the nearest
+ *              centroid (among distances equal in fp32, the smallest index).
+ *   best       device, fp32 [N] or NULL.  Written when given: the squared
+ *              distance to that centroid, ||x||^2 + ||c||^2 - 2 x.c in fp32.
+ *   N, K       > 0 and < 2^30;  d  64 or 128.
+ * Distances are formed in fp32 from the bf16 inputs (products exact, sums
+ * rounded), so points whose two nearest centroids are within that rounding
+ * may pick either.  Errors and asynchrony as attn_fwd.
+ */
+int attn_kmeans_assign(const void* x, const void* centroids, float* ws, int32_t* assign,
+                       float* best, int N, int K, int d, attn_stream_t stream);
+
+/* Scratch size (fp32 values) attn_kmeans_assign needs, or -1 for bad sizes. */
+long long attn_kmeans_workspace_floats(int N, int K);
+
+/*
  * attn_fwd_host -- the same operation on HOST buffers: copies q, k, v from
  * host to the caller's device buffers, runs attn_fwd, and copies o and lse
  * back, all enqueued on `stream` (pinned host memory makes the copies

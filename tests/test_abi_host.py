@@ -213,3 +213,18 @@ def test_splitkv_and_combine_rejections_before_any_cuda_call(lib):
     assert c(w_o, w_l, 2, 100, 80, o, l, 0, None) == -2       # d
     assert c(w_o + 8, w_l, 2, 100, 128, o, l, 0, None) == -3
     assert c(w_o, w_l, 2, 100, 128, w_o, l, 0, None) == -1    # output over a part
+
+
+def test_kmeans_rejections_before_any_cuda_call(lib):
+    f = lib.attn_kmeans_assign
+    x, c, ws, a_, b_ = A, A + (1 << 24), A + (1 << 25), A + (1 << 26), A + (1 << 27)
+    assert f(None, c, ws, a_, b_, 1000, 64, 128, None) == -1
+    assert f(x, c, ws, a_, b_, 0, 64, 128, None) == -1          # N = 0
+    assert f(x, c, ws, a_, b_, 1000, 0, 128, None) == -1        # K = 0
+    assert f(x, c, ws, a_, b_, 1000, 64, 96, None) == -2        # d
+    assert f(x + 8, c, ws, a_, b_, 1000, 64, 128, None) == -3   # misaligned x
+    assert f(x, c, ws, a_ + 2, b_, 1000, 64, 128, None) == -3   # misaligned assign
+    assert f(x, c, x, a_, b_, 1000, 64, 128, None) == -1        # scratch over the points
+    assert lib.attn_kmeans_workspace_floats(1000, 64) == 128 + 1000
+    assert lib.attn_kmeans_workspace_floats(1000, 129) == 256 + 1000
+    assert lib.attn_kmeans_workspace_floats(0, 5) == -1

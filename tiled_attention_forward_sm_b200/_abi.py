@@ -65,6 +65,10 @@ def library():
         lib.attn_fwd_varlen.argtypes = [vp] * 7 + [i] * 9 + [f, vp]
         lib.attn_fwd_splitkv.restype = i
         lib.attn_fwd_splitkv.argtypes = [vp] * 5 + [i] * 8 + [f, i, vp, vp, vp]
+        lib.attn_kmeans_assign.restype = i
+        lib.attn_kmeans_assign.argtypes = [vp, vp, vp, vp, vp, i, i, i, vp]
+        lib.attn_kmeans_workspace_floats.restype = ctypes.c_longlong
+        lib.attn_kmeans_workspace_floats.argtypes = [i, i]
         lib.attn_combine.restype = i
         lib.attn_combine.argtypes = [vp, vp, i, ctypes.c_longlong, i, vp, vp, i, vp]
         _lib = lib
@@ -316,3 +320,28 @@ def attn_combine(o_parts, lse_parts, out_dtype=torch.bfloat16, stream=None):
     if rc != ATTN_OK:
         raise AttnError(rc, "attn_combine")
     return o, lse
+
+
+def kmeans_assign(x, centroids, with_best: bool = True, stream=None):
+    """k-means assignment (see attn_kmeans_assign in the header): x bf16
+    [N, d], centroids bf16 [K, d] on the GPU.  Returns (assign int32 [N],
+    best fp32 [N] or None)."""
+    if x.dim() != 2 or centroids.dim() != 2 or x.shape[1] != centroids.shape[1]:
+        raise ValueError("x must be [N, d] and centroids [K, d]")
+    N, d = (int(v) for v in x.shape)
+    K = int(centroids.shape[0])
+    _check(x, "x", torch.bfloat16, (N, d))
+    _check(centroids, "centroids", torch.bfloat16, (K, d))
+    lib = library()
+    n_ws = int(lib.attn_kmeans_workspace_floats(N, K))
+    if n_ws < 0:
+        raise ValueError("bad sizes")
+    ws = torch.empty(n_ws, dtype=torch.float32, device=x.device)
+    assign = torch.empty(N, dtype=torch.int32, device=x.device)
+    best = torch.empty(N, dtype=torch.float32, device=x.device) if with_best else None
+    rc = lib.attn_kmeans_assign(x.data_ptr(), centroids.data_ptr(), ws.data_ptr(),
+                                assign.data_ptr(), best.data_ptr() if with_best else None,
+                                N, K, d, _stream_handle(stream))
+    if rc != ATTN_OK:
+        raise AttnError(rc, "attn_kmeans_assign")
+    return assign, best

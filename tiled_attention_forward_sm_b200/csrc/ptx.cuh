@@ -306,6 +306,12 @@ __device__ __forceinline__ float max3(float a, float b, float c) {
   return d;
 }
 
+__device__ __forceinline__ float min3(float a, float b, float c) {
+  float d;
+  asm("min.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
 // ---- packed pairs of fp32 (sm_100 f32x2 ALU forms) ------------------------
 // A pair is held in one 64-bit register: .x in the low word, .y in the high.
 __device__ __forceinline__ uint64_t f2pack(float lo, float hi) {

@@ -130,6 +130,42 @@ def make_general_inputs(w: GeneralWorkload):
     return tuple(t.to(torch.bfloat16).contiguous() for t in (q, k, v))
 
 
+@dataclass(frozen=True)
+class KMeansWorkload:
+    """A k-means assignment problem: N points, K centroids, dimension d.
+    Recipe: ``manual_seed(seed)``; centroids ~ N(0, 1) [K, d]; each point is
+    a centroid drawn uniformly plus 0.5 N(0, 1) noise; both rounded to bf16."""
+    name: str
+    N: int
+    K: int
+    d: int
+    seed: int
+
+    @property
+    def flops(self) -> float:
+        """2*N*K*d: the point-centroid products (the distance matrix's cost)."""
+        return 2.0 * self.N * self.K * self.d
+
+
+KMEANS_WORKLOADS = {
+    w.name: w for w in [
+        # the configuration the Flash-KMeans item quotes
+        KMeansWorkload("kmeans_n65536_k1024_d128", 65536, 1024, 128, 3101),
+        # a larger assignment of the same shape of problem
+        KMeansWorkload("kmeans_n1048576_k4096_d128", 1048576, 4096, 128, 3102),
+    ]
+}
+
+
+def make_kmeans_inputs(w: KMeansWorkload):
+    g = torch.Generator(device="cpu")
+    g.manual_seed(int(w.seed))
+    c = torch.randn((w.K, w.d), generator=g, dtype=torch.float32)
+    pick = torch.randint(0, w.K, (w.N,), generator=g)
+    x = c[pick] + 0.5 * torch.randn((w.N, w.d), generator=g, dtype=torch.float32)
+    return x.to(torch.bfloat16).contiguous(), c.to(torch.bfloat16).contiguous()
+
+
 def make_qkv(B: int, H: int, N: int, d: int, seed: int, q_std: float = 1.0):
     """Return bf16 CPU tensors (q, k, v), each [B, H, N, d], contiguous."""
     g = torch.Generator(device="cpu")
