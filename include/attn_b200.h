@@ -213,6 +213,28 @@ int attn_combine(const float* o_parts, const float* lse_parts, int G, long long 
                  void* o, float* lse, int o_fp32, attn_stream_t stream);
 
 /*
+ * attn_fwd_fp8 -- attention forward with FP8 (OCP E4M3) operands, head dim
+ * 128: the low-precision variant weighed on page lecompute.fr/kernel-perf/
+ * flashattention-4-limites-calcul-matriciel, section "Le FP4 ajoute un
+ * compromis numerique".  Scores are (scale * q_descale * k_descale) Q K^T;
+ * the weights are rounded to E4M3 before the second product (their row sum
+ * is kept in fp32); O = v_descale * P V / l in bf16; LSE as attn_fwd.
+ *
+ *   q, k     device, E4M3 bytes [B, H, N, 128].  Read only.
+ *   vt       device, E4M3 bytes [B, H, 128, N]: V transposed, so that both
+ *            products read K-major operands.  Read only.
+ *   o        device, bf16 [B, H, N, 128].  Written.   lse  fp32 [B, H, N].
+ *   N        > 0 and a multiple of 16 (the V^T rows must be 16-byte
+ *            aligned); B*H*N < 2^31.
+ *   scale, q_descale, k_descale, v_descale  finite and > 0.
+ * The weights' rounding (3 mantissa bits; below 2^-9 they flush to zero)
+ * is the numeric cost of the format.  Errors and asynchrony as attn_fwd.
+ */
+int attn_fwd_fp8(const void* q, const void* k, const void* vt, void* o, float* lse,
+                 int B, int H, int N, int d, int causal, float scale, float q_descale,
+                 float k_descale, float v_descale, attn_stream_t stream);
+
+/*
  * attn_kmeans_assign -- the assignment step of k-means (page lefilia.fr,
  * Flash-KMeans item, "FlashAssign"): every point goes to its nearest
  * centroid, computed tile by tile without writing the N x K distance

@@ -262,6 +262,33 @@ def lse_merge(o_parts, lse_parts):
     return o, lse
 
 
+def e4m3_bits_to_f64(bits) -> np.ndarray:
+    """Decode OCP FP8 E4M3 (``e4m3fn``) bit patterns: sign, 4 exponent bits
+    with bias 7, 3 mantissa bits; exponent 0 is subnormal (2^-6 * m/8);
+    S.1111.111 is NaN; there are no infinities."""
+    b = np.asarray(bits, dtype=np.uint8).astype(np.int64)
+    sign = np.where(b & 0x80, -1.0, 1.0)
+    e = (b >> 3) & 0xF
+    m = b & 0x7
+    val = np.where(e == 0, m / 8.0 * 2.0 ** -6, (1.0 + m / 8.0) * np.exp2(e - 7.0))
+    val = np.where((e == 15) & (m == 7), np.nan, val)
+    return sign * val
+
+
+def round_e4m3(x: np.ndarray) -> np.ndarray:
+    """Round float64 values to the nearest E4M3 value (ties to even),
+    saturating at +-448 (the largest finite value)."""
+    x = np.asarray(x, dtype=np.float64)
+    a = np.minimum(np.abs(x), 448.0)
+    # spacing of the binade holding a: 2^(max(e, -6) - 3)
+    with np.errstate(divide="ignore"):
+        e = np.floor(np.log2(np.where(a > 0, a, 1.0)))
+    e = np.maximum(e, -6.0)
+    q = np.exp2(e - 3.0)
+    r = np.round(a / q) * q          # numpy rounds halves to even
+    return np.sign(x) * np.minimum(r, 448.0)
+
+
 def bf16_bits_to_f64(bits) -> np.ndarray:
     """Exact widening of bf16 bit patterns to float64."""
     bits = np.asarray(bits, dtype=np.uint16)
@@ -280,7 +307,7 @@ def _round_bf16(x: np.ndarray) -> np.ndarray:
 
 
 def tiled_online_model(q, k, v, causal: bool, scale: float, block_n: int = 128,
-                       tau: float = 8.0, round_p_bf16: bool = False):
+                       tau: float = 8.0, round_p_bf16: bool = False, round_p=None):
     """The pages' tiled algorithm for one (b, h) pair, in fp64.
 
     Follows page "lecompute.fr/kernel-perf/flashattention-4-limites-calcul-
@@ -293,9 +320,13 @@ def tiled_online_model(q, k, v, causal: bool, scale: float, block_n: int = 128,
     maximum is kept and the tile's weights may reach 2**tau.
 
     q, k, v: float64 [N, d].  Returns (o [N, d], lse [N]) in float64.
-    With ``round_p_bf16`` the weights are rounded to bf16 before the second
-    product (what the kernel feeds its tensor cores); the row sum stays exact.
+    With ``round_p_bf16`` (or ``round_p="bf16"``) the weights are rounded to
+    bf16 before the second product (what the kernel feeds its tensor cores);
+    ``round_p="e4m3"`` rounds them to FP8 E4M3 instead (the FP8 path).  The
+    row sum stays exact.
     """
+    if round_p_bf16:
+        round_p = "bf16"
     q = np.asarray(q, dtype=np.float64)
     k = np.asarray(k, dtype=np.float64)
     v = np.asarray(v, dtype=np.float64)
@@ -320,7 +351,7 @@ def tiled_online_model(q, k, v, causal: bool, scale: float, block_n: int = 128,
             p = np.exp2(x - m_used[:, None])
         p = np.where(np.isneginf(x), 0.0, p)
         l = l * alpha + p.sum(axis=1)
-        pv = _round_bf16(p) if round_p_bf16 else p
+        pv = _round_bf16(p) if round_p == "bf16" else (round_e4m3(p) if round_p == "e4m3" else p)
         acc = acc * alpha[:, None] + pv @ v[cols]
         m = m_used
     o = acc / l[:, None]

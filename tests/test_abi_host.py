@@ -228,3 +228,15 @@ def test_kmeans_rejections_before_any_cuda_call(lib):
     assert lib.attn_kmeans_workspace_floats(1000, 64) == 128 + 1000
     assert lib.attn_kmeans_workspace_floats(1000, 129) == 256 + 1000
     assert lib.attn_kmeans_workspace_floats(0, 5) == -1
+
+
+def test_fp8_rejections_before_any_cuda_call(lib):
+    q, k, v, o, l = ptrs(128, 1, 1, 1024)
+    f = lib.attn_fwd_fp8
+    good = (1, 1, 1024, 128, 1, 0.1, 1.0, 1.0, 1.0)
+    assert f(q, k, v, o, l, 1, 1, 1000, 128, 1, 0.1, 1.0, 1.0, 1.0, None) == -2   # N % 16
+    assert f(q, k, v, o, l, 1, 1, 1024, 64, 1, 0.1, 1.0, 1.0, 1.0, None) == -2    # d
+    assert f(q, k, v, o, l, 1, 1, 1024, 128, 1, 0.1, 0.0, 1.0, 1.0, None) == -1   # descale
+    assert f(q, k, v, o, l, 1, 1, 1024, 128, 1, 0.1, 1.0, 1.0, float("nan"), None) == -1
+    assert f(q + 8, k, v, o, l, *good, None) == -3
+    assert f(q, k, v, q, l, *good, None) == -1                                    # o over q

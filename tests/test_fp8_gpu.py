@@ -1,0 +1,82 @@
+"""GPU parity of the FP8 (E4M3) attention path.
+
+Two checks per case:
+  * the implementation: against the oracle's tiled model that rounds the
+    weights to E4M3 the same way (per 128-key tile, lazy max with tau = 8),
+    |O - O_model| <= 2^-8 |O_model| + 4e-3 (the bf16 output plus rare
+    rounding flips where fp32 and fp64 weights fall on either side of an
+    E4M3 rounding boundary), |LSE - LSE_exact| <= 1e-3 (l is kept in fp32);
+  * the accuracy: against the exact definition on the same E4M3 inputs,
+    |O - O_exact| <= 2^-3 A + 2^-8 |O| + 4e-3 with A the exactly weighted
+    mean |v| of each output element (each weight within 2^-4 of itself, doubled for
+    rounding flips).
+Descale factors are powers of two so the oracle sees the same values.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import tiled_attention_forward_sm_b200 as tab
+from tiled_attention_forward_sm_b200.inputs import bf16_bits, make_qkv
+
+pytestmark = pytest.mark.gpu
+
+
+def run_case(oracle_mod, B, H, N, causal, seed, dq=0.5, dk=2.0, dv=0.25, q_std=1.0):
+    d = 128
+    scale = 1 / math.sqrt(d)
+    q, k, v = make_qkv(B, H, N, d, seed, q_std)
+    q8 = (q.float() / dq).to(torch.float8_e4m3fn)
+    k8 = (k.float() / dk).to(torch.float8_e4m3fn)
+    v8 = (v.float() / dv).to(torch.float8_e4m3fn)
+    vt8 = v8.transpose(2, 3).contiguous()
+    o, lse = tab.attn_fwd_fp8(q8.cuda(), k8.cuda(), vt8.cuda(), causal, scale, dq, dk, dv)
+    assert tab.last_device_error() == 0
+    o = o.float().cpu().numpy().astype(np.float64)
+    lse = lse.cpu().numpy().astype(np.float64)
+    # exact definition on the E4M3 values (exact in bf16; descales folded)
+    qb, kb, vb = (bf16_bits(t.float().to(torch.bfloat16)) for t in (q8, k8, v8))
+    o_ex, l_ex = oracle_mod.attn_ref(qb, kb, vb, causal, scale * dq * dk)
+    o_ex = o_ex * dv
+    Qd, Kd, Vd = (t.double().numpy() for t in (q8.float(), k8.float(), v8.float()))
+    for b in range(B):
+        for h in range(H):
+            o_m, _ = oracle_mod.tiled_online_model(Qd[b, h], Kd[b, h], Vd[b, h], causal,
+                                                   scale * dq * dk, round_p="e4m3")
+            o_m = o_m * dv
+            err = np.abs(o[b, h] - o_m)
+            assert (err <= 2.0 ** -8 * np.abs(o_m) + 4e-3).all(), \
+                f"b{b} h{h}: vs model max err {err.max():.3g}"
+            S = Qd[b, h] @ Kd[b, h].T * (scale * dq * dk)
+            if causal:
+                S = np.where(np.tril(np.ones_like(S)) > 0, S, -np.inf)
+            W = np.exp(S - S.max(1, keepdims=True))
+            W /= W.sum(1, keepdims=True)
+            A = (W @ np.abs(Vd[b, h])) * dv
+            err = np.abs(o[b, h] - o_ex[b, h])
+            assert (err <= 2.0 ** -3 * A + 2.0 ** -8 * np.abs(o_ex[b, h]) + 4e-3).all()
+    assert np.abs(lse - l_ex).max() <= 1e-3
+
+
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("N", [128, 256, 640, 1024])
+def test_fp8_matches_model_and_bound(oracle_mod, causal, N):
+    run_case(oracle_mod, 1, 3, N, causal, seed=70 + N)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_fp8_ragged_and_peaky(oracle_mod, causal):
+    run_case(oracle_mod, 2, 2, 400, causal, seed=91, q_std=3.0)
+
+
+def test_fp8_rejects_unsupported_shapes():
+    x = torch.zeros(1, 1, 100, 128, dtype=torch.uint8, device="cuda")
+    vt = torch.zeros(1, 1, 128, 100, dtype=torch.uint8, device="cuda")
+    with pytest.raises(tab.AttnError) as e:
+        tab.attn_fwd_fp8(x, x, vt)  # N = 100 is not a multiple of 16
+    assert e.value.status == -2
+    x64 = torch.zeros(1, 1, 128, 64, dtype=torch.uint8, device="cuda")
+    with pytest.raises(tab.AttnError):
+        tab.attn_fwd_fp8(x64, x64, torch.zeros(1, 1, 64, 128, dtype=torch.uint8, device="cuda"))

@@ -212,3 +212,56 @@ def test_varlen_sequences_are_independent(oracle_mod):
             full, _ = _brute(Q[t_last:t_last + 1, 0], K[cu_k[b]:cu_k[b + 1], 0],
                              V[cu_k[b]:cu_k[b + 1], 0], False, 0, scale)
             np.testing.assert_allclose(o[t_last, 0], full[0], rtol=0, atol=1e-13)
+
+
+# ------------------------------------------------------------- FP8 (E4M3) ---
+def test_e4m3_decode_matches_torch_for_every_code(oracle_mod):
+    """The oracle's E4M3 decoding from the format's definition equals
+    torch's float8_e4m3fn for all 256 codes (NaN codes included)."""
+    import torch
+    codes = np.arange(256, dtype=np.uint8)
+    mine = oracle_mod.e4m3_bits_to_f64(codes)
+    ref = torch.from_numpy(codes).view(torch.float8_e4m3fn).float().double().numpy()
+    np.testing.assert_array_equal(np.isnan(mine), np.isnan(ref))
+    ok = ~np.isnan(ref)
+    np.testing.assert_array_equal(mine[ok], ref[ok])
+
+
+def test_e4m3_rounding_matches_torch_and_saturates(oracle_mod):
+    """Round to nearest even over 20 binades (subnormals included) equals
+    torch's cast; values past 448 saturate (the kernel's satfinite)."""
+    import torch
+    rng = np.random.default_rng(0)
+    x = rng.standard_normal(200000) * np.exp2(rng.uniform(-14, 8, 200000))
+    x = np.clip(x, -447.0, 447.0)
+    ref = torch.from_numpy(x).float().to(torch.float8_e4m3fn).double().numpy()
+    np.testing.assert_array_equal(oracle_mod.round_e4m3(x), ref)
+    np.testing.assert_array_equal(oracle_mod.round_e4m3(np.array([500.0, -1e6, 448.0])),
+                                  [448.0, -448.0, 448.0])
+    # exact halfway cases go to the even neighbour
+    np.testing.assert_array_equal(oracle_mod.round_e4m3(np.array([1.0625, 1.1875, 2.0 ** -10])),
+                                  [1.0, 1.25, 0.0])
+
+
+def test_model_with_e4m3_weights_stays_inside_its_bound(oracle_mod):
+    """The tiled model with weights rounded to E4M3 differs from the exact
+    result by at most 2^-4 of the weighted mean |v| per row (each weight is
+    off by at most 2^-4 of itself in E4M3's normal range), plus the
+    flush-to-zero of weights below 2^-9, small at these sizes."""
+    from tiled_attention_forward_sm_b200.inputs import make_qkv
+    q, k, v = make_qkv(1, 1, 1024, 128, 5)
+    import torch
+    def e4(t):
+        return t[0, 0].float().to(torch.float8_e4m3fn).double().numpy()
+    Q, K, V = e4(q), e4(k), e4(v)
+    scale = 128 ** -0.5
+    for causal in (False, True):
+        o_ex, _ = oracle_mod.tiled_online_model(Q, K, V, causal, scale)
+        o_m, _ = oracle_mod.tiled_online_model(Q, K, V, causal, scale, round_p="e4m3")
+        S = Q @ K.T * scale
+        if causal:
+            S = np.where(np.tril(np.ones_like(S)) > 0, S, -np.inf)
+        W = np.exp(S - S.max(1, keepdims=True))
+        W /= W.sum(1, keepdims=True)
+        A = W @ np.abs(V)
+        assert (np.abs(o_m - o_ex) <= 2.0 ** -4 * A + 1e-3).all()

@@ -65,6 +65,8 @@ def library():
         lib.attn_fwd_varlen.argtypes = [vp] * 7 + [i] * 9 + [f, vp]
         lib.attn_fwd_splitkv.restype = i
         lib.attn_fwd_splitkv.argtypes = [vp] * 5 + [i] * 8 + [f, i, vp, vp, vp]
+        lib.attn_fwd_fp8.restype = i
+        lib.attn_fwd_fp8.argtypes = [vp] * 5 + [i] * 5 + [f, f, f, f, vp]
         lib.attn_kmeans_assign.restype = i
         lib.attn_kmeans_assign.argtypes = [vp, vp, vp, vp, vp, i, i, i, vp]
         lib.attn_kmeans_workspace_floats.restype = ctypes.c_longlong
@@ -345,3 +347,28 @@ def kmeans_assign(x, centroids, with_best: bool = True, stream=None):
     if rc != ATTN_OK:
         raise AttnError(rc, "attn_kmeans_assign")
     return assign, best
+
+
+def attn_fwd_fp8(q, k, vt, causal: bool = False, scale: float | None = None,
+                 q_descale: float = 1.0, k_descale: float = 1.0, v_descale: float = 1.0,
+                 stream=None):
+    """FP8 attention (see attn_fwd_fp8 in the header): q, k E4M3 [B,H,N,128]
+    and vt E4M3 [B,H,128,N] (V transposed) on the GPU, as float8_e4m3fn or
+    uint8 tensors.  Returns (o bf16 [B,H,N,128], lse fp32 [B,H,N])."""
+    B, H, N, d = (int(x) for x in q.shape)
+    for name, t, shape in (("q", q, (B, H, N, d)), ("k", k, (B, H, N, d)),
+                           ("vt", vt, (B, H, d, N))):
+        if t.element_size() != 1:
+            raise ValueError(f"{name} must hold 8-bit values")
+        _check(t, name, t.dtype, shape)
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    o = torch.empty((B, H, N, d), dtype=torch.bfloat16, device=q.device)
+    lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
+    rc = library().attn_fwd_fp8(q.data_ptr(), k.data_ptr(), vt.data_ptr(), o.data_ptr(),
+                                lse.data_ptr(), B, H, N, d, int(bool(causal)), float(scale),
+                                float(q_descale), float(k_descale), float(v_descale),
+                                _stream_handle(stream))
+    if rc != ATTN_OK:
+        raise AttnError(rc, "attn_fwd_fp8")
+    return o, lse

@@ -17,6 +17,7 @@
 #include "attn_fwd_kernel.cuh"
 #include "attn_fwd_wide_kernel.cuh"
 #include "kmeans_assign_kernel.cuh"
+#include "attn_fwd_fp8_kernel.cuh"
 
 namespace attn_b200 {
 
@@ -615,6 +616,99 @@ int launch_kmeans(const void* x, const void* cent, float* ws, int32_t* assign, f
 
 }  // namespace
 }  // namespace attn_b200
+
+namespace attn_b200 {
+namespace {
+
+// 3-D view of an 8-bit tensor: dims {inner, mid, outer}, boxes of 128 x 128
+// x 1 (128-byte rows, the 128-byte swizzle).
+int make_tmap_u8(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t mid, uint64_t outer) {
+  cuuint64_t dims[3] = {inner, mid, outer};
+  cuuint64_t strides[2] = {inner, inner * mid};
+  cuuint32_t box[3] = {128, 128, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(ptr), dims,
+                        strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+}  // namespace
+}  // namespace attn_b200
+
+extern "C" int attn_fwd_fp8(const void* q, const void* k, const void* vt, void* o, float* lse,
+                            int B, int H, int N, int d, int causal, float scale, float q_descale,
+                            float k_descale, float v_descale, attn_stream_t stream) {
+  if (!q || !k || !vt || !o || !lse) return ATTN_ERR_INVALID_ARG;
+  if (B <= 0 || H <= 0 || N <= 0) return ATTN_ERR_INVALID_ARG;
+  if (!scale_ok(scale) || !scale_ok(q_descale) || !scale_ok(k_descale) || !scale_ok(v_descale))
+    return ATTN_ERR_INVALID_ARG;
+  if (d != fp8::kD) return ATTN_ERR_UNSUPPORTED;
+  // V^T rows are N bytes long: the tensor map needs them 16-byte aligned.
+  if (N % 16 != 0) return ATTN_ERR_UNSUPPORTED;
+  const uint64_t rows = static_cast<uint64_t>(B) * H * N;
+  if (rows >= (1ull << 31)) return ATTN_ERR_UNSUPPORTED;
+  const uintptr_t al = reinterpret_cast<uintptr_t>(q) | reinterpret_cast<uintptr_t>(k) |
+                       reinterpret_cast<uintptr_t>(vt) | reinterpret_cast<uintptr_t>(o);
+  if (al & 15u) return ATTN_ERR_MISALIGNED;
+  if (reinterpret_cast<uintptr_t>(lse) & 3u) return ATTN_ERR_MISALIGNED;
+  const size_t ib = rows * static_cast<size_t>(d);
+  const void* outs[2] = {o, lse};
+  const size_t out_bytes[2] = {ib * 2, rows * 4};
+  const void* ins[3] = {q, k, vt};
+  const size_t in_bytes[3] = {ib, ib, ib};
+  if (!outputs_disjoint(outs, out_bytes, 2, ins, in_bytes, 3)) return ATTN_ERR_INVALID_ARG;
+  DeviceState* st = nullptr;
+  int rc = device_state(&st);
+  if (rc != ATTN_OK) return rc;
+  CUtensorMap tq, tk, tvt;
+  const uint64_t BH = static_cast<uint64_t>(B) * H;
+  if (make_tmap_u8(&tq, q, d, N, BH) || make_tmap_u8(&tk, k, d, N, BH) ||
+      make_tmap_u8(&tvt, vt, N, d, BH))
+    return ATTN_ERR_CUDA;
+  Problem p = dense_problem(q, k, vt, o, lse, B, H, N, d, causal, scale);
+  if (problem_items(p) + st->num_sms > 0x7FFFFFFFll) return ATTN_ERR_UNSUPPORTED;
+  KernelArgs args;
+  std::memset(&args, 0, sizeof args);
+  args.o = o;
+  args.lse = lse;
+  args.H = H;
+  args.H_kv = H;
+  args.q_per_kv = 1;
+  args.N_q = N;
+  args.N_k = N;
+  args.n_qpairs = ((N + kBlockM - 1) / kBlockM + 1) / 2;
+  args.n_splits = 1;
+  args.split_tiles = (N + kBlockN - 1) / kBlockN;
+  args.BH = B * H;
+  args.n_items = static_cast<int>(problem_items(p));
+  {
+    const int want = (2 * st->num_sms + args.n_qpairs - 1) / args.n_qpairs;
+    args.win_heads = want < 1 ? 1 : (want > args.BH ? args.BH : want);
+  }
+  args.scale_log2 = scale * q_descale * k_descale * 1.4426950408889634f;
+  args.status = st->status;
+  args.queue = st->queue + 2 * static_cast<int>(st->launches.fetch_add(1) % kQueueSlots);
+  auto kern = causal ? fp8::attn_fwd_fp8_kernel<true> : fp8::attn_fwd_fp8_kernel<false>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, fp8::kSmemBytes) !=
+      cudaSuccess) {
+    cudaGetLastError();
+    return ATTN_ERR_CUDA;
+  }
+  cudaLaunchConfig_t cfg;
+  std::memset(&cfg, 0, sizeof cfg);
+  const int grid = args.n_items < st->num_sms ? args.n_items : st->num_sms;
+  cfg.gridDim = dim3(static_cast<unsigned>(grid), 1, 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = fp8::kSmemBytes;
+  cfg.stream = static_cast<cudaStream_t>(stream);
+  if (cudaLaunchKernelEx(&cfg, kern, tq, tk, tvt, args, v_descale) != cudaSuccess) {
+    cudaGetLastError();
+    return ATTN_ERR_CUDA;
+  }
+  return ATTN_OK;
+}
 
 extern "C" long long attn_kmeans_workspace_floats(int N, int K) {
   if (N <= 0 || K <= 0) return -1;
