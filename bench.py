@@ -424,6 +424,98 @@ def run_general(args, w):
     }
 
 
+# ----------------------------------------------------------- FP8 path -----
+FP8_SUFFIX = "_fp8"
+
+
+def run_fp8(args, w):
+    """The FP8 attention on a square workload's shapes: the attention alone
+    (the line's value) and the bf16 -> E4M3 conversion of Q, K and V^T that
+    feeds it (conversion_ms, and the metric with the conversion included)."""
+    import tiled_attention_forward_sm_b200 as tab
+    world, rank, local = dist_env()
+    if world > 1:
+        raise SystemExit("FP8 workloads run on one GPU")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    q_h, k_h, v_h = make_workload_inputs(w)
+    q, k, v = (t.to(dev) for t in (q_h, k_h, v_h))
+    stream = torch.cuda.current_stream(dev)
+    lib = tab.library()
+    q8 = torch.empty(q.shape, dtype=torch.uint8, device=dev)
+    k8 = torch.empty_like(q8)
+    vt8 = torch.empty((w.B, w.H, w.d, w.N), dtype=torch.uint8, device=dev)
+    o = torch.empty_like(q)
+    lse = torch.empty((w.B, w.H, w.N), dtype=torch.float32, device=dev)
+    sh = stream.cuda_stream
+    BH = w.B * w.H
+    import ctypes
+
+    def convert():
+        for src, dst, tr in ((q, q8, 0), (k, k8, 0), (v, vt8, 1)):
+            rc = lib.attn_quantize_e4m3(src.data_ptr(), dst.data_ptr(), BH, w.N, w.d,
+                                        ctypes.c_float(1.0), tr, sh)
+            assert rc == 0, rc
+
+    def attend():
+        rc = lib.attn_fwd_fp8(q8.data_ptr(), k8.data_ptr(), vt8.data_ptr(), o.data_ptr(),
+                              lse.data_ptr(), w.B, w.H, w.N, w.d, int(w.causal),
+                              ctypes.c_float(w.scale), ctypes.c_float(1.0), ctypes.c_float(1.0),
+                              ctypes.c_float(1.0), sh)
+        assert rc == 0, rc
+
+    def timed(fn, steps):
+        for _ in range(args.warmup):
+            fn()
+        torch.cuda.synchronize(dev)
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(steps):
+            fn()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        return e0.elapsed_time(e1) / steps
+
+    convert()
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES", "")
+    smi_id = vis.split(",")[local].strip() if vis and len(vis.split(",")) > local else str(local)
+    sampler = ClockSampler(smi_id)
+    sampler.start()
+    ms_attn = timed(attend, args.steps)
+    clocks = sampler.stop()
+    ms_conv = timed(convert, max(1, args.steps // 4))
+    status = tab.last_device_error(stream)
+    if status != 0:
+        raise SystemExit(f"device status {status}: {tab.strerror(status)}")
+    tflops = w.flops / (ms_attn * 1e-3) / 1e12
+    peaks, peak_kind = load_peaks()
+    conv_bytes = 3 * w.rows * w.d * 3  # 2 bytes read, 1 written per element
+    return {
+        "metric": METRIC.replace("(bf16, d=128)", "(FP8 E4M3 operands, d=128)"),
+        "value": round(tflops, 2), "unit": UNIT, "n_gpus": 1, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms_attn, 4), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "e4m3",
+        "data": "synthetic (the square workload's seeded bf16 inputs, converted to E4M3)",
+        "config": {"workload": w.name + FP8_SUFFIX, "B": w.B, "H": w.H, "N": w.N, "d": w.d,
+                   "causal": w.causal, "flops_per_step": w.flops,
+                   "descales": [1.0, 1.0, 1.0],
+                   "l2": "inputs larger than L2; no flush"},
+        "roofline": {"bound": "tensor", "achieved": round(tflops, 2),
+                     "peak": 2.0 * float(peaks["bf16_tflops"]), "unit": "TFLOP/s",
+                     "frac": round(tflops / (2.0 * float(peaks["bf16_tflops"])), 4),
+                     "peak_source": f"{peak_kind} bf16 burst x 2 (the nominal fp8:bf16 ratio)",
+                     "traffic": None},
+        "conversion": {"ms": round(ms_conv, 4), "launches": 3,
+                       "gbs": round(conv_bytes / (ms_conv * 1e-3) / 1e9, 1),
+                       "hbm_frac": round(conv_bytes / (ms_conv * 1e-3) / 1e9 /
+                                         float(peaks["hbm_gbs"]), 4),
+                       "tflops_with_conversion": round(w.flops / ((ms_attn + ms_conv) * 1e-3)
+                                                       / 1e12, 2)},
+        "e2e": None, "gpu_launches": args.steps, "clocks": clocks, "kernel_sha": kernel_sha(),
+    }
+
+
 # ------------------------------------------------- k-means assignment -----
 def run_kmeans(args, w):
     import ctypes
@@ -540,14 +632,19 @@ def main():
     ap.add_argument("--impl", choices=["b200", "reference"], default="b200")
     ap.add_argument("--workload", default=BENCH_WORKLOAD,
                     choices=sorted(WORKLOADS) + sorted(GENERAL_WORKLOADS) +
-                    sorted(KMEANS_WORKLOADS))
+                    sorted(KMEANS_WORKLOADS) +
+                    sorted(n + FP8_SUFFIX for n, w_ in WORKLOADS.items() if w_.d == 128))
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
-    if args.workload in KMEANS_WORKLOADS:
+    if args.workload.endswith(FP8_SUFFIX):
+        if args.impl == "reference":
+            ap.error("--impl reference times the bf16 workloads only")
+        line = run_fp8(args, WORKLOADS[args.workload[: -len(FP8_SUFFIX)]])
+    elif args.workload in KMEANS_WORKLOADS:
         if args.impl == "reference":
             ap.error("--impl reference times the attention workloads only")
         line = run_kmeans(args, KMEANS_WORKLOADS[args.workload])

@@ -235,6 +235,18 @@ int attn_fwd_fp8(const void* q, const void* k, const void* vt, void* o, float* l
                  float k_descale, float v_descale, attn_stream_t stream);
 
 /*
+ * attn_quantize_e4m3 -- the conversion the FP8 path's inputs go through:
+ * dst = E4M3(src * inv_descale), rounded to nearest even, saturated at
+ * +-448.  src is device bf16 [BH, N, d]; dst device bytes, [BH, N, d]
+ * (transpose = 0, for Q and K) or [BH, d, N] (transpose != 0, the V^T
+ * operand; N must be a multiple of 16).  d 64 or 128; BH <= 65535; both
+ * pointers 16-byte aligned, not overlapping.  Errors and asynchrony as
+ * attn_fwd.
+ */
+int attn_quantize_e4m3(const void* src, void* dst, int BH, int N, int d, float inv_descale,
+                       int transpose, attn_stream_t stream);
+
+/*
  * attn_kmeans_assign -- the assignment step of k-means (page lefilia.fr,
  * Flash-KMeans item, "FlashAssign"): every point goes to its nearest
  * centroid, computed tile by tile without writing the N x K distance

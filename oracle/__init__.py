@@ -289,6 +289,31 @@ def round_e4m3(x: np.ndarray) -> np.ndarray:
     return np.sign(x) * np.minimum(r, 448.0)
 
 
+def e4m3_encode(x) -> np.ndarray:
+    """E4M3 bit patterns of float64 values that are already E4M3 values
+    (e.g. ``round_e4m3``'s results): sign bit, then exponent and mantissa
+    fields (subnormals for magnitudes below 2^-6; the sign of a zero is
+    kept, -0 encodes as 0x80)."""
+    x = np.asarray(x, dtype=np.float64)
+    sign = np.signbit(x).astype(np.int64) << 7
+    a = np.abs(x)
+    with np.errstate(divide="ignore"):
+        e = np.floor(np.log2(np.where(a > 0, a, 1.0))).astype(np.int64)
+    normal = a >= 2.0 ** -6
+    mant_n = np.round((a / np.exp2(e.astype(np.float64)) - 1.0) * 8).astype(np.int64)
+    code_n = ((e + 7) << 3) | mant_n
+    code_s = np.round(a / 2.0 ** -9).astype(np.int64)  # subnormal: m * 2^-9
+    code = np.where(normal, code_n, code_s)
+    code = np.where(a == 0, 0, code)
+    return (code | sign).astype(np.uint8)
+
+
+def quantize_e4m3(x_bits, inv_descale: float):
+    """E4M3 codes of bf16 values times inv_descale, rounded to nearest even
+    and saturated at +-448: the conversion the FP8 path's inputs go through."""
+    return e4m3_encode(round_e4m3(bf16_bits_to_f64(x_bits) * float(inv_descale)))
+
+
 def bf16_bits_to_f64(bits) -> np.ndarray:
     """Exact widening of bf16 bit patterns to float64."""
     bits = np.asarray(bits, dtype=np.uint16)

@@ -240,3 +240,14 @@ def test_fp8_rejections_before_any_cuda_call(lib):
     assert f(q, k, v, o, l, 1, 1, 1024, 128, 1, 0.1, 1.0, 1.0, float("nan"), None) == -1
     assert f(q + 8, k, v, o, l, *good, None) == -3
     assert f(q, k, v, q, l, *good, None) == -1                                    # o over q
+
+
+def test_quantize_rejections_before_any_cuda_call(lib):
+    f = lib.attn_quantize_e4m3
+    s, d_ = A, A + (1 << 26)
+    assert f(None, d_, 1, 128, 128, 1.0, 0, None) == -1
+    assert f(s, d_, 1, 128, 96, 1.0, 0, None) == -2         # d
+    assert f(s, d_, 1, 100, 128, 1.0, 1, None) == -2        # transposed N % 16
+    assert f(s, d_, 1, 128, 128, 0.0, 0, None) == -1        # scale
+    assert f(s + 8, d_, 1, 128, 128, 1.0, 0, None) == -3
+    assert f(s, s + 64, 1, 128, 128, 1.0, 0, None) == -1    # overlap

@@ -80,3 +80,25 @@ def test_fp8_rejects_unsupported_shapes():
     x64 = torch.zeros(1, 1, 128, 64, dtype=torch.uint8, device="cuda")
     with pytest.raises(tab.AttnError):
         tab.attn_fwd_fp8(x64, x64, torch.zeros(1, 1, 64, 128, dtype=torch.uint8, device="cuda"))
+
+
+@pytest.mark.parametrize("transpose", [False, True])
+@pytest.mark.parametrize("N,d", [(256, 128), (1040, 64), (96, 128)])
+def test_quantize_is_bit_exact(oracle_mod, transpose, N, d):
+    """The conversion kernel's E4M3 bytes equal the oracle's codes (power-of
+    -two scales: the fp32 and fp64 products agree), in either layout."""
+    B, H = 2, 3
+    x = make_qkv(B, H, N, d, seed=N + d)[0] * 3.0
+    x = x.to(torch.bfloat16)
+    for inv in (1.0, 8.0, 0.25):
+        got = tab.quantize_e4m3(x.cuda(), inv, transpose).cpu().numpy()
+        ref = oracle_mod.quantize_e4m3(bf16_bits(x), inv)
+        if transpose:
+            ref = np.ascontiguousarray(ref.transpose(0, 1, 3, 2))
+        np.testing.assert_array_equal(got, ref)
+
+
+def test_quantize_saturates_large_values(oracle_mod):
+    x = torch.tensor([[1000.0, -1000.0, 447.0, 3e-4] * 32], dtype=torch.bfloat16)
+    got = tab.quantize_e4m3(x.cuda(), 1.0).cpu().numpy()
+    np.testing.assert_array_equal(got, oracle_mod.quantize_e4m3(bf16_bits(x), 1.0))

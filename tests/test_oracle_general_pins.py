@@ -265,3 +265,23 @@ def test_model_with_e4m3_weights_stays_inside_its_bound(oracle_mod):
         W /= W.sum(1, keepdims=True)
         A = W @ np.abs(V)
         assert (np.abs(o_m - o_ex) <= 2.0 ** -4 * A + 1e-3).all()
+
+
+def test_e4m3_encoding_round_trips_every_code(oracle_mod):
+    """Encoding the decoded value of every finite code gives the code back
+    (both zeros and the subnormals included)."""
+    codes = np.arange(256, dtype=np.uint8)
+    vals = oracle_mod.e4m3_bits_to_f64(codes)
+    ok = ~np.isnan(vals)
+    np.testing.assert_array_equal(oracle_mod.e4m3_encode(vals[ok]), codes[ok])
+
+
+def test_quantize_matches_torch_cast(oracle_mod):
+    """bf16 * 2^k -> E4M3 codes equal torch's cast of the same products
+    (in range: torch's cast does not saturate)."""
+    import torch
+    x = torch.randn(50000, generator=torch.Generator().manual_seed(3)).bfloat16()
+    for inv in (1.0, 4.0, 0.125):
+        q = oracle_mod.quantize_e4m3(bf16_bits(x), inv)
+        ref = (x.float() * inv).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+        np.testing.assert_array_equal(q, ref)

@@ -67,6 +67,8 @@ def library():
         lib.attn_fwd_splitkv.argtypes = [vp] * 5 + [i] * 8 + [f, i, vp, vp, vp]
         lib.attn_fwd_fp8.restype = i
         lib.attn_fwd_fp8.argtypes = [vp] * 5 + [i] * 5 + [f, f, f, f, vp]
+        lib.attn_quantize_e4m3.restype = i
+        lib.attn_quantize_e4m3.argtypes = [vp, vp, i, i, i, f, i, vp]
         lib.attn_kmeans_assign.restype = i
         lib.attn_kmeans_assign.argtypes = [vp, vp, vp, vp, vp, i, i, i, vp]
         lib.attn_kmeans_workspace_floats.restype = ctypes.c_longlong
@@ -372,3 +374,25 @@ def attn_fwd_fp8(q, k, vt, causal: bool = False, scale: float | None = None,
     if rc != ATTN_OK:
         raise AttnError(rc, "attn_fwd_fp8")
     return o, lse
+
+
+def quantize_e4m3(x, inv_descale: float = 1.0, transpose: bool = False, stream=None):
+    """bf16 [B, H, N, d] (or [rows, d]) -> E4M3 bytes (uint8) of x * inv_descale, in the
+    same layout or, with ``transpose``, as [B, H, d, N] (see attn_quantize_e4m3)."""
+    if x.dim() == 2:
+        BH, N, d = 1, int(x.shape[0]), int(x.shape[1])
+        out_shape = (d, N) if transpose else (N, d)
+    elif x.dim() == 4:
+        B, H, N, d = (int(v) for v in x.shape)
+        BH = B * H
+        out_shape = (B, H, d, N) if transpose else (B, H, N, d)
+    else:
+        raise ValueError("x must be [rows, d] or [B, H, N, d]")
+    _check(x, "x", torch.bfloat16, x.shape)
+    out = torch.empty(out_shape, dtype=torch.uint8, device=x.device)
+    rc = library().attn_quantize_e4m3(x.data_ptr(), out.data_ptr(), BH, N, d,
+                                      float(inv_descale), int(bool(transpose)),
+                                      _stream_handle(stream))
+    if rc != ATTN_OK:
+        raise AttnError(rc, "attn_quantize_e4m3")
+    return out

@@ -18,6 +18,7 @@
 #include "attn_fwd_wide_kernel.cuh"
 #include "kmeans_assign_kernel.cuh"
 #include "attn_fwd_fp8_kernel.cuh"
+#include "quantize_kernel.cuh"
 
 namespace attn_b200 {
 
@@ -707,6 +708,39 @@ extern "C" int attn_fwd_fp8(const void* q, const void* k, const void* vt, void* 
     cudaGetLastError();
     return ATTN_ERR_CUDA;
   }
+  return ATTN_OK;
+}
+
+extern "C" int attn_quantize_e4m3(const void* src, void* dst, int BH, int N, int d,
+                                  float inv_descale, int transpose, attn_stream_t stream) {
+  if (!src || !dst || BH <= 0 || N <= 0) return ATTN_ERR_INVALID_ARG;
+  if (!std::isfinite(inv_descale) || !(inv_descale > 0.f)) return ATTN_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
+  if (transpose && N % 16 != 0) return ATTN_ERR_UNSUPPORTED;
+  const uint64_t elems = static_cast<uint64_t>(BH) * N * d;
+  if (elems >= (1ull << 40) || BH > 65535) return ATTN_ERR_UNSUPPORTED;
+  if ((reinterpret_cast<uintptr_t>(src) | reinterpret_cast<uintptr_t>(dst)) & 15u)
+    return ATTN_ERR_MISALIGNED;
+  if (ranges_overlap(src, elems * 2, dst, elems)) return ATTN_ERR_INVALID_ARG;
+  DeviceState* st = nullptr;
+  const int rc = device_state(&st);
+  if (rc != ATTN_OK) return rc;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (!transpose) {
+    const long long n16 = static_cast<long long>(elems / 16);
+    long long blocks = (n16 + 255) / 256;
+    const long long cap = 8LL * st->num_sms;
+    if (blocks > cap) blocks = cap;
+    quant::e4m3_kernel<<<static_cast<unsigned>(blocks), 256, 0, s>>>(
+        static_cast<const uint4*>(src), static_cast<uint4*>(dst), n16, inv_descale);
+  } else {
+    const dim3 grid(static_cast<unsigned>((N + 63) / 64), static_cast<unsigned>(d / 64),
+                    static_cast<unsigned>(BH));
+    quant::e4m3_transpose_kernel<<<grid, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(src),
+                                                      static_cast<uint8_t*>(dst), N, d,
+                                                      inv_descale);
+  }
+  if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
   return ATTN_OK;
 }
 
