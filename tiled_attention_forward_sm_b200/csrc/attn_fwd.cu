@@ -16,9 +16,7 @@
 #include "attn_combine_kernel.cuh"
 #include "attn_fwd_kernel.cuh"
 #include "attn_fwd_wide_kernel.cuh"
-#include "kmeans_assign_kernel.cuh"
-#include "attn_fwd_fp8_kernel.cuh"
-#include "quantize_kernel.cuh"
+#include "host_common.h"
 
 namespace attn_b200 {
 
@@ -29,8 +27,7 @@ __device__ int g_attn_status = 0;
 // finished}); the launch's last CTA resets it to zero.  Launches that run
 // at the same time use different slots as long as fewer than kQueueSlots
 // of them overlap.
-constexpr int kQueueSlots = 256;
-__device__ int g_attn_queue[2 * kQueueSlots];
+__device__ int g_attn_queue[2 * host::kQueueSlots];
 
 // Scratch of attn_fwd_noalloc: a fixed array this library owns for as long
 // as it is loaded (every GPU that loads it keeps these bytes until exit).
@@ -43,25 +40,28 @@ constexpr int kNoAllocQueueBytes = 2 * static_cast<int>(sizeof(int));
 static_assert(kNoAllocQueueBytes <= kNoAllocScratchBytes, "queue slot must fit the scratch");
 static __device__ __align__(256) int g_attn_noalloc_scratch[kNoAllocScratchBytes / sizeof(int)];
 
-namespace {
+namespace host {
 
 constexpr int kMaxDevices = 64;
-// Most key slices of one split-KV launch (and parts of one merge).
-constexpr int kMaxSplits = 256;
 
-struct DeviceState {
-  bool checked = false;
-  bool usable = false;
-  int* status = nullptr;  // device address of g_attn_status
-  int* queue = nullptr;   // device address of g_attn_queue
-  int* noalloc_scratch = nullptr;  // device address of g_attn_noalloc_scratch
-  int num_sms = 0;
-  std::atomic<unsigned> launches{0};
-};
-
+namespace {
 std::mutex g_mu;
 DeviceState g_dev[kMaxDevices];
 PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+}  // namespace
+
+int* next_queue_slot(DeviceState& st) {
+  return st.queue + 2 * static_cast<int>(st.launches.fetch_add(1) % kQueueSlots);
+}
+
+CUresult encode_tiled(CUtensorMap* m, CUtensorMapDataType type, const void* ptr,
+                      const cuuint64_t* dims, const cuuint64_t* strides, const cuuint32_t* box) {
+  cuuint32_t estr[3] = {1, 1, 1};
+  return g_encode(m, type, 3, const_cast<void*>(ptr), const_cast<cuuint64_t*>(dims),
+                  const_cast<cuuint64_t*>(strides), const_cast<cuuint32_t*>(box), estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+}
 
 // Per-device one-time set-up: capability check and the status word address.
 int device_state(DeviceState** out) {
@@ -129,12 +129,10 @@ int make_tmap_heads(CUtensorMap* m, const void* ptr, int Z, int N, int d) {
   cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2,
                            static_cast<cuuint64_t>(N) * static_cast<cuuint64_t>(d) * 2};
   cuuint32_t box[3] = {64, 128, 1};
-  cuuint32_t estr[3] = {1, 1, 1};
-  CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims,
-                        strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                        CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS ? ATTN_OK : ATTN_ERR_CUDA;
+  return encode_tiled(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, ptr, dims, strides, box) ==
+                 CUDA_SUCCESS
+             ? ATTN_OK
+             : ATTN_ERR_CUDA;
 }
 
 // Token-major 3-D view [T][Hx][d] of a packed [T, Hx, d] bf16 tensor; boxes
@@ -148,18 +146,39 @@ int make_tmap_tokens(CUtensorMap* m, const void* ptr, int T, int Hx, int d) {
   cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2,
                            static_cast<cuuint64_t>(Hx) * static_cast<cuuint64_t>(d) * 2};
   cuuint32_t box[3] = {64, 1, 128};
-  cuuint32_t estr[3] = {1, 1, 1};
-  CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims,
-                        strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                        CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS ? ATTN_OK : ATTN_ERR_CUDA;
+  return encode_tiled(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, ptr, dims, strides, box) ==
+                 CUDA_SUCCESS
+             ? ATTN_OK
+             : ATTN_ERR_CUDA;
 }
 
 bool ranges_overlap(const void* a, size_t na, const void* b, size_t nb) {
   const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
   return x < y + nb && y < x + na;
 }
+
+bool scale_ok(float scale) { return std::isfinite(scale) && scale > 0.f; }
+
+// Output buffers must not overlap the inputs or one another.
+bool outputs_disjoint(const void* const* outs, const size_t* out_bytes, int n_out,
+                      const void* const* ins, const size_t* in_bytes, int n_in) {
+  for (int i = 0; i < n_out; ++i) {
+    for (int j = 0; j < n_in; ++j)
+      if (ranges_overlap(outs[i], out_bytes[i], ins[j], in_bytes[j])) return false;
+    for (int j = i + 1; j < n_out; ++j)
+      if (ranges_overlap(outs[i], out_bytes[i], outs[j], out_bytes[j])) return false;
+  }
+  return true;
+}
+
+}  // namespace host
+
+using namespace host;
+
+namespace {
+
+// Most key slices of one split-KV launch (and parts of one merge).
+constexpr int kMaxSplits = 256;
 
 // One attention launch, in either layout (see KernelArgs).  Checked by the
 // entry points before it reaches launch().
@@ -233,9 +252,7 @@ int launch(const Problem& p, cudaStream_t stream, DeviceState& st, int* queue = 
     const int want = (2 * st.num_sms + per_head - 1) / per_head;
     args.win_heads = want < 1 ? 1 : (want > args.BH ? args.BH : want);
   }
-  args.queue = queue != nullptr
-                   ? queue
-                   : st.queue + 2 * static_cast<int>(st.launches.fetch_add(1) % kQueueSlots);
+  args.queue = queue != nullptr ? queue : next_queue_slot(st);
   args.scale_log2 = p.scale * 1.4426950408889634f;
   args.status = st.status;
 
@@ -339,20 +356,6 @@ int run_combine(const float* o_parts, const float* lse_parts, int G, long long r
 }
 
 bool head_dim_ok(int d) { return d == 64 || d == 96 || d == 128 || d == 256; }
-
-bool scale_ok(float scale) { return std::isfinite(scale) && scale > 0.f; }
-
-// Output buffers must not overlap the inputs or one another.
-bool outputs_disjoint(const void* const* outs, const size_t* out_bytes, int n_out,
-                      const void* const* ins, const size_t* in_bytes, int n_in) {
-  for (int i = 0; i < n_out; ++i) {
-    for (int j = 0; j < n_in; ++j)
-      if (ranges_overlap(outs[i], out_bytes[i], ins[j], in_bytes[j])) return false;
-    for (int j = i + 1; j < n_out; ++j)
-      if (ranges_overlap(outs[i], out_bytes[i], outs[j], out_bytes[j])) return false;
-  }
-  return true;
-}
 
 // Checks of a dense problem with per-head layout (attn_fwd, attn_fwd_chunk).
 int check_dense(const Problem& p) {
@@ -549,231 +552,6 @@ extern "C" int attn_combine(const float* o_parts, const float* lse_parts, int G,
   const int rc = device_state(&st);
   if (rc != ATTN_OK) return rc;
   return run_combine(o_parts, lse_parts, G, rows, d, o, lse, o_fp32 ? 1 : 0, stream, *st);
-}
-
-namespace attn_b200 {
-namespace {
-
-template <int D>
-int launch_kmeans(const void* x, const void* cent, float* ws, int32_t* assign, float* best,
-                  int N, int K, cudaStream_t stream, DeviceState& st) {
-  using KC = kmeans::KConfig<D>;
-  CUtensorMap tx, tc;
-  if (make_tmap_heads(&tx, x, 1, N, D) || make_tmap_heads(&tc, cent, 1, K, D)) return ATTN_ERR_CUDA;
-  const int k_tiles = (K + kmeans::kTileN - 1) / kmeans::kTileN;
-  const int64_t k_pad = static_cast<int64_t>(k_tiles) * kmeans::kTileN;
-  float* cnorm = ws;
-  float* xnorm = ws + k_pad;
-  auto norms = [&](const void* rows, int64_t n, int64_t n_pad, float* out) {
-    const int64_t blocks64 = (n_pad + 7) / 8;  // 8 warps (rows) per block
-    const int blocks = static_cast<int>(blocks64 < 8LL * st.num_sms ? blocks64 : 8LL * st.num_sms);
-    kmeans::row_norms_kernel<<<blocks, 256, 0, stream>>>(
-        static_cast<const __nv_bfloat16*>(rows), n, n_pad, D, out);
-    return cudaGetLastError() == cudaSuccess;
-  };
-  if (!norms(cent, K, k_pad, cnorm) || (best != nullptr && !norms(x, N, N, xnorm))) {
-    cudaGetLastError();
-    return ATTN_ERR_CUDA;
-  }
-  KernelArgs args;
-  std::memset(&args, 0, sizeof args);
-  args.H = 1;
-  args.H_kv = 1;
-  args.q_per_kv = 1;
-  args.N_q = N;
-  args.N_k = K;
-  args.n_qpairs = ((N + kBlockM - 1) / kBlockM + 1) / 2;
-  args.n_splits = 1;
-  args.split_tiles = k_tiles;
-  args.BH = 1;
-  args.n_items = args.n_qpairs;
-  args.win_heads = 1;
-  args.status = st.status;
-  args.queue = st.queue + 2 * static_cast<int>(st.launches.fetch_add(1) % kQueueSlots);
-  kmeans::AssignArgs out;
-  out.assign = assign;
-  out.best = best;
-  out.cnorm = cnorm;
-  out.xnorm = xnorm;
-  auto kern = kmeans::kmeans_assign_kernel<D>;
-  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, KC::kSmemBytes) !=
-      cudaSuccess) {
-    cudaGetLastError();
-    return ATTN_ERR_CUDA;
-  }
-  cudaLaunchConfig_t cfg;
-  std::memset(&cfg, 0, sizeof cfg);
-  const int grid = args.n_items < st.num_sms ? args.n_items : st.num_sms;
-  cfg.gridDim = dim3(static_cast<unsigned>(grid), 1, 1);
-  cfg.blockDim = dim3(kmeans::kThreads, 1, 1);
-  cfg.dynamicSmemBytes = KC::kSmemBytes;
-  cfg.stream = stream;
-  if (cudaLaunchKernelEx(&cfg, kern, tx, tc, args, out) != cudaSuccess) {
-    cudaGetLastError();
-    return ATTN_ERR_CUDA;
-  }
-  return ATTN_OK;
-}
-
-}  // namespace
-}  // namespace attn_b200
-
-namespace attn_b200 {
-namespace {
-
-// 3-D view of an 8-bit tensor: dims {inner, mid, outer}, boxes of 128 x 128
-// x 1 (128-byte rows, the 128-byte swizzle).
-int make_tmap_u8(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t mid, uint64_t outer) {
-  cuuint64_t dims[3] = {inner, mid, outer};
-  cuuint64_t strides[2] = {inner, inner * mid};
-  cuuint32_t box[3] = {128, 128, 1};
-  cuuint32_t estr[3] = {1, 1, 1};
-  CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(ptr), dims,
-                        strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                        CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS ? ATTN_OK : ATTN_ERR_CUDA;
-}
-
-}  // namespace
-}  // namespace attn_b200
-
-extern "C" int attn_fwd_fp8(const void* q, const void* k, const void* vt, void* o, float* lse,
-                            int B, int H, int N, int d, int causal, float scale, float q_descale,
-                            float k_descale, float v_descale, attn_stream_t stream) {
-  if (!q || !k || !vt || !o || !lse) return ATTN_ERR_INVALID_ARG;
-  if (B <= 0 || H <= 0 || N <= 0) return ATTN_ERR_INVALID_ARG;
-  if (!scale_ok(scale) || !scale_ok(q_descale) || !scale_ok(k_descale) || !scale_ok(v_descale))
-    return ATTN_ERR_INVALID_ARG;
-  if (d != fp8::kD) return ATTN_ERR_UNSUPPORTED;
-  // V^T rows are N bytes long: the tensor map needs them 16-byte aligned.
-  if (N % 16 != 0) return ATTN_ERR_UNSUPPORTED;
-  const uint64_t rows = static_cast<uint64_t>(B) * H * N;
-  if (rows >= (1ull << 31)) return ATTN_ERR_UNSUPPORTED;
-  const uintptr_t al = reinterpret_cast<uintptr_t>(q) | reinterpret_cast<uintptr_t>(k) |
-                       reinterpret_cast<uintptr_t>(vt) | reinterpret_cast<uintptr_t>(o);
-  if (al & 15u) return ATTN_ERR_MISALIGNED;
-  if (reinterpret_cast<uintptr_t>(lse) & 3u) return ATTN_ERR_MISALIGNED;
-  const size_t ib = rows * static_cast<size_t>(d);
-  const void* outs[2] = {o, lse};
-  const size_t out_bytes[2] = {ib * 2, rows * 4};
-  const void* ins[3] = {q, k, vt};
-  const size_t in_bytes[3] = {ib, ib, ib};
-  if (!outputs_disjoint(outs, out_bytes, 2, ins, in_bytes, 3)) return ATTN_ERR_INVALID_ARG;
-  DeviceState* st = nullptr;
-  int rc = device_state(&st);
-  if (rc != ATTN_OK) return rc;
-  CUtensorMap tq, tk, tvt;
-  const uint64_t BH = static_cast<uint64_t>(B) * H;
-  if (make_tmap_u8(&tq, q, d, N, BH) || make_tmap_u8(&tk, k, d, N, BH) ||
-      make_tmap_u8(&tvt, vt, N, d, BH))
-    return ATTN_ERR_CUDA;
-  Problem p = dense_problem(q, k, vt, o, lse, B, H, N, d, causal, scale);
-  if (problem_items(p) + st->num_sms > 0x7FFFFFFFll) return ATTN_ERR_UNSUPPORTED;
-  KernelArgs args;
-  std::memset(&args, 0, sizeof args);
-  args.o = o;
-  args.lse = lse;
-  args.H = H;
-  args.H_kv = H;
-  args.q_per_kv = 1;
-  args.N_q = N;
-  args.N_k = N;
-  args.n_qpairs = ((N + kBlockM - 1) / kBlockM + 1) / 2;
-  args.n_splits = 1;
-  args.split_tiles = (N + kBlockN - 1) / kBlockN;
-  args.BH = B * H;
-  args.n_items = static_cast<int>(problem_items(p));
-  {
-    const int want = (2 * st->num_sms + args.n_qpairs - 1) / args.n_qpairs;
-    args.win_heads = want < 1 ? 1 : (want > args.BH ? args.BH : want);
-  }
-  args.scale_log2 = scale * q_descale * k_descale * 1.4426950408889634f;
-  args.status = st->status;
-  args.queue = st->queue + 2 * static_cast<int>(st->launches.fetch_add(1) % kQueueSlots);
-  auto kern = causal ? fp8::attn_fwd_fp8_kernel<true> : fp8::attn_fwd_fp8_kernel<false>;
-  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, fp8::kSmemBytes) !=
-      cudaSuccess) {
-    cudaGetLastError();
-    return ATTN_ERR_CUDA;
-  }
-  cudaLaunchConfig_t cfg;
-  std::memset(&cfg, 0, sizeof cfg);
-  const int grid = args.n_items < st->num_sms ? args.n_items : st->num_sms;
-  cfg.gridDim = dim3(static_cast<unsigned>(grid), 1, 1);
-  cfg.blockDim = dim3(kThreads, 1, 1);
-  cfg.dynamicSmemBytes = fp8::kSmemBytes;
-  cfg.stream = static_cast<cudaStream_t>(stream);
-  if (cudaLaunchKernelEx(&cfg, kern, tq, tk, tvt, args, v_descale) != cudaSuccess) {
-    cudaGetLastError();
-    return ATTN_ERR_CUDA;
-  }
-  return ATTN_OK;
-}
-
-extern "C" int attn_quantize_e4m3(const void* src, void* dst, int BH, int N, int d,
-                                  float inv_descale, int transpose, attn_stream_t stream) {
-  if (!src || !dst || BH <= 0 || N <= 0) return ATTN_ERR_INVALID_ARG;
-  if (!std::isfinite(inv_descale) || !(inv_descale > 0.f)) return ATTN_ERR_INVALID_ARG;
-  if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
-  if (transpose && N % 16 != 0) return ATTN_ERR_UNSUPPORTED;
-  const uint64_t elems = static_cast<uint64_t>(BH) * N * d;
-  if (elems >= (1ull << 40) || BH > 65535) return ATTN_ERR_UNSUPPORTED;
-  if ((reinterpret_cast<uintptr_t>(src) | reinterpret_cast<uintptr_t>(dst)) & 15u)
-    return ATTN_ERR_MISALIGNED;
-  if (ranges_overlap(src, elems * 2, dst, elems)) return ATTN_ERR_INVALID_ARG;
-  DeviceState* st = nullptr;
-  const int rc = device_state(&st);
-  if (rc != ATTN_OK) return rc;
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (!transpose) {
-    const long long n16 = static_cast<long long>(elems / 16);
-    long long blocks = (n16 + 255) / 256;
-    const long long cap = 8LL * st->num_sms;
-    if (blocks > cap) blocks = cap;
-    quant::e4m3_kernel<<<static_cast<unsigned>(blocks), 256, 0, s>>>(
-        static_cast<const uint4*>(src), static_cast<uint4*>(dst), n16, inv_descale);
-  } else {
-    const dim3 grid(static_cast<unsigned>((N + 63) / 64), static_cast<unsigned>(d / 64),
-                    static_cast<unsigned>(BH));
-    quant::e4m3_transpose_kernel<<<grid, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(src),
-                                                      static_cast<uint8_t*>(dst), N, d,
-                                                      inv_descale);
-  }
-  if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
-  return ATTN_OK;
-}
-
-extern "C" long long attn_kmeans_workspace_floats(int N, int K) {
-  if (N <= 0 || K <= 0) return -1;
-  return (static_cast<long long>(K) + kmeans::kTileN - 1) / kmeans::kTileN * kmeans::kTileN + N;
-}
-
-extern "C" int attn_kmeans_assign(const void* x, const void* centroids, float* ws,
-                                  int32_t* assign, float* best, int N, int K, int d,
-                                  attn_stream_t stream) {
-  if (!x || !centroids || !ws || !assign) return ATTN_ERR_INVALID_ARG;
-  if (N <= 0 || K <= 0) return ATTN_ERR_INVALID_ARG;
-  if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
-  if (N >= (1 << 30) || K >= (1 << 30)) return ATTN_ERR_UNSUPPORTED;
-  if ((reinterpret_cast<uintptr_t>(x) | reinterpret_cast<uintptr_t>(centroids) |
-       reinterpret_cast<uintptr_t>(ws)) & 15u)
-    return ATTN_ERR_MISALIGNED;
-  if ((reinterpret_cast<uintptr_t>(assign) | reinterpret_cast<uintptr_t>(best)) & 3u)
-    return ATTN_ERR_MISALIGNED;
-  const size_t xb = static_cast<size_t>(N) * d * 2, cb = static_cast<size_t>(K) * d * 2;
-  const size_t wb = static_cast<size_t>(attn_kmeans_workspace_floats(N, K)) * 4;
-  const void* outs[3] = {ws, assign, best};
-  const size_t out_bytes[3] = {wb, static_cast<size_t>(N) * 4, best ? static_cast<size_t>(N) * 4 : 0};
-  const void* ins[2] = {x, centroids};
-  const size_t in_bytes[2] = {xb, cb};
-  if (!outputs_disjoint(outs, out_bytes, 3, ins, in_bytes, 2)) return ATTN_ERR_INVALID_ARG;
-  DeviceState* st = nullptr;
-  const int rc = device_state(&st);
-  if (rc != ATTN_OK) return rc;
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
-  return d == 128 ? launch_kmeans<128>(x, centroids, ws, assign, best, N, K, s, *st)
-                  : launch_kmeans<64>(x, centroids, ws, assign, best, N, K, s, *st);
 }
 
 // Allocation-free entry point (include/attn_b200.h): same kernel, work

@@ -994,8 +994,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 // arrives on.  After limit_ns the wait gives up, writes the timeout code to
 // the status word and returns; the CTA exits normally and the context stays
 // usable.
-__global__ void __launch_bounds__(32, 1) wait_timeout_selftest_kernel(int* status,
-                                                                    uint64_t limit_ns) {
+static __global__ void __launch_bounds__(32, 1) wait_timeout_selftest_kernel(int* status,
+                                                                           uint64_t limit_ns) {
   __shared__ uint64_t never;
   __shared__ int abort_flag;
   Shared sh = {};
