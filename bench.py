@@ -47,16 +47,19 @@ UNIT = "TFLOPS"
 FALLBACK_PEAK = {"bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "hbm_gbs": 6650.0}
 DATASHEET_BF16_TFLOPS = 2250.0
 PROFILE_FILE = os.path.join(ROOT, "profiles", "attn_fwd_b2h32n8192d128_causal.txt")
+PAIR_PROFILE_FILE = os.path.join(ROOT, "profiles", "attn_fwd_pair_b2h32n8192d128_causal.txt")
 KERNEL_SOURCES = [os.path.join(ROOT, "tiled_attention_forward_sm_b200", "csrc", f)
                   for f in ("attn_fwd_kernel.cuh", "ptx.cuh", "attn_fwd.cu")]
+PAIR_SOURCES = KERNEL_SOURCES + [os.path.join(ROOT, "tiled_attention_forward_sm_b200", "csrc", f)
+                                 for f in ("attn_fwd_pair_kernel.cuh", "pair.cu")]
 CLOCK_QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
                "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
                "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
 
-def kernel_sha() -> str:
+def kernel_sha(sources=None) -> str:
     h = hashlib.sha256()
-    for p in KERNEL_SOURCES:
+    for p in sources or KERNEL_SOURCES:
         with open(p, "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
@@ -71,18 +74,18 @@ def load_peaks():
     return dict(FALLBACK_PEAK), "fallback"
 
 
-def load_traffic(workload_name: str):
+def load_traffic(workload_name: str, profile_file: str = PROFILE_FILE, sources=None):
     """dram read+write bytes per launch from the committed ncu summary of the
     bench workload, if it was taken on the current kernel sources; else None."""
-    if workload_name != BENCH_WORKLOAD or not os.path.exists(PROFILE_FILE):
+    if workload_name != BENCH_WORKLOAD or not os.path.exists(profile_file):
         return None
     fields = {}
-    with open(PROFILE_FILE) as f:
+    with open(profile_file) as f:
         for line in f:
             if ":" in line and not line.startswith("#"):
                 k, v = line.split(":", 1)
                 fields[k.strip()] = v.strip()
-    if fields.get("kernel_sha") != kernel_sha():
+    if fields.get("kernel_sha") != kernel_sha(sources):
         return None
     try:
         return int(fields["dram_read_write_bytes_per_launch"])
@@ -202,8 +205,11 @@ def run_b200(args, w):
     lse = torch.empty((w.B, w.H, w.N), dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream(dev)
 
+    pair = args.kernel == "pair"
+    fwd_into = tab.attn_fwd_pair_into if pair else tab.attn_fwd_into
+
     def step():
-        tab.attn_fwd_into(q, k, v, o, lse, causal=w.causal, scale=w.scale, stream=stream)
+        fwd_into(q, k, v, o, lse, causal=w.causal, scale=w.scale, stream=stream)
 
     vis = os.environ.get("CUDA_VISIBLE_DEVICES", "")
     smi_id = vis.split(",")[local].strip() if vis and len(vis.split(",")) > local else str(local)
@@ -230,13 +236,26 @@ def run_b200(args, w):
     if status != 0:
         raise SystemExit(f"device status {status}: {tab.strerror(status)}")
 
-    # end to end: host buffers through the C ABI host entry point
+    # end to end: host buffers through the C ABI host entry point (the pair
+    # kernel: pinned copies in and out around attn_fwd_pair on the stream)
     q_p, k_p, v_p = (t.pin_memory() for t in (q_h, k_h, v_h))
     o_p = torch.empty_like(q_p).pin_memory()
     lse_p = torch.empty((w.B, w.H, w.N), dtype=torch.float32).pin_memory()
     e2e_steps = max(1, min(args.steps, args.e2e_steps))
+
+    def e2e_step():
+        if not pair:
+            tab.attn_fwd_host(q_p, k_p, v_p, o_p, lse_p, q, k, v, o, lse, w.causal, w.scale,
+                              stream)
+            return
+        for dst, src in ((q, q_p), (k, k_p), (v, v_p)):
+            dst.copy_(src, non_blocking=True)
+        step()
+        o_p.copy_(o, non_blocking=True)
+        lse_p.copy_(lse, non_blocking=True)
+
     for _ in range(min(args.warmup, 3)):
-        tab.attn_fwd_host(q_p, k_p, v_p, o_p, lse_p, q, k, v, o, lse, w.causal, w.scale, stream)
+        e2e_step()
     if pg:
         torch.distributed.barrier()
     torch.cuda.synchronize(dev)
@@ -244,7 +263,7 @@ def run_b200(args, w):
     f1 = torch.cuda.Event(enable_timing=True)
     f0.record(stream)
     for _ in range(e2e_steps):
-        tab.attn_fwd_host(q_p, k_p, v_p, o_p, lse_p, q, k, v, o, lse, w.causal, w.scale, stream)
+        e2e_step()
     f1.record(stream)
     torch.cuda.synchronize(dev)
     e2e_ms = f0.elapsed_time(f1) / e2e_steps
@@ -266,7 +285,8 @@ def run_b200(args, w):
     peak = float(peaks["bf16_tflops"])
     achieved = w.flops / (ms_step * 1e-3) / 1e12  # per launch, this GPU
     tb = w.rows * w.d * 2
-    traffic = load_traffic(w.name)
+    sources = PAIR_SOURCES if pair else KERNEL_SOURCES
+    traffic = load_traffic(w.name, PAIR_PROFILE_FILE if pair else PROFILE_FILE, sources)
     line = {
         "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 4),
@@ -276,7 +296,8 @@ def run_b200(args, w):
                    "causal": w.causal, "scale": w.scale, "q_std": w.q_std,
                    "flops_per_step": w.flops,
                    "l2": f"inputs larger than L2: Q+K+V {3 * tb / 1e6:.0f} MB vs 126 MB; no flush",
-                   "parallelism": f"replica x{world} (independent batches)"},
+                   "parallelism": f"replica x{world} (independent batches)",
+                   "kernel": "cta_pair (attn_fwd_pair)" if pair else "one_cta (attn_fwd)"},
         "roofline": {"bound": "tensor", "achieved": round(achieved, 2),
                      "peak": peak, "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
                      "peak_source": f"{peak_kind} bf16 burst (MEASURED_PEAKS.json)"
@@ -289,10 +310,11 @@ def run_b200(args, w):
         "e2e": {"value": round(e2e_value, 2), "unit": UNIT,
                 "h2d_bytes_per_step": 3 * tb, "d2h_bytes_per_step": tb + w.rows * 4,
                 "steps": e2e_steps, "ms_per_step": round(e2e_ms, 4),
-                "api": "attn_fwd_host (pinned host buffers, copies in the timed region)"},
+                "api": ("attn_fwd_pair_into between pinned-host copies" if pair else
+                        "attn_fwd_host (pinned host buffers, copies in the timed region)")},
         "gpu_launches": args.steps,
         "clocks": clocks,
-        "kernel_sha": kernel_sha(),
+        "kernel_sha": kernel_sha(sources),
     }
     if world == 1 and not args.no_cpu_baseline:
         bits = (bf16_bits(q_h), bf16_bits(k_h), bf16_bits(v_h))
@@ -634,6 +656,9 @@ def main():
                     choices=sorted(WORKLOADS) + sorted(GENERAL_WORKLOADS) +
                     sorted(KMEANS_WORKLOADS) +
                     sorted(n + FP8_SUFFIX for n, w_ in WORKLOADS.items() if w_.d == 128))
+    ap.add_argument("--kernel", choices=["one_cta", "pair"], default="one_cta",
+                    help="bf16 workloads at d=128: attn_fwd (one CTA per SM) or attn_fwd_pair "
+                         "(clusters of two CTAs sharing each product)")
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")

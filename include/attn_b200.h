@@ -94,6 +94,23 @@ int attn_fwd_ex(const void* q, const void* k, const void* v, void* o, float* lse
                 const attn_opts* opts, attn_stream_t stream);
 
 /*
+ * attn_fwd_pair -- attn_fwd computed by pairs of CTAs on neighbouring SMs
+ * (thread-block clusters of 2) that share each tensor-core product
+ * (tcgen05.mma.cta_group::2, M = 256 query rows): each SM stages and reads
+ * half of every K and V tile instead of all of it.  The pair form of the
+ * instructions is the one named on page lecompute.fr/en/kernel-perf/
+ * flashattention-4-gpu-blackwell, section "Blackwell deplace la limite vers
+ * les autres unites".
+ *
+ * Same arguments, results (to rounding: the same arithmetic in another
+ * order of products) and errors as attn_fwd, except that d must be 128
+ * (other head dims return ATTN_ERR_UNSUPPORTED).  Allocates nothing.
+ */
+int attn_fwd_pair(const void* q, const void* k, const void* v, void* o, float* lse,
+                  int B, int H, int N, int d, int causal, float scale,
+                  attn_stream_t stream);
+
+/*
  * attn_fwd_noalloc -- attn_fwd for callers that cannot allocate device
  * memory, e.g. code running under global-mode CUDA stream capture (where
  * cudaMalloc is refused) or inside a framework whose allocator owns all

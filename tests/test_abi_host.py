@@ -251,3 +251,17 @@ def test_quantize_rejections_before_any_cuda_call(lib):
     assert f(s, d_, 1, 128, 128, 0.0, 0, None) == -1        # scale
     assert f(s + 8, d_, 1, 128, 128, 1.0, 0, None) == -3
     assert f(s, s + 64, 1, 128, 128, 1.0, 0, None) == -1    # overlap
+
+
+def test_pair_rejections_before_any_cuda_call(lib):
+    q, k, v, o, l = ptrs(128, 1, 1, 1024)
+    f = lib.attn_fwd_pair
+    assert "attn_fwd_pair" in declared_symbols()
+    assert f(q, k, v, o, l, 1, 1, 1024, 64, 1, 0.1, None) == -2                  # d
+    assert f(q, k, v, o, l, 1, 1, 1024, 96, 0, 0.1, None) == -2
+    assert f(q, k, v, o, l, 0, 1, 1024, 128, 1, 0.1, None) == -1                 # B
+    assert f(q, k, v, o, l, 1, 1, 1024, 128, 1, float("inf"), None) == -1       # scale
+    assert f(q + 8, k, v, o, l, 1, 1, 1024, 128, 1, 0.1, None) == -3
+    assert f(q, k, v, o, l + 2, 1, 1, 1024, 128, 1, 0.1, None) == -3
+    assert f(q, k, v, q, l, 1, 1, 1024, 128, 1, 0.1, None) == -1                 # o over q
+    assert f(None, k, v, o, l, 1, 1, 1024, 128, 1, 0.1, None) == -1

@@ -47,6 +47,8 @@ def library():
         lib.attn_fwd_ex.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, f, vp, vp]
         lib.attn_fwd_noalloc.restype = i
         lib.attn_fwd_noalloc.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, f, vp]
+        lib.attn_fwd_pair.restype = i
+        lib.attn_fwd_pair.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, f, vp]
         lib.attn_fwd_host.restype = i
         lib.attn_fwd_host.argtypes = [vp] * 10 + [i, i, i, i, i, f, vp]
         lib.attn_selftest_wait_timeout.restype = i
@@ -157,6 +159,36 @@ def attn_fwd_noalloc_into(q, k, v, o, lse, causal: bool = False, scale: float | 
                                     _stream_handle(stream))
     if rc != ATTN_OK:
         raise AttnError(rc, "attn_fwd_noalloc")
+
+
+def attn_fwd_pair_into(q, k, v, o, lse, causal: bool = False, scale: float | None = None,
+                       stream=None) -> None:
+    """The CTA-pair kernel (attn_fwd_pair in the header: d = 128 only), with
+    the contract of attn_fwd_into."""
+    B, H, N, d = _shape(q)
+    for name, t in (("q", q), ("k", k), ("v", v), ("o", o)):
+        if not t.is_cuda or t.dtype != torch.bfloat16 or not t.is_contiguous() or \
+                tuple(t.shape) != (B, H, N, d):
+            raise ValueError(f"{name} must be a contiguous CUDA bf16 tensor of shape {(B, H, N, d)}")
+    if not lse.is_cuda or lse.dtype != torch.float32 or not lse.is_contiguous() or \
+            tuple(lse.shape) != (B, H, N):
+        raise ValueError(f"lse must be a contiguous CUDA fp32 tensor of shape {(B, H, N)}")
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    rc = library().attn_fwd_pair(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
+                                 lse.data_ptr(), B, H, N, d, int(bool(causal)), float(scale),
+                                 _stream_handle(stream))
+    if rc != ATTN_OK:
+        raise AttnError(rc, "attn_fwd_pair")
+
+
+def attn_fwd_pair(q, k, v, causal: bool = False, scale: float | None = None, stream=None):
+    """Return ``(o, lse)`` from the CTA-pair kernel."""
+    B, H, N, d = _shape(q)
+    o = torch.empty_like(q)
+    lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
+    attn_fwd_pair_into(q, k, v, o, lse, causal, scale, stream)
+    return o, lse
 
 
 def attn_fwd_host(q_h, k_h, v_h, o_h, lse_h, q_d, k_d, v_d, o_d, lse_d,

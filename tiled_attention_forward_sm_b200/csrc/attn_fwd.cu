@@ -124,11 +124,15 @@ int device_state(DeviceState** out) {
 // head are outside the view and read as zero, so a tile never picks up the
 // next head's rows.
 int make_tmap_heads(CUtensorMap* m, const void* ptr, int Z, int N, int d) {
+  return make_tmap_heads_rows(m, ptr, Z, N, d, 128);
+}
+
+int make_tmap_heads_rows(CUtensorMap* m, const void* ptr, int Z, int N, int d, int box_rows) {
   cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(N),
                         static_cast<cuuint64_t>(Z)};
   cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2,
                            static_cast<cuuint64_t>(N) * static_cast<cuuint64_t>(d) * 2};
-  cuuint32_t box[3] = {64, 128, 1};
+  cuuint32_t box[3] = {64, static_cast<cuuint32_t>(box_rows), 1};
   return encode_tiled(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, ptr, dims, strides, box) ==
                  CUDA_SUCCESS
              ? ATTN_OK

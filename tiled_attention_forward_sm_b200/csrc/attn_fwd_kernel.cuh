@@ -654,8 +654,9 @@ __device__ __forceinline__ float exp2_poly1(float x) {
 // One K/V step of the online softmax for one query row (one thread):
 // S_s(j) from TMEM -> running max (lazy rule) -> weights -> P_s(j) back to
 // TMEM in two published halves; m and l are the row's running max (log2
-// units) and sum.
-template <int D, bool CAUSAL, int kPolyPairs>
+// units) and sum.  PAIR: the CTA is one of a cluster pair whose rank-0 CTA
+// issues the MMAs, so P is announced on that CTA's barrier.
+template <int D, bool CAUSAL, int kPolyPairs, bool PAIR = false>
 __device__ __forceinline__ bool softmax_step(const Shared& sh, const KernelArgs& a, int s,
                                              uint32_t t_s, uint32_t t_o, int r, int lane,
                                              int key_limit, bool first, uint32_t s_parity,
@@ -782,7 +783,12 @@ __device__ __forceinline__ bool softmax_step(const Shared& sh, const KernelArgs&
     ptx::tmem_st_wait();
     ptx::tc_fence_before_sync();
     __syncwarp();
-    if (lane == 0) ptx::mbar_arrive(&sh.p_ready[2 * s + half]);
+    if (lane == 0) {
+      if constexpr (PAIR)
+        ptx::mbar_arrive_cluster(ptx::mapa(ptx::smem_u32(&sh.p_ready[2 * s + half]), 0));
+      else
+        ptx::mbar_arrive(&sh.p_ready[2 * s + half]);
+    }
     if (r == 0) ATTN_TRACE(s == 0 ? (half ? kTrSm0Pb : kTrSm0Pa) : (half ? kTrSm1Pb : kTrSm1Pa), tj);
   }
 #if ATTN_PACKED_SOFTMAX

@@ -46,6 +46,9 @@ CUresult encode_tiled(CUtensorMap* m, CUtensorMapDataType type, const void* ptr,
 // Per-head bf16 view [Z][N][d], boxes of 128 rows x 64 columns.
 int make_tmap_heads(CUtensorMap* m, const void* ptr, int Z, int N, int d);
 
+// The same view with boxes of box_rows rows x 64 columns.
+int make_tmap_heads_rows(CUtensorMap* m, const void* ptr, int Z, int N, int d, int box_rows);
+
 // Token-major bf16 view [T][Hx][d], boxes of 64 columns x 1 head x 128 tokens.
 int make_tmap_tokens(CUtensorMap* m, const void* ptr, int T, int Hx, int d);
 
