@@ -97,10 +97,11 @@ int attn_fwd_ex(const void* q, const void* k, const void* v, void* o, float* lse
  * attn_fwd_pair -- attn_fwd computed by pairs of CTAs on neighbouring SMs
  * (thread-block clusters of 2) that share each tensor-core product
  * (tcgen05.mma.cta_group::2, M = 256 query rows): each SM stages and reads
- * half of every K and V tile instead of all of it.  The pair form of the
- * instructions is the one named on page lecompute.fr/en/kernel-perf/
- * flashattention-4-gpu-blackwell, section "Blackwell deplace la limite vers
- * les autres unites".
+ * half of every K and V tile instead of all of it.  Motivation: page
+ * lecompute.fr/kernel-perf/flashattention-4-limites-calcul-matriciel,
+ * section "Blackwell deplace la limite vers les autres unites" (shared-memory
+ * reads did not keep pace with the doubled per-SM matrix rate).  Measured on
+ * B200 it is slower than attn_fwd: the P hand-off then crosses SMs.
  *
  * Same arguments, results (to rounding: the same arithmetic in another
  * order of products) and errors as attn_fwd, except that d must be 128

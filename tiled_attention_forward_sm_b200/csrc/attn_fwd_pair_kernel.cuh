@@ -1,9 +1,11 @@
 // Dense attention forward on CTA pairs (cluster of 2, tcgen05.mma.cta_group::2),
-// head dim 128, per-head layout.  Same result as attn_fwd_kernel; the page
-// lecompute.fr/en/kernel-perf/flashattention-4-gpu-blackwell (section
-// "Blackwell déplace la limite vers les autres unités") names the pair form
-// of the tensor-core instructions, whose M = 256 product reads each
-// operand half from the shared memory of the SM that holds it.
+// head dim 128, per-head layout.  Same result as attn_fwd_kernel.  The page
+// lecompute.fr/kernel-perf/flashattention-4-limites-calcul-matriciel,
+// section "Blackwell déplace la limite vers les autres unités", notes that
+// shared-memory reads did not keep pace with the doubled per-SM matrix rate
+// of B200; the pair form of the tensor-core instructions (an M = 256
+// product that reads each operand half from the shared memory of the SM
+// holding it) halves each SM's K/V staging and operand reads.
 //
 // The pair works on 4 Q tiles of one (batch, head): softmax group s of CTA
 // r (rank in the cluster) owns Q tile 4u + 2s + r, so the product for group
