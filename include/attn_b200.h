@@ -293,9 +293,14 @@ long long attn_kmeans_workspace_floats(int N, int K);
 /*
  * attn_fwd_host -- the same operation on HOST buffers: copies q, k, v from
  * host to the caller's device buffers, runs attn_fwd, and copies o and lse
- * back, all enqueued on `stream` (pinned host memory makes the copies
- * asynchronous).  Synchronises `stream` before returning, so the host
- * results are valid on return.
+ * back.  Problems of 64 MiB of inputs or more run as a pipeline over up to 8
+ * groups of heads: each group's host-to-device copies, its kernel and its
+ * device-to-host copies go to three streams the library owns (one set per
+ * device), so transfers in both directions overlap the kernels.  The work
+ * starts after everything enqueued on `stream` before the call, and `stream`
+ * continues after the last copy.  With pageable host memory the copies do
+ * not overlap.  The call returns once everything has completed, so the host
+ * results are valid on return; calls on the same device are serialised.
  *
  *   q_h, k_h, v_h   host bf16 [B,H,N,d];   o_h host bf16 [B,H,N,d];
  *   lse_h           host fp32 [B,H,N];

@@ -171,6 +171,23 @@ def test_host_entry_point_matches_device_entry_point():
     assert torch.equal(oh, o_ref.cpu()) and torch.equal(lh, l_ref.cpu())
 
 
+@pytest.mark.parametrize("causal", [False, True])
+def test_host_entry_point_pipelined_over_head_groups(causal):
+    """96 MiB of inputs: the host entry point runs as a pipeline over 8
+    groups of 4 heads; every head's result is bitwise that of the device
+    entry point on the whole tensor."""
+    B, H, N, d = 2, 16, 4096, 128
+    q, k, v = make_qkv(B, H, N, d, 13)
+    qd, kd, vd = (t.cuda() for t in (q, k, v))
+    o_ref, l_ref = tab.attn_fwd(qd, kd, vd, causal=causal)
+    qh, kh, vh = (t.pin_memory() for t in (q, k, v))
+    oh = torch.full_like(qh, float("nan")).pin_memory()
+    lh = torch.full((B, H, N), float("nan"), dtype=torch.float32).pin_memory()
+    od = torch.empty_like(qd); ld = torch.empty((B, H, N), dtype=torch.float32, device="cuda")
+    tab.attn_fwd_host(qh, kh, vh, oh, lh, qd, kd, vd, od, ld, causal=causal)
+    assert torch.equal(oh, o_ref.cpu()) and torch.equal(lh, l_ref.cpu())
+
+
 def test_rejected_arguments_launch_nothing():
     q = torch.zeros(1, 1, 128, 80, dtype=torch.bfloat16, device="cuda")  # d = 80: unsupported
     with pytest.raises(tab.AttnError) as e:

@@ -16,7 +16,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libattn_b200.so")
-SOURCES = [os.path.join(CSRC, f) for f in ("attn_fwd.cu", "fp8.cu", "kmeans.cu", "pair.cu")]
+SOURCES = [os.path.join(CSRC, f) for f in ("attn_fwd.cu", "fp8.cu", "kmeans.cu", "pair.cu", "host_io.cu")]
 HEADERS = [os.path.join(CSRC, f) for f in os.listdir(CSRC) if f.endswith((".cuh", ".h"))] + [
     os.path.join(INCLUDE, f) for f in os.listdir(INCLUDE) if f.endswith(".h")]
 

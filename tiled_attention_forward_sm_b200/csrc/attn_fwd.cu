@@ -42,8 +42,6 @@ static __device__ __align__(256) int g_attn_noalloc_scratch[kNoAllocScratchBytes
 
 namespace host {
 
-constexpr int kMaxDevices = 64;
-
 namespace {
 std::mutex g_mu;
 DeviceState g_dev[kMaxDevices];
@@ -607,32 +605,6 @@ extern "C" int attn_last_device_error(attn_stream_t stream) {
     return ATTN_ERR_CUDA;
   }
   return val;
-}
-
-extern "C" int attn_fwd_host(const void* q_h, const void* k_h, const void* v_h, void* o_h,
-                             float* lse_h, void* q_d, void* k_d, void* v_d, void* o_d,
-                             float* lse_d, int B, int H, int N, int d, int causal, float scale,
-                             attn_stream_t stream) {
-  if (!q_h || !k_h || !v_h || !o_h || !lse_h) return ATTN_ERR_INVALID_ARG;
-  int rc = attn_check_args(q_d, k_d, v_d, o_d, lse_d, B, H, N, d, scale);
-  if (rc != ATTN_OK) return rc;
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
-  const size_t rows = static_cast<size_t>(B) * H * N;
-  const size_t tb = rows * static_cast<size_t>(d) * 2;
-  if (cudaMemcpyAsync(q_d, q_h, tb, cudaMemcpyHostToDevice, s) != cudaSuccess ||
-      cudaMemcpyAsync(k_d, k_h, tb, cudaMemcpyHostToDevice, s) != cudaSuccess ||
-      cudaMemcpyAsync(v_d, v_h, tb, cudaMemcpyHostToDevice, s) != cudaSuccess) {
-    cudaGetLastError();
-    return ATTN_ERR_CUDA;
-  }
-  rc = attn_fwd(q_d, k_d, v_d, o_d, lse_d, B, H, N, d, causal, scale, stream);
-  if (rc != ATTN_OK) return rc;
-  if (cudaMemcpyAsync(o_h, o_d, tb, cudaMemcpyDeviceToHost, s) != cudaSuccess ||
-      cudaMemcpyAsync(lse_h, lse_d, rows * 4, cudaMemcpyDeviceToHost, s) != cudaSuccess) {
-    cudaGetLastError();
-    return ATTN_ERR_CUDA;
-  }
-  return attn_last_device_error(stream);
 }
 
 extern "C" const char* attn_strerror(int status) {

@@ -14,6 +14,9 @@
 namespace attn_b200 {
 namespace host {
 
+// Devices the library keeps state for (device ordinals below this).
+constexpr int kMaxDevices = 64;
+
 // Work-queue slots of the device array g_attn_queue ({next item, CTAs
 // finished} each); a launch takes the next slot round-robin.
 constexpr int kQueueSlots = 256;

@@ -17,7 +17,6 @@ namespace {
 
 using namespace host;
 
-constexpr int kMaxDevices = 64;
 // Clusters of two that fit on the device at once (0: not queried yet).
 std::atomic<int> g_pair_clusters[kMaxDevices];
 
