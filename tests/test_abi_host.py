@@ -143,6 +143,28 @@ def test_exp2_polynomial_coefficients_and_error():
                                rtol=1e-7)
 
 
+def test_exp2_degree5_polynomial_of_the_fp8_kernel():
+    """The FP8 kernel's degree-5 literals are the generator's, and the fp32
+    sequence stays within 2.5e-7 relative of 2^x (about ex2.approx's own
+    error), so E4M3 rounding of the weights flips no more often."""
+    import importlib.util
+    import numpy as np
+    gen_path = os.path.join(ROOT, "tiled_attention_forward_sm_b200", "csrc", "gen_exp2_poly.py")
+    spec = importlib.util.spec_from_file_location("gen_exp2_poly", gen_path)
+    gen = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(gen)
+    c = [float(np.float32(v)) for v in gen.remez_relative(5)]
+    src = open(os.path.join(ROOT, "tiled_attention_forward_sm_b200", "csrc",
+                            "attn_fwd_fp8_kernel.cuh")).read()
+    lits = [float(x) for x in re.findall(r"kE[0-5] = ([0-9.]+)f", src)]
+    assert len(lits) == 6
+    assert np.allclose(lits, c, rtol=0, atol=1e-10)
+    xs = np.linspace(-125.0, 8.0, 400001).astype(np.float32)
+    rel = np.abs(gen.fp32_exp2_emulation(xs, lits).astype(np.float64) /
+                 np.exp2(xs.astype(np.float64)) - 1.0)
+    assert rel.max() < 2.5e-7
+
+
 def test_selftest_rejects_bad_limit(lib):
     assert lib.attn_selftest_wait_timeout(0, None) == -1
     assert lib.attn_selftest_wait_timeout(-5, None) == -1

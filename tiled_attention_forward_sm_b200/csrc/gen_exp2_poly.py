@@ -1,10 +1,13 @@
 """Derive the coefficients of the FMA-pipe exp2 used by the softmax.
 
 2^x is split as 2^j * 2^f with j = round(x) and f = x - j in [-1/2, 1/2];
-2^f is approximated by a degree-3 polynomial c0 + c1 f + c2 f^2 + c3 f^3
-whose maximum RELATIVE error on [-1/2, 1/2] is minimised (Remez exchange
-with weight 2^-f).  Run this file to print the fp32 coefficients that
-``attn_fwd_kernel.cuh`` embeds and the resulting error bound:
+2^f is approximated by a polynomial c0 + c1 f + ... + cn f^n whose maximum
+RELATIVE error on [-1/2, 1/2] is minimised (Remez exchange with weight
+2^-f).  Two degrees are used: 3 in ``attn_fwd_kernel.cuh`` (bf16 weights,
+error far below bf16 rounding) and 5 in ``attn_fwd_fp8_kernel.cuh`` (E4M3
+weights: an error as small as the special-function unit's keeps rounding
+flips at E4M3 boundaries as rare as with ex2.approx).  Run this file to
+print the fp32 coefficients and the resulting error bounds:
 
     python tiled_attention_forward_sm_b200/csrc/gen_exp2_poly.py
 """
@@ -63,27 +66,29 @@ def fp32_exp2_emulation(x: np.ndarray, c) -> np.ndarray:
     magic = np.float32(12582912.0)
     t = (x + magic).astype(np.float32)
     f = (x - (t - magic).astype(np.float32)).astype(np.float32)
-    c0, c1, c2, c3 = (np.float32(v) for v in c)
-    p = _fma32(f, c3, c2)
-    p = _fma32(f, p, c1)
-    p = _fma32(f, p, c0)
+    c = [np.float32(v) for v in c]
+    p = _fma32(f, c[-1], c[-2])
+    for ck in reversed(c[:-2]):
+        p = _fma32(f, p, ck)
     bits = p.view(np.uint32).astype(np.uint64) + ((t.view(np.uint32).astype(np.uint64) << 23)
                                                    & 0xFFFFFFFF)
     return (bits & 0xFFFFFFFF).astype(np.uint32).view(np.float32)
 
 
 def main():
-    c = remez_relative()
-    c32 = [float(np.float32(v)) for v in c]
-    g = np.linspace(LO, HI, 1000001)
-    rel = np.abs(np.polyval(np.array(c32)[::-1], g) / 2.0 ** g - 1.0)
-    xs = np.linspace(X_MIN, 8.0, 2000001).astype(np.float32)
-    emu = fp32_exp2_emulation(xs, c32).astype(np.float64)
-    rel_emu = np.abs(emu / np.exp2(xs.astype(np.float64)) - 1.0)
-    for i, v in enumerate(c32):
-        print(f"c{i} = {v!r}  ({np.float32(v).view(np.uint32):#010x})")
-    print(f"max relative error, polynomial on [-1/2,1/2]: {rel.max():.3e}")
-    print(f"max relative error, fp32 sequence on [{X_MIN:g}, 8]: {rel_emu.max():.3e}")
+    for degree in (3, 5):
+        c = remez_relative(degree)
+        c32 = [float(np.float32(v)) for v in c]
+        g = np.linspace(LO, HI, 1000001)
+        rel = np.abs(np.polyval(np.array(c32)[::-1], g) / 2.0 ** g - 1.0)
+        xs = np.linspace(X_MIN, 8.0, 2000001).astype(np.float32)
+        emu = fp32_exp2_emulation(xs, c32).astype(np.float64)
+        rel_emu = np.abs(emu / np.exp2(xs.astype(np.float64)) - 1.0)
+        print(f"degree {degree}:")
+        for i, v in enumerate(c32):
+            print(f"  c{i} = {v!r}  ({np.float32(v).view(np.uint32):#010x})")
+        print(f"  max relative error, polynomial on [-1/2,1/2]: {rel.max():.3e}")
+        print(f"  max relative error, fp32 sequence on [{X_MIN:g}, 8]: {rel_emu.max():.3e}")
 
 
 if __name__ == "__main__":
