@@ -27,9 +27,12 @@ namespace fp8 {
 // Of every 4 quadruples of score columns, how many take their exponentials
 // from the FMA pipe (exp2_poly5) instead of the special-function unit: the
 // split of the page's section "Deplacer une partie des exponentielles".
-// Measured on B200 at d = 128: 1 of 4 is 4-5% faster than 0 (the products
-// are short in FP8, so the exponentials weigh more); 2 of 4 is slower.
-constexpr int kPolyQuads = 1;
+// Measured on B200 at d = 128, 1 of 4 is 2-3% faster in short runs but 3%
+// slower in sustained runs, where the 1 kW power limit sets the clock: the
+// polynomial costs more energy per exponential than the special-function
+// unit (median clock 1790-1810 against 1840-1905 MHz).  2 of 4 is slower
+// in both.  Hence 0.
+constexpr int kPolyQuads = 0;
 
 // exp2 on the FMA pipe for a pair of inputs, as exp2_poly2 in the bf16
 // kernel but with a degree-5 polynomial for 2^f on [-1/2, 1/2]
