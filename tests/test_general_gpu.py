@@ -137,6 +137,49 @@ def test_splitkv_matches_oracle(oracle_mod, causal, B, H, H_kv, N_q, N_k, d, n_s
           f"splitkv B{B} H{H}/{H_kv} Nq{N_q} Nk{N_k} d{d} slices{n_splits} causal={causal}")
 
 
+# Packed items are used when they number at least 2/3 of the SMs (99 of 148),
+# so every case below has 128 or more of them.
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("B,H,H_kv,N_q,N_k,n_splits", [
+    (2, 6, 2, 128, 3000, 32),  # 3 query heads per K/V head: one item holds a single head
+    (1, 8, 2, 100, 2000, 64),  # ragged query block
+    (2, 4, 1, 1, 5000, 64),    # decode: one query per head
+    (8, 32, 16, 64, 700, 1),   # 2 query heads per K/V head, no key slices
+])
+def test_query_heads_sharing_kv_are_packed(oracle_mod, causal, B, H, H_kv, N_q, N_k, n_splits):
+    """Up to 128 queries per head with K/V heads shared: each work item pairs
+    two query heads of one K/V head (one K/V stream, both softmax groups).
+    Against the oracle, for full and single-head items and key slices
+    (including slices past the last key tile, which see no key)."""
+    d = 128
+    scale = 1 / math.sqrt(d)
+    delta = N_k - N_q
+    q, k, v = draw(B, H, H_kv, N_q, N_k, d, 1300 + N_q + N_k + H, 2.0)
+    if n_splits == 1:
+        o, lse = tab.attn_fwd_chunk(q.cuda(), k.cuda(), v.cuda(), causal, delta, scale)
+    else:
+        o, lse = tab.attn_fwd_splitkv(q.cuda(), k.cuda(), v.cuda(), n_splits, causal, delta, scale)
+    assert tab.last_device_error() == 0
+    o_ref, l_ref = oracle_mod.attn_ref_general(bf16_bits(q), bf16_bits(k), bf16_bits(v), causal,
+                                               delta, scale)
+    check(o.float().cpu().numpy(), lse.cpu().numpy(), o_ref, l_ref,
+          f"packed B{B} H{H}/{H_kv} Nq{N_q} Nk{N_k} slices{n_splits} causal={causal}")
+
+
+def test_packed_heads_equal_one_head_per_item():
+    """Each query head's result does not depend on the head it shares an
+    item with: the packed launch (128 items) equals one-head launches
+    (unpacked) bitwise."""
+    B, H, H_kv, N_q, N_k, d = 64, 4, 2, 128, 1500, 128
+    q, k, v = (t.cuda() for t in draw(B, H, H_kv, N_q, N_k, d, 1400))
+    o, lse = tab.attn_fwd_chunk(q, k, v, True, N_k - N_q)
+    for h in range(H):
+        hk = h // (H // H_kv)
+        o1, l1 = tab.attn_fwd_chunk(q[:, h:h + 1].contiguous(), k[:, hk:hk + 1].contiguous(),
+                                    v[:, hk:hk + 1].contiguous(), True, N_k - N_q)
+        assert torch.equal(o[:, h:h + 1], o1) and torch.equal(lse[:, h:h + 1], l1)
+
+
 def test_splitkv_one_slice_is_attn_fwd():
     q, k, v = (t.cuda() for t in make_qkv(1, 2, 700, 128, 91))
     o1, l1 = tab.attn_fwd(q, k, v, causal=True)

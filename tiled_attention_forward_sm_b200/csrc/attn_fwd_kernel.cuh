@@ -155,6 +155,8 @@ struct KernelArgs {
   float scale_log2;   // scale * log2(e)
   int* status;        // device status word
   int* queue;         // {next item, CTAs finished}: this launch's queue slot
+  int head_pack;      // dense, N_q <= 128: an item pairs two query heads of
+                      // one K/V head (n_qpairs = head pairs per K/V head)
 };
 
 template <int D>
@@ -257,7 +259,17 @@ struct Item {
   int qz, kz;        // map coordinate of the (batch, head) of Q and of K/V
   int q_row0, k_row0;  // row coordinate of query 0 and key 0 in the maps
   int split;         // key slice (offset of the partial outputs)
+  int pack;          // 1: Q0 and Q1 are tile 0 of query heads qz and qz1
+  int qz1;           // pack: map coordinate of Q1's head (-1: no second head)
 };
+
+// Q tile index and query-head map coordinate of softmax group s's tile.
+__device__ __forceinline__ int item_qtile(const Item& it, int s) {
+  return it.pack ? 0 : 2 * it.qpair + s;
+}
+__device__ __forceinline__ int item_qz(const Item& it, int s) {
+  return (it.pack && s == 1) ? it.qz1 : it.qz;
+}
 
 // K/V tiles that Q tile `qt` of `it` visits inside the slice starting at
 // tile it.kt0 (at most split_tiles of them).
@@ -292,6 +304,33 @@ __device__ __forceinline__ bool make_item(int idx, const KernelArgs& a, int* sta
     base = idx / a.n_splits;
     split = idx - base * a.n_splits;
   }
+  if (a.head_pack) {
+    // Dense layout with one Q tile per head: item (b, K/V head hk, pair p)
+    // takes query heads hk*q_per_kv + 2p and + 2p + 1, which read the same
+    // K/V head, so one K/V stream feeds both softmax groups.
+    const int b = base / (a.H_kv * a.n_qpairs);
+    const int rem = base - b * (a.H_kv * a.n_qpairs);
+    const int hk = rem / a.n_qpairs;
+    const int pp = rem - hk * a.n_qpairs;
+    const int h0 = hk * a.q_per_kv + 2 * pp;
+    it.pack = 1;
+    it.qpair = 0;
+    it.q_row0 = 0;
+    it.q_len = a.N_q;
+    it.k_row0 = 0;
+    it.k_len = a.N_k;
+    it.qz = b * a.H + h0;
+    it.qz1 = (2 * pp + 1 < a.q_per_kv) ? it.qz + 1 : -1;
+    it.kz = b * a.H_kv + hk;
+    it.delta = a.delta;
+    it.split = split;
+    it.kt0 = split * a.split_tiles;
+    it.n0 = tiles_for<CAUSAL>(0, it, a.split_tiles);
+    it.n1 = it.qz1 >= 0 ? it.n0 : 0;
+    return true;
+  }
+  it.pack = 0;
+  it.qz1 = -1;
   const int per_win = a.win_heads * a.n_qpairs;
   const int w = base / per_win;
   const int k = base - w * per_win;
@@ -357,6 +396,8 @@ __device__ __forceinline__ bool post_item(const Shared& sh, const KernelArgs& a,
     w[10] = it->q_row0;
     w[11] = it->k_row0;
     w[12] = it->split;
+    w[13] = it->pack;
+    w[14] = it->qz1;
   }
   ptx::mbar_arrive(&sh.item_full[slot]);  // release: the writes are seen by waiters
   return true;
@@ -386,6 +427,8 @@ __device__ __forceinline__ bool read_item(const Shared& sh, const KernelArgs& a,
     it.q_row0 = w[10];
     it.k_row0 = w[11];
     it.split = w[12];
+    it.pack = w[13];
+    it.qz1 = w[14];
   }
   __syncwarp();
   if (ptx::lane_id() == 0) ptx::mbar_arrive(&sh.item_empty[slot]);
@@ -443,7 +486,7 @@ __device__ void producer_role(const Shared& sh, const KernelArgs& a, uint8_t* sm
       }
       ptx::mbar_arrive_expect_tx(&sh.q_full[s], C::kTileBytes);
       load_tile(tq, &sh.q_full[s], smem + C::kQOff + s * C::kTileBytes,
-                it.q_row0 + (2 * it.qpair + s) * kBlockM, it.qz, pol_q);
+                it.q_row0 + item_qtile(it, s) * kBlockM, item_qz(it, s), pol_q);
       ++q_loads[s];
     }
     for (int j = 0; j < n && ok; ++j) {
@@ -818,9 +861,10 @@ __device__ void softmax_role(const Shared& sh, const KernelArgs& a, uint32_t tme
   Item it;
   bool ok = true;
   for (int rr = 0; read_item(sh, a, rr, it, ok); ++rr) {
-    const int qt = 2 * it.qpair + s;
+    const int qt = item_qtile(it, s);
+    const int qz = item_qz(it, s);
     const int row = qt * kBlockM + r;  // query row in the sequence
-    if (qt * kBlockM >= it.q_len) continue;  // the item has no such tile
+    if (qt * kBlockM >= it.q_len || qz < 0) continue;  // the item has no such tile
     const int n_s = s == 0 ? it.n0 : it.n1;
     float m = -INFINITY;  // running max of scale*log2(e)*score (log2 units)
     float l = 0.f;        // running sum of weights, relative to 2^m
@@ -856,10 +900,10 @@ __device__ void softmax_role(const Shared& sh, const KernelArgs& a, uint32_t tme
     const float inv_l = empty ? 0.f : 1.f / l;
     size_t o_row, l_row;
     if (a.cu_q != nullptr) {
-      o_row = (static_cast<size_t>(it.q_row0) + row) * a.H + it.qz;
-      l_row = static_cast<size_t>(it.qz) * a.T_q + it.q_row0 + row;
+      o_row = (static_cast<size_t>(it.q_row0) + row) * a.H + qz;
+      l_row = static_cast<size_t>(qz) * a.T_q + it.q_row0 + row;
     } else {
-      o_row = static_cast<size_t>(it.qz) * a.N_q + row;
+      o_row = static_cast<size_t>(qz) * a.N_q + row;
       l_row = o_row;
     }
     o_row += static_cast<size_t>(it.split) * a.split_rows;
