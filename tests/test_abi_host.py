@@ -165,6 +165,14 @@ def test_exp2_degree5_polynomial_of_the_fp8_kernel():
     assert rel.max() < 2.5e-7
 
 
+def test_trace_reader_knows_the_kernel_events():
+    """The trace reader takes its event list from the kernel source."""
+    from tiled_attention_forward_sm_b200 import trace
+    names = trace.event_names()
+    assert names[0] == "MmaS0" and "Sm1Pb" in names and "End" in names
+    assert len(names) == len(set(names)) == 24
+
+
 def test_selftest_rejects_bad_limit(lib):
     assert lib.attn_selftest_wait_timeout(0, None) == -1
     assert lib.attn_selftest_wait_timeout(-5, None) == -1

@@ -1,6 +1,13 @@
 """Build the sm_100a shared library ``libattn_b200.so`` in place.
 
-    python -m tiled_attention_forward_sm_b200.build [--verbose]
+    python -m tiled_attention_forward_sm_b200.build [--verbose] [--trace]
+
+``--trace`` builds the timeline-tracing library ``libattn_b200_trace.so``
+instead: the attention kernel compiled with its clock64 stamps at every role
+hand-off (ATTN_TRACE_ENABLED) and the extra entry point
+``int attn_trace_set_buffer(void* dev_buf)``.  It is a debugging build, read
+by ``tiled_attention_forward_sm_b200.trace``; the product library never
+carries the stamps.
 
 Runs nvcc for ``-gencode arch=compute_100a,code=sm_100a`` with line info; the
 library is written beside this file so it travels with the source tree.
@@ -16,6 +23,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libattn_b200.so")
+TRACE_LIB = os.path.join(PKG, "libattn_b200_trace.so")
 SOURCES = [os.path.join(CSRC, f) for f in ("attn_fwd.cu", "fp8.cu", "kmeans.cu", "pair.cu", "host_io.cu")]
 HEADERS = [os.path.join(CSRC, f) for f in os.listdir(CSRC) if f.endswith((".cuh", ".h"))] + [
     os.path.join(INCLUDE, f) for f in os.listdir(INCLUDE) if f.endswith(".h")]
@@ -48,6 +56,21 @@ def build(force: bool = False, verbose: bool = False) -> str:
     return LIB
 
 
+def build_trace(force: bool = False, verbose: bool = False) -> str:
+    """The tracing library (attention entry points of attn_fwd.cu only)."""
+    src = os.path.join(CSRC, "attn_fwd.cu")
+    if (not force and os.path.exists(TRACE_LIB) and
+            all(os.path.getmtime(p) <= os.path.getmtime(TRACE_LIB) for p in [src] + HEADERS)):
+        return TRACE_LIB
+    cmd = [nvcc_path(), *NVCC_FLAGS, "-DATTN_TRACE_ENABLED", *(["-Xptxas", "-v"] if verbose else []),
+           "-o", TRACE_LIB, src]
+    subprocess.check_call(cmd)
+    return TRACE_LIB
+
+
 if __name__ == "__main__":
-    build(force=True, verbose="--verbose" in sys.argv)
-    print(LIB)
+    if "--trace" in sys.argv:
+        print(build_trace(force=True, verbose="--verbose" in sys.argv))
+    else:
+        build(force=True, verbose="--verbose" in sys.argv)
+        print(LIB)
