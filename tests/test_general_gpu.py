@@ -166,6 +166,21 @@ def test_query_heads_sharing_kv_are_packed(oracle_mod, causal, B, H, H_kv, N_q, 
           f"packed B{B} H{H}/{H_kv} Nq{N_q} Nk{N_k} slices{n_splits} causal={causal}")
 
 
+@pytest.mark.parametrize("delta", [-100, 72])
+def test_packed_heads_with_rows_that_see_no_key(oracle_mod, delta):
+    """Packed items (128 of them) under a causal offset that leaves the first
+    rows without a visible key (delta < 0), or shifts the diagonal inside
+    the tile: those rows come out as O = 0, LSE = -inf in both heads."""
+    B, H, H_kv, N_q, N_k, d = 64, 4, 2, 128, 200, 128
+    scale = 1 / math.sqrt(d)
+    q, k, v = draw(B, H, H_kv, N_q, N_k, d, 1500 + delta, 2.0)
+    o, lse = tab.attn_fwd_chunk(q.cuda(), k.cuda(), v.cuda(), True, delta, scale)
+    assert tab.last_device_error() == 0
+    o_ref, l_ref = oracle_mod.attn_ref_general(bf16_bits(q), bf16_bits(k), bf16_bits(v), True,
+                                               delta, scale)
+    check(o.float().cpu().numpy(), lse.cpu().numpy(), o_ref, l_ref, f"packed delta={delta}")
+
+
 def test_packed_heads_equal_one_head_per_item():
     """Each query head's result does not depend on the head it shares an
     item with: the packed launch (128 items) equals one-head launches
