@@ -112,6 +112,8 @@ def segments(stamps: np.ndarray, cta: int) -> dict:
         "softmax 0: second P half": med("Sm0Pa", "Sm0Pb"),
         "first P half -> PV0 issued": med("Sm0Pa", "MmaPV0a"),
         "S0 issue (8 MMAs)": med("MmaS0", "MmaS0end"),
+        "group 1 lag (sees S1 - sees S0)": med("Sm0Full", "Sm1Full"),
+        "softmax 1: sees S -> second P half": med("Sm1Full", "Sm1Pb"),
     }
 
 
