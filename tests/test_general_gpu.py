@@ -101,6 +101,50 @@ def test_varlen_matches_oracle(oracle_mod, causal, d, H, H_kv, lens_q, lens_k):
           f"varlen d{d} H{H}/{H_kv} q{lens_q} k{lens_k} causal={causal}")
 
 
+@pytest.mark.parametrize("causal", [False, True])
+def test_varlen_short_query_blocks_pack_heads(oracle_mod, causal):
+    """64 sequences of at most 128 queries (some with none) against up to
+    800 keys (some with none), 4 query heads per K/V head: two query heads
+    share each work item (256 items)."""
+    rng = np.random.default_rng(77)
+    B, H, H_kv, d = 64, 8, 2, 128
+    lens_q = rng.integers(0, 129, B)
+    lens_k = rng.integers(0, 801, B)
+    lens_q[:3] = [0, 128, 1]
+    lens_k[:3] = [10, 0, 800]
+    cu_q = np.concatenate([[0], np.cumsum(lens_q)]).astype(np.int32)
+    cu_k = np.concatenate([[0], np.cumsum(lens_k)]).astype(np.int32)
+    T_q, T_k = int(cu_q[-1]), int(cu_k[-1])
+    q = make_qkv(1, 1, T_q * H, d, 1600, 2.0)[0].reshape(T_q, H, d)
+    _, k, v = make_qkv(1, 1, T_k * H_kv, d, 1601)
+    k, v = k.reshape(T_k, H_kv, d), v.reshape(T_k, H_kv, d)
+    scale = 1 / math.sqrt(d)
+    o, lse = tab.attn_fwd_varlen(q.cuda(), k.cuda(), v.cuda(),
+                                 torch.from_numpy(cu_q).cuda(), torch.from_numpy(cu_k).cuda(),
+                                 int(lens_q.max()), int(lens_k.max()), causal, scale)
+    assert tab.last_device_error() == 0
+    o_ref, l_ref = oracle_mod.attn_ref_varlen(bf16_bits(q), bf16_bits(k), bf16_bits(v),
+                                              cu_q, cu_k, causal, scale)
+    check(o.float().cpu().numpy(), lse.cpu().numpy(), o_ref, l_ref, f"varlen packed causal={causal}")
+
+
+def test_varlen_packed_heads_bad_offsets_are_caught():
+    """Packed items (200) with one sequence longer than max_seqlen_q: that
+    sequence is skipped with ATTN_ERR_DEVICE_BOUNDS, the others computed."""
+    B, H, H_kv, d = 100, 4, 2, 128
+    lens = np.full(B, 100)
+    lens[7] = 150
+    cu = torch.from_numpy(np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)).cuda()
+    T = int(lens.sum())
+    q = make_qkv(1, 1, T * H, d, 1700)[0].reshape(T, H, d).cuda()
+    _, k, v = make_qkv(1, 1, T * H_kv, d, 1701)
+    k, v = k.reshape(T, H_kv, d).cuda(), v.reshape(T, H_kv, d).cuda()
+    o, lse = tab.attn_fwd_varlen(q, k, v, cu, cu, 128, 200, True)
+    assert tab.last_device_error() == -6
+    assert tab.last_device_error() == 0
+    assert torch.isfinite(o[:700]).all() and torch.isfinite(lse[:, :700]).all()
+
+
 def test_varlen_bad_offsets_are_caught_on_the_device():
     """A sequence longer than max_seqlen_q is skipped and reported as
     ATTN_ERR_DEVICE_BOUNDS; the other sequences are still computed, and the

@@ -206,9 +206,9 @@ struct Problem {
 };
 
 // Two query heads share one work item when every head has a single Q tile
-// and K/V heads are shared (dense layout, up to 128 queries, H / H_kv >= 2,
-// head dims handled by the two-tile kernel): both softmax groups then work,
-// and one K/V stream feeds both.  A packed item runs two tiles per step in
+// and K/V heads are shared (up to 128 queries per head, or per sequence in
+// the packed layout; H / H_kv >= 2; head dims handled by the two-tile
+// kernel): both softmax groups then work, and one K/V stream feeds both.  A packed item runs two tiles per step in
 // about 1.36x the step time of a one-tile item (measured on B200), so
 // packing pays unless it leaves too many SMs idle: it is used when the
 // packed items still number at least two thirds of the SMs.
@@ -217,7 +217,7 @@ int64_t packed_items(const Problem& p) {
   return static_cast<int64_t>(p.B) * p.H_kv * pairs * p.n_splits;
 }
 bool head_pack(const Problem& p, int num_sms) {
-  return p.cu_q == nullptr && p.N_q <= kBlockM && p.H / p.H_kv >= 2 && p.d <= 128 &&
+  return p.N_q <= kBlockM && p.H / p.H_kv >= 2 && p.d <= 128 &&
          3 * packed_items(p) >= 2 * static_cast<int64_t>(num_sms);
 }
 

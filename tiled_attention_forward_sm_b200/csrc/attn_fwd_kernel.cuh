@@ -305,24 +305,43 @@ __device__ __forceinline__ bool make_item(int idx, const KernelArgs& a, int* sta
     split = idx - base * a.n_splits;
   }
   if (a.head_pack) {
-    // Dense layout with one Q tile per head: item (b, K/V head hk, pair p)
-    // takes query heads hk*q_per_kv + 2p and + 2p + 1, which read the same
-    // K/V head, so one K/V stream feeds both softmax groups.
+    // One Q tile per head (per sequence in the packed layout): item
+    // (b, K/V head hk, pair p) takes query heads hk*q_per_kv + 2p and
+    // + 2p + 1, which read the same K/V head, so one K/V stream feeds both
+    // softmax groups.
     const int b = base / (a.H_kv * a.n_qpairs);
     const int rem = base - b * (a.H_kv * a.n_qpairs);
     const int hk = rem / a.n_qpairs;
     const int pp = rem - hk * a.n_qpairs;
     const int h0 = hk * a.q_per_kv + 2 * pp;
+    const bool two = 2 * pp + 1 < a.q_per_kv;
     it.pack = 1;
     it.qpair = 0;
-    it.q_row0 = 0;
-    it.q_len = a.N_q;
-    it.k_row0 = 0;
-    it.k_len = a.N_k;
-    it.qz = b * a.H + h0;
-    it.qz1 = (2 * pp + 1 < a.q_per_kv) ? it.qz + 1 : -1;
-    it.kz = b * a.H_kv + hk;
-    it.delta = a.delta;
+    if (a.cu_q != nullptr) {
+      const int q0 = a.cu_q[b], q1 = a.cu_q[b + 1], k0 = a.cu_k[b], k1 = a.cu_k[b + 1];
+      if (q0 < 0 || q1 < q0 || q1 > a.T_q || q1 - q0 > a.N_q || k0 < 0 || k1 < k0 ||
+          k1 > a.T_k || k1 - k0 > a.N_k) {
+        atomicCAS(status, 0, kStatusDeviceBounds);
+        return false;
+      }
+      if (q1 == q0) return false;  // a sequence without queries
+      it.q_row0 = q0;
+      it.q_len = q1 - q0;
+      it.k_row0 = k0;
+      it.k_len = k1 - k0;
+      it.qz = h0;
+      it.kz = hk;
+      it.delta = it.k_len - it.q_len;
+    } else {
+      it.q_row0 = 0;
+      it.q_len = a.N_q;
+      it.k_row0 = 0;
+      it.k_len = a.N_k;
+      it.qz = b * a.H + h0;
+      it.kz = b * a.H_kv + hk;
+      it.delta = a.delta;
+    }
+    it.qz1 = two ? it.qz + 1 : -1;
     it.split = split;
     it.kt0 = split * a.split_tiles;
     it.n0 = tiles_for<CAUSAL>(0, it, a.split_tiles);
