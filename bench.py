@@ -597,7 +597,7 @@ def run_kmeans(args, w):
                      "frac": round(tflops / float(peaks["bf16_tflops"]), 4), "traffic": None,
                      "algorithmic_bytes": bytes_alg,
                      "peak_source": f"{peak_kind} (MEASURED_PEAKS.json)"},
-        "e2e": None, "gpu_launches": 3 * args.steps, "clocks": clocks,
+        "e2e": None, "gpu_launches": 2 * args.steps, "clocks": clocks,
         "kernel_sha": kernel_sha(),
     }
 

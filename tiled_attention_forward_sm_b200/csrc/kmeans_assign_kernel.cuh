@@ -64,7 +64,8 @@ struct AssignArgs {
   int32_t* assign;      // [N] nearest centroid
   float* best;          // [N] squared distance to it (null: not written)
   const float* cnorm;   // [ceil(K/128)*128] ||c_j||^2, +inf past K
-  const float* xnorm;   // [N] ||x_i||^2 (needed only with best)
+  const __nv_bfloat16* x;  // [N, d] the points (their norms, only with best)
+  int d;
 };
 
 // ||row||^2 of bf16 rows in fp32 (one warp per row); rows in [n, n_pad)
@@ -289,7 +290,23 @@ __device__ void reduce_role(const Shared& sh, const KBars& bb, const KernelArgs&
     }
     if (row < it.q_len) {
       o.assign[row] = best_j;
-      if (o.best != nullptr) o.best[row] = fmaxf(o.xnorm[row] + best, 0.f);
+      if (o.best != nullptr) {
+        // ||x||^2 from the point's row (read back from L2, where the tile
+        // load just brought it), in fp32
+        const uint4* xr = reinterpret_cast<const uint4*>(o.x + static_cast<size_t>(row) * o.d);
+        float xn0 = 0.f, xn1 = 0.f;
+        for (int c = 0; c < o.d / 8; ++c) {
+          const uint4 u = __ldg(xr + c);
+          const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const float lo = __uint_as_float(w[k] << 16), hi = __uint_as_float(w[k] & 0xFFFF0000u);
+            xn0 = fmaf(lo, lo, xn0);
+            xn1 = fmaf(hi, hi, xn1);
+          }
+        }
+        o.best[row] = fmaxf((xn0 + xn1) + best, 0.f);
+      }
     }
   }
 }
