@@ -55,7 +55,6 @@ int launch_kmeans(const void* x, const void* cent, float* ws, int32_t* assign, f
   out.best = best;
   out.cnorm = cnorm;
   out.x = static_cast<const __nv_bfloat16*>(x);
-  out.d = D;
   auto kern = kmeans::kmeans_assign_kernel<D>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, KC::kSmemBytes) !=
       cudaSuccess) {

@@ -65,7 +65,6 @@ struct AssignArgs {
   float* best;          // [N] squared distance to it (null: not written)
   const float* cnorm;   // [ceil(K/128)*128] ||c_j||^2, +inf past K
   const __nv_bfloat16* x;  // [N, d] the points (their norms, only with best)
-  int d;
 };
 
 // ||row||^2 of bf16 rows in fp32 (one warp per row); rows in [n, n_pad)
@@ -209,8 +208,31 @@ done:
   wait_warp(sh, a.status, sh.drain, 0, true);
 }
 
+// ||x||^2 of one bf16 row of D values from global memory, in fp32; the D/8
+// 16-byte loads are independent and issue together.
+template <int D>
+__device__ __forceinline__ float row_norm(const __nv_bfloat16* x, int64_t row) {
+  const uint4* xr = reinterpret_cast<const uint4*>(x + row * D);
+  uint4 u[D / 8];
+#pragma unroll
+  for (int c = 0; c < D / 8; ++c) u[c] = __ldg(xr + c);
+  float xn0 = 0.f, xn1 = 0.f;
+#pragma unroll
+  for (int c = 0; c < D / 8; ++c) {
+    const uint32_t w[4] = {u[c].x, u[c].y, u[c].z, u[c].w};
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const float lo = __uint_as_float(w[k] << 16), hi = __uint_as_float(w[k] & 0xFFFF0000u);
+      xn0 = fmaf(lo, lo, xn0);
+      xn1 = fmaf(hi, hi, xn1);
+    }
+  }
+  return xn0 + xn1;
+}
+
 // One thread per point: v_j = ||c_j||^2 - 2 x.c_j over each centroid tile,
 // a running minimum and the smallest index that reaches it.
+template <int D>
 __device__ void reduce_role(const Shared& sh, const KBars& bb, const KernelArgs& a,
                             const AssignArgs& o, uint32_t tmem, int s, int warp_in_group) {
   const int lane = static_cast<int>(ptx::lane_id());
@@ -225,6 +247,9 @@ __device__ void reduce_role(const Shared& sh, const KBars& bb, const KernelArgs&
     const int n = s == 0 ? it.n0 : it.n1;
     float best = INFINITY;
     int best_j = 0;
+    // The point's ||x||^2 (only for the distance output), read while the
+    // first score tile is being computed.
+    const float xn = (o.best != nullptr && row < it.q_len) ? row_norm<D>(o.x, row) : 0.f;
     for (int j = 0; j < n; ++j) {
       const int b = ts & 1;
       if (!wait_warp(sh, a.status, &bb.s_full[2 * s + b], static_cast<uint32_t>((ts >> 1) & 1)))
@@ -290,23 +315,7 @@ __device__ void reduce_role(const Shared& sh, const KBars& bb, const KernelArgs&
     }
     if (row < it.q_len) {
       o.assign[row] = best_j;
-      if (o.best != nullptr) {
-        // ||x||^2 from the point's row (read back from L2, where the tile
-        // load just brought it), in fp32
-        const uint4* xr = reinterpret_cast<const uint4*>(o.x + static_cast<size_t>(row) * o.d);
-        float xn0 = 0.f, xn1 = 0.f;
-        for (int c = 0; c < o.d / 8; ++c) {
-          const uint4 u = __ldg(xr + c);
-          const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            const float lo = __uint_as_float(w[k] << 16), hi = __uint_as_float(w[k] & 0xFFFF0000u);
-            xn0 = fmaf(lo, lo, xn0);
-            xn1 = fmaf(hi, hi, xn1);
-          }
-        }
-        o.best[row] = fmaxf((xn0 + xn1) + best, 0.f);
-      }
+      if (o.best != nullptr) o.best[row] = fmaxf(xn + best, 0.f);
     }
   }
 }
@@ -372,7 +381,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem = *sh.tmem_base;
 
   if (warp < 8) {
-    reduce_role(sh, bb, args, out, tmem, warp / 4, warp % 4);
+    reduce_role<D>(sh, bb, args, out, tmem, warp / 4, warp % 4);
   } else if (warp == 8) {
     if (ptx::lane_id() == 0) producer_role<D>(sh, bb, args, smem, &tmap_x, &tmap_c);
     __syncwarp();
