@@ -555,6 +555,10 @@ def run_kmeans(args, w):
     assign = torch.empty(w.N, dtype=torch.int32, device=dev)
     best = torch.empty(w.N, dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream(dev)
+    # centroid norms + assignment; a point-norm launch too when the points
+    # fill more than four rounds of 256-point work items over the SMs
+    n_sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    launches_per_step = 3 if (w.N + 255) // 256 > 4 * n_sms else 2
 
     def step():
         rc = lib.attn_kmeans_assign(x.data_ptr(), c.data_ptr(), ws.data_ptr(), assign.data_ptr(),
@@ -597,7 +601,7 @@ def run_kmeans(args, w):
                      "frac": round(tflops / float(peaks["bf16_tflops"]), 4), "traffic": None,
                      "algorithmic_bytes": bytes_alg,
                      "peak_source": f"{peak_kind} (MEASURED_PEAKS.json)"},
-        "e2e": None, "gpu_launches": 2 * args.steps, "clocks": clocks,
+        "e2e": None, "gpu_launches": launches_per_step * args.steps, "clocks": clocks,
         "kernel_sha": kernel_sha(),
     }
 

@@ -274,8 +274,8 @@ int attn_quantize_e4m3(const void* src, void* dst, int BH, int N, int d, float i
  *   x          device, bf16 [N, d] points, contiguous.  Read only.
  *   centroids  device, bf16 [K, d], contiguous.  Read only.
  *   ws         device, fp32 scratch of attn_kmeans_workspace_floats(N, K)
- *              values (the centroid norms, padded to 128), 16-byte aligned,
- *              caller-owned; overwritten.
+ *              values (centroid norms, and point norms for large N),
+ *              16-byte aligned, caller-owned; overwritten.
  *   assign     device, int32 [N].  Written: the index of the nearest
  *              centroid (among distances equal in fp32, the smallest index).
  *   best       device, fp32 [N] or NULL.  Written when given: the squared
@@ -288,9 +288,8 @@ int attn_quantize_e4m3(const void* src, void* dst, int BH, int N, int d, float i
 int attn_kmeans_assign(const void* x, const void* centroids, float* ws, int32_t* assign,
                        float* best, int N, int K, int d, attn_stream_t stream);
 
-/* Scratch size (fp32 values) attn_kmeans_assign needs, K rounded up to a
- * multiple of 128 (N is not used; kept for callers that size by both), or
- * -1 for bad sizes. */
+/* Scratch size (fp32 values) attn_kmeans_assign needs: K rounded up to a
+ * multiple of 128, plus N; or -1 for bad sizes. */
 long long attn_kmeans_workspace_floats(int N, int K);
 
 /*

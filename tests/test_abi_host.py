@@ -255,8 +255,8 @@ def test_kmeans_rejections_before_any_cuda_call(lib):
     assert f(x + 8, c, ws, a_, b_, 1000, 64, 128, None) == -3   # misaligned x
     assert f(x, c, ws, a_ + 2, b_, 1000, 64, 128, None) == -3   # misaligned assign
     assert f(x, c, x, a_, b_, 1000, 64, 128, None) == -1        # scratch over the points
-    assert lib.attn_kmeans_workspace_floats(1000, 64) == 128
-    assert lib.attn_kmeans_workspace_floats(1000, 129) == 256
+    assert lib.attn_kmeans_workspace_floats(1000, 64) == 128 + 1000
+    assert lib.attn_kmeans_workspace_floats(1000, 129) == 256 + 1000
     assert lib.attn_kmeans_workspace_floats(0, 5) == -1
 
 

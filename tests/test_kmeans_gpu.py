@@ -88,3 +88,22 @@ def test_assign_is_deterministic():
     for _ in range(3):
         a2, b2 = tab.kmeans_assign(x.cuda(), c.cuda())
         assert torch.equal(a1, a2) and torch.equal(b1, b2)
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_assign_many_points_uses_the_norm_prologue(oracle_mod, d):
+    """Enough points for more than four rounds of work items over the SMs
+    (the point norms then come from a prologue launch rather than from the
+    assignment kernel): the same checks on sampled points, and the
+    distances agree with the in-kernel norms of the first points."""
+    N, K = 200_000, 300
+    x, c = draw(N, K, d, seed=11)
+    assign, best = tab.kmeans_assign(x.cuda(), c.cuda())
+    assert tab.last_device_error() == 0
+    rows = np.unique(np.concatenate([[0, N - 1],
+                                     np.random.default_rng(4).integers(0, N, 3000)]))
+    check(oracle_mod, x, c, assign, best, rows=rows.astype(np.int64))
+    a_small, b_small = tab.kmeans_assign(x[:5000].cuda(), c.cuda())
+    assert torch.equal(a_small, assign[:5000])
+    np.testing.assert_allclose(b_small.cpu().numpy(), best[:5000].cpu().numpy(),
+                               rtol=1e-5, atol=1e-4)

@@ -25,15 +25,25 @@ int launch_kmeans(const void* x, const void* cent, float* ws, int32_t* assign, f
   if (make_tmap_heads(&tx, x, 1, N, D) || make_tmap_heads(&tc, cent, 1, K, D)) return ATTN_ERR_CUDA;
   const int k_tiles = (K + kmeans::kTileN - 1) / kmeans::kTileN;
   const int64_t k_pad = static_cast<int64_t>(k_tiles) * kmeans::kTileN;
-  // Centroid norms (+inf past K) for every CTA; the point norms, needed only
-  // for the distances, are formed by the assignment kernel itself.
+  // Centroid norms (+inf past K) for every CTA.  The point norms (needed
+  // only for the distances) come from a prologue launch when the points fill
+  // more than four rounds of work items over the SMs; with fewer, the
+  // assignment kernel reads each point's row at the start of its item, which
+  // costs a memory latency per item but saves the launch.
   float* cnorm = ws;
-  {
-    const int64_t blocks64 = (k_pad + 7) / 8;  // 8 warps (rows) per block
+  float* xnorm = nullptr;
+  auto norms = [&](const void* rows, int64_t n, int64_t n_pad, float* out) {
+    const int64_t blocks64 = (n_pad + 7) / 8;  // 8 warps (rows) per block
     const int blocks = static_cast<int>(blocks64 < 8LL * st.num_sms ? blocks64 : 8LL * st.num_sms);
-    kmeans::row_norms_kernel<<<blocks, 256, 0, stream>>>(static_cast<const __nv_bfloat16*>(cent),
-                                                         K, k_pad, D, cnorm);
-    if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
+    kmeans::row_norms_kernel<<<blocks, 256, 0, stream>>>(
+        static_cast<const __nv_bfloat16*>(rows), n, n_pad, D, out);
+    return cudaGetLastError() == cudaSuccess;
+  };
+  const int64_t items = (static_cast<int64_t>(N) + 2 * kBlockM - 1) / (2 * kBlockM);
+  if (best != nullptr && items > 4LL * st.num_sms) xnorm = ws + k_pad;
+  if (!norms(cent, K, k_pad, cnorm) || (xnorm != nullptr && !norms(x, N, N, xnorm))) {
+    cudaGetLastError();
+    return ATTN_ERR_CUDA;
   }
   KernelArgs args;
   std::memset(&args, 0, sizeof args);
@@ -54,6 +64,7 @@ int launch_kmeans(const void* x, const void* cent, float* ws, int32_t* assign, f
   out.assign = assign;
   out.best = best;
   out.cnorm = cnorm;
+  out.xnorm = xnorm;
   out.x = static_cast<const __nv_bfloat16*>(x);
   auto kern = kmeans::kmeans_assign_kernel<D>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, KC::kSmemBytes) !=
@@ -83,7 +94,7 @@ using namespace attn_b200::host;
 
 extern "C" long long attn_kmeans_workspace_floats(int N, int K) {
   if (N <= 0 || K <= 0) return -1;
-  return (static_cast<long long>(K) + kmeans::kTileN - 1) / kmeans::kTileN * kmeans::kTileN;
+  return (static_cast<long long>(K) + kmeans::kTileN - 1) / kmeans::kTileN * kmeans::kTileN + N;
 }
 
 extern "C" int attn_kmeans_assign(const void* x, const void* centroids, float* ws,

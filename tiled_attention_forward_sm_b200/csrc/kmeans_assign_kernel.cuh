@@ -64,7 +64,8 @@ struct AssignArgs {
   int32_t* assign;      // [N] nearest centroid
   float* best;          // [N] squared distance to it (null: not written)
   const float* cnorm;   // [ceil(K/128)*128] ||c_j||^2, +inf past K
-  const __nv_bfloat16* x;  // [N, d] the points (their norms, only with best)
+  const float* xnorm;   // [N] ||x_i||^2 precomputed, or null: formed here from x
+  const __nv_bfloat16* x;  // [N, d] the points
 };
 
 // ||row||^2 of bf16 rows in fp32 (one warp per row); rows in [n, n_pad)
@@ -247,9 +248,12 @@ __device__ void reduce_role(const Shared& sh, const KBars& bb, const KernelArgs&
     const int n = s == 0 ? it.n0 : it.n1;
     float best = INFINITY;
     int best_j = 0;
-    // The point's ||x||^2 (only for the distance output), read while the
-    // first score tile is being computed.
-    const float xn = (o.best != nullptr && row < it.q_len) ? row_norm<D>(o.x, row) : 0.f;
+    // The point's ||x||^2 (only for the distance output), unless the host
+    // computed all of them in a prologue: read from the point's row while
+    // the first score tile is being computed.
+    const float xn = (o.best != nullptr && o.xnorm == nullptr && row < it.q_len)
+                         ? row_norm<D>(o.x, row)
+                         : 0.f;
     for (int j = 0; j < n; ++j) {
       const int b = ts & 1;
       if (!wait_warp(sh, a.status, &bb.s_full[2 * s + b], static_cast<uint32_t>((ts >> 1) & 1)))
@@ -315,7 +319,8 @@ __device__ void reduce_role(const Shared& sh, const KBars& bb, const KernelArgs&
     }
     if (row < it.q_len) {
       o.assign[row] = best_j;
-      if (o.best != nullptr) o.best[row] = fmaxf(xn + best, 0.f);
+      if (o.best != nullptr)
+        o.best[row] = fmaxf((o.xnorm != nullptr ? o.xnorm[row] : xn) + best, 0.f);
     }
   }
 }
