@@ -29,6 +29,7 @@ import os
 import statistics
 import subprocess
 import sys
+import tempfile
 import time
 
 import numpy as np
@@ -103,7 +104,9 @@ class ClockSampler:
         self.path = None
 
     def start(self):
-        out = os.path.join(ROOT, "gpurun_out") if os.path.isdir(os.path.join(ROOT, "gpurun_out")) else "/tmp"
+        # raw samples: ATTN_BENCH_CLOCKS_DIR if set (to keep them), else a temp dir
+        out = os.environ.get("ATTN_BENCH_CLOCKS_DIR") or tempfile.gettempdir()
+        os.makedirs(out, exist_ok=True)
         self.path = os.path.join(out, f"clocks_rank{self.gpu}_{os.getpid()}.csv")
         try:
             self.proc = subprocess.Popen(
