@@ -95,54 +95,147 @@ def load_traffic(workload_name: str, profile_file: str = PROFILE_FILE, sources=N
 
 
 # ----------------------------------------------------------------- clocks ---
-class ClockSampler:
-    """nvidia-smi sampling (100 ms) while the GPU is busy."""
+_REASON_BITS = {0x8: "hw_slowdown", 0x40: "hw_thermal_slowdown", 0x20: "sw_thermal_slowdown",
+                0x4: "sw_power_cap", 0x80: "hw_power_brake_slowdown"}
 
-    def __init__(self, gpu_id: str):
-        self.gpu = gpu_id  # nvidia-smi --id: index or UUID of the physical GPU
-        self.proc = None
-        self.path = None
+
+class ClockSampler:
+    """SM clock, power and clock-event reasons sampled every ``period_s``
+    while the GPU works, by read-only NVML queries from a thread of this
+    process (the timed region of a short run is tens of milliseconds, too
+    short for nvidia-smi's 100 ms period).  Falls back to nvidia-smi when
+    NVML cannot be used.  Nothing here changes a GPU setting."""
+
+    def __init__(self, dev: torch.device, period_s: float = 0.002):
+        self.dev = dev
+        self.period = period_s
+        self.samples = []
+        self._stop = None
+        self._thread = None
+        self._proc = None
+        self._path = None
+        self._file = None
+        self._nvml = None
+        self._handle = None
+        self.source = None
+
+    def _open_nvml(self):
+        import pynvml
+        pynvml.nvmlInit()
+        props = torch.cuda.get_device_properties(self.dev)
+        try:
+            h = pynvml.nvmlDeviceGetHandleByUUID("GPU-" + str(props.uuid))
+        except Exception:
+            bus = f"{props.pci_domain_id:08x}:{props.pci_bus_id:02x}:{props.pci_device_id:02x}.0"
+            h = pynvml.nvmlDeviceGetHandleByPciBusId(bus)
+        self._nvml, self._handle = pynvml, h
+        self.sm_max = float(pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM))
+        try:
+            self.driver = pynvml.nvmlSystemGetDriverVersion()
+            if isinstance(self.driver, bytes):
+                self.driver = self.driver.decode()
+        except Exception:
+            self.driver = None
+
+    def _loop(self):
+        nv, h = self._nvml, self._handle
+        get_reasons = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+            nv.nvmlDeviceGetCurrentClocksThrottleReasons
+        while not self._stop.is_set():
+            try:
+                self.samples.append((float(nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)),
+                                     nv.nvmlDeviceGetPowerUsage(h) / 1000.0, int(get_reasons(h))))
+            except Exception:
+                pass
+            self._stop.wait(self.period)
 
     def start(self):
-        # raw samples: ATTN_BENCH_CLOCKS_DIR if set (to keep them), else a temp dir
+        import threading
+        self.samples = []
+        try:
+            if self._nvml is None:
+                self._open_nvml()
+            self.source = f"nvml, {self.period * 1e3:g} ms"
+            self._stop = threading.Event()
+            self._thread = threading.Thread(target=self._loop, daemon=True)
+            self._thread.start()
+            return
+        except Exception:
+            self._nvml = None
+        # fallback: nvidia-smi at its 100 ms period, raw rows in a temp file
         out = os.environ.get("ATTN_BENCH_CLOCKS_DIR") or tempfile.gettempdir()
         os.makedirs(out, exist_ok=True)
-        self.path = os.path.join(out, f"clocks_rank{self.gpu}_{os.getpid()}.csv")
+        self._path = os.path.join(out, f"clocks_gpu{self.dev.index}_{os.getpid()}.csv")
+        vis = os.environ.get("CUDA_VISIBLE_DEVICES", "")
+        ids = [x.strip() for x in vis.split(",")] if vis else []
+        smi_id = ids[self.dev.index] if len(ids) > self.dev.index else str(self.dev.index)
         try:
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={CLOCK_QUERY}",
+            self._file = open(self._path, "w")
+            self._proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={smi_id}", f"--query-gpu={CLOCK_QUERY}",
                  "--format=csv,noheader,nounits", "-lms", "100"],
-                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+                stdout=self._file, stderr=subprocess.DEVNULL)
+            self.source = "nvidia-smi, 100 ms"
         except (OSError, FileNotFoundError):
-            self.proc = None
+            self._proc = None
+            if self._file:
+                self._file.close()
+                self._file = None
 
-    def stop(self):
-        if self.proc is None:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"],
-                    "samples": 0}
-        self.proc.terminate()
+    def _stop_smi(self):
+        self._proc.terminate()
         try:
-            self.proc.wait(timeout=5)
+            self._proc.wait(timeout=5)
         except subprocess.TimeoutExpired:
-            self.proc.kill()
+            self._proc.kill()
+        self._file.close()
+        self._file = None
         rows = []
-        with open(self.path) as f:
+        with open(self._path) as f:
             for line in f:
-                parts = [p.strip() for p in line.split(",")]
+                parts = [x.strip() for x in line.split(",")]
                 if len(parts) >= 9:
                     rows.append(parts)
-        if not rows:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
-        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
-        smax = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        if not os.environ.get("ATTN_BENCH_CLOCKS_DIR"):
+            os.remove(self._path)
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i] == "Active"})
-        load = [s for s in sm if s > 0.5 * max(sm)] if sm else []
-        return {"sm_mhz": statistics.median(load) if load else None,
-                "sm_max_mhz": max(smax) if smax else None,
-                "reasons": reasons, "samples": len(rows),
-                "power_w_max": max((float(r[3]) for r in rows
-                                    if r[3].replace(".", "").isdigit()), default=None)}
+        self.sm_max = max((float(r[2]) for r in rows if r[2].replace(".", "").isdigit()),
+                          default=None)
+        out = []
+        for r in rows:
+            if not r[1].replace(".", "").isdigit():
+                continue
+            bits = 0
+            for i, n in enumerate(names):
+                if r[5 + i] == "Active":
+                    bits |= {v: k for k, v in _REASON_BITS.items()}[n]
+            pw = float(r[3]) if r[3].replace(".", "").isdigit() else float("nan")
+            out.append((float(r[1]), pw, bits))
+        return out
+
+    def stop(self):
+        if self._thread is not None:
+            self._stop.set()
+            self._thread.join(timeout=5)
+            self._thread = None
+            samples = list(self.samples)
+        elif self._proc is not None:
+            samples = self._stop_smi()
+            self._proc = None
+        else:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no clock source"],
+                    "samples": 0, "source": None}
+        if not samples:
+            return {"sm_mhz": None, "sm_max_mhz": getattr(self, "sm_max", None), "reasons": [],
+                    "samples": 0, "source": self.source}
+        sm = [x[0] for x in samples]
+        load = [x for x in samples if not (x[2] & 0x1)] or samples  # drop GPU-idle samples
+        reasons = sorted({n for x in samples for b, n in _REASON_BITS.items() if x[2] & b})
+        return {"sm_mhz": statistics.median(x[0] for x in load),
+                "sm_min_mhz": min(sm), "sm_max_mhz": getattr(self, "sm_max", None),
+                "reasons": reasons, "samples": len(samples), "samples_under_load": len(load),
+                "power_w_max": max((x[1] for x in samples), default=None),
+                "source": self.source}
 
 
 # ------------------------------------------------------------ distributed ---
@@ -169,24 +262,65 @@ def row_flops(w, rows) -> float:
 
 def time_oracle(w, bits, target_s: float, seed: int = 123):
     """Run the oracle on growing seeded row batches until about target_s of
-    CPU work; return (TFLOPS, rows, seconds, threads)."""
+    CPU work; return (TFLOPS, rows, seconds, threads, last batch) where the
+    last batch is (rows, O, LSE) of the oracle's final call."""
     import oracle  # CPU baseline leg only
     qb, kb, vb = bits
     total_rows, total_t, total_f = 0, 0.0, 0.0
     batch = 1024
     k = 0
+    last = None
     while total_t < target_s and total_rows < w.rows:
         rows = oracle_sample_rows(w, batch, seed + k)
         t0 = time.perf_counter()
-        oracle.attn_ref(qb, kb, vb, w.causal, w.scale, rows=rows)
+        o_ref, lse_ref = oracle.attn_ref(qb, kb, vb, w.causal, w.scale, rows=rows)
         dt = time.perf_counter() - t0
         total_t += dt
         total_f += row_flops(w, rows)
         total_rows += len(rows)
+        last = (rows, o_ref, lse_ref)
         k += 1
         if dt < 0.5 * target_s:
             batch = min(batch * 2, 65536)
-    return total_f / total_t / 1e12, total_rows, total_t, oracle.max_threads()
+    return total_f / total_t / 1e12, total_rows, total_t, oracle.max_threads(), last
+
+
+def parity_of_rows(o, lse, w, last):
+    """Largest |O - O_oracle| and |LSE - LSE_oracle| over the oracle rows of
+    the CPU-baseline leg, against the GPU result of the last timed step, with
+    the parity tolerance (|dO| <= 2e-2 + 1e-2 |O|, |dLSE| <= 1e-3)."""
+    rows, o_ref, lse_ref = last
+    idx = torch.from_numpy(rows).to(o.device)
+    o_g = o.reshape(-1, w.d).index_select(0, idx).double().cpu().numpy()
+    l_g = lse.reshape(-1).index_select(0, idx).double().cpu().numpy()
+    d_o = np.abs(o_g - o_ref)
+    d_l = np.abs(l_g - lse_ref)
+    ok = bool((d_o <= 2e-2 + 1e-2 * np.abs(o_ref)).all() and (d_l <= 1e-3).all())
+    return {"rows": int(len(rows)), "max_abs_dO": float(d_o.max()),
+            "max_abs_dLSE": float(d_l.max()), "pass": ok}
+
+
+def versions(lib, sampler=None) -> dict:
+    v = int(lib.attn_version())
+    return {"torch": torch.__version__, "cuda_runtime": torch.version.cuda,
+            "driver": getattr(sampler, "driver", None),
+            "library": f"{v >> 16}.{(v >> 8) & 255}.{v & 255}",
+            "device": torch.cuda.get_device_name()}
+
+
+def timed_steps(step, steps: int, stream, dev):
+    """Run ``steps`` steps with a CUDA event before each and after the last,
+    all on the launching stream, synchronised on both sides.  Returns the
+    total milliseconds and the per-step list."""
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(steps + 1)]
+    torch.cuda.synchronize(dev)
+    for i in range(steps):
+        ev[i].record(stream)
+        step()
+    ev[steps].record(stream)
+    torch.cuda.synchronize(dev)
+    per = [ev[i].elapsed_time(ev[i + 1]) for i in range(steps)]
+    return ev[0].elapsed_time(ev[steps]), per
 
 
 # ------------------------------------------------------------- GPU arm -----
@@ -214,27 +348,17 @@ def run_b200(args, w):
     def step():
         fwd_into(q, k, v, o, lse, causal=w.causal, scale=w.scale, stream=stream)
 
-    vis = os.environ.get("CUDA_VISIBLE_DEVICES", "")
-    smi_id = vis.split(",")[local].strip() if vis and len(vis.split(",")) > local else str(local)
-    sampler = ClockSampler(smi_id)
+    sampler = ClockSampler(dev)
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize(dev)
     sampler.start()
     if pg:
         torch.distributed.barrier()
-    torch.cuda.synchronize(dev)
-    e0 = torch.cuda.Event(enable_timing=True)
-    e1 = torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(args.steps):
-        step()
-    e1.record(stream)
-    torch.cuda.synchronize(dev)
+    ms_total, per_step = timed_steps(step, args.steps, stream, dev)
     clocks = sampler.stop()
     if pg:
         torch.distributed.barrier()
-    ms_total = e0.elapsed_time(e1)
     status = tab.last_device_error(stream)
     if status != 0:
         raise SystemExit(f"device status {status}: {tab.strerror(status)}")
@@ -282,6 +406,9 @@ def run_b200(args, w):
         return None
 
     ms_step = ms_total / args.steps
+    if clocks.get("sm_mhz"):
+        # clock-independent size of a step: device cycles at the sampled clock
+        clocks["kcycles_per_step"] = round(ms_step * clocks["sm_mhz"], 1)
     value = world * w.flops / (ms_step * 1e-3) / 1e12
     e2e_value = world * w.flops / (e2e_ms * 1e-3) / 1e12
     peaks, peak_kind = load_peaks()
@@ -293,6 +420,9 @@ def run_b200(args, w):
     line = {
         "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 4),
+        "us_per_step": round(ms_step * 1e3, 2),
+        "step_ms": {"min": round(min(per_step), 4), "median": round(statistics.median(per_step), 4),
+                    "max": round(max(per_step), 4)},
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded N(0,1) bf16 Q/K/V, see inputs.py)",
         "config": {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d,
@@ -318,14 +448,17 @@ def run_b200(args, w):
         "gpu_launches": args.steps,
         "clocks": clocks,
         "kernel_sha": kernel_sha(sources),
+        "versions": versions(tab.library(), sampler),
     }
     if world == 1 and not args.no_cpu_baseline:
         bits = (bf16_bits(q_h), bf16_bits(k_h), bf16_bits(v_h))
-        tf, nrows, secs, cores = time_oracle(w, bits, args.cpu_seconds)
+        tf, nrows, secs, cores, last = time_oracle(w, bits, args.cpu_seconds)
         line["cpu_baseline"] = {
             "value": round(tf, 6), "unit": UNIT, "cores": cores, "kind": "oracle",
             "sample": f"{nrows} seeded random rows of {w.rows} ({secs:.1f} s); "
                       "TFLOPS from the rows' exact share of the metric FLOPs"}
+        # the timed step's output, against the oracle rows the leg computed
+        line["parity"] = parity_of_rows(o, lse, w, last)
     return line
 
 
@@ -397,9 +530,7 @@ def run_general(args, w):
                                       w.n_splits, ws_o.data_ptr(), ws_l.data_ptr(), sh)
             assert rc == 0, rc
 
-    vis = os.environ.get("CUDA_VISIBLE_DEVICES", "")
-    smi_id = vis.split(",")[local].strip() if vis and len(vis.split(",")) > local else str(local)
-    sampler = ClockSampler(smi_id)
+    sampler = ClockSampler(dev)
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize(dev)
@@ -503,9 +634,7 @@ def run_fp8(args, w):
         return e0.elapsed_time(e1) / steps
 
     convert()
-    vis = os.environ.get("CUDA_VISIBLE_DEVICES", "")
-    smi_id = vis.split(",")[local].strip() if vis and len(vis.split(",")) > local else str(local)
-    sampler = ClockSampler(smi_id)
+    sampler = ClockSampler(dev)
     sampler.start()
     ms_attn = timed(attend, args.steps)
     clocks = sampler.stop()
@@ -568,9 +697,7 @@ def run_kmeans(args, w):
                                     best.data_ptr(), w.N, w.K, w.d, stream.cuda_stream)
         assert rc == 0, rc
 
-    vis = os.environ.get("CUDA_VISIBLE_DEVICES", "")
-    smi_id = vis.split(",")[local].strip() if vis and len(vis.split(",")) > local else str(local)
-    sampler = ClockSampler(smi_id)
+    sampler = ClockSampler(dev)
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize(dev)
@@ -672,6 +799,10 @@ def main():
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
+    world = dist_env()[0]
+    if args.gpus != world:
+        ap.error(f"--gpus {args.gpus} but WORLD_SIZE is {world}: launch N > 1 ranks with "
+                 f"python -m torch.distributed.run --nproc-per-node N bench.py --gpus N")
     if args.workload.endswith(FP8_SUFFIX):
         if args.impl == "reference":
             ap.error("--impl reference times the bf16 workloads only")

@@ -32,7 +32,9 @@ extern "C" {
 
 typedef enum {
   ATTN_OK = 0,
-  ATTN_ERR_INVALID_ARG = -1,   /* null pointer, non-positive size, bad scale */
+  ATTN_ERR_INVALID_ARG = -1,   /* null pointer, non-positive size, bad scale,
+                                  or a buffer that is not device memory of the
+                                  current device */
   ATTN_ERR_UNSUPPORTED = -2,   /* d not in {64,96,128,256}, or B*H*N >= 2^31 */
   ATTN_ERR_MISALIGNED = -3,    /* a device pointer is not 16-byte aligned */
   ATTN_ERR_CUDA = -4,          /* a CUDA runtime/driver call failed */
@@ -59,6 +61,12 @@ typedef void* attn_stream_t;
  *   causal   0: every key visible; non-zero: key j visible to query i iff j <= i.
  *   scale    finite and > 0 (typically 1/sqrt(d)).
  *   stream   CUDA stream the kernel is enqueued on.
+ *
+ * Device: every buffer must be device memory (cudaMalloc or a pool over it)
+ * of the device current on the calling thread, which the stream must belong
+ * to; host, managed or another GPU's memory returns ATTN_ERR_INVALID_ARG
+ * (checked with cudaPointerGetAttributes; this holds for every entry point
+ * below that takes device buffers).
  *
  * Ownership: the caller owns every buffer; the call allocates no device
  * memory.  Asynchrony: returns once the kernel is enqueued; results are valid
@@ -113,9 +121,11 @@ int attn_fwd_pair(const void* q, const void* k, const void* v, void* o, float* l
 
 /*
  * attn_fwd_noalloc -- attn_fwd for callers that cannot allocate device
- * memory, e.g. code running under global-mode CUDA stream capture (where
- * cudaMalloc is refused) or inside a framework whose allocator owns all
- * device memory.  There is no counterpart on the source pages: it is a
+ * memory: a framework whose caching allocator has already reserved the
+ * GPU's memory (a cudaMalloc would fail, or force it to give its cache
+ * back), or a serving loop that fixed its memory budget at start-up and
+ * must keep cudaMalloc, with its implicit device synchronisation, out of
+ * its hot path.  There is no counterpart on the source pages: it is a
  * property of this library, not of the method.
  *
  * Same arguments, results and errors as attn_fwd; nothing is allocated.

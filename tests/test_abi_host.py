@@ -295,3 +295,19 @@ def test_pair_rejections_before_any_cuda_call(lib):
     assert f(q, k, v, o, l + 2, 1, 1, 1024, 128, 1, 0.1, None) == -3
     assert f(q, k, v, q, l, 1, 1, 1024, 128, 1, 0.1, None) == -1                 # o over q
     assert f(None, k, v, o, l, 1, 1, 1024, 128, 1, 0.1, None) == -1
+
+
+def test_binding_requires_one_cuda_device():
+    """The binding resolves the one device every tensor lives on and runs the
+    call with it current; tensors on two devices, or not on a GPU, are
+    refused before the library is called."""
+    import torch
+    from tiled_attention_forward_sm_b200 import _abi
+    cpu = torch.zeros(4)
+    meta = torch.zeros(4, device="meta")
+    with pytest.raises(ValueError, match="one CUDA device"):
+        _abi._device_of(cpu, meta)
+    with pytest.raises(ValueError, match="CUDA tensors"):
+        _abi._device_of(cpu, cpu)
+    with pytest.raises(ValueError, match="CUDA tensors"):
+        _abi._device_of(None, cpu, None)  # None entries are skipped

@@ -6,10 +6,21 @@ Two checks per case:
     |O - O_model| <= 2^-8 |O_model| + 4e-3 (the bf16 output plus rare
     rounding flips where fp32 and fp64 weights fall on either side of an
     E4M3 rounding boundary), |LSE - LSE_exact| <= 1e-3 (l is kept in fp32);
-  * the accuracy: against the exact definition on the same E4M3 inputs,
-    |O - O_exact| <= 2^-3 A + 2^-8 |O| + 4e-3 with A the exactly weighted
-    mean |v| of each output element (each weight within 2^-4 of itself, doubled for
-    rounding flips).
+  * the accuracy: against the exact definition on the same E4M3 inputs, a
+    bound derived per output element from the E4M3 rounding of each weight.
+    The kernel rounds p_j = 2^(x_j - m) (m its running maximum, log2 units)
+    to E4M3 and divides by the unrounded sum l = sum_j p_j.  E4M3 keeps 3
+    mantissa bits, so a weight in its normal range (p >= 2^-6) moves by at
+    most 2^-4 p; below it the spacing is 2^-9, so it moves by at most
+    min(p, 2^-10).  The lazy rule keeps m at or below the row's true
+    maximum x_max, so l >= sum_j 2^(x_j - x_max) = 1 / w_max and, in the
+    exact normalised weights w_j, |dw_j| <= max(2^-4 w_j, min(w_j,
+    2^-10 w_max)).  Hence
+    |O - O_exact| <= sum_j max(2^-4 w_j, min(w_j, 2^-10 w_max)) |v_j|
+                     + 2^-8 |O_exact| + 2e-3
+    (the last two terms: the bf16 output and the fp32 arithmetic).  A flip
+    of the fp32 weight to the other E4M3 neighbour costs only the fp32
+    error on top of the half spacing, so no factor is needed for it.
 Descale factors are powers of two so the oracle sees the same values.
 """
 import math
@@ -41,6 +52,7 @@ def run_case(oracle_mod, B, H, N, causal, seed, dq=0.5, dk=2.0, dv=0.25, q_std=1
     o_ex, l_ex = oracle_mod.attn_ref(qb, kb, vb, causal, scale * dq * dk)
     o_ex = o_ex * dv
     Qd, Kd, Vd = (t.double().numpy() for t in (q8.float(), k8.float(), v8.float()))
+    worst = []
     for b in range(B):
         for h in range(H):
             o_m, _ = oracle_mod.tiled_online_model(Qd[b, h], Kd[b, h], Vd[b, h], causal,
@@ -54,10 +66,14 @@ def run_case(oracle_mod, B, H, N, causal, seed, dq=0.5, dk=2.0, dv=0.25, q_std=1
                 S = np.where(np.tril(np.ones_like(S)) > 0, S, -np.inf)
             W = np.exp(S - S.max(1, keepdims=True))
             W /= W.sum(1, keepdims=True)
-            A = (W @ np.abs(Vd[b, h])) * dv
+            dW = np.maximum(2.0 ** -4 * W, np.minimum(W, 2.0 ** -10 * W.max(1, keepdims=True)))
+            bound = (dW @ np.abs(Vd[b, h])) * dv + 2.0 ** -8 * np.abs(o_ex[b, h]) + 2e-3
             err = np.abs(o[b, h] - o_ex[b, h])
-            assert (err <= 2.0 ** -3 * A + 2.0 ** -8 * np.abs(o_ex[b, h]) + 4e-3).all()
+            assert (err <= bound).all(), \
+                f"b{b} h{h}: vs exact {int((err > bound).sum())} elements past the E4M3 bound"
+            worst.append(float((err / np.maximum(bound, 1e-30)).max()))
     assert np.abs(lse - l_ex).max() <= 1e-3
+    return max(worst)
 
 
 @pytest.mark.parametrize("causal", [False, True])

@@ -245,26 +245,37 @@ def test_e4m3_rounding_matches_torch_and_saturates(oracle_mod):
 
 def test_model_with_e4m3_weights_stays_inside_its_bound(oracle_mod):
     """The tiled model with weights rounded to E4M3 differs from the exact
-    result by at most 2^-4 of the weighted mean |v| per row (each weight is
-    off by at most 2^-4 of itself in E4M3's normal range), plus the
-    flush-to-zero of weights below 2^-9, small at these sizes."""
+    result by at most sum_j max(2^-4 w_j, min(w_j, 2^-10 w_max)) |v_j| per
+    output element (w the exact normalised weights, w_max the row's
+    largest): a weight in E4M3's normal range (>= 2^-6 of the running scale
+    2^m) moves by at most 2^-4 of itself, a smaller one by at most the half
+    spacing 2^-10 (or itself, when it rounds to zero); the lazy rule keeps m
+    at or below the row's true maximum, so the running sum is at least
+    1 / w_max and the second term, normalised, is at most 2^-10 w_max.  This
+    is the bound the GPU test applies to the kernel; here it is checked on
+    the model, with ordinary and peaky scores."""
     from tiled_attention_forward_sm_b200.inputs import make_qkv
-    q, k, v = make_qkv(1, 1, 1024, 128, 5)
     import torch
     def e4(t):
         return t[0, 0].float().to(torch.float8_e4m3fn).double().numpy()
-    Q, K, V = e4(q), e4(k), e4(v)
-    scale = 128 ** -0.5
-    for causal in (False, True):
-        o_ex, _ = oracle_mod.tiled_online_model(Q, K, V, causal, scale)
-        o_m, _ = oracle_mod.tiled_online_model(Q, K, V, causal, scale, round_p="e4m3")
-        S = Q @ K.T * scale
-        if causal:
-            S = np.where(np.tril(np.ones_like(S)) > 0, S, -np.inf)
-        W = np.exp(S - S.max(1, keepdims=True))
-        W /= W.sum(1, keepdims=True)
-        A = W @ np.abs(V)
-        assert (np.abs(o_m - o_ex) <= 2.0 ** -4 * A + 1e-3).all()
+    for q_std, seed in ((1.0, 5), (3.0, 6)):
+        q, k, v = make_qkv(1, 1, 1024, 128, seed, q_std)
+        Q, K, V = e4(q), e4(k), e4(v)
+        scale = 128 ** -0.5
+        for causal in (False, True):
+            o_ex, _ = oracle_mod.tiled_online_model(Q, K, V, causal, scale)
+            o_m, _ = oracle_mod.tiled_online_model(Q, K, V, causal, scale, round_p="e4m3")
+            S = Q @ K.T * scale
+            if causal:
+                S = np.where(np.tril(np.ones_like(S)) > 0, S, -np.inf)
+            W = np.exp(S - S.max(1, keepdims=True))
+            W /= W.sum(1, keepdims=True)
+            dW = np.maximum(2.0 ** -4 * W, np.minimum(W, 2.0 ** -10 * W.max(1, keepdims=True)))
+            bound = dW @ np.abs(V)
+            err = np.abs(o_m - o_ex)
+            assert (err <= bound * (1 + 1e-9) + 1e-12).all()
+            # and the bound is not vacuous: the rounding uses a visible part of it
+            assert (err / np.maximum(bound, 1e-30)).max() > 0.1
 
 
 def test_e4m3_encoding_round_trips_every_code(oracle_mod):

@@ -11,7 +11,7 @@ import pytest
 import torch
 
 import tiled_attention_forward_sm_b200 as tab
-from tiled_attention_forward_sm_b200.inputs import (WORKLOADS, bf16_bits, make_qkv,
+from tiled_attention_forward_sm_b200.inputs import (WORKLOADS, bf16_bits, make_jump_qkv, make_qkv,
                                                     make_workload_inputs, sample_rows)
 
 pytestmark = pytest.mark.gpu
@@ -103,6 +103,25 @@ def test_peaky_scores_exercise_lazy_rescale(oracle_mod, causal):
     full_parity(oracle_mod, 1, 4, 1024, 128, causal, seed=77, q_std=3.0)
 
 
+@pytest.mark.parametrize("d", [64, 128, 256])
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("jump_tile,second", [(1, False), (2, True)])
+def test_lazy_rescale_at_known_rows(oracle_mod, d, causal, jump_tile, second):
+    """Constructed scores (inputs.make_jump_qkv, checked on the CPU by
+    tests/test_rescale_inputs.py): at a known K/V tile the running maximum of
+    known rows, in both Q tiles of a work item and mixed inside warps, jumps
+    by 10 (the rescale is taken: O and l scaled by 2^-10), by 7.5 (just under
+    the threshold of 8: weights up to 2^7.5 kept unrescaled) or not at all;
+    with ``second`` a further jump at the next tile rescales again.  Scale
+    ln 2 makes the raw scores log2 units.  Every element against the oracle."""
+    B, H, N = 1, 2, 640
+    scale = math.log(2.0)
+    q, k, v = make_jump_qkv(B, H, N, d, jump_tile, second, seed=400 + d + jump_tile)
+    o, lse = gpu_run(q, k, v, causal, scale)
+    o_ref, lse_ref = oracle_mod.attn_ref(bf16_bits(q), bf16_bits(k), bf16_bits(v), causal, scale)
+    check(o, lse, o_ref, lse_ref, f"jump at tile {jump_tile} d{d} causal={causal}")
+
+
 @pytest.mark.parametrize("scale", [0.01, 0.5, 2.0])
 def test_other_scales(oracle_mod, scale):
     full_parity(oracle_mod, 1, 2, 512, 128, True, seed=5, scale=scale)
@@ -119,23 +138,24 @@ def test_large_magnitude_scores(oracle_mod):
 def test_workload_sampled_rows(oracle_mod, name):
     """Full-size workloads in the launch configuration the benchmark uses;
     the oracle computes a deterministic row sample (first/last 128 rows of
-    every head, rows at every 4th tile boundary, 256 random rows)."""
+    every head, both rows at every 4th tile boundary, 256 random rows).  At
+    N = 32768 the whole sample too: the mid-sequence tiles are where the
+    work queue's order decides which CTA owns a pair."""
     w = WORKLOADS[name]
     q, k, v = make_workload_inputs(w)
     o, lse = gpu_run(q, k, v, w.causal, w.scale)
     rows = sample_rows(w, n_random=256)
-    if w.N >= 32768:
-        rows = rows[rows % w.N >= w.N - 256]  # keep the oracle to seconds: last rows
-        rows = np.concatenate([rows, np.arange(0, 128, dtype=np.int64)])
     o_ref, lse_ref = oracle_mod.attn_ref(bf16_bits(q), bf16_bits(k), bf16_bits(v), w.causal,
                                          w.scale, rows=rows)
     check(o.reshape(-1, w.d)[rows], lse.reshape(-1)[rows], o_ref, lse_ref, name)
 
 
 def test_deterministic_bitwise():
+    """No atomics touch the results: 20 launches give the same bits (the
+    work queue hands items to different CTAs from run to run)."""
     q, k, v = (t.cuda() for t in make_qkv(2, 4, 1024, 128, 9))
     o1, l1 = tab.attn_fwd(q, k, v, causal=True)
-    for _ in range(5):
+    for _ in range(20):
         o2, l2 = tab.attn_fwd(q, k, v, causal=True)
         assert torch.equal(o1, o2) and torch.equal(l1, l2)
 
@@ -203,3 +223,30 @@ def test_bounded_wait_reports_timeout_and_context_stays_usable(oracle_mod):
     assert tab.last_device_error() == -5
     assert tab.last_device_error() == 0  # read-and-clear
     full_parity(oracle_mod, 1, 2, 256, 128, True, seed=3)
+
+
+def test_buffers_not_on_the_device_are_refused_before_launch():
+    """Host memory (pinned, which CUDA can see) passed where a device buffer
+    belongs: every entry point refuses it with ATTN_ERR_INVALID_ARG before
+    encoding a tensor map, so no kernel reads it."""
+    import ctypes
+    B, H, N, d = 1, 2, 256, 128
+    q, k, v = (t.cuda() for t in make_qkv(B, H, N, d, 14))
+    o = torch.empty_like(q)
+    lse = torch.empty((B, H, N), dtype=torch.float32, device="cuda")
+    host = torch.zeros_like(q.cpu()).pin_memory()
+    lib = tab.library()
+    s = torch.cuda.current_stream().cuda_stream
+    args = (B, H, N, d, 1, ctypes.c_float(0.1), s)
+    assert lib.attn_fwd(host.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
+                        lse.data_ptr(), *args) == -1
+    assert lib.attn_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), host.data_ptr(),
+                        lse.data_ptr(), *args) == -1
+    assert lib.attn_fwd_pair(q.data_ptr(), host.data_ptr(), v.data_ptr(), o.data_ptr(),
+                             lse.data_ptr(), *args) == -1
+    assert lib.attn_fwd_noalloc(q.data_ptr(), k.data_ptr(), host.data_ptr(), o.data_ptr(),
+                                lse.data_ptr(), *args) == -1
+    assert tab.last_device_error() == 0
+    # and the same buffers on the device still work
+    tab.attn_fwd_into(q, k, v, o, lse, causal=True)
+    assert tab.last_device_error() == 0 and torch.isfinite(o).all()

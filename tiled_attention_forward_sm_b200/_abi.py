@@ -91,10 +91,28 @@ def check_args(q_ptr: int, k_ptr: int, v_ptr: int, o_ptr: int, lse_ptr: int,
     return library().attn_check_args(q_ptr, k_ptr, v_ptr, o_ptr, lse_ptr, B, H, N, d, scale)
 
 
-def _stream_handle(stream) -> int:
+def _stream_handle(stream, dev=None) -> int:
+    """The raw handle of ``stream``; None means the current stream of ``dev``
+    (or of the current device).  A torch stream of another device is
+    refused: the kernel would run on one GPU against another's memory."""
     if stream is None:
-        stream = torch.cuda.current_stream()
+        stream = torch.cuda.current_stream(dev)
+    elif dev is not None and isinstance(stream, torch.cuda.Stream) and stream.device != dev:
+        raise ValueError(f"stream is on {stream.device}, the tensors on {dev}")
     return int(stream.cuda_stream) if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def _device_of(*tensors) -> torch.device:
+    """The one CUDA device every given tensor (None entries skipped) lives
+    on.  Each call runs with that device current, so the library's
+    tensor maps, launch and stream all refer to it."""
+    devs = {t.device for t in tensors if t is not None}
+    if len(devs) != 1:
+        raise ValueError(f"tensors must all be on one CUDA device, got {sorted(map(str, devs))}")
+    dev = devs.pop()
+    if dev.type != "cuda":
+        raise ValueError(f"tensors must be CUDA tensors, got {dev}")
+    return dev
 
 
 def _shape(q: torch.Tensor):
@@ -120,11 +138,14 @@ def attn_fwd_into(q, k, v, o, lse, causal: bool = False, scale: float | None = N
         scale = 1.0 / math.sqrt(d)
     args = (q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
             B, H, N, d, int(bool(causal)), float(scale))
+    dev = _device_of(q, k, v, o, lse)
     if exp2_poly_pairs is None:
-        rc = library().attn_fwd(*args, _stream_handle(stream))
+        with torch.cuda.device(dev):
+            rc = library().attn_fwd(*args, _stream_handle(stream, dev))
     else:
         opts = AttnOpts(int(exp2_poly_pairs))
-        rc = library().attn_fwd_ex(*args, ctypes.byref(opts), _stream_handle(stream))
+        with torch.cuda.device(dev):
+            rc = library().attn_fwd_ex(*args, ctypes.byref(opts), _stream_handle(stream, dev))
     if rc != ATTN_OK:
         raise AttnError(rc, "attn_fwd")
 
@@ -154,9 +175,11 @@ def attn_fwd_noalloc_into(q, k, v, o, lse, causal: bool = False, scale: float | 
         raise ValueError(f"lse must be a contiguous CUDA fp32 tensor of shape {(B, H, N)}")
     if scale is None:
         scale = 1.0 / math.sqrt(d)
-    rc = library().attn_fwd_noalloc(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
-                                    lse.data_ptr(), B, H, N, d, int(bool(causal)), float(scale),
-                                    _stream_handle(stream))
+    dev = _device_of(q, k, v, o, lse)
+    with torch.cuda.device(dev):
+        rc = library().attn_fwd_noalloc(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
+                                        lse.data_ptr(), B, H, N, d, int(bool(causal)), float(scale),
+                                        _stream_handle(stream, dev))
     if rc != ATTN_OK:
         raise AttnError(rc, "attn_fwd_noalloc")
 
@@ -175,9 +198,11 @@ def attn_fwd_pair_into(q, k, v, o, lse, causal: bool = False, scale: float | Non
         raise ValueError(f"lse must be a contiguous CUDA fp32 tensor of shape {(B, H, N)}")
     if scale is None:
         scale = 1.0 / math.sqrt(d)
-    rc = library().attn_fwd_pair(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
-                                 lse.data_ptr(), B, H, N, d, int(bool(causal)), float(scale),
-                                 _stream_handle(stream))
+    dev = _device_of(q, k, v, o, lse)
+    with torch.cuda.device(dev):
+        rc = library().attn_fwd_pair(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
+                                     lse.data_ptr(), B, H, N, d, int(bool(causal)), float(scale),
+                                     _stream_handle(stream, dev))
     if rc != ATTN_OK:
         raise AttnError(rc, "attn_fwd_pair")
 
@@ -202,10 +227,12 @@ def attn_fwd_host(q_h, k_h, v_h, o_h, lse_h, q_d, k_d, v_d, o_d, lse_d,
             raise ValueError("host tensors must be contiguous CPU tensors")
     if scale is None:
         scale = 1.0 / math.sqrt(d)
-    rc = library().attn_fwd_host(
-        q_h.data_ptr(), k_h.data_ptr(), v_h.data_ptr(), o_h.data_ptr(), lse_h.data_ptr(),
-        q_d.data_ptr(), k_d.data_ptr(), v_d.data_ptr(), o_d.data_ptr(), lse_d.data_ptr(),
-        B, H, N, d, int(bool(causal)), float(scale), _stream_handle(stream))
+    dev = _device_of(q_d, k_d, v_d, o_d, lse_d)
+    with torch.cuda.device(dev):
+        rc = library().attn_fwd_host(
+            q_h.data_ptr(), k_h.data_ptr(), v_h.data_ptr(), o_h.data_ptr(), lse_h.data_ptr(),
+            q_d.data_ptr(), k_d.data_ptr(), v_d.data_ptr(), o_d.data_ptr(), lse_d.data_ptr(),
+            B, H, N, d, int(bool(causal)), float(scale), _stream_handle(stream, dev))
     if rc != ATTN_OK:
         raise AttnError(rc, "attn_fwd_host")
 
@@ -213,14 +240,26 @@ def attn_fwd_host(q_h, k_h, v_h, o_h, lse_h, q_d, k_d, v_d, o_d, lse_d,
 def selftest_wait_timeout(limit_us: int, stream=None) -> None:
     """Enqueue the bounded-wait self-test (see the header); the next
     last_device_error() should report the timeout status."""
-    rc = library().attn_selftest_wait_timeout(int(limit_us), _stream_handle(stream))
+    dev = _stream_device(stream)
+    with torch.cuda.device(dev):
+        rc = library().attn_selftest_wait_timeout(int(limit_us), _stream_handle(stream, dev))
     if rc != ATTN_OK:
         raise AttnError(rc, "attn_selftest_wait_timeout")
 
 
+def _stream_device(stream) -> torch.device:
+    """The device of a torch stream, else the current device."""
+    if isinstance(stream, torch.cuda.Stream):
+        return stream.device
+    return torch.device("cuda", torch.cuda.current_device())
+
+
 def last_device_error(stream=None) -> int:
-    """Synchronise the stream and return (and clear) the device status word."""
-    return int(library().attn_last_device_error(_stream_handle(stream)))
+    """Synchronise the stream and return (and clear) the device status word
+    (of the stream's device, or of the current device)."""
+    dev = _stream_device(stream)
+    with torch.cuda.device(dev):
+        return int(library().attn_last_device_error(_stream_handle(stream, dev)))
 
 
 def _check(t, name, dtype, shape):
@@ -248,10 +287,12 @@ def attn_fwd_chunk_into(q, k, v, o, lse, causal: bool = False, causal_delta: int
     _check(lse, "lse", torch.float32, (B, H, N_q))
     if scale is None:
         scale = 1.0 / math.sqrt(d)
-    rc = library().attn_fwd_chunk(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
-                                  lse.data_ptr(), B, H, H_kv, N_q, N_k, d, int(bool(causal)),
-                                  int(causal_delta), float(scale),
-                                  int(o.dtype == torch.float32), _stream_handle(stream))
+    dev = _device_of(q, k, v, o, lse)
+    with torch.cuda.device(dev):
+        rc = library().attn_fwd_chunk(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
+                                      lse.data_ptr(), B, H, H_kv, N_q, N_k, d, int(bool(causal)),
+                                      int(causal_delta), float(scale),
+                                      int(o.dtype == torch.float32), _stream_handle(stream, dev))
     if rc != ATTN_OK:
         raise AttnError(rc, "attn_fwd_chunk")
 
@@ -285,11 +326,13 @@ def attn_fwd_varlen(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q: int, max_
         scale = 1.0 / math.sqrt(d)
     o = torch.empty_like(q)
     lse = torch.empty((H, T_q), dtype=torch.float32, device=q.device)
-    rc = library().attn_fwd_varlen(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
-                                   lse.data_ptr(), cu_seqlens_q.data_ptr(),
-                                   cu_seqlens_k.data_ptr(), B, H, H_kv, int(max_seqlen_q),
-                                   int(max_seqlen_k), T_q, T_k, d, int(bool(causal)),
-                                   float(scale), _stream_handle(stream))
+    dev = _device_of(q, k, v, cu_seqlens_q, cu_seqlens_k)
+    with torch.cuda.device(dev):
+        rc = library().attn_fwd_varlen(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
+                                       lse.data_ptr(), cu_seqlens_q.data_ptr(),
+                                       cu_seqlens_k.data_ptr(), B, H, H_kv, int(max_seqlen_q),
+                                       int(max_seqlen_k), T_q, T_k, d, int(bool(causal)),
+                                       float(scale), _stream_handle(stream, dev))
     if rc != ATTN_OK:
         raise AttnError(rc, "attn_fwd_varlen")
     return o, lse
@@ -327,10 +370,12 @@ def attn_fwd_splitkv(q, k, v, n_splits: int, causal: bool = False, causal_delta:
         wp = (ws_o.data_ptr(), ws_l.data_ptr())
     else:
         wp = (None, None)
-    rc = library().attn_fwd_splitkv(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
-                                    lse.data_ptr(), B, H, H_kv, N_q, N_k, d, int(bool(causal)),
-                                    int(causal_delta), float(scale), int(n_splits), wp[0], wp[1],
-                                    _stream_handle(stream))
+    dev = _device_of(q, k, v)
+    with torch.cuda.device(dev):
+        rc = library().attn_fwd_splitkv(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
+                                        lse.data_ptr(), B, H, H_kv, N_q, N_k, d, int(bool(causal)),
+                                        int(causal_delta), float(scale), int(n_splits), wp[0], wp[1],
+                                        _stream_handle(stream, dev))
     if rc != ATTN_OK:
         raise AttnError(rc, "attn_fwd_splitkv")
     return o, lse
@@ -350,9 +395,11 @@ def attn_combine(o_parts, lse_parts, out_dtype=torch.bfloat16, stream=None):
         raise ValueError("out_dtype must be bf16 or fp32")
     o = torch.empty(tuple(o_parts.shape[1:]), dtype=out_dtype, device=o_parts.device)
     lse = torch.empty(tuple(lse_parts.shape[1:]), dtype=torch.float32, device=o_parts.device)
-    rc = library().attn_combine(o_parts.data_ptr(), lse_parts.data_ptr(), G, rows, d,
-                                o.data_ptr(), lse.data_ptr(), int(out_dtype == torch.float32),
-                                _stream_handle(stream))
+    dev = _device_of(o_parts, lse_parts)
+    with torch.cuda.device(dev):
+        rc = library().attn_combine(o_parts.data_ptr(), lse_parts.data_ptr(), G, rows, d,
+                                    o.data_ptr(), lse.data_ptr(), int(out_dtype == torch.float32),
+                                    _stream_handle(stream, dev))
     if rc != ATTN_OK:
         raise AttnError(rc, "attn_combine")
     return o, lse
@@ -375,9 +422,11 @@ def kmeans_assign(x, centroids, with_best: bool = True, stream=None):
     ws = torch.empty(n_ws, dtype=torch.float32, device=x.device)
     assign = torch.empty(N, dtype=torch.int32, device=x.device)
     best = torch.empty(N, dtype=torch.float32, device=x.device) if with_best else None
-    rc = lib.attn_kmeans_assign(x.data_ptr(), centroids.data_ptr(), ws.data_ptr(),
-                                assign.data_ptr(), best.data_ptr() if with_best else None,
-                                N, K, d, _stream_handle(stream))
+    dev = _device_of(x, centroids)
+    with torch.cuda.device(dev):
+        rc = lib.attn_kmeans_assign(x.data_ptr(), centroids.data_ptr(), ws.data_ptr(),
+                                    assign.data_ptr(), best.data_ptr() if with_best else None,
+                                    N, K, d, _stream_handle(stream, dev))
     if rc != ATTN_OK:
         raise AttnError(rc, "attn_kmeans_assign")
     return assign, best
@@ -399,10 +448,12 @@ def attn_fwd_fp8(q, k, vt, causal: bool = False, scale: float | None = None,
         scale = 1.0 / math.sqrt(d)
     o = torch.empty((B, H, N, d), dtype=torch.bfloat16, device=q.device)
     lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
-    rc = library().attn_fwd_fp8(q.data_ptr(), k.data_ptr(), vt.data_ptr(), o.data_ptr(),
-                                lse.data_ptr(), B, H, N, d, int(bool(causal)), float(scale),
-                                float(q_descale), float(k_descale), float(v_descale),
-                                _stream_handle(stream))
+    dev = _device_of(q, k, vt)
+    with torch.cuda.device(dev):
+        rc = library().attn_fwd_fp8(q.data_ptr(), k.data_ptr(), vt.data_ptr(), o.data_ptr(),
+                                    lse.data_ptr(), B, H, N, d, int(bool(causal)), float(scale),
+                                    float(q_descale), float(k_descale), float(v_descale),
+                                    _stream_handle(stream, dev))
     if rc != ATTN_OK:
         raise AttnError(rc, "attn_fwd_fp8")
     return o, lse
@@ -422,9 +473,11 @@ def quantize_e4m3(x, inv_descale: float = 1.0, transpose: bool = False, stream=N
         raise ValueError("x must be [rows, d] or [B, H, N, d]")
     _check(x, "x", torch.bfloat16, x.shape)
     out = torch.empty(out_shape, dtype=torch.uint8, device=x.device)
-    rc = library().attn_quantize_e4m3(x.data_ptr(), out.data_ptr(), BH, N, d,
-                                      float(inv_descale), int(bool(transpose)),
-                                      _stream_handle(stream))
+    dev = _device_of(x)
+    with torch.cuda.device(dev):
+        rc = library().attn_quantize_e4m3(x.data_ptr(), out.data_ptr(), BH, N, d,
+                                          float(inv_descale), int(bool(transpose)),
+                                          _stream_handle(stream, dev))
     if rc != ATTN_OK:
         raise AttnError(rc, "attn_quantize_e4m3")
     return out

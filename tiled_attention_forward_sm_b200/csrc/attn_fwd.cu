@@ -80,6 +80,7 @@ int device_state(DeviceState** out) {
     }
     st.usable = (major == 10 && minor == 0);
     st.num_sms = sms;
+    st.ordinal = dev;
     if (st.usable) {
       void* p = nullptr;
       if (cudaGetSymbolAddress(&p, g_attn_status) != cudaSuccess) {
@@ -152,6 +153,19 @@ int make_tmap_tokens(CUtensorMap* m, const void* ptr, int T, int Hx, int d) {
                  CUDA_SUCCESS
              ? ATTN_OK
              : ATTN_ERR_CUDA;
+}
+
+int check_on_device(const DeviceState& st, const void* const* ptrs, int n) {
+  for (int i = 0; i < n; ++i) {
+    if (ptrs[i] == nullptr) continue;
+    cudaPointerAttributes at;
+    if (cudaPointerGetAttributes(&at, ptrs[i]) != cudaSuccess) {
+      cudaGetLastError();
+      return ATTN_ERR_INVALID_ARG;
+    }
+    if (at.type != cudaMemoryTypeDevice || at.device != st.ordinal) return ATTN_ERR_INVALID_ARG;
+  }
+  return ATTN_OK;
 }
 
 bool ranges_overlap(const void* a, size_t na, const void* b, size_t nb) {
@@ -349,6 +363,11 @@ int run_problem(const Problem& p, int poly_pairs, attn_stream_t stream, int* que
     const int rc = device_state(&st);
     if (rc != ATTN_OK) return rc;
   }
+  {
+    const void* ptrs[7] = {p.q, p.k, p.v, p.o, p.lse, p.cu_q, p.cu_k};
+    const int rc = check_on_device(*st, ptrs, 7);
+    if (rc != ATTN_OK) return rc;
+  }
   if (problem_items(p, st->num_sms) + st->num_sms > 0x7FFFFFFFll) return ATTN_ERR_UNSUPPORTED;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   switch (p.d) {
@@ -362,6 +381,11 @@ int run_problem(const Problem& p, int poly_pairs, attn_stream_t stream, int* que
 // LSE merge of G partial results (see attn_combine_kernel.cuh).
 int run_combine(const float* o_parts, const float* lse_parts, int G, long long rows, int d,
                 void* o, float* lse, int o_f32, attn_stream_t stream, const DeviceState& st) {
+  {
+    const void* ptrs[4] = {o_parts, lse_parts, o, lse};
+    const int rc = check_on_device(st, ptrs, 4);
+    if (rc != ATTN_OK) return rc;
+  }
   const long long threads = rows * (d / 4);
   long long blocks = (threads + 255) / 256;
   const long long cap = static_cast<long long>(st.num_sms) * 8;

@@ -60,6 +60,11 @@ extern "C" int attn_fwd_fp8(const void* q, const void* k, const void* vt, void* 
   DeviceState* st = nullptr;
   int rc = device_state(&st);
   if (rc != ATTN_OK) return rc;
+  {
+    const void* ptrs[5] = {q, k, vt, o, lse};
+    rc = check_on_device(*st, ptrs, 5);
+    if (rc != ATTN_OK) return rc;
+  }
   const uint64_t BH = static_cast<uint64_t>(B) * H;
   CUtensorMap tq, tk, tvt;
   if (make_tmap_u8(&tq, q, d, N, BH) || make_tmap_u8(&tk, k, d, N, BH) ||
@@ -121,8 +126,13 @@ extern "C" int attn_quantize_e4m3(const void* src, void* dst, int BH, int N, int
     return ATTN_ERR_MISALIGNED;
   if (ranges_overlap(src, elems * 2, dst, elems)) return ATTN_ERR_INVALID_ARG;
   DeviceState* st = nullptr;
-  const int rc = device_state(&st);
+  int rc = device_state(&st);
   if (rc != ATTN_OK) return rc;
+  {
+    const void* ptrs[2] = {src, dst};
+    rc = check_on_device(*st, ptrs, 2);
+    if (rc != ATTN_OK) return rc;
+  }
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (!transpose) {
     const long long n16 = static_cast<long long>(elems / 16);

@@ -28,6 +28,7 @@ struct DeviceState {
   int* queue = nullptr;            // device address of g_attn_queue
   int* noalloc_scratch = nullptr;  // device address of g_attn_noalloc_scratch
   int num_sms = 0;
+  int ordinal = -1;                // the device's ordinal
   std::atomic<unsigned> launches{0};
 };
 
@@ -54,6 +55,12 @@ int make_tmap_heads_rows(CUtensorMap* m, const void* ptr, int Z, int N, int d, i
 
 // Token-major bf16 view [T][Hx][d], boxes of 64 columns x 1 head x 128 tokens.
 int make_tmap_tokens(CUtensorMap* m, const void* ptr, int T, int Hx, int d);
+
+// ATTN_OK when every non-null pointer is device memory of the device `st`
+// describes (the current device at set-up); ATTN_ERR_INVALID_ARG when one
+// is host memory, managed memory, another GPU's memory or unknown to CUDA:
+// the kernel would otherwise read it through a tensor map on the wrong GPU.
+int check_on_device(const DeviceState& st, const void* const* ptrs, int n);
 
 bool ranges_overlap(const void* a, size_t na, const void* b, size_t nb);
 

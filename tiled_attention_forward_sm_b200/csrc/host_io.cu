@@ -63,6 +63,11 @@ extern "C" int attn_fwd_host(const void* q_h, const void* k_h, const void* v_h, 
   DeviceState* st = nullptr;
   rc = device_state(&st);
   if (rc != ATTN_OK) return rc;
+  {
+    const void* ptrs[5] = {q_d, k_d, v_d, o_d, lse_d};
+    rc = check_on_device(*st, ptrs, 5);
+    if (rc != ATTN_OK) return rc;
+  }
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) {
     cudaGetLastError();

@@ -117,8 +117,13 @@ extern "C" int attn_kmeans_assign(const void* x, const void* centroids, float* w
   const size_t in_bytes[2] = {xb, cb};
   if (!outputs_disjoint(outs, out_bytes, 3, ins, in_bytes, 2)) return ATTN_ERR_INVALID_ARG;
   DeviceState* st = nullptr;
-  const int rc = device_state(&st);
+  int rc = device_state(&st);
   if (rc != ATTN_OK) return rc;
+  {
+    const void* ptrs[5] = {x, centroids, ws, assign, best};
+    rc = check_on_device(*st, ptrs, 5);
+    if (rc != ATTN_OK) return rc;
+  }
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   return d == 128 ? launch_kmeans<128>(x, centroids, ws, assign, best, N, K, s, *st)
                   : launch_kmeans<64>(x, centroids, ws, assign, best, N, K, s, *st);

@@ -123,8 +123,13 @@ extern "C" int attn_fwd_pair(const void* q, const void* k, const void* v, void* 
   const size_t in_bytes[3] = {ib, ib, ib};
   if (!outputs_disjoint(outs, out_bytes, 2, ins, in_bytes, 3)) return ATTN_ERR_INVALID_ARG;
   DeviceState* st = nullptr;
-  const int rc = device_state(&st);
+  int rc = device_state(&st);
   if (rc != ATTN_OK) return rc;
+  {
+    const void* ptrs[5] = {q, k, v, o, lse};
+    rc = check_on_device(*st, ptrs, 5);
+    if (rc != ATTN_OK) return rc;
+  }
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   return causal ? launch_pair<true>(q, k, v, o, lse, B, H, N, scale, s, *st)
                 : launch_pair<false>(q, k, v, o, lse, B, H, N, scale, s, *st);

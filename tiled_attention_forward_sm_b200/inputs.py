@@ -184,6 +184,65 @@ def make_workload_inputs(w: Workload):
     return make_qkv(w.B, w.H, w.N, w.d, w.seed, w.q_std)
 
 
+# Score offsets of the rows of make_jump_qkv (in units of the raw dot
+# product; with scale = ln 2 these are log2 units): the first jump lifts a
+# row's largest score by 10 (more than a lazy threshold of 8), by 7.5 (just
+# under it), or not at all.
+JUMP_OFFSETS = (10.0, 7.5, 0.0)
+
+
+def jump_offset_of_rows(N: int):
+    """Offset c of every query row of make_jump_qkv: a mix inside each warp
+    of 32 rows, except every fourth block of 32 rows, which holds one offset
+    for all its rows (a warp where every lane, or none, takes the jump)."""
+    import numpy as np
+    i = np.arange(N)
+    mixed = (7 * i + i // 32) % 3
+    uniform = (i // 128) % 3
+    pick = np.where((i // 32) % 4 == 3, uniform, mixed)
+    return np.asarray(JUMP_OFFSETS)[pick]
+
+
+def make_jump_qkv(B: int, H: int, N: int, d: int, jump_tile: int, second_jump: bool,
+                  seed: int):
+    """Inputs whose largest score per row jumps by a known amount at a known
+    K/V tile (128 keys per tile), for checking a lazy rescale of the running
+    maximum.  Every value is exact in bf16.
+
+    Query row i is [1, c_i, r_i, 0, ...] with c_i from jump_offset_of_rows
+    and r_i uniform in [-1, 1].  Key 0 (the anchor) is [2, 0, 0, ...]: raw
+    score 2.  Key 128*jump_tile is [2, 1, 0, ...]: score 2 + c_i.  With
+    second_jump, key 128*(jump_tile+1) is [2, 2, 0, ...]: score 2 + 2 c_i.
+    Every other key is [u_j, 0, w_j, 0, ...] with u_j in [-1, 1] and w_j in
+    [-1/4, 1/4]: scores in [-1.25, 1.25], below the anchor's.  V is N(0, 1).
+    The row maximum is therefore 2 until the jump key, and 2 + c_i (then
+    2 + 2 c_i) from it on, for every row that sees it."""
+    g = torch.Generator(device="cpu")
+    g.manual_seed(int(seed))
+    shape = (B, H, N, d)
+    q = torch.zeros(shape, dtype=torch.float32)
+    k = torch.zeros(shape, dtype=torch.float32)
+    c = torch.from_numpy(jump_offset_of_rows(N)).to(torch.float32)
+    q[..., 0] = 1.0
+    q[..., 1] = c
+    q[..., 2] = torch.rand((B, H, N), generator=g) * 2 - 1
+    k[..., 0] = torch.rand((B, H, N), generator=g) * 2 - 1
+    k[..., 2] = (torch.rand((B, H, N), generator=g) * 2 - 1) * 0.25
+    k[..., 0, :] = 0.0
+    k[..., 0, 0] = 2.0
+    jumps = [(jump_tile * 128, 1.0)]
+    if second_jump:
+        jumps.append(((jump_tile + 1) * 128, 2.0))
+    for row, c1 in jumps:
+        if row < N:
+            k[..., row, :] = 0.0
+            k[..., row, 0] = 2.0
+            k[..., row, 1] = c1
+    v = torch.randn(shape, generator=g, dtype=torch.float32)
+    return (q.to(torch.bfloat16).contiguous(), k.to(torch.bfloat16).contiguous(),
+            v.to(torch.bfloat16).contiguous())
+
+
 def bf16_bits(t: torch.Tensor):
     """bf16 tensor -> numpy uint16 array of its bit patterns (no copy of
     values, just a reinterpretation)."""
