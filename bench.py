@@ -99,73 +99,84 @@ _REASON_BITS = {0x8: "hw_slowdown", 0x40: "hw_thermal_slowdown", 0x20: "sw_therm
                 0x4: "sw_power_cap", 0x80: "hw_power_brake_slowdown"}
 
 
+_NVML_SAMPLER = r"""
+import os, sys, time, pynvml
+pynvml.nvmlInit()
+h = pynvml.nvmlDeviceGetHandleByUUID(sys.argv[1])
+period, path = float(sys.argv[2]), sys.argv[3]
+get = getattr(pynvml, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+    pynvml.nvmlDeviceGetCurrentClocksThrottleReasons
+drv = pynvml.nvmlSystemGetDriverVersion()
+drv = drv.decode() if isinstance(drv, bytes) else drv
+smax = pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM)
+with open(path, "w", buffering=1) as f:
+    f.write(f"ready,{smax},{drv}\n")
+    while not os.path.exists(path + ".stop"):
+        f.write(f"{pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM)},"
+                f"{pynvml.nvmlDeviceGetPowerUsage(h)},{get(h)}\n")
+        time.sleep(period)
+"""
+
+
 class ClockSampler:
     """SM clock, power and clock-event reasons sampled every ``period_s``
-    while the GPU works, by read-only NVML queries from a thread of this
-    process (the timed region of a short run is tens of milliseconds, too
-    short for nvidia-smi's 100 ms period).  Falls back to nvidia-smi when
-    NVML cannot be used.  Nothing here changes a GPU setting."""
+    while the GPU works, by read-only NVML queries in a child process (the
+    timed region of a short run lasts tens of milliseconds: too short for
+    nvidia-smi's 100 ms period, and a thread of this process would wait on
+    the interpreter lock).  Falls back to nvidia-smi when NVML cannot be
+    used.  Nothing here changes a GPU setting."""
 
-    def __init__(self, dev: torch.device, period_s: float = 0.002):
+    def __init__(self, dev: torch.device, period_s: float = 0.001):
         self.dev = dev
         self.period = period_s
-        self.samples = []
-        self._stop = None
-        self._thread = None
         self._proc = None
         self._path = None
         self._file = None
-        self._nvml = None
-        self._handle = None
+        self._kind = None
+        self.sm_max = None
+        self.driver = None
         self.source = None
 
-    def _open_nvml(self):
-        import pynvml
-        pynvml.nvmlInit()
-        props = torch.cuda.get_device_properties(self.dev)
-        try:
-            h = pynvml.nvmlDeviceGetHandleByUUID("GPU-" + str(props.uuid))
-        except Exception:
-            bus = f"{props.pci_domain_id:08x}:{props.pci_bus_id:02x}:{props.pci_device_id:02x}.0"
-            h = pynvml.nvmlDeviceGetHandleByPciBusId(bus)
-        self._nvml, self._handle = pynvml, h
-        self.sm_max = float(pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM))
-        try:
-            self.driver = pynvml.nvmlSystemGetDriverVersion()
-            if isinstance(self.driver, bytes):
-                self.driver = self.driver.decode()
-        except Exception:
-            self.driver = None
-
-    def _loop(self):
-        nv, h = self._nvml, self._handle
-        get_reasons = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
-            nv.nvmlDeviceGetCurrentClocksThrottleReasons
-        while not self._stop.is_set():
-            try:
-                self.samples.append((float(nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)),
-                                     nv.nvmlDeviceGetPowerUsage(h) / 1000.0, int(get_reasons(h))))
-            except Exception:
-                pass
-            self._stop.wait(self.period)
-
-    def start(self):
-        import threading
-        self.samples = []
-        try:
-            if self._nvml is None:
-                self._open_nvml()
-            self.source = f"nvml, {self.period * 1e3:g} ms"
-            self._stop = threading.Event()
-            self._thread = threading.Thread(target=self._loop, daemon=True)
-            self._thread.start()
-            return
-        except Exception:
-            self._nvml = None
-        # fallback: nvidia-smi at its 100 ms period, raw rows in a temp file
+    def _tmp_path(self, stem):
         out = os.environ.get("ATTN_BENCH_CLOCKS_DIR") or tempfile.gettempdir()
         os.makedirs(out, exist_ok=True)
-        self._path = os.path.join(out, f"clocks_gpu{self.dev.index}_{os.getpid()}.csv")
+        return os.path.join(out, f"{stem}_gpu{self.dev.index}_{os.getpid()}.csv")
+
+    def _start_nvml(self) -> bool:
+        props = torch.cuda.get_device_properties(self.dev)
+        self._path = self._tmp_path("clocks_nvml")
+        for p in (self._path, self._path + ".stop"):
+            if os.path.exists(p):
+                os.remove(p)
+        self._proc = subprocess.Popen(
+            [sys.executable, "-c", _NVML_SAMPLER, "GPU-" + str(props.uuid), str(self.period),
+             self._path], stdin=subprocess.DEVNULL, stdout=subprocess.DEVNULL,
+            stderr=subprocess.DEVNULL)
+        t0 = time.time()
+        while time.time() - t0 < 20:  # wait until it samples
+            if self._proc.poll() is not None:
+                return False
+            if os.path.exists(self._path):
+                with open(self._path) as f:
+                    head = f.readline()
+                if head.startswith("ready,") and head.endswith("\n"):
+                    _, smax, drv = head.strip().split(",", 2)
+                    self.sm_max, self.driver = float(smax), drv
+                    self._kind = "nvml"
+                    self.source = f"nvml in a child process, {self.period * 1e3:g} ms"
+                    return True
+            time.sleep(0.01)
+        return False
+
+    def start(self):
+        try:
+            if self._start_nvml():
+                return
+        except Exception:
+            pass
+        self._kill()
+        # fallback: nvidia-smi at its 100 ms period, raw rows in a temp file
+        self._path = self._tmp_path("clocks_smi")
         vis = os.environ.get("CUDA_VISIBLE_DEVICES", "")
         ids = [x.strip() for x in vis.split(",")] if vis else []
         smi_id = ids[self.dev.index] if len(ids) > self.dev.index else str(self.dev.index)
@@ -175,64 +186,73 @@ class ClockSampler:
                 ["nvidia-smi", f"--id={smi_id}", f"--query-gpu={CLOCK_QUERY}",
                  "--format=csv,noheader,nounits", "-lms", "100"],
                 stdout=self._file, stderr=subprocess.DEVNULL)
+            self._kind = "smi"
             self.source = "nvidia-smi, 100 ms"
         except (OSError, FileNotFoundError):
-            self._proc = None
-            if self._file:
-                self._file.close()
-                self._file = None
+            self._kill()
 
-    def _stop_smi(self):
-        self._proc.terminate()
-        try:
-            self._proc.wait(timeout=5)
-        except subprocess.TimeoutExpired:
-            self._proc.kill()
-        self._file.close()
-        self._file = None
+    def _kill(self):
+        if self._proc is not None and self._proc.poll() is None:
+            self._proc.terminate()
+            try:
+                self._proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self._proc.kill()
+        self._proc = None
+        if self._file is not None:
+            self._file.close()
+            self._file = None
+
+    def _read(self):
         rows = []
+        if self._kind == "nvml":
+            with open(self._path) as f:
+                for line in f.read().splitlines()[1:]:
+                    parts = line.split(",")
+                    if len(parts) == 3:
+                        rows.append((float(parts[0]), float(parts[1]) / 1000.0, int(parts[2])))
+            return rows
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        bit = {v: k for k, v in _REASON_BITS.items()}
         with open(self._path) as f:
             for line in f:
-                parts = [x.strip() for x in line.split(",")]
-                if len(parts) >= 9:
-                    rows.append(parts)
-        if not os.environ.get("ATTN_BENCH_CLOCKS_DIR"):
-            os.remove(self._path)
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        self.sm_max = max((float(r[2]) for r in rows if r[2].replace(".", "").isdigit()),
-                          default=None)
-        out = []
-        for r in rows:
-            if not r[1].replace(".", "").isdigit():
-                continue
-            bits = 0
-            for i, n in enumerate(names):
-                if r[5 + i] == "Active":
-                    bits |= {v: k for k, v in _REASON_BITS.items()}[n]
-            pw = float(r[3]) if r[3].replace(".", "").isdigit() else float("nan")
-            out.append((float(r[1]), pw, bits))
-        return out
+                r = [x.strip() for x in line.split(",")]
+                if len(r) < 9 or not r[1].replace(".", "").isdigit():
+                    continue
+                if r[2].replace(".", "").isdigit():
+                    self.sm_max = float(r[2])
+                bits = 0
+                for i, n in enumerate(names):
+                    if r[5 + i] == "Active":
+                        bits |= bit[n]
+                pw = float(r[3]) if r[3].replace(".", "").isdigit() else float("nan")
+                rows.append((float(r[1]), pw, bits))
+        return rows
 
     def stop(self):
-        if self._thread is not None:
-            self._stop.set()
-            self._thread.join(timeout=5)
-            self._thread = None
-            samples = list(self.samples)
-        elif self._proc is not None:
-            samples = self._stop_smi()
-            self._proc = None
-        else:
+        if self._proc is None:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no clock source"],
                     "samples": 0, "source": None}
+        if self._kind == "nvml":
+            open(self._path + ".stop", "w").close()
+            try:
+                self._proc.wait(timeout=10)
+            except subprocess.TimeoutExpired:
+                pass
+        self._kill()
+        samples = self._read()
+        if not os.environ.get("ATTN_BENCH_CLOCKS_DIR"):
+            for p in (self._path, self._path + ".stop"):
+                if os.path.exists(p):
+                    os.remove(p)
         if not samples:
-            return {"sm_mhz": None, "sm_max_mhz": getattr(self, "sm_max", None), "reasons": [],
-                    "samples": 0, "source": self.source}
+            return {"sm_mhz": None, "sm_max_mhz": self.sm_max, "reasons": [], "samples": 0,
+                    "source": self.source}
         sm = [x[0] for x in samples]
         load = [x for x in samples if not (x[2] & 0x1)] or samples  # drop GPU-idle samples
         reasons = sorted({n for x in samples for b, n in _REASON_BITS.items() if x[2] & b})
         return {"sm_mhz": statistics.median(x[0] for x in load),
-                "sm_min_mhz": min(sm), "sm_max_mhz": getattr(self, "sm_max", None),
+                "sm_min_mhz": min(sm), "sm_max_mhz": self.sm_max,
                 "reasons": reasons, "samples": len(samples), "samples_under_load": len(load),
                 "power_w_max": max((x[1] for x in samples), default=None),
                 "source": self.source}
@@ -343,10 +363,17 @@ def run_b200(args, w):
     stream = torch.cuda.current_stream(dev)
 
     pair = args.kernel == "pair"
-    fwd_into = tab.attn_fwd_pair_into if pair else tab.attn_fwd_into
+    # the timed step calls the C ABI directly (the library's boundary), with
+    # the arguments marshalled once
+    import ctypes
+    fn = tab.library().attn_fwd_pair if pair else tab.library().attn_fwd
+    cargs = (q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(), w.B, w.H,
+             w.N, w.d, int(w.causal), ctypes.c_float(w.scale), stream.cuda_stream)
 
     def step():
-        fwd_into(q, k, v, o, lse, causal=w.causal, scale=w.scale, stream=stream)
+        rc = fn(*cargs)
+        if rc != 0:
+            raise SystemExit(f"attn_fwd returned {rc}: {tab.strerror(rc)}")
 
     sampler = ClockSampler(dev)
     for _ in range(args.warmup):

@@ -356,6 +356,18 @@ const char* attn_strerror(int status);
 int attn_check_args(const void* q, const void* k, const void* v, const void* o,
                     const float* lse, int B, int H, int N, int d, float scale);
 
+/*
+ * attn_release -- drop the library's host-side cache of encoded TMA tensor
+ * maps.  Every launch needs three maps (Q, K, V views); they are cached,
+ * keyed by every argument of the encode (buffer address, extents, strides,
+ * box), so a repeated call on the same buffers skips the host work of
+ * encoding them.  A cached map is bit for bit the one a fresh encode would
+ * give, so a buffer that is freed and reallocated at the same address needs
+ * no call here; the cache only holds host memory (a few KB), which this
+ * call returns to its empty state.  Thread-safe.  Always ATTN_OK.
+ */
+int attn_release(void);
+
 /* Library version, (major << 16) | (minor << 8) | patch. */
 int attn_version(void);
 

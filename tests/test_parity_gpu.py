@@ -250,3 +250,25 @@ def test_buffers_not_on_the_device_are_refused_before_launch():
     # and the same buffers on the device still work
     tab.attn_fwd_into(q, k, v, o, lse, causal=True)
     assert tab.last_device_error() == 0 and torch.isfinite(o).all()
+
+
+def test_tensor_map_cache_follows_the_buffers(oracle_mod):
+    """Launches reuse cached tensor maps keyed by address and shape: the same
+    address with a new shape, new contents at a cached address, and calls
+    after attn_release all give the oracle's results."""
+    causal, d = True, 128
+    scale = 1 / math.sqrt(d)
+    big = torch.empty(3 * 2 * 4 * 512 * d, dtype=torch.bfloat16, device="cuda")
+    for (B, H, N, seed) in ((2, 4, 512, 21), (1, 4, 512, 22), (2, 2, 1024, 23), (2, 4, 512, 24)):
+        q, k, v = make_qkv(B, H, N, d, seed)
+        n = B * H * N * d
+        qd, kd, vd = (big[i * n:(i + 1) * n].view(B, H, N, d) for i in range(3))
+        for dst, src in ((qd, q), (kd, k), (vd, v)):
+            dst.copy_(src)
+        o, lse = tab.attn_fwd(qd, kd, vd, causal=causal, scale=scale)
+        assert tab.last_device_error() == 0
+        o_ref, l_ref = oracle_mod.attn_ref(bf16_bits(q), bf16_bits(k), bf16_bits(v), causal, scale)
+        check(o.float().cpu().numpy().astype(np.float64), lse.cpu().numpy().astype(np.float64),
+              o_ref, l_ref, f"cache B{B} H{H} N{N}")
+        if seed == 23:
+            assert tab.library().attn_release() == 0

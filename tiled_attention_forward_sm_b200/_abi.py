@@ -61,6 +61,8 @@ def library():
         lib.attn_check_args.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, f]
         lib.attn_version.restype = i
         lib.attn_version.argtypes = []
+        lib.attn_release.restype = i
+        lib.attn_release.argtypes = []
         lib.attn_fwd_chunk.restype = i
         lib.attn_fwd_chunk.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, i, i, f, i, vp]
         lib.attn_fwd_varlen.restype = i

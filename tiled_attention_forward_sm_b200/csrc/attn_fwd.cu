@@ -52,13 +52,79 @@ int* next_queue_slot(DeviceState& st) {
   return st.queue + 2 * static_cast<int>(st.launches.fetch_add(1) % kQueueSlots);
 }
 
+namespace {
+// Host-side cache of encoded tensor maps.  A map is a pure function of the
+// encode's arguments (type, address, extents, strides, box; the rest is
+// fixed below), so a hit hands back exactly what a fresh encode would: the
+// cache only saves the host time of encoding three maps per launch.  The
+// least recently used entry is replaced when it is full.
+struct TmapEntry {
+  bool used = false;
+  unsigned long long stamp = 0;
+  CUtensorMapDataType type{};
+  const void* ptr = nullptr;
+  cuuint64_t dims[3] = {0, 0, 0};
+  cuuint64_t strides[2] = {0, 0};
+  cuuint32_t box[3] = {0, 0, 0};
+  CUtensorMap map{};
+};
+constexpr int kTmapCacheEntries = 48;
+std::mutex g_tmap_mu;
+TmapEntry g_tmap[kTmapCacheEntries];
+unsigned long long g_tmap_clock = 0;
+}  // namespace
+
 CUresult encode_tiled(CUtensorMap* m, CUtensorMapDataType type, const void* ptr,
                       const cuuint64_t* dims, const cuuint64_t* strides, const cuuint32_t* box) {
+  std::lock_guard<std::mutex> lock(g_tmap_mu);
+  int victim = 0;
+  for (int i = 0; i < kTmapCacheEntries; ++i) {
+    TmapEntry& e = g_tmap[i];
+    if (e.used && e.type == type && e.ptr == ptr && e.dims[0] == dims[0] && e.dims[1] == dims[1] &&
+        e.dims[2] == dims[2] && e.strides[0] == strides[0] && e.strides[1] == strides[1] &&
+        e.box[0] == box[0] && e.box[1] == box[1] && e.box[2] == box[2]) {
+      e.stamp = ++g_tmap_clock;
+      *m = e.map;
+      return CUDA_SUCCESS;
+    }
+    if (!e.used || (g_tmap[victim].used && e.stamp < g_tmap[victim].stamp)) victim = i;
+  }
   cuuint32_t estr[3] = {1, 1, 1};
-  return g_encode(m, type, 3, const_cast<void*>(ptr), const_cast<cuuint64_t*>(dims),
-                  const_cast<cuuint64_t*>(strides), const_cast<cuuint32_t*>(box), estr,
-                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  const CUresult rc = g_encode(m, type, 3, const_cast<void*>(ptr), const_cast<cuuint64_t*>(dims),
+                               const_cast<cuuint64_t*>(strides), const_cast<cuuint32_t*>(box),
+                               estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                               CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (rc != CUDA_SUCCESS) return rc;
+  TmapEntry& e = g_tmap[victim];
+  e.used = true;
+  e.stamp = ++g_tmap_clock;
+  e.type = type;
+  e.ptr = ptr;
+  for (int k = 0; k < 3; ++k) e.dims[k] = dims[k];
+  e.strides[0] = strides[0];
+  e.strides[1] = strides[1];
+  for (int k = 0; k < 3; ++k) e.box[k] = box[k];
+  e.map = *m;
+  return CUDA_SUCCESS;
+}
+
+void tmap_cache_clear() {
+  std::lock_guard<std::mutex> lock(g_tmap_mu);
+  for (TmapEntry& e : g_tmap) e.used = false;
+}
+
+int set_smem_once(const void* kern, int bytes, const DeviceState& st,
+                  std::atomic<unsigned long long>& done) {
+  const unsigned long long bit = 1ull << st.ordinal;
+  if (done.load(std::memory_order_acquire) & bit) return ATTN_OK;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) !=
+      cudaSuccess) {
+    cudaGetLastError();
+    return ATTN_ERR_CUDA;
+  }
+  done.fetch_or(bit, std::memory_order_release);
+  return ATTN_OK;
 }
 
 // Per-device one-time set-up: capability check and the status word address.
@@ -316,11 +382,9 @@ int launch(const Problem& p, cudaStream_t stream, DeviceState& st, int* queue = 
     }();
     if (!regs_ok) return ATTN_ERR_CUDA;
   }
-  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes) !=
-      cudaSuccess) {
-    cudaGetLastError();
+  static std::atomic<unsigned long long> smem_set{0};
+  if (set_smem_once(reinterpret_cast<const void*>(kern), smem_bytes, st, smem_set) != ATTN_OK)
     return ATTN_ERR_CUDA;
-  }
   cudaLaunchConfig_t cfg;
   std::memset(&cfg, 0, sizeof cfg);
   // Persistent: one CTA per SM (at most one per work item).
@@ -674,4 +738,9 @@ extern "C" int attn_trace_set_buffer(void* dev_buf) {
 }
 #endif
 
-extern "C" int attn_version(void) { return (0 << 16) | (1 << 8) | 0; }
+extern "C" int attn_release(void) {
+  tmap_cache_clear();
+  return ATTN_OK;
+}
+
+extern "C" int attn_version(void) { return (0 << 16) | (2 << 8) | 0; }

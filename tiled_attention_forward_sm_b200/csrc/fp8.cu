@@ -95,11 +95,10 @@ extern "C" int attn_fwd_fp8(const void* q, const void* k, const void* vt, void* 
   args.status = st->status;
   args.queue = next_queue_slot(*st);
   auto kern = causal ? fp8::attn_fwd_fp8_kernel<true> : fp8::attn_fwd_fp8_kernel<false>;
-  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, fp8::kSmemBytes) !=
-      cudaSuccess) {
-    cudaGetLastError();
+  static std::atomic<unsigned long long> smem_set[2] = {{0}, {0}};
+  if (set_smem_once(reinterpret_cast<const void*>(kern), fp8::kSmemBytes, *st,
+                    smem_set[causal ? 1 : 0]) != ATTN_OK)
     return ATTN_ERR_CUDA;
-  }
   cudaLaunchConfig_t cfg;
   std::memset(&cfg, 0, sizeof cfg);
   const int grid = args.n_items < st->num_sms ? args.n_items : st->num_sms;

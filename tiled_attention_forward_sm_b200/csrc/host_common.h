@@ -43,9 +43,20 @@ int* next_queue_slot(DeviceState& st);
 // cuTensorMapEncodeTiled for a 3-D tensor with the 128-byte swizzle, no
 // interleave, zero fill out of bounds; dims/strides/box as the driver call
 // takes them (strides: the two outer ones, in bytes).  device_state() must
-// have succeeded first.
+// have succeeded first.  Encoded maps are cached host-side, keyed by every
+// argument of the encode (a map holds nothing else, so a cached map is the
+// one a fresh encode would give).
 CUresult encode_tiled(CUtensorMap* m, CUtensorMapDataType type, const void* ptr,
                       const cuuint64_t* dims, const cuuint64_t* strides, const cuuint32_t* box);
+
+// Drop every cached tensor map (attn_release); later calls encode again.
+void tmap_cache_clear();
+
+// cudaFuncSetAttribute(kern, MaxDynamicSharedMemorySize, bytes) on the
+// current device, once per device: `done` is the kernel's bit mask of the
+// devices already set (one static per kernel at the call site).
+int set_smem_once(const void* kern, int bytes, const DeviceState& st,
+                  std::atomic<unsigned long long>& done);
 
 // Per-head bf16 view [Z][N][d], boxes of 128 rows x 64 columns.
 int make_tmap_heads(CUtensorMap* m, const void* ptr, int Z, int N, int d);

@@ -67,11 +67,9 @@ int launch_kmeans(const void* x, const void* cent, float* ws, int32_t* assign, f
   out.xnorm = xnorm;
   out.x = static_cast<const __nv_bfloat16*>(x);
   auto kern = kmeans::kmeans_assign_kernel<D>;
-  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, KC::kSmemBytes) !=
-      cudaSuccess) {
-    cudaGetLastError();
+  static std::atomic<unsigned long long> smem_set{0};
+  if (set_smem_once(reinterpret_cast<const void*>(kern), KC::kSmemBytes, st, smem_set) != ATTN_OK)
     return ATTN_ERR_CUDA;
-  }
   cudaLaunchConfig_t cfg;
   std::memset(&cfg, 0, sizeof cfg);
   const int grid = args.n_items < st.num_sms ? args.n_items : st.num_sms;

@@ -30,11 +30,9 @@ int launch_pair(const void* q, const void* k, const void* v, void* o, float* lse
       make_tmap_heads_rows(&tv, v, BH, N, kD, 128))
     return ATTN_ERR_CUDA;
   auto kern = attn_fwd_pair_kernel<CAUSAL>;
-  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, pair::kSmemBytes) !=
-      cudaSuccess) {
-    cudaGetLastError();
+  static std::atomic<unsigned long long> smem_set{0};
+  if (set_smem_once(reinterpret_cast<const void*>(kern), pair::kSmemBytes, st, smem_set) != ATTN_OK)
     return ATTN_ERR_CUDA;
-  }
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = 2;
