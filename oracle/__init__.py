@@ -314,6 +314,104 @@ def quantize_e4m3(x_bits, inv_descale: float):
     return e4m3_encode(round_e4m3(bf16_bits_to_f64(x_bits) * float(inv_descale)))
 
 
+# ---------------------------------------------------------------- FP4 ---
+# The 4-bit path reads "FP4" as NVFP4: E2M1 elements (OCP microscaling
+# element type: sign, 2 exponent bits with bias 1, 1 mantissa bit; values
+# 0, 0.5, 1, 1.5, 2, 3, 4, 6) with one E4M3 scale per 16 consecutive
+# elements along the products' reduction dimension, and a per-tensor fp32
+# descale.  Page lecompute.fr/kernel-perf/flashattention-4-limites-calcul-
+# matriciel, section "Le FP4 ajoute un compromis numerique": four-bit
+# arithmetic, whose data preparation and conversion eat into the gain.
+
+NVFP4_BLOCK = 16
+
+
+def e2m1_bits_to_f64(codes) -> np.ndarray:
+    """Decode 4-bit E2M1 codes (the low nibble of each byte): bit 3 sign,
+    bits 2..1 exponent e (bias 1), bit 0 mantissa m; e = 0 is subnormal
+    (m / 2), otherwise 2^(e - 1) (1 + m / 2).  No infinities or NaN."""
+    c = np.asarray(codes, dtype=np.uint8).astype(np.int64) & 0xF
+    sign = np.where(c & 0x8, -1.0, 1.0)
+    e = (c >> 1) & 0x3
+    m = c & 0x1
+    mag = np.where(e == 0, m * 0.5, np.exp2(e - 1.0) * (1.0 + m * 0.5))
+    return sign * mag
+
+
+def round_e2m1(x) -> np.ndarray:
+    """Nearest E2M1 value of float64 inputs, ties to the even mantissa,
+    saturating at +-6.  The representable magnitudes are multiples of 0.5
+    below 2, of 1 in [2, 4) and of 2 in [4, 6]; inside each of those ranges
+    an even multiple has an even mantissa, so rounding the multiple to even
+    is rounding the mantissa to even."""
+    x = np.asarray(x, dtype=np.float64)
+    a = np.abs(x)
+    step = np.where(a < 2.0, 0.5, np.where(a < 4.0, 1.0, 2.0))
+    r = np.minimum(np.round(a / step) * step, 6.0)  # numpy rounds halves to even
+    return np.where(np.signbit(x), -r, r)
+
+
+def e2m1_encode(x) -> np.ndarray:
+    """E2M1 codes (uint8, low nibble) of values that are already E2M1
+    values; the sign of a zero is kept (-0 encodes as 0x8)."""
+    x = np.asarray(x, dtype=np.float64)
+    a = np.abs(x)
+    table = np.array([0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0])
+    idx = np.searchsorted(table, a)
+    if not np.all(table[np.minimum(idx, 7)] == a):
+        raise ValueError("e2m1_encode: value not representable in E2M1")
+    return (idx | (np.signbit(x).astype(np.int64) << 3)).astype(np.uint8)
+
+
+def nvfp4_quantize_f32(xf):
+    """NVFP4 quantisation of float32 values along their last axis (a
+    multiple of 16 long), with the steps taken in float32 as written:
+    per block of 16, amax = max |x|; the scale is amax / 6 rounded to E4M3
+    (nearest even, saturating at 448); each element is x * (1 / scale)
+    (both roundings float32) rounded to E2M1 (nearest even, saturating at
+    +-6); a block whose scale rounds to 0 stores zeros.  Returns (E2M1
+    codes [..., n], E4M3 scale codes [..., n / 16])."""
+    xf = np.asarray(xf, dtype=np.float32)
+    n = xf.shape[-1]
+    if n % NVFP4_BLOCK:
+        raise ValueError("nvfp4: the quantised axis must be a multiple of 16")
+    blk = xf.reshape(xf.shape[:-1] + (n // NVFP4_BLOCK, NVFP4_BLOCK))
+    amax = np.abs(blk).max(axis=-1)
+    s = round_e4m3((amax / np.float32(6.0)).astype(np.float32).astype(np.float64))
+    s32 = s.astype(np.float32)
+    with np.errstate(divide="ignore"):
+        inv = np.where(s32 > 0, np.float32(1.0) / np.where(s32 > 0, s32, np.float32(1.0)),
+                       np.float32(0.0)).astype(np.float32)
+    q = (blk * inv[..., None]).astype(np.float32)
+    codes = e2m1_encode(round_e2m1(q.astype(np.float64)))
+    return codes.reshape(xf.shape), e4m3_encode(s)
+
+
+def quantize_nvfp4(x_bits, inv_descale: float):
+    """NVFP4 codes of bf16 values times inv_descale (the product taken in
+    float32), quantised along the last axis: the conversion the 4-bit
+    path's inputs go through.  Returns (codes, scale codes)."""
+    xf = (bf16_bits_to_f64(x_bits).astype(np.float32) * np.float32(inv_descale)).astype(np.float32)
+    return nvfp4_quantize_f32(xf)
+
+
+def nvfp4_to_f64(codes, scale_codes, descale: float = 1.0) -> np.ndarray:
+    """Values of NVFP4 data: E2M1 value * its block's E4M3 scale * descale."""
+    v = e2m1_bits_to_f64(codes)
+    s = e4m3_bits_to_f64(scale_codes)
+    n = v.shape[-1]
+    v = v.reshape(v.shape[:-1] + (n // NVFP4_BLOCK, NVFP4_BLOCK)) * s[..., None]
+    return v.reshape(v.shape[:-2] + (n,)) * float(descale)
+
+
+def round_nvfp4_rows(p) -> np.ndarray:
+    """Values of float64 rows after NVFP4 quantisation of each row along its
+    last axis (a multiple of 16): the rounding the 4-bit path applies to the
+    softmax weights before the second product."""
+    codes, sc = nvfp4_quantize_f32(np.asarray(p, dtype=np.float64).astype(np.float32))
+    return nvfp4_to_f64(codes, sc)
+
+
 def bf16_bits_to_f64(bits) -> np.ndarray:
     """Exact widening of bf16 bit patterns to float64."""
     bits = np.asarray(bits, dtype=np.uint16)
@@ -347,8 +445,9 @@ def tiled_online_model(q, k, v, causal: bool, scale: float, block_n: int = 128,
     q, k, v: float64 [N, d].  Returns (o [N, d], lse [N]) in float64.
     With ``round_p_bf16`` (or ``round_p="bf16"``) the weights are rounded to
     bf16 before the second product (what the kernel feeds its tensor cores);
-    ``round_p="e4m3"`` rounds them to FP8 E4M3 instead (the FP8 path).  The
-    row sum stays exact.
+    ``round_p="e4m3"`` rounds them to FP8 E4M3 instead (the FP8 path), and
+    ``round_p="nvfp4"`` to NVFP4 per row in blocks of 16 keys (the 4-bit
+    path).  The row sum stays exact.
     """
     if round_p_bf16:
         round_p = "bf16"
@@ -376,7 +475,15 @@ def tiled_online_model(q, k, v, causal: bool, scale: float, block_n: int = 128,
             p = np.exp2(x - m_used[:, None])
         p = np.where(np.isneginf(x), 0.0, p)
         l = l * alpha + p.sum(axis=1)
-        pv = _round_bf16(p) if round_p == "bf16" else (round_e4m3(p) if round_p == "e4m3" else p)
+        if round_p == "bf16":
+            pv = _round_bf16(p)
+        elif round_p == "e4m3":
+            pv = round_e4m3(p)
+        elif round_p == "nvfp4":
+            pad = (-len(cols)) % NVFP4_BLOCK  # a ragged last tile: zero keys
+            pv = round_nvfp4_rows(np.pad(p, ((0, 0), (0, pad))))[:, : len(cols)]
+        else:
+            pv = p
         acc = acc * alpha[:, None] + pv @ v[cols]
         m = m_used
     o = acc / l[:, None]
