@@ -366,9 +366,20 @@ def run_b200(args, w):
     # the timed step calls the C ABI directly (the library's boundary), with
     # the arguments marshalled once
     import ctypes
-    fn = tab.library().attn_fwd_pair if pair else tab.library().attn_fwd
+    tuned = (args.exp2_poly_pairs, args.kv_stages, args.rescale_tau) != (None, None, None)
+    if pair and tuned:
+        raise SystemExit("the tuning options apply to attn_fwd, not to the pair kernel")
     cargs = (q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(), w.B, w.H,
-             w.N, w.d, int(w.causal), ctypes.c_float(w.scale), stream.cuda_stream)
+             w.N, w.d, int(w.causal), ctypes.c_float(w.scale))
+    if tuned:
+        opts = tab.AttnOpts(-1 if args.exp2_poly_pairs is None else args.exp2_poly_pairs,
+                            0 if args.kv_stages is None else args.kv_stages,
+                            -1.0 if args.rescale_tau is None else args.rescale_tau)
+        fn = tab.library().attn_fwd_ex
+        cargs = cargs + (ctypes.byref(opts), stream.cuda_stream)
+    else:
+        fn = tab.library().attn_fwd_pair if pair else tab.library().attn_fwd
+        cargs = cargs + (stream.cuda_stream,)
 
     def step():
         rc = fn(*cargs)
@@ -408,19 +419,22 @@ def run_b200(args, w):
         o_p.copy_(o, non_blocking=True)
         lse_p.copy_(lse, non_blocking=True)
 
-    for _ in range(min(args.warmup, 3)):
-        e2e_step()
-    if pg:
-        torch.distributed.barrier()
-    torch.cuda.synchronize(dev)
-    f0 = torch.cuda.Event(enable_timing=True)
-    f1 = torch.cuda.Event(enable_timing=True)
-    f0.record(stream)
-    for _ in range(e2e_steps):
-        e2e_step()
-    f1.record(stream)
-    torch.cuda.synchronize(dev)
-    e2e_ms = f0.elapsed_time(f1) / e2e_steps
+    if args.no_e2e:
+        e2e_ms = float("nan")
+    else:
+        for _ in range(min(args.warmup, 3)):
+            e2e_step()
+        if pg:
+            torch.distributed.barrier()
+        torch.cuda.synchronize(dev)
+        f0 = torch.cuda.Event(enable_timing=True)
+        f1 = torch.cuda.Event(enable_timing=True)
+        f0.record(stream)
+        for _ in range(e2e_steps):
+            e2e_step()
+        f1.record(stream)
+        torch.cuda.synchronize(dev)
+        e2e_ms = f0.elapsed_time(f1) / e2e_steps
 
     t = torch.tensor([ms_total, e2e_ms], dtype=torch.float64, device=dev)
     if pg:
@@ -457,7 +471,10 @@ def run_b200(args, w):
                    "flops_per_step": w.flops,
                    "l2": f"inputs larger than L2: Q+K+V {3 * tb / 1e6:.0f} MB vs 126 MB; no flush",
                    "parallelism": f"replica x{world} (independent batches)",
-                   "kernel": "cta_pair (attn_fwd_pair)" if pair else "one_cta (attn_fwd)"},
+                   "kernel": "cta_pair (attn_fwd_pair)" if pair else "one_cta (attn_fwd)",
+                   "tuning": None if not tuned else {
+                       "exp2_poly_pairs": args.exp2_poly_pairs, "kv_stages": args.kv_stages,
+                       "rescale_tau": args.rescale_tau}},
         "roofline": {"bound": "tensor", "achieved": round(achieved, 2),
                      "peak": peak, "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
                      "peak_source": f"{peak_kind} bf16 burst (MEASURED_PEAKS.json)"
@@ -467,11 +484,12 @@ def run_b200(args, w):
                      "frac_of_datasheet_2250": round(achieved / DATASHEET_BF16_TFLOPS, 4),
                      "traffic": traffic,
                      "algorithmic_bytes": 4 * tb + w.rows * 4},
-        "e2e": {"value": round(e2e_value, 2), "unit": UNIT,
-                "h2d_bytes_per_step": 3 * tb, "d2h_bytes_per_step": tb + w.rows * 4,
-                "steps": e2e_steps, "ms_per_step": round(e2e_ms, 4),
-                "api": ("attn_fwd_pair_into between pinned-host copies" if pair else
-                        "attn_fwd_host (pinned host buffers, copies in the timed region)")},
+        "e2e": None if args.no_e2e else {
+            "value": round(e2e_value, 2), "unit": UNIT,
+            "h2d_bytes_per_step": 3 * tb, "d2h_bytes_per_step": tb + w.rows * 4,
+            "steps": e2e_steps, "ms_per_step": round(e2e_ms, 4),
+            "api": ("attn_fwd_pair_into between pinned-host copies" if pair else
+                    "attn_fwd_host (pinned host buffers, copies in the timed region)")},
         "gpu_launches": args.steps,
         "clocks": clocks,
         "kernel_sha": kernel_sha(sources),
@@ -697,6 +715,95 @@ def run_fp8(args, w):
     }
 
 
+# ----------------------------------------------------------- FP4 path -----
+FP4_SUFFIX = "_fp4"
+
+
+def run_fp4(args, w):
+    """The 4-bit (NVFP4) attention on a square workload's shapes: the
+    attention alone (the line's value) and the bf16 -> NVFP4 conversion of
+    Q, K and V^T that feeds it (conversion_ms, and the metric with the
+    conversion included)."""
+    import ctypes
+    import tiled_attention_forward_sm_b200 as tab
+    world, rank, local = dist_env()
+    if world > 1:
+        raise SystemExit("FP4 workloads run on one GPU")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    q_h, k_h, v_h = make_workload_inputs(w)
+    q, k, v = (t.to(dev) for t in (q_h, k_h, v_h))
+    stream = torch.cuda.current_stream(dev)
+    lib = tab.library()
+    sh = stream.cuda_stream
+    BH = w.B * w.H
+    T = (w.N + 127) // 128
+    qc = torch.empty((w.B, w.H, w.N, 64), dtype=torch.uint8, device=dev)
+    kc = torch.empty_like(qc)
+    vc = torch.empty((w.B, w.H, 128, w.N // 2), dtype=torch.uint8, device=dev)
+    qs, ks, vs = (torch.empty((BH, T, 2, 512), dtype=torch.uint8, device=dev) for _ in range(3))
+    o = torch.empty_like(q)
+    lse = torch.empty((w.B, w.H, w.N), dtype=torch.float32, device=dev)
+
+    def convert():
+        for src, c, sc, tr in ((q, qc, qs, 0), (k, kc, ks, 0), (v, vc, vs, 1)):
+            rc = lib.attn_quantize_nvfp4(src.data_ptr(), c.data_ptr(), sc.data_ptr(), BH, w.N,
+                                         w.d, ctypes.c_float(1.0), tr, sh)
+            assert rc == 0, rc
+
+    cargs = (qc.data_ptr(), qs.data_ptr(), kc.data_ptr(), ks.data_ptr(), vc.data_ptr(),
+             vs.data_ptr(), o.data_ptr(), lse.data_ptr(), w.B, w.H, w.N, w.d, int(w.causal),
+             ctypes.c_float(w.scale), ctypes.c_float(1.0), ctypes.c_float(1.0),
+             ctypes.c_float(1.0), sh)
+
+    def attend():
+        rc = lib.attn_fwd_fp4(*cargs)
+        assert rc == 0, rc
+
+    def timed(fn, steps):
+        for _ in range(args.warmup):
+            fn()
+        return timed_steps(fn, steps, stream, dev)[0] / steps
+
+    convert()
+    sampler = ClockSampler(dev)
+    sampler.start()
+    ms_attn = timed(attend, args.steps)
+    clocks = sampler.stop()
+    ms_conv = timed(convert, max(1, args.steps // 4))
+    status = tab.last_device_error(stream)
+    if status != 0:
+        raise SystemExit(f"device status {status}: {tab.strerror(status)}")
+    tflops = w.flops / (ms_attn * 1e-3) / 1e12
+    peaks, peak_kind = load_peaks()
+    # per element: 2 bytes read, half a byte of codes and 1/16 byte of scale written
+    conv_bytes = 3 * w.rows * w.d * (2 + 0.5 + 1 / 16)
+    if clocks.get("sm_mhz"):
+        clocks["kcycles_per_step"] = round(ms_attn * clocks["sm_mhz"], 1)
+    return {
+        "metric": METRIC.replace("(bf16, d=128)", "(NVFP4 operands, d=128)"),
+        "value": round(tflops, 2), "unit": UNIT, "n_gpus": 1, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms_attn, 4), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "nvfp4",
+        "data": "synthetic (the square workload's seeded bf16 inputs, converted to NVFP4)",
+        "config": {"workload": w.name + FP4_SUFFIX, "B": w.B, "H": w.H, "N": w.N, "d": w.d,
+                   "causal": w.causal, "flops_per_step": w.flops, "descales": [1.0, 1.0, 1.0],
+                   "l2": "inputs larger than L2; no flush"},
+        "roofline": {"bound": "tensor", "achieved": round(tflops, 2),
+                     "peak": 4.0 * float(peaks["bf16_tflops"]), "unit": "TFLOP/s",
+                     "frac": round(tflops / (4.0 * float(peaks["bf16_tflops"])), 4),
+                     "peak_source": f"{peak_kind} bf16 burst x 4 (the nominal fp4:bf16 ratio)",
+                     "traffic": None},
+        "conversion": {"ms": round(ms_conv, 4), "launches": 3,
+                       "gbs": round(conv_bytes / (ms_conv * 1e-3) / 1e9, 1),
+                       "hbm_frac": round(conv_bytes / (ms_conv * 1e-3) / 1e9 /
+                                         float(peaks["hbm_gbs"]), 4),
+                       "tflops_with_conversion": round(w.flops / ((ms_attn + ms_conv) * 1e-3)
+                                                       / 1e12, 2)},
+        "e2e": None, "gpu_launches": args.steps, "clocks": clocks, "kernel_sha": kernel_sha(),
+    }
+
+
 # ------------------------------------------------- k-means assignment -----
 def run_kmeans(args, w):
     import ctypes
@@ -816,13 +923,22 @@ def main():
     ap.add_argument("--workload", default=BENCH_WORKLOAD,
                     choices=sorted(WORKLOADS) + sorted(GENERAL_WORKLOADS) +
                     sorted(KMEANS_WORKLOADS) +
-                    sorted(n + FP8_SUFFIX for n, w_ in WORKLOADS.items() if w_.d == 128))
+                    sorted(n + FP8_SUFFIX for n, w_ in WORKLOADS.items() if w_.d == 128) +
+                    sorted(n + FP4_SUFFIX for n, w_ in WORKLOADS.items() if w_.d == 128))
     ap.add_argument("--kernel", choices=["one_cta", "pair"], default="one_cta",
                     help="bf16 workloads at d=128: attn_fwd (one CTA per SM) or attn_fwd_pair "
                          "(clusters of two CTAs sharing each product)")
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true",
+                    help="skip the end-to-end (host buffers) measurement")
+    ap.add_argument("--exp2-poly-pairs", type=int, default=None,
+                    help="attn_fwd_ex option: exponential pairs of every 4 on the FMA polynomial")
+    ap.add_argument("--kv-stages", type=int, default=None,
+                    help="attn_fwd_ex option: K/V ring depth (2..5 at d = 128)")
+    ap.add_argument("--rescale-tau", type=float, default=None,
+                    help="attn_fwd_ex option: lazy-rescale threshold (0..16, log2 units)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -830,7 +946,11 @@ def main():
     if args.gpus != world:
         ap.error(f"--gpus {args.gpus} but WORLD_SIZE is {world}: launch N > 1 ranks with "
                  f"python -m torch.distributed.run --nproc-per-node N bench.py --gpus N")
-    if args.workload.endswith(FP8_SUFFIX):
+    if args.workload.endswith(FP4_SUFFIX):
+        if args.impl == "reference":
+            ap.error("--impl reference times the bf16 workloads only")
+        line = run_fp4(args, WORKLOADS[args.workload[: -len(FP4_SUFFIX)]])
+    elif args.workload.endswith(FP8_SUFFIX):
         if args.impl == "reference":
             ap.error("--impl reference times the bf16 workloads only")
         line = run_fp8(args, WORKLOADS[args.workload[: -len(FP8_SUFFIX)]])

@@ -82,15 +82,39 @@ int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
 /*
  * Tuning options for attn_fwd_ex.  Every option only changes how the same
  * result is computed (rounding differs within the documented tolerance).
+ * Start from attn_opts_default() and set the fields you need.
  *   exp2_poly_pairs  of every 4 pairs of score columns, how many take their
  *                    exponential from an FMA-pipe polynomial instead of the
  *                    special-function unit (the split described on the page's
  *                    section "Deplacer une partie des exponentielles");
  *                    0, 1 or 2, or -1 for the library default.
+ *   kv_stages        depth of the shared-memory ring that K and V tiles flow
+ *                    through (page lecompute.fr/en/kernel-perf/flapping-
+ *                    airplanes-thunderkittens-megakernels, section "Prepare
+ *                    the next operation without overwriting the current
+ *                    one"): 0 for the default (4 at d = 96 and 128, 8 at
+ *                    d = 64), or 2, 3, 4 or 5 at d = 128 with the default
+ *                    exponential split (other head dims or splits return
+ *                    ATTN_ERR_UNSUPPORTED; 1 or more than 5 return
+ *                    ATTN_ERR_INVALID_ARG).
+ *   rescale_tau      the lazy-rescale threshold, in log2 units of the
+ *                    scores (section "Deplacer une partie des
+ *                    exponentielles": some rescalings are skipped under a
+ *                    condition): the running maximum moves only when a
+ *                    tile's maximum exceeds it by more than rescale_tau, so
+ *                    weights stay below 2^rescale_tau.  -1 for the default
+ *                    (8), or 0 .. 16 (0: rescale whenever the maximum
+ *                    grows); d <= 128 only (ATTN_ERR_UNSUPPORTED at d = 256).
+ *                    Note 0 is a valid threshold, not the default.
  */
 typedef struct {
   int exp2_poly_pairs;
+  int kv_stages;
+  float rescale_tau;
 } attn_opts;
+
+/* Every option at its default: {-1, 0, -1.f}. */
+attn_opts attn_opts_default(void);
 
 /*
  * attn_fwd_ex -- attn_fwd with tuning options (opts may be NULL: defaults).
@@ -273,6 +297,59 @@ int attn_fwd_fp8(const void* q, const void* k, const void* vt, void* o, float* l
  */
 int attn_quantize_e4m3(const void* src, void* dst, int BH, int N, int d, float inv_descale,
                        int transpose, attn_stream_t stream);
+
+/*
+ * attn_fwd_fp4 -- 4-bit (NVFP4) attention forward, d = 128 (page
+ * lecompute.fr/kernel-perf/flashattention-4-limites-calcul-matriciel,
+ * section "Le FP4 ajoute un compromis numerique": four-bit products, whose
+ * data preparation eats into the gain).  Both products are block-scaled
+ * 4-bit tensor-core MMAs: E2M1 elements with one E4M3 scale per 16
+ * elements of the reduction axis, fp32 accumulation.  The softmax weights
+ * are rounded to the same format (per row and 16 keys: scale =
+ * E4M3(max / 6), codes = E2M1(p / scale)); the row sum uses the unrounded
+ * fp32 weights.  O is bf16 and LSE fp32 as in attn_fwd, of the scores
+ * scale * q_descale * k_descale * (Q K^T), with O scaled by v_descale.
+ *
+ *   q, k      device, E2M1 codes [B, H, N, 64] bytes (two per byte, the
+ *             lower-indexed element in the lower nibble), from
+ *             attn_quantize_nvfp4(transpose = 0).
+ *   q_sf, k_sf  device, their E4M3 scales, attn_nvfp4_scale_bytes(B*H, N)
+ *             bytes, from the same call.
+ *   vt        device, E2M1 codes of V transposed per head, [B, H, 128, N/2]
+ *             bytes; vt_sf its scales; from attn_quantize_nvfp4(transpose).
+ *   o, lse    as attn_fwd (bf16 [B, H, N, 128]; fp32 [B, H, N]).  Written.
+ *   N         > 0 and a multiple of 32 (V^T rows of N/2 bytes must be
+ *             16-byte aligned); d must be 128: otherwise ATTN_ERR_UNSUPPORTED.
+ *   descales  finite and > 0.
+ * Every pointer 16-byte aligned (lse 4); outputs must not overlap inputs.
+ * Causal mask, errors, asynchrony and ownership as attn_fwd.
+ */
+int attn_fwd_fp4(const void* q, const void* q_sf, const void* k, const void* k_sf,
+                 const void* vt, const void* vt_sf, void* o, float* lse, int B, int H, int N,
+                 int d, int causal, float scale, float q_descale, float k_descale,
+                 float v_descale, attn_stream_t stream);
+
+/*
+ * attn_quantize_nvfp4 -- the conversion the 4-bit path's inputs go through.
+ * x = src * inv_descale (float32); per 16 consecutive elements along d
+ * (transpose = 0: Q and K, codes [BH, N, 64] bytes) or along the keys
+ * (transpose != 0: V, codes of V^T [BH, 128, N/2] bytes, N a multiple of
+ * 32): scale = E4M3(amax / 6) (nearest even, saturating at 448),
+ * code = E2M1(x * (1 / scale)) (nearest even, saturating at +-6; zero codes
+ * where the scale is 0).  The scales go to `scales`
+ * (attn_nvfp4_scale_bytes(BH, N) bytes), per head and 128-row tile of the
+ * product's operand in the order the block-scaled MMA reads them: two
+ * 512-byte blocks (the first and second 64 elements of the reduction axis),
+ * row m's four scales at byte 16 (m % 32) + 4 (m / 32) of a block.
+ * src device bf16 [BH, N, 128]; d must be 128; src and codes 16-byte
+ * aligned; no overlaps.  Errors and asynchrony as attn_fwd.
+ */
+int attn_quantize_nvfp4(const void* src, void* codes, void* scales, int BH, int N, int d,
+                        float inv_descale, int transpose, attn_stream_t stream);
+
+/* Bytes of one NVFP4 scale array for BH heads of N rows (or keys): -1 for
+ * non-positive sizes. */
+long long attn_nvfp4_scale_bytes(int BH, int N);
 
 /*
  * attn_kmeans_assign -- the assignment step of k-means (page lefilia.fr,

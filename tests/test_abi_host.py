@@ -109,9 +109,22 @@ def test_fwd_ex_rejects_bad_option_before_any_cuda_call(lib):
     import ctypes
     p = ptrs()
     for bad in (-2, 3, 100):
-        opts = tab.AttnOpts(bad)
+        opts = tab.AttnOpts(bad, 0)
         rc = lib.attn_fwd_ex(*p, 1, 1, 128, 128, 0, 0.1, ctypes.byref(opts), None)
         assert rc == -1
+    for bad in (-1, 1, 6):  # ring depths
+        opts = tab.AttnOpts(-1, bad)
+        assert lib.attn_fwd_ex(*p, 1, 1, 128, 128, 0, 0.1, ctypes.byref(opts), None) == -1
+    # depths other than the default only at d = 128 with the default split
+    assert lib.attn_fwd_ex(*p, 1, 1, 128, 64, 0, 0.1, ctypes.byref(tab.AttnOpts(-1, 3)), None) == -2
+    assert lib.attn_fwd_ex(*p, 1, 1, 128, 128, 0, 0.1, ctypes.byref(tab.AttnOpts(1, 3)), None) == -2
+    for bad in (-0.5, 16.5, float("nan"), float("inf")):  # rescale thresholds
+        opts = tab.AttnOpts(-1, 0, bad)
+        assert lib.attn_fwd_ex(*p, 1, 1, 128, 128, 0, 0.1, ctypes.byref(opts), None) == -1
+    assert lib.attn_fwd_ex(*p, 1, 1, 128, 256, 0, 0.1, ctypes.byref(tab.AttnOpts(-1, 0, 4.0)),
+                           None) == -2
+    d = lib.attn_opts_default()
+    assert (d.exp2_poly_pairs, d.kv_stages, d.rescale_tau) == (-1, 0, -1.0)
 
 
 def test_exp2_polynomial_coefficients_and_error():
@@ -311,3 +324,11 @@ def test_binding_requires_one_cuda_device():
         _abi._device_of(cpu, cpu)
     with pytest.raises(ValueError, match="CUDA tensors"):
         _abi._device_of(None, cpu, None)  # None entries are skipped
+
+
+def test_product_library_carries_no_test_hooks(lib):
+    """The abort-path hooks exist only in the test library."""
+    assert not hasattr(lib, "attn_test_set_hooks")
+    if os.path.exists(tab_build.TEST_HOOKS_LIB):
+        import ctypes
+        assert hasattr(ctypes.CDLL(tab_build.TEST_HOOKS_LIB), "attn_test_set_hooks")

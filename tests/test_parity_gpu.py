@@ -19,9 +19,10 @@ pytestmark = pytest.mark.gpu
 ATOL_O, RTOL_O, ATOL_LSE = 2e-2, 1e-2, 1e-3
 
 
-def gpu_run(q, k, v, causal, scale, poly=None):
+def gpu_run(q, k, v, causal, scale, poly=None, stages=None):
     qd, kd, vd = (t.cuda() for t in (q, k, v))
-    o, lse = tab.attn_fwd(qd, kd, vd, causal=causal, scale=scale, exp2_poly_pairs=poly)
+    o, lse = tab.attn_fwd(qd, kd, vd, causal=causal, scale=scale, exp2_poly_pairs=poly,
+                          kv_stages=stages)
     assert tab.last_device_error() == 0
     return o.float().cpu().numpy().astype(np.float64), lse.cpu().numpy().astype(np.float64)
 
@@ -36,10 +37,11 @@ def check(o_gpu, lse_gpu, o_ref, lse_ref, what=""):
     return err_o.max(), err_l.max()
 
 
-def full_parity(oracle_mod, B, H, N, d, causal, seed, q_std=1.0, scale=None, poly=None):
+def full_parity(oracle_mod, B, H, N, d, causal, seed, q_std=1.0, scale=None, poly=None,
+                stages=None):
     scale = 1 / math.sqrt(d) if scale is None else scale
     q, k, v = make_qkv(B, H, N, d, seed, q_std)
-    o, lse = gpu_run(q, k, v, causal, scale, poly)
+    o, lse = gpu_run(q, k, v, causal, scale, poly, stages)
     o_ref, lse_ref = oracle_mod.attn_ref(bf16_bits(q), bf16_bits(k), bf16_bits(v), causal, scale)
     return check(o, lse, o_ref, lse_ref, f"B{B} H{H} N{N} d{d} causal={causal}")
 
@@ -91,6 +93,28 @@ def test_exp2_split_variants(oracle_mod, poly, d, causal):
     full_parity(oracle_mod, 1, 3, 640, d, causal, seed=31 + poly, q_std=3.0, poly=poly)
 
 
+@pytest.mark.parametrize("stages", [2, 3, 4, 5])
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("N", [200, 1000])
+def test_kv_ring_depths(oracle_mod, stages, causal, N):
+    """Every depth of the K/V ring (page lecompute.fr/en/kernel-perf/flapping-
+    airplanes-thunderkittens-megakernels, section "Prepare the next operation
+    without overwriting the current one": a stage is refilled only after its
+    last reader is done) gives the oracle's result; a ring of 2 stages holds
+    exactly one K and one V tile, so every refill waits on the previous
+    step's release.  Ragged lengths, several work items per CTA."""
+    full_parity(oracle_mod, 2, 5, N, 128, causal, seed=60 + stages + N, q_std=2.0, stages=stages)
+
+
+def test_kv_ring_depths_are_bitwise_equal():
+    """The ring depth changes when tiles arrive, not what is computed."""
+    q, k, v = (t.cuda() for t in make_qkv(2, 4, 1024, 128, 61))
+    o4, l4 = tab.attn_fwd(q, k, v, causal=True)
+    for st in (2, 3, 5):
+        o, l = tab.attn_fwd(q, k, v, causal=True, kv_stages=st)
+        assert torch.equal(o, o4) and torch.equal(l, l4)
+
+
 @pytest.mark.parametrize("name", ["b1h2n256d64", "b4h16n2048d128_causal"])
 def test_workload_full(oracle_mod, name):
     w = WORKLOADS[name]
@@ -120,6 +144,32 @@ def test_lazy_rescale_at_known_rows(oracle_mod, d, causal, jump_tile, second):
     o, lse = gpu_run(q, k, v, causal, scale)
     o_ref, lse_ref = oracle_mod.attn_ref(bf16_bits(q), bf16_bits(k), bf16_bits(v), causal, scale)
     check(o, lse, o_ref, lse_ref, f"jump at tile {jump_tile} d{d} causal={causal}")
+
+
+@pytest.mark.parametrize("tau", [0.0, 4.0, 16.0])
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("causal", [False, True])
+def test_rescale_thresholds(oracle_mod, tau, d, causal):
+    """Any lazy-rescale threshold gives the oracle's result (0: an eager
+    rescale whenever the maximum grows; 16: weights up to 2^16 kept
+    unrescaled), on the constructed jumps and on peaky random scores."""
+    B, H, N = 1, 2, 640
+    scale = math.log(2.0)
+    q, k, v = make_jump_qkv(B, H, N, d, 2, True, seed=450 + d)
+    qd, kd, vd = (t.cuda() for t in (q, k, v))
+    o, lse = tab.attn_fwd(qd, kd, vd, causal=causal, scale=scale, rescale_tau=tau)
+    assert tab.last_device_error() == 0
+    o_ref, lse_ref = oracle_mod.attn_ref(bf16_bits(q), bf16_bits(k), bf16_bits(v), causal, scale)
+    check(o.float().cpu().numpy().astype(np.float64), lse.cpu().numpy().astype(np.float64),
+          o_ref, lse_ref, f"tau {tau}")
+    q, k, v = make_qkv(1, 3, 640, d, 470 + d, q_std=3.0)
+    qd, kd, vd = (t.cuda() for t in (q, k, v))
+    o, lse = tab.attn_fwd(qd, kd, vd, causal=causal, rescale_tau=tau)
+    assert tab.last_device_error() == 0
+    o_ref, lse_ref = oracle_mod.attn_ref(bf16_bits(q), bf16_bits(k), bf16_bits(v), causal,
+                                         1 / math.sqrt(d))
+    check(o.float().cpu().numpy().astype(np.float64), lse.cpu().numpy().astype(np.float64),
+          o_ref, lse_ref, f"tau {tau} peaky")
 
 
 @pytest.mark.parametrize("scale", [0.01, 0.5, 2.0])

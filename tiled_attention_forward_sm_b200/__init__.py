@@ -9,15 +9,15 @@ the calls raise.
 from __future__ import annotations
 
 from ._abi import (ATTN_OK, AttnError, AttnOpts, attn_combine, attn_fwd, attn_fwd_chunk,
-                   attn_fwd_fp8, attn_fwd_pair, attn_fwd_pair_into,
+                   attn_fwd_fp4, attn_fwd_fp8, attn_fwd_pair, attn_fwd_pair_into,
                    attn_fwd_chunk_into, attn_fwd_host, attn_fwd_into, attn_fwd_noalloc_into,
                    attn_fwd_splitkv, attn_fwd_varlen, check_args, kmeans_assign,
-                   last_device_error, library, library_path, quantize_e4m3,
+                   last_device_error, library, library_path, quantize_e4m3, quantize_nvfp4,
                    selftest_wait_timeout, splitkv_slices, strerror)
 
 __all__ = ["ATTN_OK", "AttnError", "AttnOpts", "attn_combine", "attn_fwd", "attn_fwd_chunk",
-           "attn_fwd_fp8", "attn_fwd_pair", "attn_fwd_pair_into",
+           "attn_fwd_fp4", "attn_fwd_fp8", "attn_fwd_pair", "attn_fwd_pair_into",
            "attn_fwd_chunk_into", "attn_fwd_host", "attn_fwd_into", "attn_fwd_noalloc_into",
            "attn_fwd_splitkv", "attn_fwd_varlen", "check_args", "kmeans_assign",
-           "last_device_error", "library", "quantize_e4m3",
+           "last_device_error", "library", "quantize_e4m3", "quantize_nvfp4",
            "library_path", "selftest_wait_timeout", "splitkv_slices", "strerror"]

@@ -19,7 +19,11 @@ _lib = None
 
 class AttnOpts(ctypes.Structure):
     """Mirror of attn_opts in include/attn_b200.h."""
-    _fields_ = [("exp2_poly_pairs", ctypes.c_int)]
+    _fields_ = [("exp2_poly_pairs", ctypes.c_int), ("kv_stages", ctypes.c_int),
+                ("rescale_tau", ctypes.c_float)]
+
+    def __init__(self, exp2_poly_pairs: int = -1, kv_stages: int = 0, rescale_tau: float = -1.0):
+        super().__init__(exp2_poly_pairs, kv_stages, rescale_tau)
 
 
 class AttnError(RuntimeError):
@@ -63,6 +67,8 @@ def library():
         lib.attn_version.argtypes = []
         lib.attn_release.restype = i
         lib.attn_release.argtypes = []
+        lib.attn_opts_default.restype = AttnOpts
+        lib.attn_opts_default.argtypes = []
         lib.attn_fwd_chunk.restype = i
         lib.attn_fwd_chunk.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, i, i, f, i, vp]
         lib.attn_fwd_varlen.restype = i
@@ -73,6 +79,12 @@ def library():
         lib.attn_fwd_fp8.argtypes = [vp] * 5 + [i] * 5 + [f, f, f, f, vp]
         lib.attn_quantize_e4m3.restype = i
         lib.attn_quantize_e4m3.argtypes = [vp, vp, i, i, i, f, i, vp]
+        lib.attn_fwd_fp4.restype = i
+        lib.attn_fwd_fp4.argtypes = [vp] * 8 + [i] * 5 + [f, f, f, f, vp]
+        lib.attn_quantize_nvfp4.restype = i
+        lib.attn_quantize_nvfp4.argtypes = [vp, vp, vp, i, i, i, f, i, vp]
+        lib.attn_nvfp4_scale_bytes.restype = ctypes.c_longlong
+        lib.attn_nvfp4_scale_bytes.argtypes = [i, i]
         lib.attn_kmeans_assign.restype = i
         lib.attn_kmeans_assign.argtypes = [vp, vp, vp, vp, vp, i, i, i, vp]
         lib.attn_kmeans_workspace_floats.restype = ctypes.c_longlong
@@ -124,10 +136,12 @@ def _shape(q: torch.Tensor):
 
 
 def attn_fwd_into(q, k, v, o, lse, causal: bool = False, scale: float | None = None,
-                  stream=None, exp2_poly_pairs: int | None = None) -> None:
+                  stream=None, exp2_poly_pairs: int | None = None,
+                  kv_stages: int | None = None, rescale_tau: float | None = None) -> None:
     """Enqueue the forward pass writing into ``o`` (bf16 [B,H,N,d]) and ``lse``
     (fp32 [B,H,N]).  Inputs: CUDA bf16 contiguous [B,H,N,d] tensors.
-    ``exp2_poly_pairs`` (0..2) selects the attn_fwd_ex tuning option."""
+    ``exp2_poly_pairs`` (0..2), ``kv_stages`` (2..5 at d = 128) and
+    ``rescale_tau`` (0..16, d <= 128) select the attn_fwd_ex tuning options."""
     B, H, N, d = _shape(q)
     for name, t, dt in (("q", q, torch.bfloat16), ("k", k, torch.bfloat16),
                         ("v", v, torch.bfloat16), ("o", o, torch.bfloat16)):
@@ -141,11 +155,13 @@ def attn_fwd_into(q, k, v, o, lse, causal: bool = False, scale: float | None = N
     args = (q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
             B, H, N, d, int(bool(causal)), float(scale))
     dev = _device_of(q, k, v, o, lse)
-    if exp2_poly_pairs is None:
+    if exp2_poly_pairs is None and kv_stages is None and rescale_tau is None:
         with torch.cuda.device(dev):
             rc = library().attn_fwd(*args, _stream_handle(stream, dev))
     else:
-        opts = AttnOpts(int(exp2_poly_pairs))
+        opts = AttnOpts(-1 if exp2_poly_pairs is None else int(exp2_poly_pairs),
+                        0 if kv_stages is None else int(kv_stages),
+                        -1.0 if rescale_tau is None else float(rescale_tau))
         with torch.cuda.device(dev):
             rc = library().attn_fwd_ex(*args, ctypes.byref(opts), _stream_handle(stream, dev))
     if rc != ATTN_OK:
@@ -153,13 +169,14 @@ def attn_fwd_into(q, k, v, o, lse, causal: bool = False, scale: float | None = N
 
 
 def attn_fwd(q, k, v, causal: bool = False, scale: float | None = None, stream=None,
-             exp2_poly_pairs: int | None = None):
+             exp2_poly_pairs: int | None = None, kv_stages: int | None = None,
+             rescale_tau: float | None = None):
     """Return ``(o, lse)`` for CUDA bf16 [B,H,N,d] inputs (enqueued on the
     current or given stream)."""
     B, H, N, d = _shape(q)
     o = torch.empty_like(q)
     lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
-    attn_fwd_into(q, k, v, o, lse, causal, scale, stream, exp2_poly_pairs)
+    attn_fwd_into(q, k, v, o, lse, causal, scale, stream, exp2_poly_pairs, kv_stages, rescale_tau)
     return o, lse
 
 
@@ -483,3 +500,53 @@ def quantize_e4m3(x, inv_descale: float = 1.0, transpose: bool = False, stream=N
     if rc != ATTN_OK:
         raise AttnError(rc, "attn_quantize_e4m3")
     return out
+
+
+def quantize_nvfp4(x, inv_descale: float = 1.0, transpose: bool = False, stream=None):
+    """bf16 [B, H, N, 128] -> NVFP4 (see attn_quantize_nvfp4): returns
+    (codes uint8 [B, H, N, 64], or [B, H, 128, N // 2] with ``transpose``,
+    scales uint8 [B * H, ceil(N / 128), 2, 512])."""
+    if x.dim() != 4:
+        raise ValueError("x must be [B, H, N, d]")
+    B, H, N, d = (int(v) for v in x.shape)
+    _check(x, "x", torch.bfloat16, x.shape)
+    codes = torch.empty((B, H, d, N // 2) if transpose else (B, H, N, d // 2), dtype=torch.uint8,
+                        device=x.device)
+    scales = torch.empty((B * H, (N + 127) // 128, 2, 512), dtype=torch.uint8, device=x.device)
+    dev = _device_of(x)
+    with torch.cuda.device(dev):
+        rc = library().attn_quantize_nvfp4(x.data_ptr(), codes.data_ptr(), scales.data_ptr(),
+                                           B * H, N, d, float(inv_descale), int(bool(transpose)),
+                                           _stream_handle(stream, dev))
+    if rc != ATTN_OK:
+        raise AttnError(rc, "attn_quantize_nvfp4")
+    return codes, scales
+
+
+def attn_fwd_fp4(q, q_sf, k, k_sf, vt, vt_sf, causal: bool = False, scale: float | None = None,
+                 q_descale: float = 1.0, k_descale: float = 1.0, v_descale: float = 1.0,
+                 stream=None):
+    """4-bit attention (see attn_fwd_fp4 in the header) on the outputs of
+    quantize_nvfp4: q, k codes [B, H, N, 64], vt codes [B, H, 128, N // 2],
+    and their scales.  Returns (o bf16 [B, H, N, 128], lse fp32 [B, H, N])."""
+    B, H, N, half = (int(v) for v in q.shape)
+    d = 2 * half
+    for name, t, shape in (("q", q, (B, H, N, half)), ("k", k, (B, H, N, half)),
+                           ("vt", vt, (B, H, d, N // 2))):
+        _check(t, name, torch.uint8, shape)
+    for name, t in (("q_sf", q_sf), ("k_sf", k_sf), ("vt_sf", vt_sf)):
+        _check(t, name, torch.uint8, (B * H, (N + 127) // 128, 2, 512))
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    o = torch.empty((B, H, N, d), dtype=torch.bfloat16, device=q.device)
+    lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
+    dev = _device_of(q, q_sf, k, k_sf, vt, vt_sf)
+    with torch.cuda.device(dev):
+        rc = library().attn_fwd_fp4(q.data_ptr(), q_sf.data_ptr(), k.data_ptr(), k_sf.data_ptr(),
+                                    vt.data_ptr(), vt_sf.data_ptr(), o.data_ptr(), lse.data_ptr(),
+                                    B, H, N, d, int(bool(causal)), float(scale), float(q_descale),
+                                    float(k_descale), float(v_descale),
+                                    _stream_handle(stream, dev))
+    if rc != ATTN_OK:
+        raise AttnError(rc, "attn_fwd_fp4")
+    return o, lse

@@ -2,6 +2,13 @@
 
     python -m tiled_attention_forward_sm_b200.build [--verbose] [--trace]
 
+``--test-hooks`` builds ``libattn_b200_testhooks.so``: the attention and FP8
+entry points compiled with ATTN_TEST_HOOKS, which adds
+``int attn_test_set_hooks(unsigned long long wait_limit_ns, int withhold_load)``
+(a shorter bounded-wait limit and one K/V load that CTA 0 skips, so that a
+wait runs out and the kernels' abort path runs; see the GPU test of the
+abort path).  The product library never carries these hooks.
+
 ``--trace`` builds the timeline-tracing library ``libattn_b200_trace.so``
 instead: the attention kernel compiled with its clock64 stamps at every role
 hand-off (ATTN_TRACE_ENABLED) and the extra entry point
@@ -24,7 +31,9 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libattn_b200.so")
 TRACE_LIB = os.path.join(PKG, "libattn_b200_trace.so")
-SOURCES = [os.path.join(CSRC, f) for f in ("attn_fwd.cu", "fp8.cu", "kmeans.cu", "pair.cu", "host_io.cu")]
+TEST_HOOKS_LIB = os.path.join(PKG, "libattn_b200_testhooks.so")
+SOURCES = [os.path.join(CSRC, f) for f in ("attn_fwd.cu", "fp8.cu", "fp4.cu", "kmeans.cu", "pair.cu",
+                                           "host_io.cu")]
 HEADERS = [os.path.join(CSRC, f) for f in os.listdir(CSRC) if f.endswith((".cuh", ".h"))] + [
     os.path.join(INCLUDE, f) for f in os.listdir(INCLUDE) if f.endswith(".h")]
 
@@ -68,8 +77,21 @@ def build_trace(force: bool = False, verbose: bool = False) -> str:
     return TRACE_LIB
 
 
+def build_test_hooks(force: bool = False) -> str:
+    """The test-hooks library (attention and FP8 entry points)."""
+    srcs = [os.path.join(CSRC, f) for f in ("attn_fwd.cu", "fp8.cu")]
+    if (not force and os.path.exists(TEST_HOOKS_LIB) and
+            all(os.path.getmtime(p) <= os.path.getmtime(TEST_HOOKS_LIB) for p in srcs + HEADERS)):
+        return TEST_HOOKS_LIB
+    cmd = [nvcc_path(), *NVCC_FLAGS, "-DATTN_TEST_HOOKS", "-o", TEST_HOOKS_LIB, *srcs]
+    subprocess.check_call(cmd)
+    return TEST_HOOKS_LIB
+
+
 if __name__ == "__main__":
-    if "--trace" in sys.argv:
+    if "--test-hooks" in sys.argv:
+        print(build_test_hooks(force=True))
+    elif "--trace" in sys.argv:
         print(build_trace(force=True, verbose="--verbose" in sys.argv))
     else:
         build(force=True, verbose="--verbose" in sys.argv)

@@ -62,6 +62,7 @@ struct TmapEntry {
   bool used = false;
   unsigned long long stamp = 0;
   CUtensorMapDataType type{};
+  CUtensorMapSwizzle swizzle{};
   const void* ptr = nullptr;
   cuuint64_t dims[3] = {0, 0, 0};
   cuuint64_t strides[2] = {0, 0};
@@ -75,12 +76,14 @@ unsigned long long g_tmap_clock = 0;
 }  // namespace
 
 CUresult encode_tiled(CUtensorMap* m, CUtensorMapDataType type, const void* ptr,
-                      const cuuint64_t* dims, const cuuint64_t* strides, const cuuint32_t* box) {
+                      const cuuint64_t* dims, const cuuint64_t* strides, const cuuint32_t* box,
+                      CUtensorMapSwizzle swizzle) {
   std::lock_guard<std::mutex> lock(g_tmap_mu);
   int victim = 0;
   for (int i = 0; i < kTmapCacheEntries; ++i) {
     TmapEntry& e = g_tmap[i];
-    if (e.used && e.type == type && e.ptr == ptr && e.dims[0] == dims[0] && e.dims[1] == dims[1] &&
+    if (e.used && e.type == type && e.swizzle == swizzle && e.ptr == ptr &&
+        e.dims[0] == dims[0] && e.dims[1] == dims[1] &&
         e.dims[2] == dims[2] && e.strides[0] == strides[0] && e.strides[1] == strides[1] &&
         e.box[0] == box[0] && e.box[1] == box[1] && e.box[2] == box[2]) {
       e.stamp = ++g_tmap_clock;
@@ -92,7 +95,7 @@ CUresult encode_tiled(CUtensorMap* m, CUtensorMapDataType type, const void* ptr,
   cuuint32_t estr[3] = {1, 1, 1};
   const CUresult rc = g_encode(m, type, 3, const_cast<void*>(ptr), const_cast<cuuint64_t*>(dims),
                                const_cast<cuuint64_t*>(strides), const_cast<cuuint32_t*>(box),
-                               estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                               estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle,
                                CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (rc != CUDA_SUCCESS) return rc;
@@ -100,6 +103,7 @@ CUresult encode_tiled(CUtensorMap* m, CUtensorMapDataType type, const void* ptr,
   e.used = true;
   e.stamp = ++g_tmap_clock;
   e.type = type;
+  e.swizzle = swizzle;
   e.ptr = ptr;
   for (int k = 0; k < 3; ++k) e.dims[k] = dims[k];
   e.strides[0] = strides[0];
@@ -259,6 +263,11 @@ using namespace host;
 
 namespace {
 
+// Default share of exponentials computed by the FMA polynomial (pairs per 4):
+// measured on B200, the special-function unit alone is fastest for this
+// kernel (see the exp2 split sweep in the design notes).
+constexpr int kDefaultPolyPairs = 0;
+
 // Most key slices of one split-KV launch (and parts of one merge).
 constexpr int kMaxSplits = 256;
 
@@ -309,8 +318,9 @@ int64_t problem_items(const Problem& p, int num_sms) {
   return static_cast<int64_t>(p.B) * p.H * pairs * p.n_splits;
 }
 
-template <int D, bool CAUSAL, int kPolyPairs>
-int launch(const Problem& p, cudaStream_t stream, DeviceState& st, int* queue = nullptr) {
+template <int D, bool CAUSAL, int kPolyPairs, int STAGES = 0>
+int launch(const Problem& p, cudaStream_t stream, DeviceState& st, int* queue = nullptr,
+           float tau = kRescaleTau) {
   CUtensorMap tq, tk, tv;
   if (p.cu_q != nullptr) {
     if (make_tmap_tokens(&tq, p.q, p.T_q, p.H, D) || make_tmap_tokens(&tk, p.k, p.T_k, p.H_kv, D) ||
@@ -356,6 +366,7 @@ int launch(const Problem& p, cudaStream_t stream, DeviceState& st, int* queue = 
   }
   args.queue = queue != nullptr ? queue : next_queue_slot(st);
   args.scale_log2 = p.scale * 1.4426950408889634f;
+  args.rescale_tau = tau;
   args.status = st.status;
 
   // d = 256 runs the wide kernel (one Q tile at a time, 256-column O).
@@ -366,9 +377,9 @@ int launch(const Problem& p, cudaStream_t stream, DeviceState& st, int* queue = 
     threads = wide::kThreads;
     smem_bytes = wide::kSmemBytes;
   } else {
-    kern = attn_fwd_kernel<D, CAUSAL, kPolyPairs>;
+    kern = attn_fwd_kernel<D, CAUSAL, kPolyPairs, STAGES>;
     threads = kThreads;
-    smem_bytes = Config<D>::kSmemBytes;
+    smem_bytes = Config<D, STAGES>::kSmemBytes;
     // The kernel's register split (setmaxnreg) hands the softmax warpgroups
     // registers released by the producer/MMA warpgroup; it is only valid if
     // the kernel was built with the full per-thread budget it assumes.
@@ -400,28 +411,40 @@ int launch(const Problem& p, cudaStream_t stream, DeviceState& st, int* queue = 
   return ATTN_OK;
 }
 
-// Default share of exponentials computed by the FMA polynomial (pairs per 4):
-// measured on B200, the special-function unit alone is fastest for this
-// kernel (see the exp2 split sweep in the design notes).
-constexpr int kDefaultPolyPairs = 0;
+// How a launch computes (attn_opts, checked): the exponential split and
+// the K/V ring depth (0: the head dim's default; 2..5 at d = 128 with the
+// default split).
+struct Tuning {
+  int poly_pairs = kDefaultPolyPairs;
+  int kv_stages = 0;
+  float rescale_tau = kRescaleTau;
+};
 
 template <int D, bool CAUSAL>
-int launch_poly(int poly_pairs, const Problem& p, cudaStream_t s, DeviceState& st, int* queue) {
-  switch (poly_pairs) {
-    case 0: return launch<D, CAUSAL, 0>(p, s, st, queue);
-    case 2: return launch<D, CAUSAL, 2>(p, s, st, queue);
-    default: return launch<D, CAUSAL, 1>(p, s, st, queue);
+int launch_poly(const Tuning& t, const Problem& p, cudaStream_t s, DeviceState& st, int* queue) {
+  if constexpr (D == 128) {
+    switch (t.kv_stages) {
+      case 2: return launch<D, CAUSAL, 0, 2>(p, s, st, queue, t.rescale_tau);
+      case 3: return launch<D, CAUSAL, 0, 3>(p, s, st, queue, t.rescale_tau);
+      case 5: return launch<D, CAUSAL, 0, 5>(p, s, st, queue, t.rescale_tau);
+      default: break;
+    }
+  }
+  switch (t.poly_pairs) {
+    case 0: return launch<D, CAUSAL, 0>(p, s, st, queue, t.rescale_tau);
+    case 2: return launch<D, CAUSAL, 2>(p, s, st, queue, t.rescale_tau);
+    default: return launch<D, CAUSAL, 1>(p, s, st, queue, t.rescale_tau);
   }
 }
 
 template <int D>
-int launch_d(int poly_pairs, const Problem& p, cudaStream_t s, DeviceState& st, int* queue) {
-  return p.causal ? launch_poly<D, true>(poly_pairs, p, s, st, queue)
-                  : launch_poly<D, false>(poly_pairs, p, s, st, queue);
+int launch_d(const Tuning& t, const Problem& p, cudaStream_t s, DeviceState& st, int* queue) {
+  return p.causal ? launch_poly<D, true>(t, p, s, st, queue)
+                  : launch_poly<D, false>(t, p, s, st, queue);
 }
 
 // Launch a checked problem on the calling thread's device.
-int run_problem(const Problem& p, int poly_pairs, attn_stream_t stream, int* queue = nullptr,
+int run_problem(const Problem& p, const Tuning& tune, attn_stream_t stream, int* queue = nullptr,
                 DeviceState* st = nullptr) {
   if (st == nullptr) {
     const int rc = device_state(&st);
@@ -435,10 +458,10 @@ int run_problem(const Problem& p, int poly_pairs, attn_stream_t stream, int* que
   if (problem_items(p, st->num_sms) + st->num_sms > 0x7FFFFFFFll) return ATTN_ERR_UNSUPPORTED;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   switch (p.d) {
-    case 256: return launch_d<256>(poly_pairs, p, s, *st, queue);
-    case 128: return launch_d<128>(poly_pairs, p, s, *st, queue);
-    case 96: return launch_d<96>(poly_pairs, p, s, *st, queue);
-    default: return launch_d<64>(poly_pairs, p, s, *st, queue);
+    case 256: return launch_d<256>(tune, p, s, *st, queue);
+    case 128: return launch_d<128>(tune, p, s, *st, queue);
+    case 96: return launch_d<96>(tune, p, s, *st, queue);
+    default: return launch_d<64>(tune, p, s, *st, queue);
   }
 }
 
@@ -530,21 +553,39 @@ extern "C" int attn_fwd(const void* q, const void* k, const void* v, void* o, fl
   const Problem p = dense_problem(q, k, v, o, lse, B, H, N, d, causal, scale);
   const int rc = check_dense(p);
   if (rc != ATTN_OK) return rc;
-  return run_problem(p, kDefaultPolyPairs, stream);
+  return run_problem(p, Tuning{}, stream);
+}
+
+extern "C" attn_opts attn_opts_default(void) {
+  attn_opts o;
+  o.exp2_poly_pairs = -1;
+  o.kv_stages = 0;
+  o.rescale_tau = -1.f;
+  return o;
 }
 
 extern "C" int attn_fwd_ex(const void* q, const void* k, const void* v, void* o, float* lse, int B,
                            int H, int N, int d, int causal, float scale, const attn_opts* opts,
                            attn_stream_t stream) {
-  int poly = kDefaultPolyPairs;
+  Tuning t;
   if (opts) {
     if (opts->exp2_poly_pairs < -1 || opts->exp2_poly_pairs > 2) return ATTN_ERR_INVALID_ARG;
-    if (opts->exp2_poly_pairs >= 0) poly = opts->exp2_poly_pairs;
+    if (opts->exp2_poly_pairs >= 0) t.poly_pairs = opts->exp2_poly_pairs;
+    if (opts->kv_stages < 0 || opts->kv_stages == 1 || opts->kv_stages > 5)
+      return ATTN_ERR_INVALID_ARG;
+    t.kv_stages = opts->kv_stages == kDefaultStagesD128 ? 0 : opts->kv_stages;
+    if (t.kv_stages != 0 && (d != 128 || t.poly_pairs != kDefaultPolyPairs))
+      return ATTN_ERR_UNSUPPORTED;
+    if (opts->rescale_tau != -1.f) {  // -1: the default
+      if (!(opts->rescale_tau >= 0.f && opts->rescale_tau <= 16.f)) return ATTN_ERR_INVALID_ARG;
+      if (d > 128) return ATTN_ERR_UNSUPPORTED;
+      t.rescale_tau = opts->rescale_tau;
+    }
   }
   const Problem p = dense_problem(q, k, v, o, lse, B, H, N, d, causal, scale);
   const int rc = check_dense(p);
   if (rc != ATTN_OK) return rc;
-  return run_problem(p, poly, stream);
+  return run_problem(p, t, stream);
 }
 
 extern "C" int attn_fwd_chunk(const void* q, const void* k, const void* v, void* o, float* lse,
@@ -557,7 +598,7 @@ extern "C" int attn_fwd_chunk(const void* q, const void* k, const void* v, void*
   p.o_f32 = o_fp32 ? 1 : 0;
   const int rc = check_dense(p);
   if (rc != ATTN_OK) return rc;
-  return run_problem(p, kDefaultPolyPairs, stream);
+  return run_problem(p, Tuning{}, stream);
 }
 
 extern "C" int attn_fwd_varlen(const void* q, const void* k, const void* v, void* o, float* lse,
@@ -594,7 +635,7 @@ extern "C" int attn_fwd_varlen(const void* q, const void* k, const void* v, void
   p.cu_k = cu_seqlens_k;
   p.T_q = total_q;
   p.T_k = total_k;
-  return run_problem(p, kDefaultPolyPairs, stream);
+  return run_problem(p, Tuning{}, stream);
 }
 
 extern "C" int attn_fwd_splitkv(const void* q, const void* k, const void* v, void* o, float* lse,
@@ -611,7 +652,7 @@ extern "C" int attn_fwd_splitkv(const void* q, const void* k, const void* v, voi
   const int tiles = (N_k + kBlockN - 1) / kBlockN;
   const int split_tiles = (tiles + n_splits - 1) / n_splits;
   const int used = (tiles + split_tiles - 1) / split_tiles;  // slices that hold keys
-  if (used <= 1) return run_problem(p, kDefaultPolyPairs, stream);
+  if (used <= 1) return run_problem(p, Tuning{}, stream);
   if (!ws_o || !ws_lse) return ATTN_ERR_INVALID_ARG;
   if (reinterpret_cast<uintptr_t>(ws_o) & 15u) return ATTN_ERR_MISALIGNED;
   if (reinterpret_cast<uintptr_t>(ws_lse) & 3u) return ATTN_ERR_MISALIGNED;
@@ -635,7 +676,7 @@ extern "C" int attn_fwd_splitkv(const void* q, const void* k, const void* v, voi
   part.n_splits = used;
   part.split_tiles = split_tiles;
   part.split_rows = static_cast<long long>(rows);
-  rc = run_problem(part, kDefaultPolyPairs, stream, nullptr, st);
+  rc = run_problem(part, Tuning{}, stream, nullptr, st);
   if (rc != ATTN_OK) return rc;
   return run_combine(ws_o, ws_lse, used, static_cast<long long>(rows), d, o, lse, 0, stream, *st);
 }
@@ -683,7 +724,7 @@ extern "C" int attn_fwd_noalloc(const void* q, const void* k, const void* v, voi
     cudaGetLastError();
     return ATTN_ERR_CUDA;
   }
-  return run_problem(p, kDefaultPolyPairs, stream, st->noalloc_scratch, st);
+  return run_problem(p, Tuning{}, stream, st->noalloc_scratch, st);
 }
 
 extern "C" int attn_selftest_wait_timeout(int limit_us, attn_stream_t stream) {
@@ -735,6 +776,26 @@ extern "C" const char* attn_strerror(int status) {
 extern "C" int attn_trace_set_buffer(void* dev_buf) {
   unsigned long long* p = static_cast<unsigned long long*>(dev_buf);
   return cudaMemcpyToSymbol(g_trace_buf, &p, sizeof p) == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+#endif
+
+#ifdef ATTN_TEST_HOOKS
+// Test builds only: the limit of every bounded wait in the attention kernels
+// (nanoseconds, 0 for the default of 2 s) and the index of a K/V load that
+// CTA 0's producer withholds (-1: none).  A withheld load makes a consumer's
+// wait run out: the kernel then reports ATTN_ERR_DEVICE_TIMEOUT and leaves
+// through its abort path (every role stops, loads and MMAs in flight drain,
+// Tensor Memory is freed).  No fault, trap or endless wait is involved.
+extern "C" int attn_test_set_hooks(unsigned long long wait_limit_ns, int withhold_load) {
+  if (wait_limit_ns == 0) wait_limit_ns = kWaitLimitNs;
+  if (cudaMemcpyToSymbol(g_test_wait_limit_ns, &wait_limit_ns, sizeof wait_limit_ns) !=
+          cudaSuccess ||
+      cudaMemcpyToSymbol(g_test_withhold_load, &withhold_load, sizeof withhold_load) !=
+          cudaSuccess) {
+    cudaGetLastError();
+    return ATTN_ERR_CUDA;
+  }
+  return host::fp8_test_set_hooks(wait_limit_ns, withhold_load);
 }
 #endif
 

@@ -132,6 +132,10 @@ __device__ void producer_role(const Shared& sh, const Bars& bb, const KernelArgs
           ok = false;
           break;
         }
+        if (withhold_load(issued)) {  // test builds only
+          ++issued;
+          continue;
+        }
         ptx::mbar_arrive_expect_tx(&bb.kv_full[st], kTileBytes);
         if (which == 0)
           ptx::tma_load_3d(tk, &bb.kv_full[st], smem + kKVOff + st * kTileBytes, 0,

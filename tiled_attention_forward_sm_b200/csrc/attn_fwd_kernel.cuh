@@ -64,16 +64,33 @@ constexpr int kStatusDeviceBounds = -6;
 // status word and the CTA's abort flag, and every role then leaves its loop.
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s
 
+#ifdef ATTN_TEST_HOOKS
+// Test builds only (the product library never defines ATTN_TEST_HOOKS): the
+// limit of every bounded wait, and one K/V tile load that the producer of
+// CTA 0 skips (its index among that CTA's K/V loads; -1 for none), so that
+// a consumer's wait runs out and the kernel's abort path runs, with no
+// fault anywhere.  Every translation unit has its own copy; the test
+// library's attn_test_set_hooks sets all of them.
+static __device__ unsigned long long g_test_wait_limit_ns = kWaitLimitNs;
+static __device__ int g_test_withhold_load = -1;
+__device__ __forceinline__ uint64_t wait_limit_ns() { return g_test_wait_limit_ns; }
+__device__ __forceinline__ bool withhold_load(int issued) {
+  return blockIdx.x == 0 && issued == g_test_withhold_load;
+}
+#else
+__device__ __forceinline__ constexpr uint64_t wait_limit_ns() { return kWaitLimitNs; }
+__device__ __forceinline__ constexpr bool withhold_load(int) { return false; }
+#endif
+
 // Softmax arithmetic form: packed f32x2 FMA/ADD (1) or scalar FMA/ADD (0).
 // Measured on B200 the packed form is faster.
 #ifndef ATTN_PACKED_SOFTMAX
 #define ATTN_PACKED_SOFTMAX 1
 #endif
 
-// K/V ring depth for d = 128 (each stage holds one 128 x 128 bf16 tile).
-#ifndef ATTN_KV_STAGES_D128
-#define ATTN_KV_STAGES_D128 4
-#endif
+// Default K/V ring depth for d = 96 and 128 (each stage holds one 128-row
+// tile, 32 KB); d = 64 tiles are half as large and take 8 stages.
+constexpr int kDefaultStagesD128 = 4;
 
 // Work items announced by the producer to the MMA and softmax warps through
 // a small ring in shared memory (kItemWords ints per slot).
@@ -95,7 +112,10 @@ static_assert(kRegSplitTotal <= kThreads * 168, "register split exceeds the laun
 
 // Lazy-rescale threshold in log2 units: the running maximum is raised only
 // when a tile's maximum exceeds it by more than this, so every weight stays
-// at most 2^8 (fp32 row sums and bf16 weights stay far from overflow).
+// at most 2^8 (fp32 row sums and bf16 weights stay far from overflow).  The
+// two-tile kernel takes it from KernelArgs::rescale_tau (attn_fwd_ex can
+// change it, 0 meaning an eager rescale whenever the maximum grows); the
+// other kernels use this value.
 constexpr float kRescaleTau = 8.0f;
 
 // Optional timeline tracing (compiled in only with ATTN_TRACE_ENABLED; the
@@ -153,22 +173,25 @@ struct KernelArgs {
   int n_items;        // BH * n_qpairs * n_splits work items (some may be empty)
   int win_heads;      // heads per scheduling window (item order, see make_item)
   float scale_log2;   // scale * log2(e)
+  float rescale_tau;  // lazy-rescale threshold (log2 units) of softmax_step
   int* status;        // device status word
   int* queue;         // {next item, CTAs finished}: this launch's queue slot
   int head_pack;      // dense, N_q <= 128: an item pairs two query heads of
                       // one K/V head (n_qpairs = head pairs per K/V head)
 };
 
-template <int D>
+// STAGES: K/V ring depth, 0 for the default of the head dim.
+template <int D, int STAGES = 0>
 struct Config {
   static_assert(D == 64 || D == 96 || D == 128, "head dim");
+  static_assert(STAGES == 0 || (STAGES >= 2 && STAGES <= 5 && D > 64), "ring depth");
   // A tile is kBoxes 64-column TMA boxes of 128 rows; at D = 96 the second
   // box's columns 96..127 lie outside the tensor and arrive as zeros (the
   // products below never read them: QK stops at K = D, PV's N is D).
   static constexpr int kBoxes = (D + 63) / 64;
   static constexpr int kBoxBytes = kBlockM * 64 * 2;         // 16 KB
   static constexpr int kTileBytes = kBoxes * kBoxBytes;      // one 128 x 64*kBoxes tile
-  static constexpr int kStages = D > 64 ? ATTN_KV_STAGES_D128 : 8;  // K/V ring depth
+  static constexpr int kStages = STAGES > 0 ? STAGES : (D > 64 ? kDefaultStagesD128 : 8);
   static constexpr int kQOff = 0;
   static constexpr int kKVOff = 2 * kTileBytes;
   static constexpr int kBarOff = kKVOff + kStages * kTileBytes;
@@ -205,11 +228,13 @@ __device__ __forceinline__ void raise_status(const Shared& sh, int* status, int 
 }
 
 // Single-thread bounded wait.  A drain wait (for this thread's own copies or
-// MMAs in flight) ignores the abort flag but keeps the time limit.
+// MMAs in flight) ignores the abort flag but keeps the time limit (0: the
+// kernel's limit).
 __device__ __forceinline__ bool wait_one(const Shared& sh, int* status, uint64_t* bar,
                                          uint32_t parity, bool drain = false,
-                                         uint64_t limit_ns = kWaitLimitNs) {
+                                         uint64_t limit_ns = 0) {
   if (ptx::mbar_try_wait(bar, parity)) return true;
+  if (limit_ns == 0) limit_ns = wait_limit_ns();
   const uint64_t t0 = ptx::globaltimer_ns();
   for (uint32_t it = 1;; ++it) {
     if (ptx::mbar_try_wait(bar, parity)) return true;
@@ -227,7 +252,8 @@ __device__ __forceinline__ bool wait_one(const Shared& sh, int* status, uint64_t
 // whose next instructions are warp-collective tcgen05 loads/stores.
 __device__ __forceinline__ bool wait_warp(const Shared& sh, int* status, uint64_t* bar,
                                           uint32_t parity, bool drain = false,
-                                          uint64_t limit_ns = kWaitLimitNs) {
+                                          uint64_t limit_ns = 0) {
+  if (limit_ns == 0) limit_ns = wait_limit_ns();
   uint64_t t0 = 0;
   for (uint32_t it = 0;; ++it) {
     const bool ok = ptx::mbar_try_wait(bar, parity);
@@ -455,11 +481,11 @@ __device__ __forceinline__ bool read_item(const Shared& sh, const KernelArgs& a,
 }
 
 // ----------------------------------------------------------------- producer
-template <int D, bool CAUSAL>
+template <int D, bool CAUSAL, int STAGES = 0>
 __device__ void producer_role(const Shared& sh, const KernelArgs& a, uint8_t* smem,
                               const CUtensorMap* tq, const CUtensorMap* tk,
                               const CUtensorMap* tv) {
-  using C = Config<D>;
+  using C = Config<D, STAGES>;
   const uint64_t pol_q = ptx::policy_evict_first();
   const uint64_t pol_kv = ptx::policy_evict_last();
   const bool packed = a.cu_q != nullptr;
@@ -513,6 +539,10 @@ __device__ void producer_role(const Shared& sh, const KernelArgs& a, uint8_t* sm
         const int st = issued % C::kStages;
         const uint32_t ph = (issued / C::kStages) & 1;
         if (!wait_one(sh, a.status, &sh.kv_empty[st], ph ^ 1)) { ok = false; break; }
+        if (withhold_load(issued)) {  // test builds only
+          ++issued;
+          continue;
+        }
         uint8_t* dst = smem + C::kKVOff + st * C::kTileBytes;
         ATTN_TRACE(which == 0 ? kTrProdK : kTrProdV, r == 0 ? j : -1);
         ptx::mbar_arrive_expect_tx(&sh.kv_full[st], C::kTileBytes);
@@ -540,9 +570,9 @@ __device__ void producer_role(const Shared& sh, const KernelArgs& a, uint8_t* sm
 // are built once and advanced by constant offsets (the start-address field
 // is the low 14 bits, in 16-byte units; no carry can leave it because
 // shared memory is below 256 KB).
-template <int D, bool CAUSAL>
+template <int D, bool CAUSAL, int STAGES = 0>
 __device__ void mma_role(const Shared& sh, const KernelArgs& a, uint8_t* smem, uint32_t tmem) {
-  using C = Config<D>;
+  using C = Config<D, STAGES>;
   const uint32_t t_s[2] = {tmem + 0, tmem + 128};
   const uint32_t t_o[2] = {tmem + 256, tmem + 384};
   // K-major (Q, K): SBO = 1024 B between 8-row groups; MN-major (V):
@@ -770,7 +800,7 @@ __device__ __forceinline__ bool softmax_step(const Shared& sh, const KernelArgs&
   // Lazy rescale: raise the running max only when it moves by > tau.
   float alpha = 1.f;
   bool rescale = false;
-  if (tile_max - m > kRescaleTau) {  // also true on the first tile (m = -inf)
+  if (tile_max - m > a.rescale_tau) {  // also true on the first tile (m = -inf)
     alpha = ptx::ex2_approx(m - tile_max);  // 0 on the first tile
     m = tile_max;
     rescale = !first;
@@ -963,12 +993,12 @@ __device__ void softmax_role(const Shared& sh, const KernelArgs& a, uint32_t tme
 }
 
 // ------------------------------------------------------------------- kernel
-template <int D, bool CAUSAL, int kPolyPairs>
+template <int D, bool CAUSAL, int kPolyPairs, int STAGES = 0>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap_q,
                     const __grid_constant__ CUtensorMap tmap_k,
                     const __grid_constant__ CUtensorMap tmap_v, const KernelArgs args) {
-  using C = Config<D>;
+  using C = Config<D, STAGES>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -1033,10 +1063,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     ptx::setmaxnreg_inc<kRegsSoftmax>();
     softmax_role<D, CAUSAL, kPolyPairs>(sh, args, tmem, warp / 4, warp % 4);
   } else if (warp == 8) {
-    if (ptx::lane_id() == 0) producer_role<D, CAUSAL>(sh, args, smem, &tmap_q, &tmap_k, &tmap_v);
+    if (ptx::lane_id() == 0)
+      producer_role<D, CAUSAL, STAGES>(sh, args, smem, &tmap_q, &tmap_k, &tmap_v);
     __syncwarp();
   } else if (warp == 9) {
-    mma_role<D, CAUSAL>(sh, args, smem, tmem);
+    mma_role<D, CAUSAL, STAGES>(sh, args, smem, tmem);
   }
 
   ptx::tc_fence_before_sync();

@@ -91,6 +91,10 @@ __device__ void producer_role(const Shared& sh, const Bars& bb, const KernelArgs
     const int st = issued % kStages;
     const uint32_t ph = (issued / kStages) & 1;
     if (!wait_one(sh, a.status, &bb.kv_empty[st], ph ^ 1)) return false;
+    if (withhold_load(issued)) {  // test builds only
+      ++issued;
+      return true;
+    }
     ptx::mbar_arrive_expect_tx(&bb.kv_full[st], kTileBytes);
     load_tile(is_v ? tv : tk, &bb.kv_full[st], smem + kKVOff + st * kTileBytes,
               it.k_row0 + (it.kt0 + j) * kBlockN, it.kz, pol_kv);

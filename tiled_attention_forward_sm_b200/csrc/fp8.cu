@@ -33,6 +33,23 @@ int make_tmap_u8(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t mid, 
 }  // namespace attn_b200
 
 using namespace attn_b200;
+
+#ifdef ATTN_TEST_HOOKS
+namespace attn_b200 {
+namespace host {
+int fp8_test_set_hooks(unsigned long long wait_limit_ns, int withhold_load) {
+  if (cudaMemcpyToSymbol(g_test_wait_limit_ns, &wait_limit_ns, sizeof wait_limit_ns) !=
+          cudaSuccess ||
+      cudaMemcpyToSymbol(g_test_withhold_load, &withhold_load, sizeof withhold_load) !=
+          cudaSuccess) {
+    cudaGetLastError();
+    return ATTN_ERR_CUDA;
+  }
+  return ATTN_OK;
+}
+}  // namespace host
+}  // namespace attn_b200
+#endif
 using namespace attn_b200::host;
 
 extern "C" int attn_fwd_fp8(const void* q, const void* k, const void* vt, void* o, float* lse,

@@ -40,14 +40,22 @@ int device_state(DeviceState** out);
 // Device address of the next work-queue slot for one launch.
 int* next_queue_slot(DeviceState& st);
 
-// cuTensorMapEncodeTiled for a 3-D tensor with the 128-byte swizzle, no
+// cuTensorMapEncodeTiled for a 3-D tensor with the 128-byte swizzle (or the
+// one given), no
 // interleave, zero fill out of bounds; dims/strides/box as the driver call
 // takes them (strides: the two outer ones, in bytes).  device_state() must
 // have succeeded first.  Encoded maps are cached host-side, keyed by every
 // argument of the encode (a map holds nothing else, so a cached map is the
 // one a fresh encode would give).
 CUresult encode_tiled(CUtensorMap* m, CUtensorMapDataType type, const void* ptr,
-                      const cuuint64_t* dims, const cuuint64_t* strides, const cuuint32_t* box);
+                      const cuuint64_t* dims, const cuuint64_t* strides, const cuuint32_t* box,
+                      CUtensorMapSwizzle swizzle = CU_TENSOR_MAP_SWIZZLE_128B);
+
+#ifdef ATTN_TEST_HOOKS
+// Test builds only: set the bounded-wait limit and the withheld K/V load
+// (see g_test_withhold_load) of the FP8 translation unit's kernels.
+int fp8_test_set_hooks(unsigned long long wait_limit_ns, int withhold_load);
+#endif
 
 // Drop every cached tensor map (attn_release); later calls encode again.
 void tmap_cache_clear();

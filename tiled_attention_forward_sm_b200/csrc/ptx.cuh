@@ -95,6 +95,18 @@ __device__ __forceinline__ void tma_load_2d(const CUtensorMap* map, uint64_t* ba
       : "memory");
 }
 
+// Untiled bulk copy of `bytes` bytes (a multiple of 16; both addresses
+// 16-byte aligned) from global to this CTA's shared memory, completing its
+// bytes on `bar`.  No cluster multicast.
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes,
+                                          uint64_t* bar, uint64_t cache_policy) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1], %2, [%3], %4;" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_u32(bar)), "l"(cache_policy)
+      : "memory");
+}
+
 // 3-D tiled load; coordinates innermost first.  Out-of-range elements of
 // the box read as zero.
 __device__ __forceinline__ void tma_load_3d(const CUtensorMap* map, uint64_t* bar, void* dst,
@@ -392,6 +404,12 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t* r) {
 }
 
 // 16 columns per call.
+__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t* r) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(
+                   taddr),
+               ATTN_W8(r, 0)
+               : "memory");
+}
 __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t* r) {
   asm volatile(
       "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
@@ -436,6 +454,13 @@ __device__ __forceinline__ void setmaxnreg_dec() {
 __device__ __forceinline__ float ex2_approx(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// Approximate reciprocal (special-function unit, within 1 ulp).
+__device__ __forceinline__ float rcp_approx(float x) {
+  float y;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
 }
 
@@ -494,6 +519,124 @@ __device__ __forceinline__ uint32_t pack_e4m3x4(float a, float b, float c, float
       : "=r"(r)
       : "f"(a), "f"(b), "f"(c), "f"(d));
   return r;
+}
+
+// ------------------------------------------------ 4-bit (NVFP4) operands
+// Eight floats to E2M1 (round to nearest even, saturating at +-6), packed
+// first value in the lowest nibble.  cvt packs its first source into the
+// upper nibble of each byte.
+__device__ __forceinline__ uint32_t pack_e2m1x8(float v0, float v1, float v2, float v3, float v4,
+                                                float v5, float v6, float v7) {
+  uint32_t r;
+  asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b2, %6, %5;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b3, %8, %7;\n\t"
+      "mov.b32 %0, {b0, b1, b2, b3};\n\t}"
+      : "=r"(r)
+      : "f"(v0), "f"(v1), "f"(v2), "f"(v3), "f"(v4), "f"(v5), "f"(v6), "f"(v7));
+  return r;
+}
+
+// One float to its E4M3 code (round to nearest even, saturating at 448).
+__device__ __forceinline__ uint32_t f32_to_e4m3(float x) {
+  uint16_t r;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(0.f), "f"(x));
+  return r & 0xFFu;
+}
+
+// The value of an E4M3 code (low byte), exactly (through f16).
+__device__ __forceinline__ float e4m3_to_f32(uint32_t code) {
+  uint32_t h2;
+  float f;
+  asm("{\n\t.reg .b16 lo, hi;\n\tmov.b32 {lo, hi}, %1;\n\tcvt.rn.f16x2.e4m3x2 %0, lo;\n\t}"
+      : "=r"(h2)
+      : "r"(code & 0xFFu));
+  asm("{\n\t.reg .f16 a, b;\n\tmov.b32 {a, b}, %1;\n\tcvt.f32.f16 %0, a;\n\t}"
+      : "=f"(f)
+      : "r"(h2));
+  return f;
+}
+
+// Make this thread's generic-proxy writes to shared memory visible to the
+// async proxy (TMA stores, tcgen05.cp, tcgen05.mma operand reads).
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// Shared-memory matrix descriptor with the 64-byte swizzle (layout type 4),
+// for K-major tiles whose rows are 64 bytes (128 E2M1 values): 8-row groups
+// of 512 B (SBO); the tile base must be 512-byte aligned.  Same fields as
+// sdesc_sw128.
+__device__ __forceinline__ uint64_t sdesc_sw64(uint32_t smem_addr, uint32_t sbo_bytes) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((smem_addr & 0x3FFFFu) >> 4);
+  d |= static_cast<uint64_t>(1) << 16;  // leading byte offset: unused (16 B)
+  d |= static_cast<uint64_t>((sbo_bytes >> 4) & 0x3FFFu) << 32;
+  d |= static_cast<uint64_t>(1) << 46;
+  d |= static_cast<uint64_t>(4) << 61;
+  return d;
+}
+
+// Descriptor of an unswizzled block of 32 rows x 16 bytes stored row after
+// row (four 8-row core matrices, 128 B apart): the source of tcgen05.cp
+// 32x128b.
+__device__ __forceinline__ uint64_t sdesc_rows16(uint32_t smem_addr) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((smem_addr & 0x3FFFFu) >> 4);
+  d |= static_cast<uint64_t>(128 >> 4) << 16;
+  d |= static_cast<uint64_t>(128 >> 4) << 32;
+  d |= static_cast<uint64_t>(1) << 46;
+  return d;
+}
+
+// Copy 32 rows x 128 bits from shared memory into TMEM columns [c, c+4) of
+// lanes 0-31 and, replicated, of the other three lane quarters (.warpx4):
+// the layout the block-scaled MMA reads its scale factors in.  Executed by
+// the warp, issued by one elected lane (the lane that issues the MMAs).
+__device__ __forceinline__ void tmem_cp_32x128b_x4_elect(uint32_t taddr, uint64_t sdesc) {
+  asm volatile(
+      "{\n\t.reg .pred e;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "@e tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;\n\t}" ::"r"(taddr),
+      "l"(sdesc)
+      : "memory");
+}
+
+// Block-scaled 4-bit products, kind::mxf4nvf4 with one UE4M3 scale per 16
+// elements of K (scale_vec::4X), E2M1 A and B, fp32 D, K = 64 per MMA.
+// sfa/sfb: TMEM addresses of the A and B scale-factor columns.
+__device__ __forceinline__ void mma_fp4_ss_elect(uint32_t d_tmem, uint64_t a_desc,
+                                                 uint64_t b_desc, uint32_t idesc, uint32_t sfa,
+                                                 uint32_t sfb, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p, e;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "setp.ne.b32 p, %6, 0;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.scale_vec::4X [%0], %1, %2, %3, "
+      "[%4], [%5], p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(sfa), "r"(sfb), "r"(accumulate)
+      : "memory");
+}
+__device__ __forceinline__ void mma_fp4_ts_elect(uint32_t d_tmem, uint32_t a_tmem,
+                                                 uint64_t b_desc, uint32_t idesc, uint32_t sfa,
+                                                 uint32_t sfb, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p, e;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "setp.ne.b32 p, %6, 0;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.scale_vec::4X [%0], [%1], %2, %3, "
+      "[%4], [%5], p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(sfa), "r"(sfb), "r"(accumulate)
+      : "memory");
+}
+
+// Instruction descriptor of the block-scaled 4-bit MMA: [7,10) A format and
+// [10,13) B format (1 = E2M1), bits 15/16 K-major, [17,23) N>>3, bit 23 scale
+// format (0 = UE4M3), [24,29) M>>4, scale-factor ids 0, K = 64.
+__host__ __device__ constexpr uint32_t idesc_nvfp4_f32(uint32_t M, uint32_t N) {
+  return (1u << 7) | (1u << 10) | ((N >> 3) << 17) | ((M >> 4) << 24);
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
