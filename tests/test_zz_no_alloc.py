@@ -10,6 +10,7 @@ device array, cleared on every call.  This file is collected last so that a
 run stopping at the first failure has already run every other test.
 """
 import ctypes
+import gc
 import math
 
 import numpy as np
@@ -72,13 +73,21 @@ def test_noalloc_takes_no_device_memory(d):
     scale = 1.0 / math.sqrt(d)
     assert _noalloc_call(lib, q, k, v, o, lse, True, scale) == 0
     torch.cuda.synchronize()
-    free0, _ = torch.cuda.mem_get_info()
-    alloc0 = torch.cuda.memory_allocated()
-    for _ in range(3):
-        assert _noalloc_call(lib, q, k, v, o, lse, True, scale) == 0
-    torch.cuda.synchronize()
-    free1, _ = torch.cuda.mem_get_info()
-    assert torch.cuda.memory_allocated() == alloc0
+    # tensors of earlier tests that the garbage collector frees would move
+    # the counters: collect first, and not while measuring
+    gc.collect()
+    gc.disable()
+    try:
+        free0, _ = torch.cuda.mem_get_info()
+        alloc0 = torch.cuda.memory_allocated()
+        for _ in range(3):
+            assert _noalloc_call(lib, q, k, v, o, lse, True, scale) == 0
+        torch.cuda.synchronize()
+        free1, _ = torch.cuda.mem_get_info()
+        alloc1 = torch.cuda.memory_allocated()
+    finally:
+        gc.enable()
+    assert alloc1 == alloc0
     assert free1 == free0
     assert tab.last_device_error() == 0
 
