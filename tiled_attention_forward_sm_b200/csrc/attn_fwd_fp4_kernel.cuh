@@ -32,9 +32,12 @@
 //   [256,384)  O (fp32)
 //   [384,400)  Q scale factors, two slots of 8 columns (Q tiles alternate)
 //   [400,464)  K or V scale factors, one slot of 8 columns per ring stage
-// Roles (6 warps): warps 0-3 softmax (one thread per query row, lazy O
-// rescale, epilogue), warp 4 TMA producer, warp 5 TMEM allocator and MMA
-// issuer.
+// Roles (10 warps): warps 0-7 softmax, two threads per query row: warp w
+// reads TMEM lanes 32 (w % 4) .. + 31 and keys 64 (w / 4) .. + 63 of every
+// score tile (the two halves of a row exchange their maxima through shared
+// memory, so both take the same lazy decision; each rescales, quantises and
+// stores its half of P and of O), warp 8 TMA producer, warp 9 TMEM
+// allocator and MMA issuer.
 #pragma once
 
 #include "attn_fwd_kernel.cuh"
@@ -43,7 +46,7 @@ namespace attn_b200 {
 namespace fp4 {
 
 constexpr int kD = 128;
-constexpr int kThreads = 192;
+constexpr int kThreads = 320;
 constexpr int kRowBytes = kD / 2;                    // 64 B: one row of 128 E2M1 codes
 constexpr int kCodeBytes = kBlockM * kRowBytes;      // 8 KB per 128-row tile
 constexpr int kScaleBytes = 1024;                    // 2 blocks of 512 B per tile
@@ -52,16 +55,19 @@ constexpr int kStages = 8;                           // K / V^T ring depth
 constexpr int kQOff = 0;                             // one Q buffer (codes + scales)
 constexpr int kKVOff = kSlotBytes;
 constexpr int kPScaleOff = kKVOff + kStages * kSlotBytes;  // P scales, 2 buffers x 1 KB
-constexpr int kBarOff = kPScaleOff + 2 * kScaleBytes;
+// exchange of the two half-rows' values (row maxima, then row sums): 2
+// parities x 2 halves x 128 rows, fp32
+constexpr int kXchOff = kPScaleOff + 2 * kScaleBytes;
+constexpr int kBarOff = kXchOff + 4 * 128 * 4;
 // barriers: q_full, q_empty, kv_full[S], kv_empty[S], s_full[2],
 // p_ready[2 buffers][2 halves], pv_done, o_ready, drain, item_full[R],
-// item_empty[R]
-constexpr int kNumBars = 2 + 2 * kStages + 2 + 4 + 1 + 1 + 1 + 2 * kItemSlots;
+// item_empty[R], xch[4 lane quarters]
+constexpr int kNumBars = 2 + 2 * kStages + 2 + 4 + 1 + 1 + 1 + 2 * kItemSlots + 4;
 constexpr int kMiscOff = kBarOff + kNumBars * 8;
 constexpr int kRingOff = kMiscOff + 16;
 constexpr int kSmemBytes = kRingOff + 4 * kItemWords * kItemSlots + 1024;  // + alignment slack
 static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
-constexpr int kReaders = 5;  // item-ring readers: the MMA warp and 4 softmax warps
+constexpr int kReaders = 9;  // item-ring readers: the MMA warp and 8 softmax warps
 constexpr uint32_t kIdesc = ptx::idesc_nvfp4_f32(128, 128);  // QK and PV: M = N = 128
 constexpr uint32_t kTmemO = 256;
 constexpr uint32_t kTmemQsf = 384;   // + 8 * (Q tile parity)
@@ -87,6 +93,7 @@ struct Bars {
   uint64_t* p_ready;   // [2 buffers][2 halves]
   uint64_t* pv_done;   // PV of a K/V tile complete (one phase per tile)
   uint64_t* o_ready;   // the Q tile's last PV complete
+  uint64_t* xch;       // [4] the two warps of a lane quarter have posted their half-rows
 };
 
 __device__ __forceinline__ int tile_n(const Item& it, int s) { return s == 0 ? it.n0 : it.n1; }
@@ -281,15 +288,34 @@ template <bool CAUSAL>
 __device__ void softmax_role(const Shared& sh, const Bars& bb, const KernelArgs& a,
                              const Fp4Args& f, uint8_t* smem, uint32_t tmem, int warp) {
   const int lane = static_cast<int>(ptx::lane_id());
-  const int r = warp * 32 + lane;
-  const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
-  const uint32_t t_o = tmem + lane_off + kTmemO;
-  // this row's word in each 512-byte scale block: byte 16 (r % 32) + 4 (r / 32)
-  uint32_t* ps_word = reinterpret_cast<uint32_t*>(smem + kPScaleOff + 16 * lane + 4 * warp);
+  const int quarter = warp & 3;  // TMEM lanes of this warp
+  const int h = warp >> 2;       // key half of every tile (and column half of O)
+  const int r = quarter * 32 + lane;
+  const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
+  const uint32_t t_o = tmem + lane_off + kTmemO + 64u * h;
+  // this row's word in its half's 512-byte scale block: byte 16 (r % 32) + 4 (r / 32)
+  uint32_t* ps_word = reinterpret_cast<uint32_t*>(smem + kPScaleOff + 512 * h + 16 * lane +
+                                                  4 * quarter);
+  float* xbuf = reinterpret_cast<float*>(smem + kXchOff);  // [parity][half][row]
+  uint64_t* xbar = &bb.xch[quarter];
   const float sl2 = a.scale_log2;
   const uint64_t sl2x2 = ptx::f2pack(sl2, sl2);
   int g = 0;   // K/V tiles consumed (S buffer g % 2)
   int eo = 0;  // Q tiles with at least one K/V tile finished
+  int xc = 0;  // exchanges with the other half of the row
+  // Post this half-row's value and take the other half's (both warps of the
+  // lane quarter arrive on xbar; bounded wait).  A partner is at most one
+  // exchange behind, so slots alternate by the exchange's parity.
+  auto exchange = [&](float v, float& other) -> bool {
+    float* slots = xbuf + (xc & 1) * 256;
+    slots[h * 128 + r] = v;
+    __syncwarp();
+    if (lane == 0) ptx::mbar_arrive(xbar);
+    if (!wait_warp(sh, a.status, xbar, static_cast<uint32_t>(xc & 1))) return false;
+    ++xc;
+    other = slots[(1 - h) * 128 + r];
+    return true;
+  };
 
   Item it;
   bool ok = true;
@@ -301,49 +327,47 @@ __device__ void softmax_role(const Shared& sh, const Bars& bb, const KernelArgs&
       const int n = tile_n(it, s);
       float m = -INFINITY, l = 0.f;
       for (int j = 0; j < n; ++j) {
-        const int key0 = (it.kt0 + j) * kBlockN;
-        int key_limit = it.k_len - key0;
+        const int key0 = (it.kt0 + j) * kBlockN + 64 * h;
+        int key_limit = it.k_len - key0;  // keys of this half visible to the row
         if (CAUSAL) {
           const long long lim = static_cast<long long>(row) + it.delta + 1 - key0;
           if (lim < key_limit) key_limit = lim < -1 ? -1 : static_cast<int>(lim);
         }
         const int b = g & 1;
-        const uint32_t t_s = tmem + lane_off + 128u * b;
+        const uint32_t t_s = tmem + lane_off + 128u * b + 64u * h;
         if (!wait_warp(sh, a.status, &bb.s_full[b], static_cast<uint32_t>((g >> 1) & 1))) return;
         ptx::tc_fence_after_sync();
-        const bool masked = __any_sync(0xffffffffu, key_limit < kBlockN);
-        uint32_t sr[128];
+        const bool masked = __any_sync(0xffffffffu, key_limit < 64);
+        uint32_t sr[64];
         ptx::tmem_ld32(t_s + 0, sr + 0);
         ptx::tmem_ld32(t_s + 32, sr + 32);
-        ptx::tmem_ld32(t_s + 64, sr + 64);
-        ptx::tmem_ld32(t_s + 96, sr + 96);
         ptx::tmem_ld_wait_tie(sr + 0);
         ptx::reg_tie32(sr + 32);
-        ptx::reg_tie32(sr + 64);
-        ptx::reg_tie32(sr + 96);
-        float x[128];
+        float x[64];
 #pragma unroll
-        for (int c = 0; c < 128; ++c) x[c] = __uint_as_float(sr[c]);
+        for (int c = 0; c < 64; ++c) x[c] = __uint_as_float(sr[c]);
         if (masked) {
 #pragma unroll
-          for (int c = 0; c < 128; ++c)
+          for (int c = 0; c < 64; ++c)
             if (c >= key_limit) x[c] = -INFINITY;
         }
         float mx[8];
 #pragma unroll
         for (int k = 0; k < 8; ++k) mx[k] = x[k];
 #pragma unroll
-        for (int c = 8; c + 16 <= 128; c += 16) {
+        for (int c = 8; c + 16 <= 64; c += 16) {
 #pragma unroll
           for (int k = 0; k < 8; ++k) mx[k] = ptx::max3(mx[k], x[c + 2 * k], x[c + 2 * k + 1]);
         }
 #pragma unroll
-        for (int k = 0; k < 4; ++k) mx[k] = ptx::max3(mx[k], x[120 + 2 * k], x[121 + 2 * k]);
-        const float tile_max = ptx::max3(ptx::max3(mx[0], mx[1], mx[2]),
-                                         ptx::max3(mx[3], mx[4], mx[5]), fmaxf(mx[6], mx[7])) *
-                               sl2;
-        // Lazy rescale, as in attn_fwd_kernel.cuh; O may be touched only
-        // once the previous tile's PV has completed.
+        for (int k = 0; k < 4; ++k) mx[k] = ptx::max3(mx[k], x[56 + 2 * k], x[57 + 2 * k]);
+        const float half_max = ptx::max3(ptx::max3(mx[0], mx[1], mx[2]),
+                                         ptx::max3(mx[3], mx[4], mx[5]), fmaxf(mx[6], mx[7]));
+        float other_max;
+        if (!exchange(half_max, other_max)) return;
+        const float tile_max = fmaxf(half_max, other_max) * sl2;
+        // Lazy rescale, the same decision in both halves of the row; O may
+        // be touched only once the previous tile's PV has completed.
         float alpha = 1.f;
         bool rescale = false;
         if (tile_max - m > kRescaleTau) {
@@ -355,7 +379,7 @@ __device__ void softmax_role(const Shared& sh, const Bars& bb, const KernelArgs&
           if (!wait_warp(sh, a.status, bb.pv_done, static_cast<uint32_t>((g - 1) & 1))) return;
           ptx::tc_fence_after_sync();
 #pragma unroll 1
-          for (int c0 = 0; c0 < kD; c0 += 32) {
+          for (int c0 = 0; c0 < 64; c0 += 32) {
             uint32_t ov[32];
             ptx::tmem_ld32(t_o + c0, ov);
             ptx::tmem_ld_wait_tie(ov);
@@ -368,37 +392,33 @@ __device__ void softmax_role(const Shared& sh, const Bars& bb, const KernelArgs&
         const uint64_t negm2 = ptx::f2pack(negm, negm);
         uint64_t sa = ptx::f2pack(0.f, 0.f), sb = sa;
 #pragma unroll
-        for (int half = 0; half < 2; ++half) {
-          // weights of keys [64 half, 64 half + 64), kept in x
-#pragma unroll
-          for (int q = 0; q < 32; ++q) {
-            const int c = 64 * half + 2 * q;
-            const uint64_t y2 = ptx::ffma2(ptx::f2pack(x[c], x[c + 1]), sl2x2, negm2);
-            float y0, y1;
-            ptx::f2unpack(y2, y0, y1);
-            const uint64_t p2 = ptx::f2pack(ptx::ex2_approx(y0), ptx::ex2_approx(y1));
-            if (q & 1) sb = ptx::fadd2(sb, p2);
-            else sa = ptx::fadd2(sa, p2);
-            ptx::f2unpack(p2, x[c], x[c + 1]);
-          }
-          // four 16-key blocks: 8 words of codes, 4 scale bytes
-          uint32_t pk[8];
-          uint32_t sw = 0;
-#pragma unroll
-          for (int blk = 0; blk < 4; ++blk) {
-            const uint32_t sc = quantize_block16(x + 64 * half + 16 * blk, pk[2 * blk], pk[2 * blk + 1]);
-            sw |= sc << (8 * blk);
-          }
-          // codes -> TMEM columns [8 half, 8 half + 8) of the S buffer,
-          // scales -> this row's word of the buffer's scale block `half`
-          ptx::tmem_st8(t_s + 8 * half, pk);
-          ps_word[(b * kScaleBytes + 512 * half) / 4] = sw;
-          ptx::tmem_st_wait();
-          ptx::fence_proxy_async_smem();
-          ptx::tc_fence_before_sync();
-          __syncwarp();
-          if (lane == 0) ptx::mbar_arrive(&bb.p_ready[2 * b + half]);
+        for (int q = 0; q < 32; ++q) {
+          const int c = 2 * q;
+          const uint64_t y2 = ptx::ffma2(ptx::f2pack(x[c], x[c + 1]), sl2x2, negm2);
+          float y0, y1;
+          ptx::f2unpack(y2, y0, y1);
+          const uint64_t p2 = ptx::f2pack(ptx::ex2_approx(y0), ptx::ex2_approx(y1));
+          if (q & 1) sb = ptx::fadd2(sb, p2);
+          else sa = ptx::fadd2(sa, p2);
+          ptx::f2unpack(p2, x[c], x[c + 1]);
         }
+        // four 16-key blocks: 8 words of codes, 4 scale bytes
+        uint32_t pk[8];
+        uint32_t sw = 0;
+#pragma unroll
+        for (int blk = 0; blk < 4; ++blk) {
+          const uint32_t sc = quantize_block16(x + 16 * blk, pk[2 * blk], pk[2 * blk + 1]);
+          sw |= sc << (8 * blk);
+        }
+        // codes -> TMEM columns [8 h, 8 h + 8) of the S buffer, scales ->
+        // this row's word of the buffer's scale block h
+        ptx::tmem_st8(tmem + lane_off + 128u * b + 8u * h, pk);
+        ps_word[(b * kScaleBytes) / 4] = sw;
+        ptx::tmem_st_wait();
+        ptx::fence_proxy_async_smem();
+        ptx::tc_fence_before_sync();
+        __syncwarp();
+        if (lane == 0) ptx::mbar_arrive(&bb.p_ready[2 * b + h]);
         float la0, la1, lb0, lb1;
         ptx::f2unpack(sa, la0, la1);
         ptx::f2unpack(sb, lb0, lb1);
@@ -406,7 +426,11 @@ __device__ void softmax_role(const Shared& sh, const Bars& bb, const KernelArgs&
         ++g;
       }
 
-      // Epilogue: O v_descale / l -> bf16 rows; LSE = (m + log2 l) ln 2.
+      // Epilogue: the row sum of both halves; this half's 64 columns of
+      // O v_descale / l -> bf16; LSE = (m + log2 l) ln 2 (written by half 0).
+      float l_other = 0.f;
+      if (!exchange(l, l_other)) return;
+      l += l_other;
       if (n > 0) {
         if (!wait_warp(sh, a.status, bb.o_ready, static_cast<uint32_t>(eo & 1))) return;
         ++eo;
@@ -416,9 +440,9 @@ __device__ void softmax_role(const Shared& sh, const Bars& bb, const KernelArgs&
       const bool empty = m == -INFINITY;
       const float fo = empty ? 0.f : f.v_descale / l;
       const size_t o_row = static_cast<size_t>(it.qz) * a.N_q + row;
-      __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(a.o) + o_row * kD;
+      __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(a.o) + o_row * kD + 64 * h;
 #pragma unroll 1
-      for (int c0 = 0; c0 < kD; c0 += 32) {
+      for (int c0 = 0; c0 < 64; c0 += 32) {
         uint32_t ov[32];
         if (n > 0) {
           ptx::tmem_ld32(t_o + c0, ov);
@@ -438,7 +462,7 @@ __device__ void softmax_role(const Shared& sh, const Bars& bb, const KernelArgs&
         for (int v = 0; v < 4; ++v)
           dst[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
       }
-      if (row_ok) a.lse[o_row] = empty ? -INFINITY : (m + log2f(l)) * 0.69314718055994531f;
+      if (row_ok && h == 0) a.lse[o_row] = empty ? -INFINITY : (m + log2f(l)) * 0.69314718055994531f;
     }
   }
 }
@@ -463,8 +487,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   bb.p_ready = bb.s_full + 2;
   bb.pv_done = bb.p_ready + 4;
   bb.o_ready = bb.pv_done + 1;
+  bb.xch = bb.o_ready + 1;
   Shared sh = {};
-  sh.drain = bb.o_ready + 1;
+  sh.drain = bb.xch + 4;
   sh.item_full = sh.drain + 1;
   sh.item_empty = sh.item_full + kItemSlots;
   sh.tmem_base = reinterpret_cast<uint32_t*>(smem + kMiscOff);
@@ -483,6 +508,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int i = 0; i < 4; ++i) ptx::mbar_init(&bb.p_ready[i], 4);
     ptx::mbar_init(bb.pv_done, 1);
     ptx::mbar_init(bb.o_ready, 1);
+    for (int i = 0; i < 4; ++i) ptx::mbar_init(&bb.xch[i], 2);
     ptx::mbar_init(sh.drain, 1);
     for (int i = 0; i < kItemSlots; ++i) {
       ptx::mbar_init(&sh.item_full[i], 1);
@@ -491,12 +517,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     *sh.abort_flag = 0;
     ptx::fence_barrier_init();
   }
-  if (warp == 4 && ptx::lane_id() == 0) {
+  if (warp == 8 && ptx::lane_id() == 0) {
     ptx::prefetch_tmap(&tmap_q);
     ptx::prefetch_tmap(&tmap_k);
     ptx::prefetch_tmap(&tmap_vt);
   }
-  if (warp == 5) {
+  if (warp == 9) {
     ptx::tmem_alloc(sh.tmem_base, 512);
     ptx::tmem_relinquish();
   }
@@ -505,9 +531,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   ptx::tc_fence_after_sync();
   const uint32_t tmem = *sh.tmem_base;
 
-  if (warp < 4) {
+  if (warp < 8) {
     softmax_role<CAUSAL>(sh, bb, args, fargs, smem, tmem, warp);
-  } else if (warp == 4) {
+  } else if (warp == 8) {
     if (ptx::lane_id() == 0)
       producer_role<CAUSAL>(sh, bb, args, fargs, smem, &tmap_q, &tmap_k, &tmap_vt);
     __syncwarp();
@@ -524,7 +550,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       atomicExch(args.queue + 1, 0);
     }
   }
-  if (warp == 5) {
+  if (warp == 9) {
     ptx::tc_fence_after_sync();
     ptx::tmem_dealloc(tmem, 512);
   }
