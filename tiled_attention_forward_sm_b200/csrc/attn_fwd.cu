@@ -358,7 +358,9 @@ int launch(const Problem& p, cudaStream_t stream, DeviceState& st, int* queue = 
   args.n_items = static_cast<int>(problem_items(p, st.num_sms));
   // Scheduling window: enough heads that a window holds about two rounds of
   // items (so its light tail evens out the CTAs), few enough that the
-  // window's K/V stays in L2 while its CTAs run.
+  // window's K/V stays in L2 while its CTAs run.  This is the largest
+  // window; the kernel cuts the heads into windows of equal size to within
+  // one head (item_window).
   {
     const int per_head = args.n_qpairs * args.n_splits;
     const int want = (2 * st.num_sms + per_head - 1) / per_head;

@@ -313,12 +313,31 @@ __device__ __forceinline__ int tiles_for(int qt, const Item& it, int split_tiles
   return n <= 0 ? 0 : (n > split_tiles ? split_tiles : static_cast<int>(n));
 }
 
+// Scheduling window of the item with head-major index `base` (units of
+// n_per_head items per head): heads are cut into ceil(BH / win_heads)
+// windows of equal size to within one head (the first ones one head
+// larger), so the last window is as large as the others and its heaviest
+// items do not start after every other CTA has run dry.  Returns the
+// window's first head h0 and head count wh; base - h0 * n_per_head indexes
+// the item inside it.
+__device__ __forceinline__ void item_window(int base, int BH, int win_heads, int n_per_head,
+                                            int& h0, int& wh) {
+  const int n_win = (BH + win_heads - 1) / win_heads;
+  const int wsz = BH / n_win, wrem = BH - wsz * n_win;  // wrem windows of wsz + 1 heads
+  const int hpos = base / n_per_head;
+  const int big = wrem * (wsz + 1);
+  const int w = hpos < big ? hpos / (wsz + 1) : wrem + (hpos - big) / wsz;
+  h0 = w * wsz + (w < wrem ? w : wrem);
+  wh = wsz + (w < wrem ? 1 : 0);
+}
+
 // Item numbering: items are (head, Q tile pair, key slice) with the slice
-// innermost.  Heads are taken in windows of win_heads; inside a window the
-// pairs are numbered heaviest first under the causal mask (pair-major over
-// the window's heads).  Items handed out in this order keep the CTAs that
-// run together on a few heads, whose K/V then stays in L2, while the light
-// pairs at the end of each window even out the CTAs' finishing times.
+// innermost.  Heads are taken in windows of at most win_heads (item_window);
+// inside a window the pairs are numbered heaviest first under the causal
+// mask (pair-major over the window's heads).  Items handed out in this
+// order keep the CTAs that run together on a few heads, whose K/V then
+// stays in L2, while the light pairs at the end of each window even out the
+// CTAs' finishing times.
 // Returns false for an item with no query rows (a pair past the end of a
 // shorter sequence) or, after raising the bounds status, for a sequence
 // whose offsets do not fit the buffers.
@@ -376,11 +395,9 @@ __device__ __forceinline__ bool make_item(int idx, const KernelArgs& a, int* sta
   }
   it.pack = 0;
   it.qz1 = -1;
-  const int per_win = a.win_heads * a.n_qpairs;
-  const int w = base / per_win;
-  const int k = base - w * per_win;
-  const int h0 = w * a.win_heads;
-  const int wh = (a.BH - h0) < a.win_heads ? (a.BH - h0) : a.win_heads;
+  int h0, wh;
+  item_window(base, a.BH, a.win_heads, a.n_qpairs, h0, wh);
+  const int k = base - h0 * a.n_qpairs;
   const int qp_idx = k / wh;
   const int bh = h0 + (k - qp_idx * wh);
   const int b = bh / a.H, h = bh - b * a.H;

@@ -111,11 +111,9 @@ __device__ __forceinline__ bool wait_one_cl(const Shared& sh, int* status, uint6
 // the K/V tiles of the products for tiles (4u, 4u+1) and (4u+2, 4u+3).
 template <bool CAUSAL>
 __device__ __forceinline__ bool make_item_pair(int idx, const KernelArgs& a, Item& it) {
-  const int per_win = a.win_heads * a.n_qpairs;
-  const int w = idx / per_win;
-  const int k = idx - w * per_win;
-  const int h0 = w * a.win_heads;
-  const int wh = (a.BH - h0) < a.win_heads ? (a.BH - h0) : a.win_heads;
+  int h0, wh;
+  item_window(idx, a.BH, a.win_heads, a.n_qpairs, h0, wh);
+  const int k = idx - h0 * a.n_qpairs;
   const int qd_idx = k / wh;
   const int bh = h0 + (k - qd_idx * wh);
   const int b = bh / a.H, h = bh - b * a.H;
