@@ -328,12 +328,54 @@ def versions(lib, sampler=None) -> dict:
             "device": torch.cuda.get_device_name()}
 
 
-def timed_steps(step, steps: int, stream, dev):
-    """Run ``steps`` steps with a CUDA event before each and after the last,
-    all on the launching stream, synchronised on both sides.  Returns the
-    total milliseconds and the per-step list."""
-    ev = [torch.cuda.Event(enable_timing=True) for _ in range(steps + 1)]
+L2_BYTES = 126e6
+
+
+class L2Flush:
+    """Timing hygiene for inputs that fit in L2 (126 MB): a write of 256 MB
+    between timed steps evicts them, so every step reads its inputs from
+    HBM.  The write runs between the step's events, outside the timed
+    interval.  For inputs larger than L2 it does nothing."""
+
+    def __init__(self, input_bytes: float, dev):
+        self.input_bytes = float(input_bytes)
+        self.active = self.input_bytes < L2_BYTES
+        self.buf = (torch.empty(int(2 * 128 * 2**20) // 4, dtype=torch.int32, device=dev)
+                    if self.active else None)
+        self.n = 0
+
+    def __call__(self):
+        if self.active:
+            self.n += 1
+            self.buf.fill_(self.n)
+
+    def note(self) -> str:
+        mb = self.input_bytes / 1e6
+        if self.active:
+            return (f"inputs {mb:.1f} MB fit in L2 (126 MB): L2 flushed between timed steps "
+                    "by a 256 MB write outside each step's events")
+        return f"inputs larger than L2: {mb:.0f} MB vs 126 MB; no flush"
+
+
+def timed_steps(step, steps: int, stream, dev, flush=None):
+    """Run ``steps`` steps on the launching stream, synchronised on both
+    sides.  Without a flush: one event before each step and one after the
+    last (back-to-back steps).  With an L2 flush: the flush runs before each
+    step, outside that step's pair of events, and the total is the sum of
+    the steps.  Returns the total milliseconds and the per-step list."""
     torch.cuda.synchronize(dev)
+    if flush is not None and flush.active:
+        ev0 = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+        ev1 = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+        for i in range(steps):
+            flush()
+            ev0[i].record(stream)
+            step()
+            ev1[i].record(stream)
+        torch.cuda.synchronize(dev)
+        per = [ev0[i].elapsed_time(ev1[i]) for i in range(steps)]
+        return sum(per), per
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(steps + 1)]
     for i in range(steps):
         ev[i].record(stream)
         step()
@@ -389,11 +431,12 @@ def run_b200(args, w):
     sampler = ClockSampler(dev)
     for _ in range(args.warmup):
         step()
+    flush = L2Flush(3 * w.rows * w.d * 2, dev)
     torch.cuda.synchronize(dev)
     sampler.start()
     if pg:
         torch.distributed.barrier()
-    ms_total, per_step = timed_steps(step, args.steps, stream, dev)
+    ms_total, per_step = timed_steps(step, args.steps, stream, dev, flush)
     clocks = sampler.stop()
     if pg:
         torch.distributed.barrier()
@@ -469,7 +512,7 @@ def run_b200(args, w):
         "config": {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d,
                    "causal": w.causal, "scale": w.scale, "q_std": w.q_std,
                    "flops_per_step": w.flops,
-                   "l2": f"inputs larger than L2: Q+K+V {3 * tb / 1e6:.0f} MB vs 126 MB; no flush",
+                   "l2": flush.note(),
                    "parallelism": f"replica x{world} (independent batches)",
                    "kernel": "cta_pair (attn_fwd_pair)" if pair else "one_cta (attn_fwd)",
                    "tuning": None if not tuned else {
@@ -500,7 +543,8 @@ def run_b200(args, w):
         tf, nrows, secs, cores, last = time_oracle(w, bits, args.cpu_seconds)
         line["cpu_baseline"] = {
             "value": round(tf, 6), "unit": UNIT, "cores": cores, "kind": "oracle",
-            "sample": f"{nrows} seeded random rows of {w.rows} ({secs:.1f} s); "
+            "sample": f"{nrows} row evaluations in seeded batches of distinct rows (a row "
+                      f"may recur across batches) out of {w.rows} rows ({secs:.1f} s); "
                       "TFLOPS from the rows' exact share of the metric FLOPs"}
         # the timed step's output, against the oracle rows the leg computed
         line["parity"] = parity_of_rows(o, lse, w, last)
@@ -578,20 +622,14 @@ def run_general(args, w):
     sampler = ClockSampler(dev)
     for _ in range(args.warmup):
         step()
+    flush = L2Flush(2 * (q.numel() + k.numel() + v.numel()), dev)
     torch.cuda.synchronize(dev)
     sampler.start()
-    e0 = torch.cuda.Event(enable_timing=True)
-    e1 = torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(args.steps):
-        step()
-    e1.record(stream)
-    torch.cuda.synchronize(dev)
+    ms_step = timed_steps(step, args.steps, stream, dev, flush)[0] / args.steps
     clocks = sampler.stop()
     status = tab.last_device_error(stream)
     if status != 0:
         raise SystemExit(f"device status {status}: {tab.strerror(status)}")
-    ms_step = e0.elapsed_time(e1) / args.steps
     flops = 4.0 * w.d * visible_pairs(w)
     bytes_alg = 2 * (q.numel() + k.numel() + v.numel() + o.numel()) + 4 * lse.numel()
     peaks, peak_kind = load_peaks()
@@ -612,8 +650,7 @@ def run_general(args, w):
     cfg["workload"] = cfg.pop("name")
     if w.kind == "varlen":
         cfg["lens"] = list(w.lens_q)
-    cfg.update({"flops_per_step": flops, "l2": "inputs larger than L2; no flush"
-                if bytes_alg > 126e6 else "inputs fit in L2 (126 MB); no flush"})
+    cfg.update({"flops_per_step": flops, "l2": flush.note()})
     return {
         "metric": METRIC, "value": round(tflops, 2), "unit": UNIT, "n_gpus": 1,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 4),
@@ -665,25 +702,19 @@ def run_fp8(args, w):
                               ctypes.c_float(1.0), sh)
         assert rc == 0, rc
 
-    def timed(fn, steps):
+    def timed(fn, steps, flush):
         for _ in range(args.warmup):
             fn()
-        torch.cuda.synchronize(dev)
-        e0 = torch.cuda.Event(enable_timing=True)
-        e1 = torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        for _ in range(steps):
-            fn()
-        e1.record(stream)
-        torch.cuda.synchronize(dev)
-        return e0.elapsed_time(e1) / steps
+        return timed_steps(fn, steps, stream, dev, flush)[0] / steps
 
+    flush_attn = L2Flush(3 * w.rows * w.d, dev)       # E4M3 Q, K, V^T
+    flush_conv = L2Flush(3 * w.rows * w.d * 2, dev)   # their bf16 sources
     convert()
     sampler = ClockSampler(dev)
     sampler.start()
-    ms_attn = timed(attend, args.steps)
+    ms_attn = timed(attend, args.steps, flush_attn)
     clocks = sampler.stop()
-    ms_conv = timed(convert, max(1, args.steps // 4))
+    ms_conv = timed(convert, max(1, args.steps // 4), flush_conv)
     status = tab.last_device_error(stream)
     if status != 0:
         raise SystemExit(f"device status {status}: {tab.strerror(status)}")
@@ -699,7 +730,7 @@ def run_fp8(args, w):
         "config": {"workload": w.name + FP8_SUFFIX, "B": w.B, "H": w.H, "N": w.N, "d": w.d,
                    "causal": w.causal, "flops_per_step": w.flops,
                    "descales": [1.0, 1.0, 1.0],
-                   "l2": "inputs larger than L2; no flush"},
+                   "l2": flush_attn.note()},
         "roofline": {"bound": "tensor", "achieved": round(tflops, 2),
                      "peak": 2.0 * float(peaks["bf16_tflops"]), "unit": "TFLOP/s",
                      "frac": round(tflops / (2.0 * float(peaks["bf16_tflops"])), 4),
@@ -760,17 +791,20 @@ def run_fp4(args, w):
         rc = lib.attn_fwd_fp4(*cargs)
         assert rc == 0, rc
 
-    def timed(fn, steps):
+    def timed(fn, steps, flush):
         for _ in range(args.warmup):
             fn()
-        return timed_steps(fn, steps, stream, dev)[0] / steps
+        return timed_steps(fn, steps, stream, dev, flush)[0] / steps
 
+    # E2M1 codes (half a byte per element) and their E4M3 scales
+    flush_attn = L2Flush(3 * (w.rows * w.d // 2 + BH * T * 1024), dev)
+    flush_conv = L2Flush(3 * w.rows * w.d * 2, dev)   # the bf16 sources
     convert()
     sampler = ClockSampler(dev)
     sampler.start()
-    ms_attn = timed(attend, args.steps)
+    ms_attn = timed(attend, args.steps, flush_attn)
     clocks = sampler.stop()
-    ms_conv = timed(convert, max(1, args.steps // 4))
+    ms_conv = timed(convert, max(1, args.steps // 4), flush_conv)
     status = tab.last_device_error(stream)
     if status != 0:
         raise SystemExit(f"device status {status}: {tab.strerror(status)}")
@@ -788,7 +822,7 @@ def run_fp4(args, w):
         "data": "synthetic (the square workload's seeded bf16 inputs, converted to NVFP4)",
         "config": {"workload": w.name + FP4_SUFFIX, "B": w.B, "H": w.H, "N": w.N, "d": w.d,
                    "causal": w.causal, "flops_per_step": w.flops, "descales": [1.0, 1.0, 1.0],
-                   "l2": "inputs larger than L2; no flush"},
+                   "l2": flush_attn.note()},
         "roofline": {"bound": "tensor", "achieved": round(tflops, 2),
                      "peak": 4.0 * float(peaks["bf16_tflops"]), "unit": "TFLOP/s",
                      "frac": round(tflops / (4.0 * float(peaks["bf16_tflops"])), 4),
@@ -834,20 +868,14 @@ def run_kmeans(args, w):
     sampler = ClockSampler(dev)
     for _ in range(args.warmup):
         step()
+    flush = L2Flush(2 * (x.numel() + c.numel()), dev)
     torch.cuda.synchronize(dev)
     sampler.start()
-    e0 = torch.cuda.Event(enable_timing=True)
-    e1 = torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(args.steps):
-        step()
-    e1.record(stream)
-    torch.cuda.synchronize(dev)
+    ms_step = timed_steps(step, args.steps, stream, dev, flush)[0] / args.steps
     clocks = sampler.stop()
     status = tab.last_device_error(stream)
     if status != 0:
         raise SystemExit(f"device status {status}: {tab.strerror(status)}")
-    ms_step = e0.elapsed_time(e1) / args.steps
     bytes_alg = 2 * (x.numel() + c.numel()) + 8 * w.N
     tflops = w.flops / (ms_step * 1e-3) / 1e12
     peaks, peak_kind = load_peaks()
@@ -858,8 +886,7 @@ def run_kmeans(args, w):
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded centroids and points around them, see inputs.py)",
         "config": {"workload": w.name, "N": w.N, "K": w.K, "d": w.d, "flops_per_step": w.flops,
-                   "l2": "inputs fit in L2 (126 MB); no flush" if bytes_alg < 126e6
-                   else "inputs larger than L2; no flush"},
+                   "l2": flush.note()},
         "roofline": {"bound": "tensor", "achieved": round(tflops, 2),
                      "peak": float(peaks["bf16_tflops"]), "unit": "TFLOP/s",
                      "frac": round(tflops / float(peaks["bf16_tflops"]), 4), "traffic": None,
