@@ -40,7 +40,10 @@ typedef enum {
   ATTN_ERR_CUDA = -4,          /* a CUDA runtime/driver call failed */
   ATTN_ERR_DEVICE_TIMEOUT = -5,/* a bounded wait inside the kernel ran out */
   ATTN_ERR_DEVICE_BOUNDS = -6, /* device-side check: sequence offsets do not
-                                  fit the buffers (attn_fwd_varlen) */
+                                  fit the buffers (attn_fwd_varlen); in the
+                                  bounds-checked debug build also a tile
+                                  coordinate or output index outside the
+                                  launch's tensors */
   ATTN_ERR_NO_DEVICE = -7      /* no usable sm_100 device is current */
 } attn_status;
 

@@ -43,57 +43,46 @@ def library():
         if not os.path.exists(LIB):
             raise RuntimeError(
                 f"CUDA library {LIB} not built; run python -m tiled_attention_forward_sm_b200.build")
-        lib = ctypes.CDLL(LIB)
-        vp, i, f = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
-        lib.attn_fwd.restype = i
-        lib.attn_fwd.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, f, vp]
-        lib.attn_fwd_ex.restype = i
-        lib.attn_fwd_ex.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, f, vp, vp]
-        lib.attn_fwd_noalloc.restype = i
-        lib.attn_fwd_noalloc.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, f, vp]
-        lib.attn_fwd_pair.restype = i
-        lib.attn_fwd_pair.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, f, vp]
-        lib.attn_fwd_host.restype = i
-        lib.attn_fwd_host.argtypes = [vp] * 10 + [i, i, i, i, i, f, vp]
-        lib.attn_selftest_wait_timeout.restype = i
-        lib.attn_selftest_wait_timeout.argtypes = [i, vp]
-        lib.attn_last_device_error.restype = i
-        lib.attn_last_device_error.argtypes = [vp]
-        lib.attn_strerror.restype = ctypes.c_char_p
-        lib.attn_strerror.argtypes = [i]
-        lib.attn_check_args.restype = i
-        lib.attn_check_args.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, f]
-        lib.attn_version.restype = i
-        lib.attn_version.argtypes = []
-        lib.attn_release.restype = i
-        lib.attn_release.argtypes = []
-        lib.attn_opts_default.restype = AttnOpts
-        lib.attn_opts_default.argtypes = []
-        lib.attn_fwd_chunk.restype = i
-        lib.attn_fwd_chunk.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, i, i, f, i, vp]
-        lib.attn_fwd_varlen.restype = i
-        lib.attn_fwd_varlen.argtypes = [vp] * 7 + [i] * 9 + [f, vp]
-        lib.attn_fwd_splitkv.restype = i
-        lib.attn_fwd_splitkv.argtypes = [vp] * 5 + [i] * 8 + [f, i, vp, vp, vp]
-        lib.attn_fwd_fp8.restype = i
-        lib.attn_fwd_fp8.argtypes = [vp] * 5 + [i] * 5 + [f, f, f, f, vp]
-        lib.attn_quantize_e4m3.restype = i
-        lib.attn_quantize_e4m3.argtypes = [vp, vp, i, i, i, f, i, vp]
-        lib.attn_fwd_fp4.restype = i
-        lib.attn_fwd_fp4.argtypes = [vp] * 8 + [i] * 5 + [f, f, f, f, vp]
-        lib.attn_quantize_nvfp4.restype = i
-        lib.attn_quantize_nvfp4.argtypes = [vp, vp, vp, i, i, i, f, i, vp]
-        lib.attn_nvfp4_scale_bytes.restype = ctypes.c_longlong
-        lib.attn_nvfp4_scale_bytes.argtypes = [i, i]
-        lib.attn_kmeans_assign.restype = i
-        lib.attn_kmeans_assign.argtypes = [vp, vp, vp, vp, vp, i, i, i, vp]
-        lib.attn_kmeans_workspace_floats.restype = ctypes.c_longlong
-        lib.attn_kmeans_workspace_floats.argtypes = [i, i]
-        lib.attn_combine.restype = i
-        lib.attn_combine.argtypes = [vp, vp, i, ctypes.c_longlong, i, vp, vp, i, vp]
-        _lib = lib
+        _lib = configure(ctypes.CDLL(LIB))
     return _lib
 
+
+def configure(lib):
+    """Declare the C ABI's signatures on a ctypes handle of the library (or
+    of one of its debugging builds, which export a subset of the entry
+    points: a symbol a build does not export is left undeclared)."""
+    vp, i, f = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
+    sigs = {  # name: (return type, argument types)
+        "attn_fwd": (i, [vp, vp, vp, vp, vp, i, i, i, i, i, f, vp]),
+        "attn_fwd_ex": (i, [vp, vp, vp, vp, vp, i, i, i, i, i, f, vp, vp]),
+        "attn_fwd_noalloc": (i, [vp, vp, vp, vp, vp, i, i, i, i, i, f, vp]),
+        "attn_fwd_pair": (i, [vp, vp, vp, vp, vp, i, i, i, i, i, f, vp]),
+        "attn_fwd_host": (i, [vp] * 10 + [i, i, i, i, i, f, vp]),
+        "attn_selftest_wait_timeout": (i, [i, vp]),
+        "attn_last_device_error": (i, [vp]),
+        "attn_strerror": (ctypes.c_char_p, [i]),
+        "attn_check_args": (i, [vp, vp, vp, vp, vp, i, i, i, i, f]),
+        "attn_version": (i, []),
+        "attn_release": (i, []),
+        "attn_opts_default": (AttnOpts, []),
+        "attn_fwd_chunk": (i, [vp, vp, vp, vp, vp, i, i, i, i, i, i, i, i, f, i, vp]),
+        "attn_fwd_varlen": (i, [vp] * 7 + [i] * 9 + [f, vp]),
+        "attn_fwd_splitkv": (i, [vp] * 5 + [i] * 8 + [f, i, vp, vp, vp]),
+        "attn_fwd_fp8": (i, [vp] * 5 + [i] * 5 + [f, f, f, f, vp]),
+        "attn_quantize_e4m3": (i, [vp, vp, i, i, i, f, i, vp]),
+        "attn_fwd_fp4": (i, [vp] * 8 + [i] * 5 + [f, f, f, f, vp]),
+        "attn_quantize_nvfp4": (i, [vp, vp, vp, i, i, i, f, i, vp]),
+        "attn_nvfp4_scale_bytes": (ctypes.c_longlong, [i, i]),
+        "attn_kmeans_assign": (i, [vp, vp, vp, vp, vp, i, i, i, vp]),
+        "attn_kmeans_workspace_floats": (ctypes.c_longlong, [i, i]),
+        "attn_combine": (i, [vp, vp, i, ctypes.c_longlong, i, vp, vp, i, vp]),
+    }
+    for name, (restype, argtypes) in sigs.items():
+        if hasattr(lib, name):
+            fn = getattr(lib, name)
+            fn.restype = restype
+            fn.argtypes = argtypes
+    return lib
 
 def strerror(status: int) -> str:
     return library().attn_strerror(int(status)).decode()

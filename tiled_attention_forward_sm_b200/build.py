@@ -9,6 +9,15 @@ entry points compiled with ATTN_TEST_HOOKS, which adds
 wait runs out and the kernels' abort path runs; see the GPU test of the
 abort path).  The product library never carries these hooks.
 
+``--checked`` builds ``libattn_b200_checked.so``: the same entry points as
+the test-hooks library compiled with ATTN_BOUNDS_CHECKS as well, so that
+every tensor-map coordinate and every O / LSE store index is checked against
+the launch's tensor extents before the access (a failed check writes
+ATTN_ERR_DEVICE_BOUNDS to the status word and skips the access), plus
+``int attn_test_set_bad_kv_head(int offset)`` to plant one bad K/V head
+index that the check must catch.  A debugging build; the product library
+carries neither the checks nor the hook.
+
 ``--trace`` builds the timeline-tracing library ``libattn_b200_trace.so``
 instead: the attention kernel compiled with its clock64 stamps at every role
 hand-off (ATTN_TRACE_ENABLED) and the extra entry point
@@ -32,6 +41,7 @@ INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libattn_b200.so")
 TRACE_LIB = os.path.join(PKG, "libattn_b200_trace.so")
 TEST_HOOKS_LIB = os.path.join(PKG, "libattn_b200_testhooks.so")
+CHECKED_LIB = os.path.join(PKG, "libattn_b200_checked.so")
 SOURCES = [os.path.join(CSRC, f) for f in ("attn_fwd.cu", "fp8.cu", "fp4.cu", "kmeans.cu", "pair.cu",
                                            "host_io.cu")]
 HEADERS = [os.path.join(CSRC, f) for f in os.listdir(CSRC) if f.endswith((".cuh", ".h"))] + [
@@ -88,9 +98,23 @@ def build_test_hooks(force: bool = False) -> str:
     return TEST_HOOKS_LIB
 
 
+def build_checked(force: bool = False) -> str:
+    """The bounds-checked test library (attention and FP8 entry points)."""
+    srcs = [os.path.join(CSRC, f) for f in ("attn_fwd.cu", "fp8.cu")]
+    if (not force and os.path.exists(CHECKED_LIB) and
+            all(os.path.getmtime(p) <= os.path.getmtime(CHECKED_LIB) for p in srcs + HEADERS)):
+        return CHECKED_LIB
+    cmd = [nvcc_path(), *NVCC_FLAGS, "-DATTN_TEST_HOOKS", "-DATTN_BOUNDS_CHECKS", "-o",
+           CHECKED_LIB, *srcs]
+    subprocess.check_call(cmd)
+    return CHECKED_LIB
+
+
 if __name__ == "__main__":
     if "--test-hooks" in sys.argv:
         print(build_test_hooks(force=True))
+    elif "--checked" in sys.argv:
+        print(build_checked(force=True))
     elif "--trace" in sys.argv:
         print(build_trace(force=True, verbose="--verbose" in sys.argv))
     else:

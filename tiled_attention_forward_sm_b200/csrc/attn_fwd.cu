@@ -355,6 +355,7 @@ int launch(const Problem& p, cudaStream_t stream, DeviceState& st, int* queue = 
   args.split_rows = p.split_rows;
   args.o_f32 = p.o_f32;
   args.BH = args.head_pack ? p.B * p.H_kv : p.B * p.H;  // units of the item windows
+  args.B = p.B;
   args.n_items = static_cast<int>(problem_items(p, st.num_sms));
   // Scheduling window: enough heads that a window holds about two rounds of
   // items (so its light tail evens out the CTAs), few enough that the
@@ -798,6 +799,19 @@ extern "C" int attn_test_set_hooks(unsigned long long wait_limit_ns, int withhol
     return ATTN_ERR_CUDA;
   }
   return host::fp8_test_set_hooks(wait_limit_ns, withhold_load);
+}
+#endif
+
+#if defined(ATTN_BOUNDS_CHECKS) && defined(ATTN_TEST_HOOKS)
+// Checked test builds only: an offset added to the K/V head of CTA 0's first
+// item (0 for none), which the producer's bounds check must catch before
+// any load of that head is issued.
+extern "C" int attn_test_set_bad_kv_head(int offset) {
+  if (cudaMemcpyToSymbol(g_test_bad_kv_head, &offset, sizeof offset) != cudaSuccess) {
+    cudaGetLastError();
+    return ATTN_ERR_CUDA;
+  }
+  return ATTN_OK;
 }
 #endif
 

@@ -82,6 +82,22 @@ __device__ __forceinline__ constexpr uint64_t wait_limit_ns() { return kWaitLimi
 __device__ __forceinline__ constexpr bool withhold_load(int) { return false; }
 #endif
 
+// Checked builds (ATTN_BOUNDS_CHECKS, libattn_b200_checked.so only) test
+// every tensor-map coordinate and every O / LSE store index against the
+// extents of the launch's tensors before the access is issued.  A failed
+// check writes the bounds status, raises the CTA's abort flag and skips the
+// access; nothing traps.  With the test hooks as well, the producer of CTA 0
+// can be told to add an offset to its first item's K/V head, which a
+// checked build must catch before any load of that head is issued.
+#if defined(ATTN_BOUNDS_CHECKS) && defined(ATTN_TEST_HOOKS)
+static __device__ int g_test_bad_kv_head = 0;
+__device__ __forceinline__ int test_bad_kv_head() {
+  return blockIdx.x == 0 ? g_test_bad_kv_head : 0;
+}
+#else
+__device__ __forceinline__ constexpr int test_bad_kv_head() { return 0; }
+#endif
+
 // Softmax arithmetic form: packed f32x2 FMA/ADD (1) or scalar FMA/ADD (0).
 // Measured on B200 the packed form is faster.
 #ifndef ATTN_PACKED_SOFTMAX
@@ -169,7 +185,8 @@ struct KernelArgs {
   int split_tiles;    // K/V tiles per slice
   long long split_rows;  // rows of one slice of the outputs (0 without slices)
   int o_f32;          // store O as fp32 instead of bf16
-  int BH;             // B * H
+  int BH;             // B * H (B * H_kv when two query heads share an item)
+  int B;              // batch (sequences in the packed layout)
   int n_items;        // BH * n_qpairs * n_splits work items (some may be empty)
   int win_heads;      // heads per scheduling window (item order, see make_item)
   float scale_log2;   // scale * log2(e)
@@ -225,6 +242,38 @@ struct Shared {
 __device__ __forceinline__ void raise_status(const Shared& sh, int* status, int code) {
   *sh.abort_flag = 1;
   atomicCAS(status, 0, code);
+}
+
+// In checked builds: ok, or the bounds status written and the abort flag
+// raised (the caller then skips the access).  Elsewhere: true.
+__device__ __forceinline__ bool in_bounds(const Shared& sh, int* status, bool ok) {
+#ifdef ATTN_BOUNDS_CHECKS
+  if (!ok) raise_status(sh, status, kStatusDeviceBounds);
+  return ok;
+#else
+  (void)sh;
+  (void)status;
+  (void)ok;
+  return true;
+#endif
+}
+
+// Tile coordinates inside the tensor maps: the first row (token) of a tile
+// lies inside the tensor and the head exists.  Rows of a tile past the end
+// of a ragged sequence are the maps' zero fill, not an error.
+__device__ __forceinline__ bool q_tile_ok(const KernelArgs& a, long long row, int z) {
+  if (a.cu_q != nullptr) return row >= 0 && row < a.T_q && z >= 0 && z < a.H;
+  return row >= 0 && row < a.N_q && z >= 0 && z < a.B * a.H;
+}
+__device__ __forceinline__ bool kv_tile_ok(const KernelArgs& a, long long row, int z) {
+  if (a.cu_q != nullptr) return row >= 0 && row < a.T_k && z >= 0 && z < a.H_kv;
+  return row >= 0 && row < a.N_k && z >= 0 && z < a.B * a.H_kv;
+}
+// O rows (of D values) and LSE entries of the launch's outputs.
+__device__ __forceinline__ long long out_rows(const KernelArgs& a) {
+  const long long one = a.cu_q != nullptr ? static_cast<long long>(a.T_q) * a.H
+                                          : static_cast<long long>(a.B) * a.H * a.N_q;
+  return a.n_splits > 1 ? a.n_splits * a.split_rows : one;
 }
 
 // Single-thread bounded wait.  A drain wait (for this thread's own copies or
@@ -531,6 +580,7 @@ __device__ void producer_role(const Shared& sh, const KernelArgs& a, uint8_t* sm
     }
   };
   bool have = claim();
+  if (have) it.kz += test_bad_kv_head();  // test builds only
   for (int r = 0; ok; ++r) {
     if (!have) {
       post_item(sh, a, r, nullptr);
@@ -546,9 +596,14 @@ __device__ void producer_role(const Shared& sh, const KernelArgs& a, uint8_t* sm
         ok = false;
         break;
       }
+      const int q_row = it.q_row0 + item_qtile(it, s) * kBlockM;
+      if (!in_bounds(sh, a.status, q_tile_ok(a, q_row, item_qz(it, s)))) {
+        ok = false;
+        break;
+      }
       ptx::mbar_arrive_expect_tx(&sh.q_full[s], C::kTileBytes);
-      load_tile(tq, &sh.q_full[s], smem + C::kQOff + s * C::kTileBytes,
-                it.q_row0 + item_qtile(it, s) * kBlockM, item_qz(it, s), pol_q);
+      load_tile(tq, &sh.q_full[s], smem + C::kQOff + s * C::kTileBytes, q_row, item_qz(it, s),
+                pol_q);
       ++q_loads[s];
     }
     for (int j = 0; j < n && ok; ++j) {
@@ -561,10 +616,11 @@ __device__ void producer_role(const Shared& sh, const KernelArgs& a, uint8_t* sm
           continue;
         }
         uint8_t* dst = smem + C::kKVOff + st * C::kTileBytes;
+        const int kv_row = it.k_row0 + (it.kt0 + j) * kBlockN;
+        if (!in_bounds(sh, a.status, kv_tile_ok(a, kv_row, it.kz))) { ok = false; break; }
         ATTN_TRACE(which == 0 ? kTrProdK : kTrProdV, r == 0 ? j : -1);
         ptx::mbar_arrive_expect_tx(&sh.kv_full[st], C::kTileBytes);
-        load_tile(which == 0 ? tk : tv, &sh.kv_full[st], dst,
-                  it.k_row0 + (it.kt0 + j) * kBlockN, it.kz, pol_kv);
+        load_tile(which == 0 ? tk : tv, &sh.kv_full[st], dst, kv_row, it.kz, pol_kv);
         ++issued;
       }
     }
@@ -974,6 +1030,9 @@ __device__ void softmax_role(const Shared& sh, const KernelArgs& a, uint32_t tme
     }
     o_row += static_cast<size_t>(it.split) * a.split_rows;
     l_row += static_cast<size_t>(it.split) * a.split_rows;
+    const bool store = row_ok && in_bounds(sh, a.status,
+                                           static_cast<long long>(o_row) < out_rows(a) &&
+                                               static_cast<long long>(l_row) < out_rows(a));
 #pragma unroll 1
     for (int c0 = 0; c0 < D; c0 += 32) {
       uint32_t ov[32];
@@ -987,7 +1046,7 @@ __device__ void softmax_role(const Shared& sh, const KernelArgs& a, uint32_t tme
 #pragma unroll
         for (int c = 0; c < 32; ++c) ov[c] = 0u;
       }
-      if (!row_ok) continue;
+      if (!store) continue;
       if (a.o_f32) {
         uint4* dst = reinterpret_cast<uint4*>(static_cast<float*>(a.o) + o_row * D + c0);
 #pragma unroll
@@ -1005,7 +1064,7 @@ __device__ void softmax_role(const Shared& sh, const KernelArgs& a, uint32_t tme
           dst[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
       }
     }
-    if (row_ok) a.lse[l_row] = empty ? -INFINITY : (m + log2f(l)) * 0.69314718055994531f;
+    if (store) a.lse[l_row] = empty ? -INFINITY : (m + log2f(l)) * 0.69314718055994531f;
   }
 }
 

@@ -95,9 +95,11 @@ __device__ void producer_role(const Shared& sh, const Bars& bb, const KernelArgs
       ++issued;
       return true;
     }
+    const int kv_row = it.k_row0 + (it.kt0 + j) * kBlockN;
+    if (!in_bounds(sh, a.status, kv_tile_ok(a, kv_row, it.kz))) return false;
     ptx::mbar_arrive_expect_tx(&bb.kv_full[st], kTileBytes);
-    load_tile(is_v ? tv : tk, &bb.kv_full[st], smem + kKVOff + st * kTileBytes,
-              it.k_row0 + (it.kt0 + j) * kBlockN, it.kz, pol_kv);
+    load_tile(is_v ? tv : tk, &bb.kv_full[st], smem + kKVOff + st * kTileBytes, kv_row, it.kz,
+              pol_kv);
     ++issued;
     return true;
   };
@@ -109,6 +111,7 @@ __device__ void producer_role(const Shared& sh, const Bars& bb, const KernelArgs
     }
   };
   bool have = claim();
+  if (have) it.kz += test_bad_kv_head();  // test builds only
   for (int r = 0; ok; ++r) {
     if (!have) {
       post_item(sh, a, r, nullptr);
@@ -124,9 +127,13 @@ __device__ void producer_role(const Shared& sh, const Bars& bb, const KernelArgs
         ok = false;
         break;
       }
+      const int q_row = it.q_row0 + (2 * it.qpair + s) * kBlockM;
+      if (!in_bounds(sh, a.status, q_tile_ok(a, q_row, it.qz))) {
+        ok = false;
+        break;
+      }
       ptx::mbar_arrive_expect_tx(bb.q_full, kTileBytes);
-      load_tile(tq, bb.q_full, smem + kQOff, it.q_row0 + (2 * it.qpair + s) * kBlockM, it.qz,
-                pol_q);
+      load_tile(tq, bb.q_full, smem + kQOff, q_row, it.qz, pol_q);
       ++q_loads;
       ok = push(false, 0) && (n < 2 || push(false, 1));
       for (int j = 0; j < n && ok; ++j) ok = push(true, j) && (j + 2 >= n || push(false, j + 2));
@@ -366,6 +373,9 @@ __device__ void softmax_role(const Shared& sh, const Bars& bb, const KernelArgs&
       }
       o_row += static_cast<size_t>(it.split) * a.split_rows;
       l_row += static_cast<size_t>(it.split) * a.split_rows;
+      const bool store = row_ok && in_bounds(sh, a.status,
+                                             static_cast<long long>(o_row) < out_rows(a) &&
+                                                 static_cast<long long>(l_row) < out_rows(a));
 #pragma unroll 1
       for (int c0 = 0; c0 < kD; c0 += 32) {
         uint32_t ov[32];
@@ -379,7 +389,7 @@ __device__ void softmax_role(const Shared& sh, const Bars& bb, const KernelArgs&
 #pragma unroll
           for (int c = 0; c < 32; ++c) ov[c] = 0u;
         }
-        if (!row_ok) continue;
+        if (!store) continue;
         if (a.o_f32) {
           uint4* dst = reinterpret_cast<uint4*>(static_cast<float*>(a.o) + o_row * kD + c0);
 #pragma unroll
@@ -397,7 +407,7 @@ __device__ void softmax_role(const Shared& sh, const Bars& bb, const KernelArgs&
             dst[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
         }
       }
-      if (row_ok) a.lse[l_row] = empty ? -INFINITY : (m + log2f(l)) * 0.69314718055994531f;
+      if (store) a.lse[l_row] = empty ? -INFINITY : (m + log2f(l)) * 0.69314718055994531f;
     }
   }
 }
