@@ -879,9 +879,16 @@ __device__ __forceinline__ bool softmax_step(const Shared& sh, const KernelArgs&
     rescale = !first;
   }
   // O_s *= alpha for the rows whose max moved (PV_s(j-1) is complete: its
-  // commit preceded the one that published S_s(j)).  Done before any P is
-  // published, so the first half of PV_s(j) sees the rescaled O.
-  if (__any_sync(0xffffffffu, rescale)) {
+  // commit preceded the one that published S_s(j)), before any P is
+  // published, so the first half of PV_s(j) sees the rescaled O.  Where:
+  // under the causal mask after the first half's weights, which the
+  // warp-wide vote then overlaps (1.7% faster on B2 H32 N8192, 5% at
+  // N 32768, 0.6% slower with peaky scores); without the mask before them
+  // (the late form is 0.3-0.7% faster there with ordinary scores but 1.5%
+  // slower with peaky ones, whose frequent rescales it leaves exposed).
+  constexpr bool kLateRescale = CAUSAL;
+  const bool any_rescale = __any_sync(0xffffffffu, rescale);
+  if (!kLateRescale && any_rescale) {
 #pragma unroll 1
     for (int c0 = 0; c0 < D; c0 += 32) {
       uint32_t ov[32];
@@ -892,6 +899,19 @@ __device__ __forceinline__ bool softmax_step(const Shared& sh, const KernelArgs&
       ptx::tmem_st32(t_o + c0, ov);
     }
   }
+  // (the late form in 16-column pieces: half of P and the second half's
+  // scores still hold registers)
+  auto rescale_o_late = [&]() {
+#pragma unroll 1
+    for (int c0 = 0; c0 < D; c0 += 16) {
+      uint32_t ov[16];
+      ptx::tmem_ld16(t_o + c0, ov);
+      ptx::tmem_ld_wait_tie16(ov);
+#pragma unroll
+      for (int c = 0; c < 16; ++c) ov[c] = __float_as_uint(__uint_as_float(ov[c]) * alpha);
+      ptx::tmem_st16(t_o + c0, ov);
+    }
+  };
   const uint64_t sl2x2 = ptx::f2pack(sl2, sl2);
   // A row that has seen no visible key yet keeps m = -inf; its weights are
   // then computed against 0 (all masked scores give 0, never NaN).
@@ -942,6 +962,7 @@ __device__ __forceinline__ bool softmax_step(const Shared& sh, const KernelArgs&
 #endif
       pk[q] = ptx::pack_bf16x2(p0, p1);
     }
+    if (kLateRescale && half == 0 && any_rescale) rescale_o_late();
     // P_s keys [64*half, 64*half+64) as bf16 pairs over TMEM columns
     // [32*half, 32*half+32) of the S_s region; publish this half at once.
     ptx::tmem_st32(t_s + 32 * half, pk);

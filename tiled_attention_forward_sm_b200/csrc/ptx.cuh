@@ -418,6 +418,22 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t* r) {
       : "memory");
 }
 
+// 16 columns per call.
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t* r) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+      : ATTN_R8(r, 0), ATTN_R8(r, 8)
+      : "r"(taddr)
+      : "memory");
+}
+
+// Wait for this thread's outstanding TMEM loads, the 16 registers of the
+// most recent 16-column load tied to the wait.
+__device__ __forceinline__ void tmem_ld_wait_tie16(uint32_t* r) {
+  asm volatile("tcgen05.wait::ld.sync.aligned;" : ATTN_T8(r, 0), ATTN_T8(r, 8) : : "memory");
+}
+
 // Wait for this thread's outstanding TMEM loads.  The 32 registers of the
 // most recent load are tied to the wait so no use of them can be scheduled
 // before it.
