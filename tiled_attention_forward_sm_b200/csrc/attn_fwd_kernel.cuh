@@ -51,6 +51,7 @@
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cstdint>
+#include <type_traits>
 
 #include "ptx.cuh"
 
@@ -125,6 +126,15 @@ constexpr int kRegsSoftmax = 200;
 constexpr int kRegsOther = 104;
 constexpr int kRegSplitTotal = 256 * kRegsSoftmax + 128 * kRegsOther;
 static_assert(kRegSplitTotal <= kThreads * 168, "register split exceeds the launch budget");
+
+// Keys of a score tile in the first published part of P (a multiple of 16,
+// one PV MMA per 16 keys); the second part holds the remaining 48.  The
+// uneven split leaves three PV MMAs, not four, between the last part's
+// announcement and the next S of the same Q tile, while the first part's
+// five MMAs run during the second part's exponentials (+1.1-1.5% with
+// peaky scores, unchanged elsewhere; 96 + 32 is slower).
+constexpr int kPFirstKeys = 80;
+static_assert(kPFirstKeys % 16 == 0 && kPFirstKeys > 0 && kPFirstKeys < 128, "P split");
 
 // Lazy-rescale threshold in log2 units: the running maximum is raised only
 // when a tile's maximum exceeds it by more than this, so every weight stays
@@ -666,13 +676,14 @@ __device__ void mma_role(const Shared& sh, const KernelArgs& a, uint8_t* smem, u
       ptx::mma_ss_elect(t_s[s], qd + off, kd + off, C::kIdescQK, kk > 0 ? 1u : 0u);
     }
   };
-  // O_s (+)= P_s V over keys [64*half, 64*half + 64): P from TMEM (8 columns
-  // per 16 keys), V MN-major (2 KB per 16 keys)
+  // O_s (+)= P_s V over the keys of one published part of P (half 0: keys
+  // [0, kPFirstKeys), half 1: the rest): P from TMEM (8 columns per 16
+  // keys), V MN-major (2 KB per 16 keys)
   auto issue_pv_half = [&](int s, int half, int stage, uint32_t accumulate) {
     const uint64_t vd = v_desc + stage * kTileUnits;
+    constexpr int kKa = kPFirstKeys / 16;  // MMAs of the first part
 #pragma unroll
-    for (int k4 = 0; k4 < 4; ++k4) {
-      const int kk = 4 * half + k4;
+    for (int kk = half ? kKa : 0; kk < (half ? 8 : kKa); ++kk) {
       ptx::mma_ts_elect(t_o[s], t_s[s] + 8 * kk, vd + static_cast<uint64_t>((kk * 2048) >> 4),
                         C::kIdescPV, (accumulate | static_cast<uint32_t>(kk > 0)));
     }
@@ -816,10 +827,27 @@ __device__ __forceinline__ float exp2_poly1(float x) {
   return __uint_as_float(__float_as_uint(p) + (__float_as_uint(t) << 23));
 }
 
+// N consecutive TMEM columns of this thread's lane from pk, in stores of 32,
+// 16 and 8 columns (N a multiple of 8).
+template <int N>
+__device__ __forceinline__ void store_cols(uint32_t taddr, const uint32_t* pk) {
+  if constexpr (N >= 32) {
+    ptx::tmem_st32(taddr, pk);
+    store_cols<N - 32>(taddr + 32, pk + 32);
+  } else if constexpr (N >= 16) {
+    ptx::tmem_st16(taddr, pk);
+    store_cols<N - 16>(taddr + 16, pk + 16);
+  } else if constexpr (N >= 8) {
+    ptx::tmem_st8(taddr, pk);
+    store_cols<N - 8>(taddr + 8, pk + 8);
+  }
+}
+
 // One K/V step of the online softmax for one query row (one thread):
 // S_s(j) from TMEM -> running max (lazy rule) -> weights -> P_s(j) back to
-// TMEM in two published halves; m and l are the row's running max (log2
-// units) and sum.  PAIR: the CTA is one of a cluster pair whose rank-0 CTA
+// TMEM in two published parts (keys [0, kPFirstKeys) and the rest); m and
+// l are the row's running max (log2 units) and sum.  PAIR: the CTA is one
+// of a cluster pair whose rank-0 CTA
 // issues the MMAs, so P is announced on that CTA's barrier.
 template <int D, bool CAUSAL, int kPolyPairs, bool PAIR = false>
 __device__ __forceinline__ bool softmax_step(const Shared& sh, const KernelArgs& a, int s,
@@ -925,12 +953,15 @@ __device__ __forceinline__ bool softmax_step(const Shared& sh, const KernelArgs&
 #else
   float ls0 = 0.f, ls1 = 0.f, ls2 = 0.f, ls3 = 0.f;
 #endif
+  // the two published parts of P: pairs [0, kPa) and [kPa, 64)
+  auto part = [&](auto half_c) {
+    constexpr int half = decltype(half_c)::value;
+    constexpr int kPa = kPFirstKeys / 2;
+    constexpr int q0 = half ? kPa : 0, q1 = half ? 64 : kPa;
+    uint32_t pk[q1 - q0];
 #pragma unroll
-  for (int half = 0; half < 2; ++half) {
-    uint32_t pk[32];
-#pragma unroll
-    for (int q = 0; q < 32; ++q) {
-      const int c = 64 * half + 2 * q;
+    for (int q = q0; q < q1; ++q) {
+      const int c = 2 * q;
 #if ATTN_PACKED_SOFTMAX
       const uint64_t y2 = ptx::ffma2(ptx::f2pack(x[c], x[c + 1]), sl2x2, negm2);
       uint64_t p2;
@@ -960,12 +991,14 @@ __device__ __forceinline__ bool softmax_step(const Shared& sh, const KernelArgs&
       }
       if (q & 1) { ls2 += p0; ls3 += p1; } else { ls0 += p0; ls1 += p1; }
 #endif
-      pk[q] = ptx::pack_bf16x2(p0, p1);
+      pk[q - q0] = ptx::pack_bf16x2(p0, p1);
     }
-    if (kLateRescale && half == 0 && any_rescale) rescale_o_late();
-    // P_s keys [64*half, 64*half+64) as bf16 pairs over TMEM columns
-    // [32*half, 32*half+32) of the S_s region; publish this half at once.
-    ptx::tmem_st32(t_s + 32 * half, pk);
+    if constexpr (half == 0) {
+      if (kLateRescale && any_rescale) rescale_o_late();
+    }
+    // P_s keys [2 q0, 2 q1) as bf16 pairs over TMEM columns [q0, q1) of the
+    // S_s region, in stores of 32, 16 and 8 columns; publish this part.
+    store_cols<q1 - q0>(t_s + q0, pk);
     ptx::tmem_st_wait();
     ptx::tc_fence_before_sync();
     __syncwarp();
@@ -976,7 +1009,9 @@ __device__ __forceinline__ bool softmax_step(const Shared& sh, const KernelArgs&
         ptx::mbar_arrive(&sh.p_ready[2 * s + half]);
     }
     if (r == 0) ATTN_TRACE(s == 0 ? (half ? kTrSm0Pb : kTrSm0Pa) : (half ? kTrSm1Pb : kTrSm1Pa), tj);
-  }
+  };
+  part(std::integral_constant<int, 0>{});
+  part(std::integral_constant<int, 1>{});
 #if ATTN_PACKED_SOFTMAX
   float la0, la1, lb0, lb1;
   ptx::f2unpack(lsum2a, la0, la1);

@@ -304,11 +304,13 @@ __device__ void mma_role(const Shared& sh, const KernelArgs& a, uint8_t* smem, u
       ptx::mma_pair_ss_elect(t_s[s], qd + qo, kd + ko, kIdescQK, kk > 0 ? 1u : 0u);
     }
   };
+  // (the parts of P that the shared softmax step publishes: keys
+  // [0, kPFirstKeys) and the rest)
   auto issue_pv_half = [&](int s, int half, int stage, uint32_t accumulate) {
     const uint64_t vd = v_desc + stage * kStageUnits;
+    constexpr int kKa = kPFirstKeys / 16;
 #pragma unroll
-    for (int k4 = 0; k4 < 4; ++k4) {
-      const int kk = 4 * half + k4;
+    for (int kk = half ? kKa : 0; kk < (half ? 8 : kKa); ++kk) {
       ptx::mma_pair_ts_elect(t_o[s], t_s[s] + 8 * kk, vd + static_cast<uint64_t>((kk * 2048) >> 4),
                              kIdescPV, (accumulate | static_cast<uint32_t>(kk > 0)));
     }
