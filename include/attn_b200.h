@@ -106,8 +106,10 @@ int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
  *                    condition): the running maximum moves only when a
  *                    tile's maximum exceeds it by more than rescale_tau, so
  *                    weights stay below 2^rescale_tau.  -1 for the default
- *                    (8), or 0 .. 16 (0: rescale whenever the maximum
- *                    grows); d <= 128 only (ATTN_ERR_UNSUPPORTED at d = 256).
+ *                    (12: bf16 weights up to 2^12 with fp32 sums are far
+ *                    from overflow), or 0 .. 16 (0: rescale whenever the
+ *                    maximum grows); d <= 128 only (ATTN_ERR_UNSUPPORTED at
+ *                    d = 256, whose kernel also uses 12).
  *                    Note 0 is a valid threshold, not the default.
  */
 typedef struct {

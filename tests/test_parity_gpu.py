@@ -134,8 +134,8 @@ def test_lazy_rescale_at_known_rows(oracle_mod, d, causal, jump_tile, second):
     """Constructed scores (inputs.make_jump_qkv, checked on the CPU by
     tests/test_rescale_inputs.py): at a known K/V tile the running maximum of
     known rows, in both Q tiles of a work item and mixed inside warps, jumps
-    by 10 (the rescale is taken: O and l scaled by 2^-10), by 7.5 (just under
-    the threshold of 8: weights up to 2^7.5 kept unrescaled) or not at all;
+    by the default threshold + 2 (the rescale is taken), by the threshold
+    - 0.5 (just under it: weights that large kept unrescaled) or not at all;
     with ``second`` a further jump at the next tile rescales again.  Scale
     ln 2 makes the raw scores log2 units.  Every element against the oracle."""
     B, H, N = 1, 2, 640

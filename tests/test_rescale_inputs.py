@@ -4,8 +4,9 @@ The GPU test that uses them (tests/test_parity_gpu.py,
 test_lazy_rescale_at_known_rows) is only as strong as the construction, so
 this file checks, on the exact bf16 values, that:
   * every row's running maximum jumps by exactly the intended amount at the
-    intended K/V tile (more than the threshold of 8, just under it, or not
-    at all), in both 128-row Q tiles of a work item and under the causal mask;
+    intended K/V tile (more than the bf16 kernels' default threshold, just
+    under it, or not at all), in both 128-row Q tiles of a work item and
+    under the causal mask;
   * a lazy-rescale step with a plausible mistake (the rescale factor's sign
     flipped, the rescale of O skipped, or applied to the other Q tile's rows)
     moves the result outside the parity tolerance at those rows, while the
@@ -22,11 +23,12 @@ import math
 import numpy as np
 import pytest
 
-from tiled_attention_forward_sm_b200.inputs import (JUMP_OFFSETS, bf16_bits, jump_offset_of_rows,
-                                                    make_jump_qkv)
+from tiled_attention_forward_sm_b200.inputs import (DEFAULT_RESCALE_TAU, JUMP_OFFSETS, bf16_bits,
+                                                    jump_offset_of_rows, make_jump_qkv)
 
 ATOL_O, RTOL_O = 2e-2, 1e-2
-TAU = 8.0
+TAU = DEFAULT_RESCALE_TAU
+UNDER = JUMP_OFFSETS[1]  # the jump just under the threshold
 SCALE = math.log(2.0)  # scale * log2(e) = 1: raw scores are log2 units
 
 
@@ -95,8 +97,9 @@ def test_jump_rows_take_the_intended_branch(causal, jump_tile, second):
         assert (at[~sees] == -np.inf).all() or not causal
         # both branches occur in both Q tiles of some work item
         taken = sees & (at - before > TAU)
-        under = sees & (c == 7.5)
-        assert (at[under] - before[under] == 7.5).all()
+        under = sees & (c == UNDER)
+        assert UNDER < TAU < JUMP_OFFSETS[0]
+        assert (at[under] - before[under] == UNDER).all()
         pair_rows = [(rows // 128) % 2 == s for s in (0, 1)]
         for s in (0, 1):
             assert (taken & pair_rows[s]).any() and (under & pair_rows[s]).any()
@@ -121,3 +124,15 @@ def test_planted_rescale_mistakes_leave_the_tolerance(oracle_mod, causal, mistak
     bad = _tiled(Q, K, V, causal, mistake)
     out = np.abs(bad - o_ref) > ATOL_O + RTOL_O * np.abs(o_ref)
     assert out.any(), f"planted mistake {mistake} stays inside the tolerance"
+
+
+def test_default_threshold_matches_the_kernel():
+    """The inputs' threshold mirrors the bf16 kernels' default (the constant
+    in the kernel source), so the constructed jumps straddle the threshold
+    the product uses."""
+    import os
+    import re
+    src = open(os.path.join(os.path.dirname(__file__), "..", "tiled_attention_forward_sm_b200",
+                            "csrc", "attn_fwd_kernel.cuh")).read()
+    value = float(re.search(r"constexpr float kRescaleTauBf16 = ([0-9.]+)f;", src).group(1))
+    assert value == DEFAULT_RESCALE_TAU

@@ -320,7 +320,7 @@ int64_t problem_items(const Problem& p, int num_sms) {
 
 template <int D, bool CAUSAL, int kPolyPairs, int STAGES = 0>
 int launch(const Problem& p, cudaStream_t stream, DeviceState& st, int* queue = nullptr,
-           float tau = kRescaleTau) {
+           float tau = kRescaleTauBf16) {
   CUtensorMap tq, tk, tv;
   if (p.cu_q != nullptr) {
     if (make_tmap_tokens(&tq, p.q, p.T_q, p.H, D) || make_tmap_tokens(&tk, p.k, p.T_k, p.H_kv, D) ||
@@ -420,7 +420,7 @@ int launch(const Problem& p, cudaStream_t stream, DeviceState& st, int* queue = 
 struct Tuning {
   int poly_pairs = kDefaultPolyPairs;
   int kv_stages = 0;
-  float rescale_tau = kRescaleTau;
+  float rescale_tau = kRescaleTauBf16;
 };
 
 template <int D, bool CAUSAL>

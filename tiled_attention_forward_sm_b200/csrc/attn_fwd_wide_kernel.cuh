@@ -295,7 +295,7 @@ __device__ void softmax_role(const Shared& sh, const Bars& bb, const KernelArgs&
         // once the previous tile's PV has completed (g - 1 PVs done).
         float alpha = 1.f;
         bool rescale = false;
-        if (tile_max - m > kRescaleTau) {
+        if (tile_max - m > kRescaleTauBf16) {
           alpha = ptx::ex2_approx(m - tile_max);
           m = tile_max;
           rescale = j > 0;

@@ -84,7 +84,7 @@ int launch_pair(const void* q, const void* k, const void* v, void* o, float* lse
     args.win_heads = static_cast<int>(want < 1 ? 1 : (want > BH ? BH : want));
   }
   args.scale_log2 = scale * 1.4426950408889634f;
-  args.rescale_tau = kRescaleTau;
+  args.rescale_tau = kRescaleTauBf16;
   args.status = st.status;
   args.queue = next_queue_slot(st);
   const int64_t grid_clusters = n_items < clusters ? n_items : clusters;

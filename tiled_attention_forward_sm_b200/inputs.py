@@ -184,11 +184,15 @@ def make_workload_inputs(w: Workload):
     return make_qkv(w.B, w.H, w.N, w.d, w.seed, w.q_std)
 
 
+# The bf16 kernels' default lazy-rescale threshold (log2 units), mirrored
+# from the kernel source (a CPU test checks the two agree).
+DEFAULT_RESCALE_TAU = 12.0
+
 # Score offsets of the rows of make_jump_qkv (in units of the raw dot
 # product; with scale = ln 2 these are log2 units): the first jump lifts a
-# row's largest score by 10 (more than a lazy threshold of 8), by 7.5 (just
-# under it), or not at all.
-JUMP_OFFSETS = (10.0, 7.5, 0.0)
+# row's largest score by the default threshold + 2 (the rescale is taken),
+# by the threshold - 0.5 (just under it), or not at all.  All exact in bf16.
+JUMP_OFFSETS = (DEFAULT_RESCALE_TAU + 2.0, DEFAULT_RESCALE_TAU - 0.5, 0.0)
 
 
 def jump_offset_of_rows(N: int):
