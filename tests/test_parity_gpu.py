@@ -64,7 +64,7 @@ def test_ragged_lengths(oracle_mod, d, causal, N):
     full_parity(oracle_mod, 2, 3, N, d, causal, seed=900 + N + d, q_std=2.0)
 
 
-@pytest.mark.parametrize("d", [96, 128, 256])
+@pytest.mark.parametrize("d", [64, 96, 128, 256])
 @pytest.mark.parametrize("causal", [False, True])
 def test_ragged_length_writes_nothing_past_the_rows(causal, d):
     """B*H heads of N = 200 rows, packed back to back inside guard bands: no
@@ -113,6 +113,24 @@ def test_kv_ring_depths_are_bitwise_equal():
     for st in (2, 3, 5):
         o, l = tab.attn_fwd(q, k, v, causal=True, kv_stages=st)
         assert torch.equal(o, o4) and torch.equal(l, l4)
+
+
+@pytest.mark.parametrize("d", [64, 96, 128])
+@pytest.mark.parametrize("N", [1, 33, 161, 1000])
+def test_store_paths_are_bitwise_equal(d, N):
+    """Without the causal mask O leaves through per-warp shared-memory boxes
+    and TMA stores by default, and through per-row stores with the 5-stage
+    ring (no room for the boxes; d = 128) or as fp32: the same values, last
+    tiles whose warps hold no row, some rows or all rows included."""
+    q, k, v = (t.cuda() for t in make_qkv(2, 3, N, d, 62 + N + d))
+    o, lse = tab.attn_fwd(q, k, v, causal=False)
+    assert tab.last_device_error() == 0
+    if d == 128:
+        o5, l5 = tab.attn_fwd(q, k, v, causal=False, kv_stages=5)
+        assert torch.equal(o, o5) and torch.equal(lse, l5)
+    o32, l32 = tab.attn_fwd_chunk(q, k, v, causal=False, out_dtype=torch.float32)
+    assert torch.equal(lse, l32)
+    assert torch.equal(o, o32.to(torch.bfloat16))
 
 
 @pytest.mark.parametrize("name", ["b1h2n256d64", "b4h16n2048d128_causal"])

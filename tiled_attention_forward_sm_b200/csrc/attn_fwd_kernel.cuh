@@ -214,8 +214,10 @@ struct KernelArgs {
                       // one K/V head (n_qpairs = head pairs per K/V head)
 };
 
-// STAGES: K/V ring depth, 0 for the default of the head dim.
-template <int D, int STAGES = 0>
+// STAGES: K/V ring depth, 0 for the default of the head dim.  TMA_O: the
+// epilogue stores O through shared memory and TMA where there is room (the
+// kernel asks for it without the causal mask, see softmax_role).
+template <int D, int STAGES = 0, bool TMA_O = false>
 struct Config {
   static_assert(D == 64 || D == 96 || D == 128, "head dim");
   static_assert(STAGES == 0 || (STAGES >= 2 && STAGES <= 5 && D > 64), "ring depth");
@@ -228,14 +230,23 @@ struct Config {
   static constexpr int kStages = STAGES > 0 ? STAGES : (D > 64 ? kDefaultStagesD128 : 8);
   static constexpr int kQOff = 0;
   static constexpr int kKVOff = 2 * kTileBytes;
-  static constexpr int kBarOff = kKVOff + kStages * kTileBytes;
   // barriers: q_full[2], q_empty[2], kv_full[S], kv_empty[S], s_full[2],
   // p_ready[2 tiles][2 halves], o_final[2], drain, item_full[R], item_empty[R]
   static constexpr int kNumBars = 4 + 2 * kStages + 2 + 4 + 2 + 1 + 2 * kItemSlots;
+  // barriers, misc (tmem base, abort flag), the item ring, alignment slack
+  static constexpr int kTailBytes = kNumBars * 8 + 16 + 4 * kItemWords * kItemSlots + 1024;
+  // O staging for the epilogue's TMA stores: one 64-column box of 32 rows
+  // (4 KB) per softmax warp, 32 KB in all, where it fits beside the K/V ring
+  // (not beside a 5-stage ring at d > 64; the epilogue then stores rows
+  // directly).
+  static constexpr int kOOff = kKVOff + kStages * kTileBytes;
+  static constexpr int kOWarpBytes = kBoxBytes / 4;
+  static constexpr bool kOStage = TMA_O && kOOff + 8 * kOWarpBytes + kTailBytes <= 227 * 1024;
+  static constexpr int kBarOff = kOOff + (kOStage ? 8 * kOWarpBytes : 0);
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;
-  // misc: tmem base, abort flag; then the item ring
   static constexpr int kRingOff = kMiscOff + 16;
   static constexpr int kSmemBytes = kRingOff + 4 * kItemWords * kItemSlots + 1024;  // + alignment slack
+  static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
   static constexpr uint32_t kIdescQK = ptx::idesc_bf16_f32(128, kBlockN, 0, 0);
   static constexpr uint32_t kIdescPV = ptx::idesc_bf16_f32(128, D, 0, 1);
 };
@@ -568,7 +579,7 @@ template <int D, bool CAUSAL, int STAGES = 0>
 __device__ void producer_role(const Shared& sh, const KernelArgs& a, uint8_t* smem,
                               const CUtensorMap* tq, const CUtensorMap* tk,
                               const CUtensorMap* tv) {
-  using C = Config<D, STAGES>;
+  using C = Config<D, STAGES, !CAUSAL>;
   const uint64_t pol_q = ptx::policy_evict_first();
   const uint64_t pol_kv = ptx::policy_evict_last();
   const bool packed = a.cu_q != nullptr;
@@ -662,7 +673,7 @@ __device__ void producer_role(const Shared& sh, const KernelArgs& a, uint8_t* sm
 // shared memory is below 256 KB).
 template <int D, bool CAUSAL, int STAGES = 0>
 __device__ void mma_role(const Shared& sh, const KernelArgs& a, uint8_t* smem, uint32_t tmem) {
-  using C = Config<D, STAGES>;
+  using C = Config<D, STAGES, !CAUSAL>;
   const uint32_t t_s[2] = {tmem + 0, tmem + 128};
   const uint32_t t_o[2] = {tmem + 256, tmem + 384};
   // K-major (Q, K): SBO = 1024 B between 8-row groups; MN-major (V):
@@ -1032,9 +1043,21 @@ __device__ __forceinline__ bool softmax_step(const Shared& sh, const KernelArgs&
 
 // One thread per query row; warp w of the group reads TMEM lanes
 // [32*(w%4), 32*(w%4)+32), so row r = 32*(w%4) + lane is the tile row.
-template <int D, bool CAUSAL, int kPolyPairs>
+//
+// Without the causal mask both Q tiles of an item visit the same K/V tiles,
+// so the two groups reach their epilogues together.  Row-per-thread stores
+// from both (each warp store touching 32 rows) then fill the SM's
+// load/store queue for microseconds, and the MMA warp's next barrier
+// operations wait behind them.  There (bf16 per-head output, no key slices,
+// staging room) the epilogue hands O to TMA stores instead: each warp writes
+// its 32 rows of a 64-column box into its own 128-byte-swizzled staging box,
+// and lane 0 stores the box.  Rows past the end of the sequence fall outside
+// the tensor map and are not written.  Otherwise each thread stores its row.
+template <int D, bool CAUSAL, int kPolyPairs, int STAGES>
 __device__ void softmax_role(const Shared& sh, const KernelArgs& a, uint32_t tmem, int s,
-                             int warp_in_group) {
+                             int warp_in_group, uint8_t* o_stage, const CUtensorMap* tmap_o) {
+  using C = Config<D, STAGES, !CAUSAL>;
+  const bool tma_o = C::kOStage && !a.o_f32 && a.cu_q == nullptr && a.split_rows == 0;
   const int lane = static_cast<int>(ptx::lane_id());
   const int r = warp_in_group * 32 + lane;
   const uint32_t lane_off = static_cast<uint32_t>(warp_in_group * 32) << 16;
@@ -1096,35 +1119,90 @@ __device__ void softmax_role(const Shared& sh, const KernelArgs& a, uint32_t tme
     const bool store = row_ok && in_bounds(sh, a.status,
                                            static_cast<long long>(o_row) < out_rows(a) &&
                                                static_cast<long long>(l_row) < out_rows(a));
+    if (tma_o) {
+      // Box b holds columns [64b, 64b+64) of this warp's 32 rows.  The next
+      // box's TMEM loads are in flight while this one is staged and stored;
+      // the staging box is rewritten only after the previous store has read
+      // it.
+      const uint32_t row_addr = ptx::smem_u32(o_stage) + static_cast<uint32_t>(lane) * 128u;
+      const uint32_t sw = static_cast<uint32_t>(lane & 7);  // 128-byte swizzle
+      uint32_t ov0[32], ov1[32];
+      auto load_box = [&](int b) {
+        if (n_s > 0) {
+          ptx::tmem_ld32(t_o + 64 * b, ov0);
+          ptx::tmem_ld32(t_o + 64 * b + 32, ov1);
+        } else {
+#pragma unroll
+          for (int c = 0; c < 32; ++c) ov0[c] = ov1[c] = 0u;
+        }
+      };
+      auto wait_box = [&]() {
+        if (n_s > 0) {
+          ptx::tmem_ld_wait_tie(ov0);
+          ptx::reg_tie32(ov1);
+        }
+      };
+      load_box(0);
+      wait_box();
 #pragma unroll 1
-    for (int c0 = 0; c0 < D; c0 += 32) {
-      uint32_t ov[32];
-      if (n_s > 0) {
-        ptx::tmem_ld32(t_o + c0, ov);
-        ptx::tmem_ld_wait_tie(ov);
+      for (int b = 0; b < C::kBoxes; ++b) {
+        uint32_t pk[32];
 #pragma unroll
-        for (int c = 0; c < 32; ++c)
-          ov[c] = __float_as_uint(empty ? 0.f : __uint_as_float(ov[c]) * inv_l);
-      } else {
+        for (int c = 0; c < 16; ++c) {
+          pk[c] = ptx::pack_bf16x2(empty ? 0.f : __uint_as_float(ov0[2 * c]) * inv_l,
+                                   empty ? 0.f : __uint_as_float(ov0[2 * c + 1]) * inv_l);
+          pk[16 + c] = ptx::pack_bf16x2(empty ? 0.f : __uint_as_float(ov1[2 * c]) * inv_l,
+                                        empty ? 0.f : __uint_as_float(ov1[2 * c + 1]) * inv_l);
+        }
+        if (b + 1 < C::kBoxes) load_box(b + 1);
+        // (returns at once when no store is outstanding)
+        if (lane == 0) ptx::bulk_wait_read_all();
+        __syncwarp();
 #pragma unroll
-        for (int c = 0; c < 32; ++c) ov[c] = 0u;
+        for (int c = 0; c < 8; ++c)
+          ptx::st_shared_v4(row_addr + ((static_cast<uint32_t>(c) ^ sw) << 4), pk[4 * c],
+                            pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+        ptx::fence_proxy_async_smem();
+        __syncwarp();
+        const int row0 = qt * kBlockM + 32 * warp_in_group;
+        if (lane == 0 && row0 < it.q_len) {
+          ptx::tma_store_3d(tmap_o, o_stage, 64 * b, row0, qz);
+          ptx::bulk_commit_group();
+        }
+        if (b + 1 < C::kBoxes) wait_box();
       }
-      if (!store) continue;
-      if (a.o_f32) {
-        uint4* dst = reinterpret_cast<uint4*>(static_cast<float*>(a.o) + o_row * D + c0);
+    } else {
+#pragma unroll 1
+      for (int c0 = 0; c0 < D; c0 += 32) {
+        uint32_t ov[32];
+        if (n_s > 0) {
+          ptx::tmem_ld32(t_o + c0, ov);
+          ptx::tmem_ld_wait_tie(ov);
 #pragma unroll
-        for (int v = 0; v < 8; ++v)
-          dst[v] = make_uint4(ov[4 * v], ov[4 * v + 1], ov[4 * v + 2], ov[4 * v + 3]);
-      } else {
-        uint32_t pk[16];
+          for (int c = 0; c < 32; ++c)
+            ov[c] = __float_as_uint(empty ? 0.f : __uint_as_float(ov[c]) * inv_l);
+        } else {
 #pragma unroll
-        for (int c = 0; c < 16; ++c)
-          pk[c] = ptx::pack_bf16x2(__uint_as_float(ov[2 * c]), __uint_as_float(ov[2 * c + 1]));
-        uint4* dst =
-            reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.o) + o_row * D + c0);
+          for (int c = 0; c < 32; ++c) ov[c] = 0u;
+        }
+        if (!store) continue;
+        if (a.o_f32) {
+          uint4* dst = reinterpret_cast<uint4*>(static_cast<float*>(a.o) + o_row * D + c0);
 #pragma unroll
-        for (int v = 0; v < 4; ++v)
-          dst[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+          for (int v = 0; v < 8; ++v)
+            dst[v] = make_uint4(ov[4 * v], ov[4 * v + 1], ov[4 * v + 2], ov[4 * v + 3]);
+        } else {
+          uint32_t pk[16];
+#pragma unroll
+          for (int c = 0; c < 16; ++c)
+            pk[c] =
+                ptx::pack_bf16x2(__uint_as_float(ov[2 * c]), __uint_as_float(ov[2 * c + 1]));
+          uint4* dst =
+              reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.o) + o_row * D + c0);
+#pragma unroll
+          for (int v = 0; v < 4; ++v)
+            dst[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+        }
       }
     }
     if (store) a.lse[l_row] = empty ? -INFINITY : (m + log2f(l)) * 0.69314718055994531f;
@@ -1136,8 +1214,9 @@ template <int D, bool CAUSAL, int kPolyPairs, int STAGES = 0>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap_q,
                     const __grid_constant__ CUtensorMap tmap_k,
-                    const __grid_constant__ CUtensorMap tmap_v, const KernelArgs args) {
-  using C = Config<D, STAGES>;
+                    const __grid_constant__ CUtensorMap tmap_v,
+                    const __grid_constant__ CUtensorMap tmap_o, const KernelArgs args) {
+  using C = Config<D, STAGES, !CAUSAL>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -1200,7 +1279,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   // its share before the CTA-wide barrier above.
   if (warp < 8) {
     ptx::setmaxnreg_inc<kRegsSoftmax>();
-    softmax_role<D, CAUSAL, kPolyPairs>(sh, args, tmem, warp / 4, warp % 4);
+    softmax_role<D, CAUSAL, kPolyPairs, STAGES>(
+        sh, args, tmem, warp / 4, warp % 4,
+        C::kOStage ? smem + C::kOOff + warp * C::kOWarpBytes : nullptr,
+        C::kOStage ? &tmap_o : nullptr);
+    // the staging boxes are read before the CTA exits
+    if constexpr (C::kOStage) ptx::bulk_wait_read_all();
   } else if (warp == 8) {
     if (ptx::lane_id() == 0)
       producer_role<D, CAUSAL, STAGES>(sh, args, smem, &tmap_q, &tmap_k, &tmap_v);
