@@ -67,7 +67,11 @@ constexpr int kTileBytes = kBlockM * kD;  // 16 KB: 128 rows of 128 E4M3 values
 constexpr int kStages = 8;                // K / V^T ring depth
 constexpr int kQOff = 0;
 constexpr int kKVOff = 2 * kTileBytes;
-constexpr int kBarOff = kKVOff + kStages * kTileBytes;
+// O staging for the epilogue's TMA stores without the causal mask: one
+// 64-column bf16 box of 32 rows (4 KB) per softmax warp.
+constexpr int kOOff = kKVOff + kStages * kTileBytes;
+constexpr int kOWarpBytes = 4096;
+constexpr int kBarOff = kOOff + 8 * kOWarpBytes;
 // barriers: q_full[2], q_empty[2], kv_full[S], kv_empty[S], s_full[2],
 // p_ready[2 tiles][2 halves], o_final[2], drain, item_full[R], item_empty[R]
 constexpr int kNumBars = 4 + 2 * kStages + 2 + 4 + 2 + 1 + 2 * kItemSlots;
@@ -254,9 +258,13 @@ done:
   wait_warp(sh, a.status, sh.drain, 0, true);
 }
 
+// The epilogue follows the bf16 kernel's: without the causal mask the two
+// groups finish an item together, so O leaves through this warp's staging
+// box and a TMA store per 64 columns instead of row-per-thread stores.
 template <bool CAUSAL>
 __device__ void softmax_role(const Shared& sh, const Bars& bb, const KernelArgs& a,
-                             float v_descale, uint32_t tmem, int s, int warp_in_group) {
+                             float v_descale, uint32_t tmem, int s, int warp_in_group,
+                             uint8_t* o_stage, const CUtensorMap* tmap_o) {
   const int lane = static_cast<int>(ptx::lane_id());
   const int r = warp_in_group * 32 + lane;
   const uint32_t lane_off = static_cast<uint32_t>(warp_in_group * 32) << 16;
@@ -385,6 +393,57 @@ __device__ void softmax_role(const Shared& sh, const Bars& bb, const KernelArgs&
     const float f = empty ? 0.f : v_descale / l;
     const size_t o_row = static_cast<size_t>(it.qz) * a.N_q + row;
     __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(a.o) + o_row * kD;
+    if constexpr (!CAUSAL) {
+      const uint32_t row_addr = ptx::smem_u32(o_stage) + static_cast<uint32_t>(lane) * 128u;
+      const uint32_t sw = static_cast<uint32_t>(lane & 7);  // 128-byte swizzle
+      uint32_t ov0[32], ov1[32];
+      auto load_box = [&](int b) {
+        if (n_s > 0) {
+          ptx::tmem_ld32(t_o + 64 * b, ov0);
+          ptx::tmem_ld32(t_o + 64 * b + 32, ov1);
+        } else {
+#pragma unroll
+          for (int c = 0; c < 32; ++c) ov0[c] = ov1[c] = 0u;
+        }
+      };
+      auto wait_box = [&]() {
+        if (n_s > 0) {
+          ptx::tmem_ld_wait_tie(ov0);
+          ptx::reg_tie32(ov1);
+        }
+      };
+      load_box(0);
+      wait_box();
+#pragma unroll 1
+      for (int b = 0; b < kD / 64; ++b) {
+        uint32_t pk[32];
+#pragma unroll
+        for (int c = 0; c < 16; ++c) {
+          pk[c] = ptx::pack_bf16x2(__uint_as_float(ov0[2 * c]) * f,
+                                   __uint_as_float(ov0[2 * c + 1]) * f);
+          pk[16 + c] = ptx::pack_bf16x2(__uint_as_float(ov1[2 * c]) * f,
+                                        __uint_as_float(ov1[2 * c + 1]) * f);
+        }
+        if (b + 1 < kD / 64) load_box(b + 1);
+        // the box is rewritten once the previous store has read it
+        if (lane == 0) ptx::bulk_wait_read_all();
+        __syncwarp();
+#pragma unroll
+        for (int c = 0; c < 8; ++c)
+          ptx::st_shared_v4(row_addr + ((static_cast<uint32_t>(c) ^ sw) << 4), pk[4 * c],
+                            pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+        ptx::fence_proxy_async_smem();
+        __syncwarp();
+        const int row0 = qt * kBlockM + 32 * warp_in_group;
+        if (lane == 0 && row0 < it.q_len) {
+          ptx::tma_store_3d(tmap_o, o_stage, 64 * b, row0, it.qz);
+          ptx::bulk_commit_group();
+        }
+        if (b + 1 < kD / 64) wait_box();
+      }
+      if (row_ok) a.lse[o_row] = empty ? -INFINITY : (m + log2f(l)) * 0.69314718055994531f;
+      continue;
+    }
 #pragma unroll 1
     for (int c0 = 0; c0 < kD; c0 += 32) {
       uint32_t ov[32];
@@ -413,7 +472,8 @@ template <bool CAUSAL>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_fwd_fp8_kernel(const __grid_constant__ CUtensorMap tmap_q,
                         const __grid_constant__ CUtensorMap tmap_k,
-                        const __grid_constant__ CUtensorMap tmap_vt, const KernelArgs args,
+                        const __grid_constant__ CUtensorMap tmap_vt,
+                        const __grid_constant__ CUtensorMap tmap_o, const KernelArgs args,
                         float v_descale) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -474,7 +534,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp < 8) {
     ptx::setmaxnreg_inc<kRegsSoftmax>();
-    softmax_role<CAUSAL>(sh, bb, args, v_descale, tmem, warp / 4, warp % 4);
+    softmax_role<CAUSAL>(sh, bb, args, v_descale, tmem, warp / 4, warp % 4,
+                         smem + kOOff + warp * kOWarpBytes, &tmap_o);
+    // the staging boxes are read before the CTA exits
+    if constexpr (!CAUSAL) ptx::bulk_wait_read_all();
   } else if (warp == 8) {
     if (ptx::lane_id() == 0) producer_role<CAUSAL>(sh, bb, args, smem, &tmap_q, &tmap_k, &tmap_vt);
     __syncwarp();

@@ -83,9 +83,13 @@ extern "C" int attn_fwd_fp8(const void* q, const void* k, const void* vt, void* 
     if (rc != ATTN_OK) return rc;
   }
   const uint64_t BH = static_cast<uint64_t>(B) * H;
-  CUtensorMap tq, tk, tvt;
+  CUtensorMap tq, tk, tvt, to;
   if (make_tmap_u8(&tq, q, d, N, BH) || make_tmap_u8(&tk, k, d, N, BH) ||
       make_tmap_u8(&tvt, vt, N, d, BH))
+    return ATTN_ERR_CUDA;
+  // O (bf16), boxes of 32 rows: the epilogue's TMA stores without the mask
+  to = tq;
+  if (!causal && make_tmap_heads_rows(&to, o, static_cast<int>(BH), N, d, 32))
     return ATTN_ERR_CUDA;
   const int64_t n_qpairs = ((static_cast<int64_t>(N) + kBlockM - 1) / kBlockM + 1) / 2;
   const int64_t n_items = static_cast<int64_t>(BH) * n_qpairs;
@@ -123,7 +127,7 @@ extern "C" int attn_fwd_fp8(const void* q, const void* k, const void* vt, void* 
   cfg.blockDim = dim3(kThreads, 1, 1);
   cfg.dynamicSmemBytes = fp8::kSmemBytes;
   cfg.stream = static_cast<cudaStream_t>(stream);
-  if (cudaLaunchKernelEx(&cfg, kern, tq, tk, tvt, args, v_descale) != cudaSuccess) {
+  if (cudaLaunchKernelEx(&cfg, kern, tq, tk, tvt, to, args, v_descale) != cudaSuccess) {
     cudaGetLastError();
     return ATTN_ERR_CUDA;
   }
