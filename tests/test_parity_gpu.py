@@ -133,6 +133,20 @@ def test_store_paths_are_bitwise_equal(d, N):
     assert torch.equal(o, o32.to(torch.bfloat16))
 
 
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("N", [1, 33, 161, 1000])
+def test_wide_store_paths_are_bitwise_equal(causal, N):
+    """d = 256: bf16 O always leaves through two staging boxes per warp and
+    TMA stores (a box rewritten once the store two boxes back has read it);
+    fp32 O through per-row stores.  Same values."""
+    q, k, v = (t.cuda() for t in make_qkv(2, 3, N, 256, 63 + N))
+    o, lse = tab.attn_fwd(q, k, v, causal=causal)
+    assert tab.last_device_error() == 0
+    o32, l32 = tab.attn_fwd_chunk(q, k, v, causal=causal, out_dtype=torch.float32)
+    assert torch.equal(lse, l32)
+    assert torch.equal(o, o32.to(torch.bfloat16))
+
+
 @pytest.mark.parametrize("name", ["b1h2n256d64", "b4h16n2048d128_causal"])
 def test_workload_full(oracle_mod, name):
     w = WORKLOADS[name]

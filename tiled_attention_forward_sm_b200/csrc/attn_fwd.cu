@@ -333,11 +333,11 @@ int launch(const Problem& p, cudaStream_t stream, DeviceState& st, int* queue = 
       return ATTN_ERR_CUDA;
   }
   // O's map (boxes of 32 rows, one softmax warp's share of a tile) for the
-  // epilogue's TMA stores of bf16 per-head output without key slices and
-  // without the causal mask; in every other case the kernel stores rows
-  // itself and never reads it.
+  // epilogue's TMA stores of bf16 per-head output without key slices: in
+  // the wide kernel always, in the two-tile kernel without the causal mask.
+  // In every other case the kernel stores rows itself and never reads it.
   to = tq;
-  if constexpr (D != wide::kD && !CAUSAL) {
+  if constexpr (D == wide::kD || !CAUSAL) {
     if (p.cu_q == nullptr && !p.o_f32 && p.split_rows == 0 &&
         make_tmap_heads_rows(&to, p.o, p.B * p.H, p.N_q, D, 32))
       return ATTN_ERR_CUDA;
@@ -383,16 +383,15 @@ int launch(const Problem& p, cudaStream_t stream, DeviceState& st, int* queue = 
   args.status = st.status;
 
   // d = 256 runs the wide kernel (one Q tile at a time, 256-column O).
-  // The wide kernel takes Q, K, V maps; the two-tile kernel also O's.
-  void (*kern3)(CUtensorMap, CUtensorMap, CUtensorMap, KernelArgs) = nullptr;
-  void (*kern4)(CUtensorMap, CUtensorMap, CUtensorMap, CUtensorMap, KernelArgs) = nullptr;
+  // Both kernels take the maps of Q, K, V and O.
+  void (*kern)(CUtensorMap, CUtensorMap, CUtensorMap, CUtensorMap, KernelArgs);
   int threads, smem_bytes;
   if constexpr (D == wide::kD) {
-    kern3 = wide::attn_fwd_wide_kernel<CAUSAL, kPolyPairs>;
+    kern = wide::attn_fwd_wide_kernel<CAUSAL, kPolyPairs>;
     threads = wide::kThreads;
     smem_bytes = wide::kSmemBytes;
   } else {
-    kern4 = attn_fwd_kernel<D, CAUSAL, kPolyPairs, STAGES>;
+    kern = attn_fwd_kernel<D, CAUSAL, kPolyPairs, STAGES>;
     threads = kThreads;
     smem_bytes = Config<D, STAGES, !CAUSAL>::kSmemBytes;
     // The kernel's register split (setmaxnreg) hands the softmax warpgroups
@@ -400,7 +399,7 @@ int launch(const Problem& p, cudaStream_t stream, DeviceState& st, int* queue = 
     // the kernel was built with the full per-thread budget it assumes.
     static const bool regs_ok = [&] {
       cudaFuncAttributes fa;
-      if (cudaFuncGetAttributes(&fa, kern4) != cudaSuccess) {
+      if (cudaFuncGetAttributes(&fa, kern) != cudaSuccess) {
         cudaGetLastError();
         return false;
       }
@@ -409,9 +408,8 @@ int launch(const Problem& p, cudaStream_t stream, DeviceState& st, int* queue = 
     if (!regs_ok) return ATTN_ERR_CUDA;
   }
   static std::atomic<unsigned long long> smem_set{0};
-  const void* fn = kern4 != nullptr ? reinterpret_cast<const void*>(kern4)
-                                     : reinterpret_cast<const void*>(kern3);
-  if (set_smem_once(fn, smem_bytes, st, smem_set) != ATTN_OK) return ATTN_ERR_CUDA;
+  if (set_smem_once(reinterpret_cast<const void*>(kern), smem_bytes, st, smem_set) != ATTN_OK)
+    return ATTN_ERR_CUDA;
   cudaLaunchConfig_t cfg;
   std::memset(&cfg, 0, sizeof cfg);
   // Persistent: one CTA per SM (at most one per work item).
@@ -420,9 +418,7 @@ int launch(const Problem& p, cudaStream_t stream, DeviceState& st, int* queue = 
   cfg.blockDim = dim3(static_cast<unsigned>(threads), 1, 1);
   cfg.dynamicSmemBytes = static_cast<size_t>(smem_bytes);
   cfg.stream = stream;
-  const cudaError_t e = kern4 != nullptr ? cudaLaunchKernelEx(&cfg, kern4, tq, tk, tv, to, args)
-                                          : cudaLaunchKernelEx(&cfg, kern3, tq, tk, tv, args);
-  if (e != cudaSuccess) {
+  if (cudaLaunchKernelEx(&cfg, kern, tq, tk, tv, to, args) != cudaSuccess) {
     cudaGetLastError();
     return ATTN_ERR_CUDA;
   }

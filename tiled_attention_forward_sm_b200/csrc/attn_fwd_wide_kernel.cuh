@@ -36,7 +36,15 @@ constexpr int kTileBytes = kBoxes * kBoxBytes;     // 64 KB: one 128 x 256 bf16 
 constexpr int kStages = 2;                         // K/V ring depth
 constexpr int kQOff = 0;                           // one Q buffer
 constexpr int kKVOff = kTileBytes;
-constexpr int kBarOff = kKVOff + kStages * kTileBytes;
+// O staging for the epilogue's TMA stores (bf16 per-head output without key
+// slices): two 64-column boxes of 32 rows (2 x 4 KB) per softmax warp.  A
+// warp store of row-per-thread output touches 32 rows, so one 256-column
+// tile took 4 x 32 such instructions of 32 lines each through the load/store
+// unit; through shared memory and TMA the same tile costs 8-row conflict-free
+// 16-byte stores and 16 bulk stores.
+constexpr int kOOff = kKVOff + kStages * kTileBytes;
+constexpr int kOWarpBytes = 8192;
+constexpr int kBarOff = kOOff + 4 * kOWarpBytes;
 // barriers: q_full, q_empty, kv_full[S], kv_empty[S], s_full[2],
 // p_ready[2 buffers][2 halves], pv_done, o_ready, drain, item_full[R],
 // item_empty[R]
@@ -230,7 +238,9 @@ done:
 // ---------------------------------------------------------------- softmax
 template <bool CAUSAL, int kPolyPairs>
 __device__ void softmax_role(const Shared& sh, const Bars& bb, const KernelArgs& a,
-                             uint32_t tmem, int warp) {
+                             uint32_t tmem, int warp, uint8_t* o_stage,
+                             const CUtensorMap* tmap_o) {
+  const bool tma_o = !a.o_f32 && a.cu_q == nullptr && a.split_rows == 0;
   const int lane = static_cast<int>(ptx::lane_id());
   const int r = warp * 32 + lane;
   const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
@@ -376,6 +386,60 @@ __device__ void softmax_role(const Shared& sh, const Bars& bb, const KernelArgs&
       const bool store = row_ok && in_bounds(sh, a.status,
                                              static_cast<long long>(o_row) < out_rows(a) &&
                                                  static_cast<long long>(l_row) < out_rows(a));
+      if (tma_o) {
+        // Box b (columns [64b, 64b+64)) of this warp's 32 rows goes through
+        // staging box b % 2 and one TMA store; a staging box is rewritten
+        // once the store two boxes back has read it.
+        uint32_t ov0[32], ov1[32];
+        auto load_box = [&](int b) {
+          if (n > 0) {
+            ptx::tmem_ld32(t_o + 64 * b, ov0);
+            ptx::tmem_ld32(t_o + 64 * b + 32, ov1);
+          } else {
+#pragma unroll
+            for (int c = 0; c < 32; ++c) ov0[c] = ov1[c] = 0u;
+          }
+        };
+        auto wait_box = [&]() {
+          if (n > 0) {
+            ptx::tmem_ld_wait_tie(ov0);
+            ptx::reg_tie32(ov1);
+          }
+        };
+        const uint32_t sw = static_cast<uint32_t>(lane & 7);
+        const int row0 = qt * kBlockM + 32 * warp;
+        load_box(0);
+        wait_box();
+#pragma unroll 1
+        for (int b = 0; b < kBoxes; ++b) {
+          uint32_t pk[32];
+#pragma unroll
+          for (int c = 0; c < 16; ++c) {
+            pk[c] = ptx::pack_bf16x2(empty ? 0.f : __uint_as_float(ov0[2 * c]) * inv_l,
+                                     empty ? 0.f : __uint_as_float(ov0[2 * c + 1]) * inv_l);
+            pk[16 + c] = ptx::pack_bf16x2(empty ? 0.f : __uint_as_float(ov1[2 * c]) * inv_l,
+                                          empty ? 0.f : __uint_as_float(ov1[2 * c + 1]) * inv_l);
+          }
+          if (b + 1 < kBoxes) load_box(b + 1);
+          if (lane == 0) ptx::bulk_wait_read_but_one();
+          __syncwarp();
+          uint8_t* box = o_stage + (b & 1) * 4096;
+          const uint32_t row_addr = ptx::smem_u32(box) + static_cast<uint32_t>(lane) * 128u;
+#pragma unroll
+          for (int c = 0; c < 8; ++c)
+            ptx::st_shared_v4(row_addr + ((static_cast<uint32_t>(c) ^ sw) << 4), pk[4 * c],
+                              pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+          ptx::fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0 && row0 < it.q_len) {
+            ptx::tma_store_3d(tmap_o, box, 64 * b, row0, it.qz);
+            ptx::bulk_commit_group();
+          }
+          if (b + 1 < kBoxes) wait_box();
+        }
+        if (store) a.lse[l_row] = empty ? -INFINITY : (m + log2f(l)) * 0.69314718055994531f;
+        continue;
+      }
 #pragma unroll 1
       for (int c0 = 0; c0 < kD; c0 += 32) {
         uint32_t ov[32];
@@ -417,7 +481,8 @@ template <bool CAUSAL, int kPolyPairs>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_fwd_wide_kernel(const __grid_constant__ CUtensorMap tmap_q,
                          const __grid_constant__ CUtensorMap tmap_k,
-                         const __grid_constant__ CUtensorMap tmap_v, const KernelArgs args) {
+                         const __grid_constant__ CUtensorMap tmap_v,
+                         const __grid_constant__ CUtensorMap tmap_o, const KernelArgs args) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -474,7 +539,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem = *sh.tmem_base;
 
   if (warp < 4) {
-    softmax_role<CAUSAL, kPolyPairs>(sh, bb, args, tmem, warp);
+    softmax_role<CAUSAL, kPolyPairs>(sh, bb, args, tmem, warp, smem + kOOff + warp * kOWarpBytes,
+                                     &tmap_o);
+    // the staging boxes are read before the CTA exits
+    ptx::bulk_wait_read_all();
   } else if (warp == 4) {
     if (ptx::lane_id() == 0) producer_role<CAUSAL>(sh, bb, args, smem, &tmap_q, &tmap_k, &tmap_v);
     __syncwarp();
