@@ -78,9 +78,14 @@ extern "C" int attn_fwd_fp4(const void* q, const void* q_sf, const void* k, cons
     rc = check_on_device(*st, ptrs, 8);
     if (rc != ATTN_OK) return rc;
   }
-  CUtensorMap tq, tk, tvt;
+  CUtensorMap tq, tk, tvt, to;
   if (make_tmap_e2m1(&tq, q, fp4::kD / 2, N, BH) || make_tmap_e2m1(&tk, k, fp4::kD / 2, N, BH) ||
       make_tmap_e2m1(&tvt, vt, N / 2, fp4::kD, BH))
+    return ATTN_ERR_CUDA;
+  // O (bf16), boxes of 32 rows x 64 columns: the epilogue's TMA stores
+  // without the causal mask (otherwise unused)
+  to = tq;
+  if (!causal && make_tmap_heads_rows(&to, o, static_cast<int>(BH), N, fp4::kD, 32))
     return ATTN_ERR_CUDA;
   const int64_t n_qpairs = ((static_cast<int64_t>(N) + kBlockM - 1) / kBlockM + 1) / 2;
   const int64_t n_items = static_cast<int64_t>(BH) * n_qpairs;
@@ -124,7 +129,7 @@ extern "C" int attn_fwd_fp4(const void* q, const void* q_sf, const void* k, cons
   cfg.blockDim = dim3(fp4::kThreads, 1, 1);
   cfg.dynamicSmemBytes = fp4::kSmemBytes;
   cfg.stream = static_cast<cudaStream_t>(stream);
-  if (cudaLaunchKernelEx(&cfg, kern, tq, tk, tvt, args, fa) != cudaSuccess) {
+  if (cudaLaunchKernelEx(&cfg, kern, tq, tk, tvt, to, args, fa) != cudaSuccess) {
     cudaGetLastError();
     return ATTN_ERR_CUDA;
   }
