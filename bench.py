@@ -941,6 +941,60 @@ def run_reference(args, w):
     }
 
 
+def run_copy_rates(args, w):
+    """Plain pinned-memory copy rates for the bytes the e2e leg moves per step
+    (Q, K, V in; O and LSE out): the floor under the e2e figure on this machine.
+    Host-to-device and device-to-host alone, then both at once on two
+    streams; CUDA events on the current stream, after warm-up."""
+    world, rank, local = dist_env()
+    if world > 1:
+        raise SystemExit("--copy-rates runs on one GPU")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    n_in = 3 * w.rows * w.d * 2
+    n_out = w.rows * w.d * 2 + w.rows * 4
+    h_in = torch.empty(n_in, dtype=torch.uint8, pin_memory=True)
+    d_in = torch.empty(n_in, dtype=torch.uint8, device=dev)
+    h_out = torch.empty(n_out, dtype=torch.uint8, pin_memory=True)
+    d_out = torch.empty(n_out, dtype=torch.uint8, device=dev)
+    s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    cur = torch.cuda.current_stream(dev)
+
+    def both():
+        ev = torch.cuda.Event()
+        ev.record(cur)
+        s_in.wait_event(ev)
+        s_out.wait_event(ev)
+        with torch.cuda.stream(s_in):
+            d_in.copy_(h_in, non_blocking=True)
+        with torch.cuda.stream(s_out):
+            h_out.copy_(d_out, non_blocking=True)
+        cur.wait_stream(s_in)
+        cur.wait_stream(s_out)
+
+    def ms(fn):
+        for _ in range(args.warmup):
+            fn()
+        torch.cuda.synchronize(dev)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(cur)
+        for _ in range(args.steps):
+            fn()
+        e1.record(cur)
+        torch.cuda.synchronize(dev)
+        return e0.elapsed_time(e1) / args.steps
+
+    t_in = ms(lambda: d_in.copy_(h_in, non_blocking=True))
+    t_out = ms(lambda: h_out.copy_(d_out, non_blocking=True))
+    t_both = ms(both)
+    return {"copy_rates": {"workload": w.name, "h2d_bytes": n_in, "d2h_bytes": n_out,
+                           "h2d_ms": round(t_in, 4), "h2d_GBps": round(n_in / t_in / 1e6, 1),
+                           "d2h_ms": round(t_out, 4), "d2h_GBps": round(n_out / t_out / 1e6, 1),
+                           "both_ms": round(t_both, 4),
+                           "metric_at_both_ms": round(w.flops / t_both / 1e9, 2),
+                           "unit": "TFLOPS", "steps": args.steps, "warmup": args.warmup}}
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -966,6 +1020,9 @@ def main():
                     help="attn_fwd_ex option: K/V ring depth (2..5 at d = 128)")
     ap.add_argument("--rescale-tau", type=float, default=None,
                     help="attn_fwd_ex option: lazy-rescale threshold (0..16, log2 units)")
+    ap.add_argument("--copy-rates", action="store_true",
+                    help="print the pinned host<->device copy rates for the workload's e2e bytes "
+                         "instead of timing the attention")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -973,7 +1030,9 @@ def main():
     if args.gpus != world:
         ap.error(f"--gpus {args.gpus} but WORLD_SIZE is {world}: launch N > 1 ranks with "
                  f"python -m torch.distributed.run --nproc-per-node N bench.py --gpus N")
-    if args.workload.endswith(FP4_SUFFIX):
+    if args.copy_rates:
+        line = run_copy_rates(args, WORKLOADS[args.workload])
+    elif args.workload.endswith(FP4_SUFFIX):
         if args.impl == "reference":
             ap.error("--impl reference times the bf16 workloads only")
         line = run_fp4(args, WORKLOADS[args.workload[: -len(FP4_SUFFIX)]])

@@ -409,10 +409,11 @@ int attn_fwd_host(const void* q_h, const void* k_h, const void* v_h, void* o_h, 
                   attn_stream_t stream);
 
 /*
- * attn_last_device_error -- synchronises `stream`, then reads and clears the
- * device status word written by kernels on the current device (ATTN_OK if no
- * kernel reported an error).  Returns ATTN_ERR_CUDA if synchronisation or
- * the read fails.
+ * attn_last_device_error -- reads and clears the device status word written
+ * by kernels on the current device, behind the work already enqueued on
+ * `stream`, and synchronises `stream` once (ATTN_OK if no kernel reported an
+ * error).  Work on other streams is not waited for: join it into `stream`
+ * first.  Returns ATTN_ERR_CUDA if the read or the synchronisation fails.
  */
 int attn_last_device_error(attn_stream_t stream);
 

@@ -756,14 +756,14 @@ extern "C" int attn_last_device_error(attn_stream_t stream) {
   DeviceState* st = nullptr;
   int rc = device_state(&st);
   if (rc != ATTN_OK) return rc;
-  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) {
-    cudaGetLastError();
-    return ATTN_ERR_CUDA;
-  }
+  // Read and clear on `stream`, behind everything already queued there, and
+  // synchronise once (two synchronous symbol copies on the legacy stream
+  // would each wait for the whole device).
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
   int val = 0;
-  const int zero = 0;
-  if (cudaMemcpyFromSymbol(&val, g_attn_status, sizeof(int)) != cudaSuccess ||
-      cudaMemcpyToSymbol(g_attn_status, &zero, sizeof(int)) != cudaSuccess) {
+  if (cudaMemcpyAsync(&val, st->status, sizeof(int), cudaMemcpyDeviceToHost, s) != cudaSuccess ||
+      cudaMemsetAsync(st->status, 0, sizeof(int), s) != cudaSuccess ||
+      cudaStreamSynchronize(s) != cudaSuccess) {
     cudaGetLastError();
     return ATTN_ERR_CUDA;
   }

@@ -441,28 +441,28 @@ __device__ void softmax_role(const Shared& sh, const Bars& bb, const KernelArgs&
         }
         if (b + 1 < kD / 64) wait_box();
       }
-      if (row_ok) a.lse[o_row] = empty ? -INFINITY : (m + log2f(l)) * 0.69314718055994531f;
-      continue;
-    }
+    } else {
 #pragma unroll 1
-    for (int c0 = 0; c0 < kD; c0 += 32) {
-      uint32_t ov[32];
-      if (n_s > 0) {
-        ptx::tmem_ld32(t_o + c0, ov);
-        ptx::tmem_ld_wait_tie(ov);
-      } else {
+      for (int c0 = 0; c0 < kD; c0 += 32) {
+        uint32_t ov[32];
+        if (n_s > 0) {
+          ptx::tmem_ld32(t_o + c0, ov);
+          ptx::tmem_ld_wait_tie(ov);
+        } else {
 #pragma unroll
-        for (int c = 0; c < 32; ++c) ov[c] = 0u;
+          for (int c = 0; c < 32; ++c) ov[c] = 0u;
+        }
+        if (!row_ok) continue;
+        uint32_t pk[16];
+#pragma unroll
+        for (int c = 0; c < 16; ++c)
+          pk[c] = ptx::pack_bf16x2(__uint_as_float(ov[2 * c]) * f,
+                                   __uint_as_float(ov[2 * c + 1]) * f);
+        uint4* dst = reinterpret_cast<uint4*>(orow + c0);
+#pragma unroll
+        for (int v = 0; v < 4; ++v)
+          dst[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
       }
-      if (!row_ok) continue;
-      uint32_t pk[16];
-#pragma unroll
-      for (int c = 0; c < 16; ++c)
-        pk[c] = ptx::pack_bf16x2(__uint_as_float(ov[2 * c]) * f, __uint_as_float(ov[2 * c + 1]) * f);
-      uint4* dst = reinterpret_cast<uint4*>(orow + c0);
-#pragma unroll
-      for (int v = 0; v < 4; ++v)
-        dst[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
     }
     if (row_ok) a.lse[o_row] = empty ? -INFINITY : (m + log2f(l)) * 0.69314718055994531f;
   }

@@ -90,6 +90,26 @@ extern "C" int attn_fwd_host(const void* q_h, const void* k_h, const void* v_h, 
   const size_t total = static_cast<size_t>(BH) * head_bytes * 3;
   int n_chunks = total >= (64ull << 20) ? kHostChunksMax : 1;
   if (n_chunks > BH) n_chunks = BH;
+  if (n_chunks == 1) {
+    // One group: copies in, the kernel and copies out in order on the
+    // caller's stream, with no cross-stream events.
+    const size_t bytes = static_cast<size_t>(BH) * head_bytes;
+    const size_t rows = static_cast<size_t>(BH) * head_rows;
+    if (cudaMemcpyAsync(q_d, q_h, bytes, cudaMemcpyHostToDevice, s) != cudaSuccess ||
+        cudaMemcpyAsync(k_d, k_h, bytes, cudaMemcpyHostToDevice, s) != cudaSuccess ||
+        cudaMemcpyAsync(v_d, v_h, bytes, cudaMemcpyHostToDevice, s) != cudaSuccess) {
+      cudaGetLastError();
+      return ATTN_ERR_CUDA;
+    }
+    rc = attn_fwd(q_d, k_d, v_d, o_d, lse_d, B, H, N, d, causal, scale, stream);
+    if (rc != ATTN_OK) return rc;
+    if (cudaMemcpyAsync(o_h, o_d, bytes, cudaMemcpyDeviceToHost, s) != cudaSuccess ||
+        cudaMemcpyAsync(lse_h, lse_d, rows * 4, cudaMemcpyDeviceToHost, s) != cudaSuccess) {
+      cudaGetLastError();
+      return ATTN_ERR_CUDA;
+    }
+    return attn_last_device_error(stream);
+  }
   const uint8_t* qh = static_cast<const uint8_t*>(q_h);
   const uint8_t* kh = static_cast<const uint8_t*>(k_h);
   const uint8_t* vh = static_cast<const uint8_t*>(v_h);
