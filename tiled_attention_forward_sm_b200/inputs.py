@@ -108,6 +108,12 @@ GENERAL_WORKLOADS = {
         # 16 sequences of 512..8192 tokens (seeded), packed without padding
         GeneralWorkload("varlen_b16h16_d128_causal", "varlen", 16, 16, 16, max(_LENS),
                         max(_LENS), 128, True, 2103, lens_q=_LENS, lens_k=_LENS),
+        # head dim 256 at the bench workload's shape (the d = 256 kernel), with
+        # and without the mask
+        GeneralWorkload("square_b2h32n8192d256_causal", "chunk", 2, 32, 32, 8192, 8192, 256,
+                        True, 2104),
+        GeneralWorkload("square_b2h32n8192d256", "chunk", 2, 32, 32, 8192, 8192, 256, False,
+                        2105),
     ]
 }
 
