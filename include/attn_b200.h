@@ -76,7 +76,12 @@ typedef void* attn_stream_t;
  * after the stream reaches that point.  Errors: argument and precondition
  * failures return a negative status before anything is enqueued; a failed
  * launch returns ATTN_ERR_CUDA.  A device-side timeout is reported later by
- * attn_last_device_error().
+ * attn_last_device_error().  Stream capture: once a first call with the same
+ * head dim, mask and options has run on the device (it sets up the device
+ * state and the kernel's shared-memory attribute), the call can be captured
+ * into a CUDA graph.  The captured launch keeps the work-queue slot it took
+ * at capture time and its last CTA resets it, so replays in stream order are
+ * correct; replays that may overlap on the GPU need separate captures.
  */
 int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
              int B, int H, int N, int d, int causal, float scale,

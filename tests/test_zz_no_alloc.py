@@ -99,3 +99,61 @@ def test_noalloc_rejects_bad_arguments_like_attn_fwd():
     o = torch.zeros_like(q)
     assert _noalloc_call(lib, q, q, q, o, lse, False, 0.1) == -2  # d = 80 is unsupported
     assert tab.last_device_error() == 0
+
+
+@pytest.mark.parametrize("causal,d", [(True, 128), (False, 128), (False, 256)])
+def test_noalloc_captured_in_a_cuda_graph(causal, d):
+    """attn_fwd_noalloc inside stream capture (torch.cuda.graph, global
+    capture mode): after a first call on the device, the call captures a
+    memset of the scratch counter and the kernel, and each replay on new
+    contents of the same buffers equals attn_fwd bitwise."""
+    B, H, N = 1, 4, 1000
+    scale = 1.0 / math.sqrt(d)
+    q, k, v = (t.cuda() for t in make_qkv(B, H, N, d, seed=900 + d))
+    o = torch.empty_like(q)
+    lse = torch.empty((B, H, N), dtype=torch.float32, device="cuda")
+    lib = tab.library()
+    assert _noalloc_call(lib, q, k, v, o, lse, causal, scale) == 0  # first call: device set-up
+    torch.cuda.synchronize()
+    assert tab.last_device_error() == 0
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        rc = _noalloc_call(lib, q, k, v, o, lse, causal, scale)
+    assert rc == 0
+    for trial in range(3):
+        qn, kn, vn = make_qkv(B, H, N, d, seed=910 + d + trial)
+        q.copy_(qn)
+        k.copy_(kn)
+        v.copy_(vn)
+        o.fill_(float("nan"))
+        graph.replay()
+        torch.cuda.synchronize()
+        assert tab.last_device_error() == 0
+        o_ref, l_ref = tab.attn_fwd(q, k, v, causal=causal, scale=scale)
+        assert torch.equal(o, o_ref) and torch.equal(lse, l_ref), f"replay {trial}"
+    del graph
+
+
+def test_attn_fwd_captured_in_a_cuda_graph():
+    """attn_fwd itself also captures after a first call on the device: the
+    launch takes its work-queue slot at capture time, every replay reuses
+    it, and the launch's last CTA resets it, so replays in stream order stay
+    correct (bitwise equal to eager calls)."""
+    B, H, N, d, causal = 2, 4, 2048, 128, True
+    q, k, v = (t.cuda() for t in make_qkv(B, H, N, d, seed=930))
+    o = torch.empty_like(q)
+    lse = torch.empty((B, H, N), dtype=torch.float32, device="cuda")
+    tab.attn_fwd_into(q, k, v, o, lse, causal=causal)
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        tab.attn_fwd_into(q, k, v, o, lse, causal=causal)
+    for trial in range(3):
+        for dst, src in zip((q, k, v), make_qkv(B, H, N, d, seed=931 + trial)):
+            dst.copy_(src)
+        graph.replay()
+        torch.cuda.synchronize()
+        assert tab.last_device_error() == 0
+        o_ref, l_ref = tab.attn_fwd(q, k, v, causal=causal)
+        assert torch.equal(o, o_ref) and torch.equal(lse, l_ref), f"replay {trial}"
+    del graph
